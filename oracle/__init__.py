@@ -1,0 +1,227 @@
+"""CPU oracle for the co-activation dispatch/combine path (numpy front end).
+
+TEST INFRASTRUCTURE ONLY: imported by the tests, by the smoke check and by the
+benchmark's CPU-baseline leg -- never by the library.  The arithmetic lives in
+`coact_oracle.c` (plain single-threaded C, compiled here with gcc); this module only
+allocates numpy arrays and marshals them.  It shares no code with the CUDA library.
+
+Parity pins: see tests/test_oracle_pins.py.  Each function below names the page
+passage its definition follows (in the C source).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "coact_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+FLAG_ID_RANGE, FLAG_DUP_ID, FLAG_CAPACITY, FLAG_SRC_RANK = 1, 2, 4, 8
+N_STATS = 8
+STAT_NAMES = ("naive_rows", "dedup_rows", "remote_rows", "crossnode_rows",
+              "node_dedup_crossnode_rows", "local_served_asg", "remote_asg", "crossnode_asg")
+
+
+def build(force: bool = False) -> str:
+    """Compile coact_oracle.c into liboracle.so (plain gcc, no fast-math, no FP contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-Wall", "-ffp-contract=off",
+                               "-fno-fast-math", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _get():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I64, I32 = ctypes.c_int64, ctypes.c_int
+            _lib.oracle_count.argtypes = [P, I64, I32, I32, P, P]
+            _lib.oracle_count_cross.argtypes = [P, I32, I32, P, I32, I32, I64, P, P]
+            _lib.oracle_plan.argtypes = [P, I64, I32, I32, P, I32, P, I32, P, P, P, P, P, P, P,
+                                         I64, P, P, P, P]
+            _lib.oracle_gather.argtypes = [P, I64, P, I64, P]
+            _lib.oracle_gather.restype = None
+            _lib.oracle_combine_f64.argtypes = [P, I64, P, P, I64, I32, I64, P]
+            _lib.oracle_combine_f64.restype = None
+            _lib.oracle_combine_f32chain.argtypes = [P, I64, P, P, I64, I32, I64, P]
+            _lib.oracle_combine_f32chain.restype = None
+            _lib.oracle_bf16_rne_array.argtypes = [P, P, I64]
+            _lib.oracle_bf16_rne_array.restype = None
+            _lib.oracle_expand_identity.argtypes = [P, I64, P, P, I64, P]
+            _lib.oracle_expand_identity.restype = I64
+            _lib.oracle_naive_combine_identity_f32.argtypes = [P, P, I64, I32, I64, P]
+            _lib.oracle_naive_combine_identity_f32.restype = None
+            _lib.oracle_predict_home.argtypes = [P, I64, I32, I32, P, I32, P, I32, P]
+        return _lib
+
+
+def _p(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(np.asarray(a), dtype=dtype)
+
+
+def _bits(a) -> np.ndarray:
+    """bf16 data as uint16 bit patterns (accepts uint16/int16 numpy or a torch bf16 tensor)."""
+    if hasattr(a, "view") and hasattr(a, "dtype") and str(a.dtype) == "torch.bfloat16":
+        import torch
+        return a.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    a = np.asarray(a)
+    if a.dtype == np.int16:
+        a = a.view(np.uint16)
+    return np.ascontiguousarray(a, dtype=np.uint16)
+
+
+# ----------------------------------------------------------------------------- counting
+
+
+def count(ids, E: int, pair=None, loads=None):
+    """Co-activation pair counts [E,E] and loads [E] (int64, accumulated).  Returns
+    (pair, loads, flags)."""
+    ids = _c(ids, np.int32)
+    N, k = ids.shape
+    pair = np.zeros((E, E), np.int64) if pair is None else pair
+    loads = np.zeros(E, np.int64) if loads is None else loads
+    f = _get().oracle_count(_p(ids), N, k, E, _p(pair), _p(loads))
+    return pair, loads, f
+
+
+def count_cross(ids1, E1: int, ids2, E2: int, C12=None, loads1=None):
+    """Cross-layer counts C12 [E1,E2] and layer-1 loads (int64, accumulated)."""
+    ids1, ids2 = _c(ids1, np.int32), _c(ids2, np.int32)
+    N, k1 = ids1.shape
+    k2 = ids2.shape[1]
+    C12 = np.zeros((E1, E2), np.int64) if C12 is None else C12
+    loads1 = np.zeros(E1, np.int64) if loads1 is None else loads1
+    f = _get().oracle_count_cross(_p(ids1), k1, E1, _p(ids2), k2, E2, N, _p(C12), _p(loads1))
+    return C12, loads1, f
+
+
+# ----------------------------------------------------------------------------- plan
+
+
+def plan(ids, E: int, expert_rank, R: int, rank_node=None, n_nodes: int = 1, src_rank=None,
+         row_capacity: Optional[int] = None) -> dict:
+    """Deduplicated dispatch plan; returns a dict of numpy arrays plus 'flags' and 'D'."""
+    ids = _c(ids, np.int32)
+    N, k = ids.shape
+    er = _c(expert_rank, np.int32)
+    rn = None if rank_node is None else _c(rank_node, np.int32)
+    sr = None if src_rank is None else _c(src_rank, np.int32)
+    cap = N * min(k, R) if row_capacity is None else int(row_capacity)
+    out = {
+        "rank_counts": np.zeros(R, np.int32),
+        "rank_offsets": np.zeros(R + 1, np.int32),
+        "asg_offsets": np.zeros(R + 1, np.int32),
+        "rank_mask": np.zeros(N, np.uint64),
+        "row_token": np.full(max(cap, 0), -1, np.int32),
+        "row_kmask": np.zeros(max(cap, 0), np.uint8),
+        "send_row": np.zeros((N, k), np.int32),
+        "comb_row": np.zeros((N, k), np.int32),
+        "stats": np.zeros(N_STATS, np.int64),
+        "src_dst": np.zeros((R, R), np.int32),
+    }
+    f = _get().oracle_plan(_p(ids), N, k, E, _p(er), R, _p(rn), n_nodes, _p(sr),
+                           _p(out["rank_counts"]), _p(out["rank_offsets"]),
+                           _p(out["asg_offsets"]), _p(out["rank_mask"]), _p(out["row_token"]),
+                           _p(out["row_kmask"]), cap, _p(out["send_row"]), _p(out["comb_row"]),
+                           _p(out["stats"]), _p(out["src_dst"]))
+    out["flags"] = f
+    out["D"] = int(out["rank_offsets"][R])
+    out["row_capacity"] = cap
+    return out
+
+
+# ----------------------------------------------------------------------------- rows
+
+
+def gather(x, row_token, D: int) -> np.ndarray:
+    """send[d] = x[row_token[d]] for d < D (uint16 bf16 bits [D, H])."""
+    xb = _bits(x)
+    H = xb.shape[1]
+    rt = _c(row_token, np.int32)
+    send = np.zeros((D, H), np.uint16)
+    _get().oracle_gather(_p(xb), H, _p(rt), D, _p(send))
+    return send
+
+
+def combine_f64(y, gates, comb_row) -> np.ndarray:
+    """out[t] = sum_j gate[t,j] * y[comb_row[t,j]] in float64 ([N, H])."""
+    yb = _bits(y)
+    g = _c(gates, np.float32)
+    cr = _c(comb_row, np.int32)
+    N, k = g.shape
+    H = yb.shape[1]
+    out = np.zeros((N, H), np.float64)
+    _get().oracle_combine_f64(_p(yb), yb.shape[0], _p(g), _p(cr), N, k, H, _p(out))
+    return out
+
+
+def combine_f32chain(y, gates, comb_row) -> np.ndarray:
+    """The fixed-order fp32 fma chain (ascending j from +0) ([N, H] float32)."""
+    yb = _bits(y)
+    g = _c(gates, np.float32)
+    cr = _c(comb_row, np.int32)
+    N, k = g.shape
+    H = yb.shape[1]
+    out = np.zeros((N, H), np.float32)
+    _get().oracle_combine_f32chain(_p(yb), yb.shape[0], _p(g), _p(cr), N, k, H, _p(out))
+    return out
+
+
+def bf16_rne(a) -> np.ndarray:
+    """float32 -> bf16 bits, round to nearest even (the oracle's own definition)."""
+    a = _c(a, np.float32)
+    out = np.zeros(a.shape, np.uint16)
+    _get().oracle_bf16_rne_array(_p(a), _p(out), a.size)
+    return out
+
+
+def expand_identity(x, row_token, row_kmask, D: int) -> np.ndarray:
+    """Identity-expert outputs in expanded receive order ([sum popcount(row_kmask[:D]), H])."""
+    xb = _bits(x)
+    H = xb.shape[1]
+    rt = _c(row_token, np.int32)
+    km = _c(row_kmask, np.uint8)
+    n = int(sum(bin(int(v)).count("1") for v in km[:D]))
+    y = np.zeros((n, H), np.uint16)
+    got = _get().oracle_expand_identity(_p(xb), H, _p(rt), _p(km), D, _p(y))
+    assert got == n
+    return y
+
+
+def naive_combine_identity_f32(x, gates) -> np.ndarray:
+    """Non-deduplicated combine with identity experts (fp32 chain), [N, H] float32."""
+    xb = _bits(x)
+    g = _c(gates, np.float32)
+    N, k = g.shape
+    H = xb.shape[1]
+    out = np.zeros((N, H), np.float32)
+    _get().oracle_naive_combine_identity_f32(_p(xb), _p(g), N, k, H, _p(out))
+    return out
+
+
+def predict_home(ids1, E1: int, C12, expert_rank2, R: int):
+    """Predicted layer-2 home rank per token (int32 [N]) and flags."""
+    ids1 = _c(ids1, np.int32)
+    N, k1 = ids1.shape
+    C = _c(C12, np.int64)
+    E2 = C.shape[1]
+    er2 = _c(expert_rank2, np.int32)
+    home = np.zeros(N, np.int32)
+    f = _get().oracle_predict_home(_p(ids1), N, k1, E1, _p(C), E2, _p(er2), R, _p(home))
+    return home, f

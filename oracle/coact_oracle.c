@@ -1,0 +1,389 @@
+/*
+ * coact_oracle.c -- plain, slow, single-threaded CPU oracle for the co-activation
+ * dispatch/combine path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or load this
+ * file: only the tests, the smoke check and the benchmark's CPU-baseline leg use it.
+ * It shares no code, header, table or helper with the CUDA library.
+ *
+ * Every function is the plain definition of what the method computes, written as
+ * straight loops, with no blocking, fusion or reordering.  Sources (web pages):
+ *   [Cobalt]  "Cobalt: efficient distributed MoE training using expert co-activation"
+ *             (arxivdaily 2609.36959), English abstract: expert pairs co-activated by
+ *             single tokens; per-expert workload statistics; routing tokens to fewer
+ *             remote nodes; all-to-all token exchange under EP.
+ *   [Zyphra]  correlated expert placement / token shuffling (arxivdaily 2610.09372),
+ *             English abstract: "a dispatcher that sends each token to each GPU once",
+ *             dispatch then combine, expert pairs selected together, next-layer
+ *             prediction, locally served token--expert assignments, and routing
+ *             decisions left unchanged by both methods.
+ * Where the pages leave a step open, the reading taken is stated at the function.
+ *
+ * Floating point: the pages fix no precision.  The combine reference is computed in
+ * float64 (oracle_combine_f64).  oracle_combine_f32chain additionally spells out the
+ * fixed-order fp32 accumulation the library specifies (acc = fma(g_j, y_j, acc) for
+ * j = 0..k-1 from +0), so that order can be checked bit for bit.
+ *
+ * Error flags returned (bit-or): 1 = expert id out of range, 2 = repeated id within a
+ * token, 4 = row capacity exceeded, 8 = source rank out of range.  A token with an
+ * invalid id or source rank is skipped entirely (it contributes nothing).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OF_ID_RANGE 1
+#define OF_DUP_ID 2
+#define OF_CAPACITY 4
+#define OF_SRC_RANK 8
+
+/* Flags for token t: ids in [0,E) and pairwise distinct. */
+static int token_flags(const int32_t *ids, int64_t t, int k, int E) {
+    int f = 0;
+    for (int j = 0; j < k; ++j) {
+        int32_t a = ids[t * k + j];
+        if (a < 0 || a >= E) f |= OF_ID_RANGE;
+        for (int jj = 0; jj < j; ++jj)
+            if (ids[t * k + jj] == a) f |= OF_DUP_ID;
+    }
+    return f;
+}
+
+/*
+ * Co-activation pair counts and per-expert loads.
+ * [Cobalt] "many pairs of experts are frequently co-activated by individual tokens";
+ * "per-expert workload statistics".  [Zyphra] "expert pairs ... selected together".
+ *   pair[a*E+b] += #{t : a and b both among token t's k experts, a != b}
+ *   loads[e]    += #{(t,j) : ids[t,j] == e}
+ * Reading: unordered distinct pairs, so the E x E matrix is symmetric with a zero
+ * diagonal and its strict upper triangle gains N*k*(k-1)/2; loads are kept apart.
+ * Counts accumulate into the caller's arrays.  loads may be NULL.
+ */
+int oracle_count(const int32_t *ids, int64_t N, int k, int E, int64_t *pair, int64_t *loads) {
+    int flags = 0;
+    for (int64_t t = 0; t < N; ++t) {
+        int f = token_flags(ids, t, k, E);
+        flags |= f;
+        if (f) continue;
+        for (int j = 0; j < k; ++j) {
+            int32_t a = ids[t * k + j];
+            if (loads) loads[a] += 1;
+            for (int jj = 0; jj < k; ++jj) {
+                if (jj == j) continue;
+                int32_t b = ids[t * k + jj];
+                pair[(int64_t)a * E + b] += 1;
+            }
+        }
+    }
+    return flags;
+}
+
+/*
+ * Cross-layer counts.  [Zyphra] "the experts a token selects at one layer predict the
+ * experts it selects at the next layer".
+ *   C12[a*E2+b] += #{(t,j,j') : ids1[t,j] == a, ids2[t,j'] == b}
+ * Not symmetric; a == b is a legitimate entry.  loads1 (may be NULL) gains the
+ * layer-1 loads.  A token is skipped if either layer's ids are invalid.
+ */
+int oracle_count_cross(const int32_t *ids1, int k1, int E1, const int32_t *ids2, int k2, int E2,
+                       int64_t N, int64_t *C12, int64_t *loads1) {
+    int flags = 0;
+    for (int64_t t = 0; t < N; ++t) {
+        int f = token_flags(ids1, t, k1, E1) | token_flags(ids2, t, k2, E2);
+        flags |= f;
+        if (f) continue;
+        for (int j = 0; j < k1; ++j) {
+            int32_t a = ids1[t * k1 + j];
+            if (loads1) loads1[a] += 1;
+            for (int jj = 0; jj < k2; ++jj) C12[(int64_t)a * E2 + ids2[t * k2 + jj]] += 1;
+        }
+    }
+    return flags;
+}
+
+/*
+ * Deduplicated dispatch plan.  [Zyphra] "a dispatcher that sends each token to each
+ * GPU once" (rows), [Cobalt] "routes tokens to fewer remote nodes" (node statistics)
+ * and all-to-all exchange of tokens under EP.
+ *
+ * Inputs: ids [N,k]; expert_rank [E] (expert -> logical rank); rank_node [R] (rank ->
+ * node, NULL = one node); src_rank [N] (token's home rank, NULL = contiguous shards
+ * floor(t*R/N)).
+ * Definitions (rank(j) = expert_rank[ids[t,j]]):
+ *   rank_mask[t]  = OR_j 1<<rank(j)
+ *   kmask(t,r)    = OR_{j : rank(j) == r} 1<<j        (mask over the token's k slots)
+ *   rank_counts[r]= #{t : r in rank_mask[t]}           (rows sent to r)
+ *   asg(r)        = sum_t popcount(kmask(t,r))         (token-expert assignments on r)
+ *   rank_offsets / asg_offsets = exclusive prefix sums over r, with totals at [R]
+ * Row order inside rank r's segment: ascending token index (reading: "stable"; with
+ * contiguous source shards this is the all-to-all receive order).  Walking r = 0..R-1
+ * and t = 0..N-1:
+ *   row_token[pos] = t, row_kmask[pos] = kmask(t,r)   (pos < row_capacity; else flag 4)
+ *   send_row[t,j]  = pos for the smallest slot j with rank(j) == r, -1 for r's other slots
+ *   comb_row[t,j]  = next assignment row of r, slots in ascending j
+ * so the expert outputs sit in "expanded receive order": rank segments, send rows in
+ * order, one row per set slot in ascending j.
+ * Statistics (int64 [8]):
+ *   0 naive rows N*k          1 dedup rows D = rank_offsets[R]
+ *   2 remote rows     = sum_t popcount(rank_mask[t] without src[t])
+ *   3 cross-node rows = sum_t #{r in rank_mask[t] : node(r) != node(src[t])}
+ *   4 node-dedup cross-node rows = sum_t #{nodes n != node(src[t]) touched by t}
+ *   5 local-served assignments = #{(t,j) : rank(j) == src[t]}
+ *   6 remote assignments = N*k - stat5
+ *   7 cross-node assignments = #{(t,j) : node(rank(j)) != node(src[t])}
+ * src_dst [R*R] (may be NULL): src_dst[s*R+r] = #{t : src[t] == s, r in rank_mask[t]}.
+ * rank_mask [N] (may be NULL) is written as uint64.
+ * Invalid tokens (bad id, repeated id, bad expert_rank entry, bad src) contribute
+ * nothing; their send_row / comb_row entries are -1.
+ */
+int oracle_plan(const int32_t *ids, int64_t N, int k, int E, const int32_t *expert_rank, int R,
+                const int32_t *rank_node, int n_nodes, const int32_t *src_rank,
+                int32_t *rank_counts, int32_t *rank_offsets, int32_t *asg_offsets,
+                uint64_t *rank_mask_out, int32_t *row_token, uint8_t *row_kmask,
+                int64_t row_capacity, int32_t *send_row, int32_t *comb_row, int64_t *stats,
+                int32_t *src_dst) {
+    int flags = 0;
+    (void)n_nodes;
+    for (int64_t i = 0; i < N * k; ++i) { send_row[i] = -1; comb_row[i] = -1; }
+    for (int s = 0; s < 8; ++s) stats[s] = 0;
+    if (src_dst) for (int64_t i = 0; i < (int64_t)R * R; ++i) src_dst[i] = 0;
+
+    /* per-token source rank and validity (an invalid token contributes nothing) */
+    int64_t *src = (int64_t *)malloc((size_t)(N > 0 ? N : 1) * sizeof(int64_t));
+    char *valid = (char *)malloc((size_t)(N > 0 ? N : 1));
+    for (int64_t t = 0; t < N; ++t) {
+        int f = token_flags(ids, t, k, E);
+        src[t] = src_rank ? src_rank[t] : (t * R) / N;
+        if (!(f & OF_ID_RANGE))
+            for (int j = 0; j < k; ++j) {
+                int32_t r = expert_rank[ids[t * k + j]];
+                if (r < 0 || r >= R) f |= OF_ID_RANGE;
+            }
+        if (src[t] < 0 || src[t] >= R) f |= OF_SRC_RANK;
+        flags |= f;
+        valid[t] = (char)(f == 0);
+        uint64_t m = 0;
+        if (valid[t])
+            for (int j = 0; j < k; ++j) m |= 1ull << expert_rank[ids[t * k + j]];
+        if (rank_mask_out) rank_mask_out[t] = m;
+    }
+
+    /* counts and exclusive offsets, by a loop over r */
+    int64_t row_acc = 0, asg_acc = 0;
+    for (int r = 0; r < R; ++r) {
+        int64_t rows = 0, asg = 0;
+        for (int64_t t = 0; t < N; ++t) {
+            if (!valid[t]) continue;
+            int in = 0;
+            for (int j = 0; j < k; ++j)
+                if (expert_rank[ids[t * k + j]] == r) { in = 1; asg += 1; }
+            rows += in;
+        }
+        rank_counts[r] = (int32_t)rows;
+        rank_offsets[r] = (int32_t)row_acc;
+        asg_offsets[r] = (int32_t)asg_acc;
+        row_acc += rows;
+        asg_acc += asg;
+    }
+    rank_offsets[R] = (int32_t)row_acc;
+    asg_offsets[R] = (int32_t)asg_acc;
+
+    /* stable positions: walk ranks, then tokens in ascending order */
+    for (int r = 0; r < R; ++r) {
+        int64_t pos = rank_offsets[r];
+        int64_t apos = asg_offsets[r];
+        for (int64_t t = 0; t < N; ++t) {
+            if (!valid[t]) continue;
+            uint32_t km = 0;
+            for (int j = 0; j < k; ++j)
+                if (expert_rank[ids[t * k + j]] == r) km |= 1u << j;
+            if (!km) continue;
+            int first = 1;
+            for (int j = 0; j < k; ++j) {
+                if (!(km & (1u << j))) continue;
+                if (first) {
+                    send_row[t * k + j] = pos < row_capacity ? (int32_t)pos : -1;
+                    first = 0;
+                }
+                comb_row[t * k + j] = (int32_t)apos;
+                apos += 1;
+            }
+            if (pos < row_capacity) {
+                row_token[pos] = (int32_t)t;
+                row_kmask[pos] = (uint8_t)km;
+            } else {
+                flags |= OF_CAPACITY;
+            }
+            if (src_dst) src_dst[src[t] * R + r] += 1;
+            pos += 1;
+        }
+    }
+
+    /* statistics, from the sets of ranks and nodes each token touches */
+    stats[0] = N * (int64_t)k;
+    stats[1] = row_acc;
+    for (int64_t t = 0; t < N; ++t) {
+        if (!valid[t]) continue;
+        char rank_set[64] = {0}, node_set[64] = {0};
+        int node_src = rank_node ? rank_node[src[t]] : 0;
+        for (int j = 0; j < k; ++j) {
+            int32_t r = expert_rank[ids[t * k + j]];
+            int nd = rank_node ? rank_node[r] : 0;
+            rank_set[r] = 1;
+            node_set[nd] = 1;
+            if (r == src[t]) stats[5] += 1;
+            if (nd != node_src) stats[7] += 1;
+        }
+        for (int r = 0; r < R; ++r) {
+            if (!rank_set[r]) continue;
+            if (r != src[t]) stats[2] += 1;
+            if ((rank_node ? rank_node[r] : 0) != node_src) stats[3] += 1;
+        }
+        for (int nd = 0; nd < 64; ++nd)
+            if (node_set[nd] && nd != node_src) stats[4] += 1;
+    }
+    stats[6] = asg_acc - stats[5];   /* every assignment of a valid token that is not local */
+    free(src);
+    free(valid);
+    return flags;
+}
+
+/* Gathered send buffer: send[d] = x[row_token[d]] for d < D (bf16 rows copied as bits). */
+void oracle_gather(const uint16_t *x, int64_t H, const int32_t *row_token, int64_t D,
+                   uint16_t *send) {
+    for (int64_t d = 0; d < D; ++d)
+        memcpy(send + d * H, x + (int64_t)row_token[d] * H, (size_t)H * sizeof(uint16_t));
+}
+
+/* bf16 bits -> float: the bf16 pattern is the top half of the float32 pattern. */
+static float bf16_to_f32(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/*
+ * float32 -> bf16, IEEE round to nearest, ties to even, from the definition: keep
+ * the top 16 bits; look at the 16 dropped bits; round up if they exceed half an ulp,
+ * or equal half an ulp and the kept part is odd.  A carry out of the mantissa rolls
+ * into the exponent (and up to infinity), which is the correct IEEE result.  NaN
+ * stays NaN (quiet bit set).
+ */
+uint16_t oracle_bf16_rne(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu))
+        return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t kept = u >> 16;
+    uint32_t dropped = u & 0xffffu;
+    if (dropped > 0x8000u || (dropped == 0x8000u && (kept & 1u))) kept += 1;
+    return (uint16_t)kept;
+}
+
+void oracle_bf16_rne_array(const float *in, uint16_t *out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_rne(in[i]);
+}
+
+/*
+ * Weighted combine in float64.  [Zyphra] dispatch tokens to their experts "and then
+ * combine the results":
+ *   out[t][h] = sum_j gate[t,j] * y[comb_row[t,j]][h]
+ * y is bf16 [n_rows, H] in expanded receive order.  Rows with comb_row < 0 or
+ * >= n_rows are skipped (invalid tokens).
+ */
+void oracle_combine_f64(const uint16_t *y, int64_t n_rows, const float *gates,
+                        const int32_t *comb_row, int64_t N, int k, int64_t H, double *out) {
+    for (int64_t t = 0; t < N; ++t)
+        for (int64_t h = 0; h < H; ++h) {
+            double acc = 0.0;
+            for (int j = 0; j < k; ++j) {
+                int64_t row = comb_row[t * k + j];
+                if (row < 0 || row >= n_rows) continue;
+                acc += (double)gates[t * k + j] * (double)bf16_to_f32(y[row * H + h]);
+            }
+            out[t * H + h] = acc;
+        }
+}
+
+/*
+ * The library's specified fp32 accumulation, spelled out: acc starts at +0.0f and
+ * takes one fused multiply-add per slot in ascending j (C99 fmaf: one rounding).
+ */
+void oracle_combine_f32chain(const uint16_t *y, int64_t n_rows, const float *gates,
+                             const int32_t *comb_row, int64_t N, int k, int64_t H, float *out) {
+    for (int64_t t = 0; t < N; ++t)
+        for (int64_t h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int j = 0; j < k; ++j) {
+                int64_t row = comb_row[t * k + j];
+                if (row < 0 || row >= n_rows) continue;
+                acc = fmaf(gates[t * k + j], bf16_to_f32(y[row * H + h]), acc);
+            }
+            out[t * H + h] = acc;
+        }
+}
+
+/*
+ * Expert outputs of *identity* experts in expanded receive order: for each send row d
+ * in order and each set slot of row_kmask[d] in ascending order, one copy of
+ * x[row_token[d]].  Returns the number of rows written.
+ */
+int64_t oracle_expand_identity(const uint16_t *x, int64_t H, const int32_t *row_token,
+                               const uint8_t *row_kmask, int64_t D, uint16_t *y) {
+    int64_t a = 0;
+    for (int64_t d = 0; d < D; ++d)
+        for (int j = 0; j < 8; ++j)
+            if (row_kmask[d] & (1u << j)) {
+                memcpy(y + a * H, x + (int64_t)row_token[d] * H, (size_t)H * sizeof(uint16_t));
+                a += 1;
+            }
+    return a;
+}
+
+/*
+ * Naive (non-deduplicated) combine with identity experts: one row per (t,j), so
+ * every slot's output is x[t]; same fp32 chain as above.  [Zyphra] "neither method
+ * changes the models' underlying routing decisions": the deduplicated combine must
+ * equal this bit for bit.
+ */
+void oracle_naive_combine_identity_f32(const uint16_t *x, const float *gates, int64_t N, int k,
+                                       int64_t H, float *out) {
+    for (int64_t t = 0; t < N; ++t)
+        for (int64_t h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int j = 0; j < k; ++j) acc = fmaf(gates[t * k + j], bf16_to_f32(x[t * H + h]), acc);
+            out[t * H + h] = acc;
+        }
+}
+
+/*
+ * Token shuffling's home prediction.  [Zyphra] each token moves "to the GPU predicted
+ * to hold its next-layer experts".  Reading: score(t,r) = sum over the token's layer-1
+ * experts a of the calibration counts C12[a][b] summed over the layer-2 experts b
+ * placed on rank r; the predicted home is the rank with the largest score, ties to the
+ * lowest rank.  Tokens with invalid ids get home -1 and flag 1/2.
+ */
+int oracle_predict_home(const int32_t *ids1, int64_t N, int k1, int E1, const int64_t *C12,
+                        int E2, const int32_t *expert_rank2, int R, int32_t *home) {
+    int flags = 0;
+    for (int64_t t = 0; t < N; ++t) {
+        int f = token_flags(ids1, t, k1, E1);
+        flags |= f;
+        if (f) { home[t] = -1; continue; }
+        int best = 0;
+        int64_t best_score = -1;
+        for (int r = 0; r < R; ++r) {
+            int64_t score = 0;
+            for (int j = 0; j < k1; ++j) {
+                int32_t a = ids1[t * k1 + j];
+                for (int b = 0; b < E2; ++b)
+                    if (expert_rank2[b] == r) score += C12[(int64_t)a * E2 + b];
+            }
+            if (score > best_score) { best_score = score; best = r; }
+        }
+        home[t] = best;
+    }
+    return flags;
+}
