@@ -1,0 +1,274 @@
+"""Python binding of libcoact.so, the B200 co-activation dispatch/combine library.
+
+Thin marshalling only: every entry point takes torch CUDA tensors, checks dtype /
+shape / contiguity, and passes data pointers and the current CUDA stream to the C ABI
+declared in include/coact.h.  All computation happens in the library's CUDA kernels;
+there is no CPU fallback, and importing this module fails loudly if the library has
+not been built (python co_activation_b200/build.py).
+
+Entry points (same names as the C ABI):
+  coact_count, plan_dispatch, dispatch_gather, combine_scatter, predict_home
+plus allocation helpers (`alloc_plan`, `plan_workspace`) that only create torch tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.environ.get("COACT_LIB", os.path.join(_PKG, "libcoact.so"))
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libcoact.so not found at {LIB_PATH}: build it first with "
+        "`python co_activation_b200/build.py` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+EFLAG_ID_RANGE, EFLAG_DUP_ID, EFLAG_CAPACITY, EFLAG_SRC_RANK, EFLAG_ROW_RANGE, EFLAG_TIMEOUT = (
+    1, 2, 4, 8, 16, 32)
+NUM_STATS = 8
+STAT_NAMES = ("naive_rows", "dedup_rows", "remote_rows", "crossnode_rows",
+              "node_dedup_crossnode_rows", "local_served_asg", "remote_asg", "crossnode_asg")
+MAX_K, MAX_E, MAX_R = 8, 1024, 64
+
+_P, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+_lib.coact_strerror.argtypes = [_I32]
+_lib.coact_strerror.restype = ctypes.c_char_p
+_lib.coact_abi_version.restype = _I32
+_lib.coact_count.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _I32, _P, _P, _P, _P]
+_lib.plan_dispatch_workspace_bytes.argtypes = [_I64, _I32, _I32, _I32]
+_lib.plan_dispatch_workspace_bytes.restype = _SZ
+_lib.plan_dispatch.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _P, _P, _P, _P,
+                               _P, _I64, _P, _P, _P, _P, _P, _SZ, _P, _P]
+_lib.dispatch_gather.argtypes = [_P, _I64, _I64, _P, _I32, _P, _I64, _P, _P]
+_lib.combine_scatter.argtypes = [_P, _I64, _P, _P, _I64, _I32, _I64, _P, _I32, _P, _P]
+_lib.predict_home_workspace_bytes.argtypes = [_I32, _I32]
+_lib.predict_home_workspace_bytes.restype = _SZ
+_lib.predict_home.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _SZ, _P, _P]
+for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "combine_scatter", "predict_home"):
+    getattr(_lib, _f).restype = _I32
+
+ABI_SYMBOLS = ("coact_strerror", "coact_abi_version", "coact_count", "plan_dispatch_workspace_bytes",
+               "plan_dispatch", "dispatch_gather", "combine_scatter",
+               "predict_home_workspace_bytes", "predict_home")
+
+
+class CoactError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {_lib.coact_strerror(status).decode()} (status {status})")
+        self.status = status
+
+
+def abi_version() -> int:
+    return _lib.coact_abi_version()
+
+
+def strerror(status: int) -> str:
+    return _lib.coact_strerror(status).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise CoactError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _need(t: Optional[torch.Tensor], name: str, dtype, shape=None, optional=False):
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _bits16(t: torch.Tensor) -> torch.Tensor:
+    """bf16 tensors are passed by bit pattern (uint16 in the ABI)."""
+    if t.dtype != torch.bfloat16:
+        raise ValueError(f"expected a bfloat16 tensor, got {t.dtype}")
+    return t
+
+
+# ----------------------------------------------------------------------------- entry points
+
+
+def coact_count(ids: torch.Tensor, E: int, pair: torch.Tensor, loads: Optional[torch.Tensor] = None,
+                ids2: Optional[torch.Tensor] = None, E2: Optional[int] = None,
+                err_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    """pair[a,b] += tokens selecting both a and b (a != b); loads[e] += selections of e.
+    Cross mode (ids2 given): pair[a,b] += slot pairs with ids[t,.] == a, ids2[t,.] == b."""
+    N, k = ids.shape
+    _need(ids, "ids", torch.int32)
+    if ids2 is None:
+        _need(pair, "pair", torch.int64, (E, E))
+        k2, E2_ = 0, 0
+    else:
+        if E2 is None:
+            raise ValueError("E2 is required with ids2")
+        _need(ids2, "ids2", torch.int32)
+        if ids2.shape[0] != N:
+            raise ValueError("ids and ids2 must have the same number of tokens")
+        _need(pair, "pair", torch.int64, (E, E2))
+        k2, E2_ = ids2.shape[1], E2
+    _need(loads, "loads", torch.int64, (E,), optional=True)
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.coact_count(_ptr(ids), N, k, E, _ptr(ids2), k2, E2_, _ptr(pair), _ptr(loads),
+                            _ptr(err_flag), _stream(stream)), "coact_count")
+
+
+def plan_workspace_bytes(N: int, k: int, E: int, R: int) -> int:
+    return int(_lib.plan_dispatch_workspace_bytes(N, k, E, R))
+
+
+@dataclasses.dataclass
+class Plan:
+    """Output buffers of plan_dispatch (torch CUDA tensors)."""
+    rank_counts: torch.Tensor
+    rank_offsets: torch.Tensor
+    asg_offsets: torch.Tensor
+    rank_mask: Optional[torch.Tensor]
+    row_token: torch.Tensor
+    row_kmask: torch.Tensor
+    send_row: torch.Tensor
+    comb_row: torch.Tensor
+    stats: torch.Tensor
+    src_dst: Optional[torch.Tensor]
+    workspace: torch.Tensor
+
+    @property
+    def row_capacity(self) -> int:
+        return self.row_token.shape[0]
+
+
+def alloc_plan(N: int, k: int, E: int, R: int, device="cuda", row_capacity: Optional[int] = None,
+               with_rank_mask: bool = True, with_src_dst: bool = True) -> Plan:
+    """Allocates plan_dispatch's outputs and workspace.  row_capacity defaults to
+    N*min(k, R), the size that can never overflow."""
+    cap = N * min(k, R) if row_capacity is None else int(row_capacity)
+    dev = torch.device(device)
+    i32 = dict(dtype=torch.int32, device=dev)
+    ws = torch.empty(max(plan_workspace_bytes(N, k, E, R), 16), dtype=torch.uint8, device=dev)
+    return Plan(rank_counts=torch.empty(R, **i32), rank_offsets=torch.empty(R + 1, **i32),
+                asg_offsets=torch.empty(R + 1, **i32),
+                rank_mask=torch.empty(N, dtype=torch.int64, device=dev) if with_rank_mask else None,
+                row_token=torch.empty(cap, **i32),
+                row_kmask=torch.empty(cap, dtype=torch.uint8, device=dev),
+                send_row=torch.empty((N, k), **i32), comb_row=torch.empty((N, k), **i32),
+                stats=torch.empty(NUM_STATS, dtype=torch.int64, device=dev),
+                src_dst=torch.empty((R, R), **i32) if with_src_dst else None, workspace=ws)
+
+
+def plan_dispatch(ids: torch.Tensor, E: int, expert_rank: torch.Tensor, R: int, plan: Plan,
+                  rank_node: Optional[torch.Tensor] = None, n_nodes: int = 1,
+                  src_rank: Optional[torch.Tensor] = None,
+                  err_flag: Optional[torch.Tensor] = None, stream=None) -> Plan:
+    """Deduplicated dispatch layout into `plan`'s buffers (see include/coact.h)."""
+    N, k = ids.shape
+    _need(ids, "ids", torch.int32)
+    _need(expert_rank, "expert_rank", torch.int32, (E,))
+    _need(rank_node, "rank_node", torch.int32, (R,), optional=True)
+    _need(src_rank, "src_rank", torch.int32, (N,), optional=True)
+    _need(plan.rank_counts, "rank_counts", torch.int32, (R,))
+    _need(plan.rank_offsets, "rank_offsets", torch.int32, (R + 1,))
+    _need(plan.asg_offsets, "asg_offsets", torch.int32, (R + 1,))
+    _need(plan.rank_mask, "rank_mask", torch.int64, (N,), optional=True)
+    _need(plan.row_token, "row_token", torch.int32)
+    _need(plan.row_kmask, "row_kmask", torch.uint8, (plan.row_token.shape[0],))
+    _need(plan.send_row, "send_row", torch.int32, (N, k))
+    _need(plan.comb_row, "comb_row", torch.int32, (N, k))
+    _need(plan.stats, "stats", torch.int64, (NUM_STATS,))
+    _need(plan.src_dst, "src_dst", torch.int32, (R, R), optional=True)
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    ws = plan.workspace
+    _check(_lib.plan_dispatch(
+        _ptr(ids), N, k, E, _ptr(expert_rank), R, _ptr(rank_node), n_nodes, _ptr(src_rank),
+        _ptr(plan.rank_counts), _ptr(plan.rank_offsets), _ptr(plan.asg_offsets),
+        _ptr(plan.rank_mask), _ptr(plan.row_token), _ptr(plan.row_kmask), plan.row_capacity,
+        _ptr(plan.send_row), _ptr(plan.comb_row), _ptr(plan.stats), _ptr(plan.src_dst),
+        _ptr(ws), ws.numel() * ws.element_size(), _ptr(err_flag), _stream(stream)),
+        "plan_dispatch")
+    return plan
+
+
+def dispatch_gather(x: torch.Tensor, send_row: torch.Tensor, send: torch.Tensor,
+                    err_flag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """send[send_row[t, j]] = x[t] for every send_row entry >= 0 (bf16 rows)."""
+    N, H = x.shape
+    _need(_bits16(x), "x", torch.bfloat16)
+    _need(send_row, "send_row", torch.int32)
+    if send_row.shape[0] != N:
+        raise ValueError("send_row must have one row per token")
+    _need(_bits16(send), "send", torch.bfloat16)
+    if send.shape[1] != H:
+        raise ValueError("send rows must have x's hidden size")
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.dispatch_gather(_ptr(x), N, H, _ptr(send_row), send_row.shape[1], _ptr(send),
+                                send.shape[0], _ptr(err_flag), _stream(stream)), "dispatch_gather")
+    return send
+
+
+def combine_scatter(y: torch.Tensor, gates: torch.Tensor, comb_row: torch.Tensor,
+                    out: torch.Tensor, err_flag: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """out[t] = sum_j gates[t,j] * y[comb_row[t,j]] (fp32 fma chain in ascending j;
+    out is bf16 or fp32)."""
+    N, k = gates.shape
+    _need(_bits16(y), "y", torch.bfloat16)
+    H = y.shape[1]
+    _need(gates, "gates", torch.float32)
+    _need(comb_row, "comb_row", torch.int32, (N, k))
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out must be bfloat16 or float32")
+    _need(out, "out", out.dtype, (N, H))
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.combine_scatter(_ptr(y), y.shape[0], _ptr(gates), _ptr(comb_row), N, k, H,
+                                _ptr(out), 1 if out.dtype == torch.float32 else 0,
+                                _ptr(err_flag), _stream(stream)), "combine_scatter")
+    return out
+
+
+def predict_workspace_bytes(E1: int, R: int) -> int:
+    return int(_lib.predict_home_workspace_bytes(E1, R))
+
+
+def predict_home(ids1: torch.Tensor, E1: int, C12: torch.Tensor, expert_rank2: torch.Tensor, R: int,
+                 home: torch.Tensor, workspace: Optional[torch.Tensor] = None,
+                 err_flag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """home[t] = argmax_r sum_j sum_{b on r} C12[ids1[t,j], b] (ties -> lowest r)."""
+    N, k1 = ids1.shape
+    _need(ids1, "ids1", torch.int32)
+    _need(C12, "C12", torch.int64)
+    E2 = C12.shape[1]
+    if C12.shape[0] != E1:
+        raise ValueError("C12 must be [E1, E2]")
+    _need(expert_rank2, "expert_rank2", torch.int32, (E2,))
+    _need(home, "home", torch.int32, (N,))
+    if workspace is None:
+        workspace = torch.empty(max(predict_workspace_bytes(E1, R), 16), dtype=torch.uint8,
+                                device=ids1.device)
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.predict_home(_ptr(ids1), N, k1, E1, _ptr(C12), E2, _ptr(expert_rank2), R,
+                             _ptr(home), _ptr(workspace), workspace.numel(), _ptr(err_flag),
+                             _stream(stream)), "predict_home")
+    return home

@@ -1,0 +1,51 @@
+// Status strings, ABI version and the per-device attribute cache.
+#include "common.cuh"
+
+namespace coact {
+
+namespace {
+std::atomic<int> g_sm_count[kMaxDevices];
+std::atomic<int> g_smem_optin[kMaxDevices];
+std::atomic<int> g_smem_sm[kMaxDevices];
+}  // namespace
+
+int device_info(DeviceInfo *out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return COACT_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return COACT_ERR_CUDA;
+    int sms = g_sm_count[dev].load(std::memory_order_relaxed);
+    int smem = g_smem_optin[dev].load(std::memory_order_relaxed);
+    int smem_sm = g_smem_sm[dev].load(std::memory_order_relaxed);
+    if (sms <= 0 || smem <= 0 || smem_sm <= 0) {
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+                cudaSuccess ||
+            cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+                cudaSuccess)
+            return COACT_ERR_CUDA;
+        g_sm_count[dev].store(sms, std::memory_order_relaxed);
+        g_smem_optin[dev].store(smem, std::memory_order_relaxed);
+        g_smem_sm[dev].store(smem_sm, std::memory_order_relaxed);
+    }
+    out->device = dev;
+    out->sm_count = sms;
+    out->smem_optin = smem;
+    out->smem_per_sm = smem_sm;
+    return COACT_OK;
+}
+
+}  // namespace coact
+
+extern "C" const char *coact_strerror(int status) {
+    switch (status) {
+        case COACT_OK: return "ok";
+        case COACT_ERR_INVALID: return "invalid argument (NULL pointer, negative size or misaligned buffer)";
+        case COACT_ERR_UNSUPPORTED: return "argument outside the supported limits";
+        case COACT_ERR_CUDA: return "CUDA launch or attribute query failed";
+        case COACT_ERR_WORKSPACE: return "workspace missing or too small";
+        case COACT_ERR_TIMEOUT: return "a bounded device wait gave up";
+        default: return "unknown status";
+    }
+}
+
+extern "C" int coact_abi_version(void) { return COACT_ABI_VERSION; }

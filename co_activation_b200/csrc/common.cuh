@@ -1,0 +1,123 @@
+// Internal helpers shared by the library's kernels (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "coact.h"
+
+namespace coact {
+
+constexpr int kWarp = 32;
+
+// ------------------------------------------------------------------ device helpers
+
+__device__ __forceinline__ void raise_flag(int32_t *err, int bits) {
+    if (bits && err) atomicOr(err, bits);
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+    unsigned m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// bf16 bit pattern -> fp32 (exact: bf16 is the top half of an fp32).
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Streaming 16-byte global accesses: data touched once, do not keep it in L1.
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_stream(uint4 *p, const uint4 &v) {
+    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Loads token t's K expert ids (row t of an int32 [N, K] array) and returns the
+// validation bits: COACT_EFLAG_ID_RANGE for an id outside [0, E), COACT_EFLAG_DUP_ID
+// for an id that repeats within the token.  0 means the token is valid.
+template <int K>
+__device__ __forceinline__ int load_ids(const int32_t *__restrict__ ids, int64_t t, int E,
+                                        int (&e)[K]) {
+    int f = 0;
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+        e[j] = __ldg(ids + t * K + j);
+        if ((unsigned)e[j] >= (unsigned)E) f |= COACT_EFLAG_ID_RANGE;
+    }
+#pragma unroll
+    for (int j = 1; j < K; ++j)
+#pragma unroll
+        for (int jj = 0; jj < j; ++jj)
+            if (e[j] == e[jj]) f |= COACT_EFLAG_DUP_ID;
+    return f;
+}
+
+// OR of `bits` over the warp, raised once by lane 0 (all lanes must call).
+__device__ __forceinline__ void raise_flag_warp(int32_t *err, int bits) {
+    const unsigned all = __reduce_or_sync(0xffffffffu, (unsigned)bits);
+    if (all && (threadIdx.x & 31) == 0 && err) atomicOr(err, (int)all);
+}
+
+// ------------------------------------------------------------------ host helpers
+
+// Per-device attributes, queried once per device.
+struct DeviceInfo {
+    int device;
+    int sm_count;
+    int smem_optin;   // max dynamic shared memory per block (opt-in)
+    int smem_per_sm;  // shared memory per SM
+};
+int device_info(DeviceInfo *out);  // returns COACT_OK or COACT_ERR_CUDA
+
+constexpr int kMaxDevices = 64;
+
+// Largest dynamic shared-memory size already opted in, per device, for one kernel.
+struct SmemOptIn {
+    std::atomic<int> bytes[kMaxDevices];
+};
+
+// Opts `kernel` in to `bytes` of dynamic shared memory on the current device once;
+// later calls only read the cache, so a stream capture sees launches alone.
+template <typename F>
+int ensure_smem(F kernel, size_t bytes, SmemOptIn &cache, const DeviceInfo &di) {
+    if (bytes <= 48 * 1024) return COACT_OK;
+    if (bytes > (size_t)di.smem_optin) return COACT_ERR_UNSUPPORTED;
+    std::atomic<int> &slot = cache.bytes[di.device];
+    if (slot.load(std::memory_order_relaxed) >= (int)bytes) return COACT_OK;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+        cudaSuccess)
+        return COACT_ERR_CUDA;
+    slot.store((int)bytes, std::memory_order_relaxed);
+    return COACT_OK;
+}
+
+// Resident blocks per SM for a kernel limited by threads and shared memory (the
+// library's kernels use few enough registers that registers never bind).
+inline int blocks_per_sm(int threads, size_t smem, const DeviceInfo &di) {
+    int by_threads = 2048 / threads;
+    int by_smem = smem ? (int)(di.smem_per_sm / (smem + 1024)) : 32;
+    int b = by_threads < by_smem ? by_threads : by_smem;
+    b = b < 32 ? b : 32;
+    return b > 0 ? b : 1;
+}
+
+inline int launch_status() {
+    return cudaGetLastError() == cudaSuccess ? COACT_OK : COACT_ERR_CUDA;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace coact

@@ -1,0 +1,290 @@
+// dispatch_gather: fill the per-rank send buffers, token-major.
+//
+// Cobalt (arxivdaily 2609.36959) and Zyphra (arxivdaily 2610.09372), English
+// abstracts: tokens are exchanged by all-to-all so each reaches the ranks that hold its
+// experts -- with the deduplicated dispatcher, each rank once.  Here a rank's send
+// segment is a region of this GPU's memory.
+//
+// Each x row is read from HBM once and written to every distinct destination row, so
+// the algorithmic traffic is (N + D) * H * 2 bytes (+ N*k*4 for send_row).
+//  * k_gather_bulk -- TMA bulk copies.  One warp per CTA; lane 0 streams rows into a
+//    ring of shared-memory stages with cp.async.bulk (global -> shared, completion on
+//    an mbarrier), then lanes j < k each issue the cp.async.bulk store of the staged
+//    row to destination j.  The hardware copy engine moves whole 0.5-14 KB rows with a
+//    handful of instructions; many small CTAs per SM keep enough bytes in flight.
+//    No multicast: every load reads this GPU's own memory once.
+//  * k_gather_v16 -- one warp per token, 16-byte vector loads into registers and
+//    streaming 16-byte stores to each destination.  Used for unaligned rows and short
+//    rows where staging does not pay.
+// All mbarrier waits are bounded by a wall-clock limit; on expiry the kernel raises
+// COACT_EFLAG_TIMEOUT, drains its own copies and returns.
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace coact {
+namespace {
+
+// ------------------------------------------------------------------ vector path
+
+template <int UNROLL>
+__global__ void __launch_bounds__(256)
+    k_gather_v16(const uint4 *__restrict__ x, int64_t N, int64_t H16,
+                 const int32_t *__restrict__ send_row, int k, uint4 *__restrict__ send,
+                 int64_t cap, int32_t *__restrict__ err) {
+    const int lane = threadIdx.x & 31;
+    const int64_t gwarp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    int flags = 0;
+    for (int64_t t = gwarp; t < N; t += nwarps) {
+        // destinations: lane j < k reads send_row[t, j]; broadcast by shuffles below
+        int dl = -1;
+        if (lane < k) {
+            dl = __ldg(send_row + t * k + lane);
+            if (dl >= 0 && (int64_t)dl >= cap) {
+                flags |= COACT_EFLAG_ROW_RANGE;
+                dl = -1;
+            }
+        }
+        const unsigned dmask = __ballot_sync(0xffffffffu, dl >= 0);
+        const uint4 *src = x + t * H16;
+        for (int64_t c0 = 0; c0 < H16; c0 += 32 * UNROLL) {
+            uint4 v[UNROLL];
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const int64_t c = c0 + u * 32 + lane;
+                if (c < H16) v[u] = ld_stream(src + c);
+            }
+            unsigned m = dmask;
+            while (m) {
+                const int j = __ffs(m) - 1;
+                m &= m - 1;
+                const int d = __shfl_sync(0xffffffffu, dl, j);
+                uint4 *dst = send + (int64_t)d * H16;
+#pragma unroll
+                for (int u = 0; u < UNROLL; ++u) {
+                    const int64_t c = c0 + u * 32 + lane;
+                    if (c < H16) st_stream(dst + c, v[u]);
+                }
+            }
+        }
+    }
+    raise_flag_warp(err, flags);
+}
+
+// ------------------------------------------------------------------ bulk (TMA) path
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Waits for phase `parity` of the mbarrier; gives up after `limit_ns` of wall clock.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63) == 63 && globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst_smem, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst_smem),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src_smem, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                 "r"(src_smem), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate copy
+constexpr int kBulkHeader = 128;                   // mbarriers live in the first 128 bytes
+
+// One warp per CTA.  Token i of this CTA is t = blockIdx.x + i * gridDim.x and uses
+// stage i % S.  Lane 0 owns the mbarriers and the loads; lane j < k owns the store of
+// destination j and its bulk groups.
+template <int S>
+__global__ void __launch_bounds__(32)
+    k_gather_bulk(const uint16_t *__restrict__ x, int64_t N, uint32_t row_bytes,
+                  const int32_t *__restrict__ send_row, int k, uint16_t *__restrict__ send,
+                  int64_t cap, int32_t *__restrict__ err) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int lane = threadIdx.x;
+    const uint32_t bars = smem_u32(smem);
+    const uint32_t bufs = smem_u32(smem + kBulkHeader);
+    const int64_t first = blockIdx.x, step = gridDim.x;
+    const int64_t n_mine = N > first ? (N - 1 - first) / step + 1 : 0;
+    const char *xb = reinterpret_cast<const char *>(x);
+    char *sb = reinterpret_cast<char *>(send);
+
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < S; ++s) mbar_init(bars + 8 * s, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int64_t i = 0; i < n_mine && i < S; ++i) {
+            const uint32_t bar = bars + 8 * (uint32_t)i;
+            mbar_expect_tx(bar, row_bytes);
+            bulk_load(bufs + (uint32_t)i * row_bytes, xb + (first + i * step) * (int64_t)row_bytes,
+                      row_bytes, bar);
+        }
+    }
+    __syncwarp();
+
+    int flags = 0;
+    int64_t loaded = n_mine < S ? n_mine : S;  // tokens whose load was issued
+    int dnext = (lane < k && n_mine > 0) ? __ldg(send_row + first * k + lane) : -1;
+    int64_t i = 0;
+    for (; i < n_mine; ++i) {
+        const int s = (int)(i % S);
+        const uint32_t parity = (uint32_t)((i / S) & 1);
+        const int d = dnext;
+        if (lane < k && i + 1 < n_mine) dnext = __ldg(send_row + (first + (i + 1) * step) * k + lane);
+        bool ready = true;
+        if (lane == 0) ready = mbar_wait_bounded(bars + 8 * s, parity, kWaitLimitNs);
+        ready = __shfl_sync(0xffffffffu, ready, 0);
+        if (!ready) {
+            flags |= COACT_EFLAG_TIMEOUT;
+            break;
+        }
+        // every lane observes the completed phase before reading the stage
+        mbar_try_wait(bars + 8 * s, parity);
+        fence_proxy_async_smem();
+        if (lane < k && d >= 0) {
+            if ((int64_t)d < cap) {
+                bulk_store(sb + (int64_t)d * row_bytes, bufs + (uint32_t)s * row_bytes, row_bytes);
+            } else {
+                flags |= COACT_EFLAG_ROW_RANGE;
+            }
+        }
+        bulk_commit();
+        // token i-1's stores have finished reading its stage once at most the newest
+        // group (token i's) is outstanding; refill that stage with token i-1+S
+        bulk_wait_read<1>();
+        __syncwarp();
+        if (lane == 0 && i >= 1 && loaded < n_mine) {
+            const int sp = (int)((i - 1) % S);
+            const uint32_t bar = bars + 8 * sp;
+            mbar_expect_tx(bar, row_bytes);
+            bulk_load(bufs + (uint32_t)sp * row_bytes,
+                      xb + (first + loaded * step) * (int64_t)row_bytes, row_bytes, bar);
+            ++loaded;
+        }
+        __syncwarp();
+    }
+    if (i < n_mine && lane == 0) {
+        // gave up: wait (bounded) for the loads still in flight before the CTA exits
+        for (int64_t q = i; q < loaded; ++q)
+            mbar_wait_bounded(bars + 8 * (uint32_t)(q % S), (uint32_t)((q / S) & 1), kWaitLimitNs);
+    }
+    bulk_wait_all();
+    raise_flag_warp(err, flags);
+}
+
+template <int S>
+int launch_bulk(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row, int k,
+                uint16_t *send, int64_t cap, int32_t *err, cudaStream_t st, const DeviceInfo &di) {
+    const uint32_t row_bytes = (uint32_t)(H * 2);
+    const size_t smem = kBulkHeader + (size_t)S * row_bytes;
+    auto kern = k_gather_bulk<S>;
+    static SmemOptIn opt;
+    if (int s = ensure_smem(kern, smem, opt, di)) return s;
+    const int per_sm = blocks_per_sm(32, smem, di);
+    // at least S tokens per CTA so the ring fills, but every SM busy
+    const int64_t want = std::max<int64_t>(1, ceil_div(N, 2 * S));
+    const int blocks = (int)std::min<int64_t>(want, (int64_t)per_sm * di.sm_count);
+    kern<<<blocks, 32, smem, st>>>(x, N, row_bytes, send_row, k, send, cap, err);
+    return launch_status();
+}
+
+int launch_v16(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row, int k,
+               uint16_t *send, int64_t cap, int32_t *err, cudaStream_t st, const DeviceInfo &di) {
+    const int64_t H16 = H / 8;
+    const int64_t warps_needed = N;
+    const int blocks = (int)std::max<int64_t>(
+        1, std::min<int64_t>(ceil_div(warps_needed, 8), (int64_t)di.sm_count * 8));
+    const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+    uint4 *sv = reinterpret_cast<uint4 *>(send);
+    if (H16 <= 32)
+        k_gather_v16<1><<<blocks, 256, 0, st>>>(xv, N, H16, send_row, k, sv, cap, err);
+    else if (H16 <= 128)
+        k_gather_v16<4><<<blocks, 256, 0, st>>>(xv, N, H16, send_row, k, sv, cap, err);
+    else
+        k_gather_v16<8><<<blocks, 256, 0, st>>>(xv, N, H16, send_row, k, sv, cap, err);
+    return launch_status();
+}
+
+}  // namespace
+}  // namespace coact
+
+using namespace coact;
+
+extern "C" int dispatch_gather(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row,
+                               int k, uint16_t *send, int64_t row_capacity, int32_t *err_flag,
+                               coact_stream_t stream) {
+    if (N < 0 || H < 0 || row_capacity < 0) return COACT_ERR_INVALID;
+    if (k < 1 || k > COACT_MAX_K) return COACT_ERR_UNSUPPORTED;
+    if (H % 8 != 0) return COACT_ERR_UNSUPPORTED;
+    if (N == 0 || H == 0) return COACT_OK;
+    if (!x || !send_row || (row_capacity > 0 && !send)) return COACT_ERR_INVALID;
+    if (!aligned16(x) || (send && !aligned16(send))) return COACT_ERR_INVALID;
+    if (N > (int64_t)INT32_MAX / k || row_capacity > (int64_t)INT32_MAX) return COACT_ERR_UNSUPPORTED;
+    DeviceInfo di;
+    if (int s = device_info(&di)) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t row_bytes = H * 2;
+    bool bulk = row_bytes >= 1024 && row_bytes <= 32768;
+#if defined(COACT_GATHER_PATH)
+    bulk = bulk && COACT_GATHER_PATH != 0;  // experiment builds only
+#endif
+    if (bulk) {
+        if (row_bytes <= 4096) return launch_bulk<8>(x, N, H, send_row, k, send, row_capacity, err_flag, st, di);
+        return launch_bulk<4>(x, N, H, send_row, k, send, row_capacity, err_flag, st, di);
+    }
+    return launch_v16(x, N, H, send_row, k, send, row_capacity, err_flag, st, di);
+}

@@ -1,0 +1,520 @@
+// plan_dispatch: the deduplicated dispatch layout.
+//
+// Zyphra (arxivdaily 2610.09372), English abstract: "a dispatcher that sends each token
+// to each GPU once" -- one send row per (token, destination rank) instead of one per
+// (token, expert).  Cobalt (arxivdaily 2609.36959), English abstract: routing tokens to
+// fewer remote nodes -- node-level statistics of the same plan.
+//
+// Three launches, none of which waits on another block:
+//  1. k_plan_tiles   one thread per token, 256-token tiles: per-token rank mask, per-tile
+//                    per-rank row and assignment counts (warp ballots / redux, no
+//                    atomics) and per-tile statistics partials.
+//  2. k_plan_scan    R + 1 blocks: block r turns rank r's per-tile counts into exclusive
+//                    per-tile bases (in place) and a total; the last block reduces the
+//                    statistics partials and clears src_dst.
+//  3. k_plan_scatter one thread per token again: rank offsets from the totals, stable
+//                    in-tile positions from per-rank ballots (rows) and 4-bit ballot
+//                    prefix sums (assignments), then row_token / row_kmask / send_row /
+//                    comb_row / rank_mask, and the src x dst split matrix.
+// Positions depend only on token order, so every output is deterministic.
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace coact {
+namespace {
+
+constexpr int kTile = 256;                 // tokens per tile, one per thread
+constexpr int kTileWarps = kTile / 32;
+constexpr int kScanThreads = 1024;
+constexpr int kStatSlots = 6;              // per-tile partials (see TileStat)
+enum TileStat { TS_REMOTE_ROWS, TS_XNODE_ROWS, TS_NODE_ROWS, TS_LOCAL_ASG, TS_XNODE_ASG, TS_VALID_ASG };
+
+struct Workspace {
+    int32_t *tile_rows;   // [R][n_tiles]  counts, then exclusive bases (in place)
+    int32_t *tile_asg;    // [R][n_tiles]
+    int64_t *tile_stats;  // [n_tiles][kStatSlots]
+    int32_t *tot;         // [2R] rows per rank, assignments per rank
+};
+
+inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+size_t workspace_layout(int64_t N, int R, Workspace *ws, void *base) {
+    const int64_t n_tiles = ceil_div(N, kTile);
+    const size_t b_rows = align256(sizeof(int32_t) * (size_t)R * n_tiles);
+    const size_t b_stats = align256(sizeof(int64_t) * kStatSlots * (size_t)n_tiles);
+    const size_t b_tot = align256(sizeof(int32_t) * 2 * (size_t)R);
+    if (ws) {
+        char *p = static_cast<char *>(base);
+        ws->tile_rows = reinterpret_cast<int32_t *>(p);
+        ws->tile_asg = reinterpret_cast<int32_t *>(p + b_rows);
+        ws->tile_stats = reinterpret_cast<int64_t *>(p + 2 * b_rows);
+        ws->tot = reinterpret_cast<int32_t *>(p + 2 * b_rows + b_stats);
+    }
+    return 2 * b_rows + b_stats + b_tot;
+}
+
+// Token t's per-slot ranks and home rank; returns validation bits (0 = valid).
+template <int K>
+__device__ __forceinline__ int load_token(const int32_t *__restrict__ ids,
+                                          const int32_t *__restrict__ expert_rank,
+                                          const int32_t *__restrict__ src_rank, int64_t t,
+                                          int64_t N, int E, int R, int (&rk)[K], int &src) {
+    int e[K];
+    int f = load_ids<K>(ids, t, E, e);
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+        rk[j] = (f & COACT_EFLAG_ID_RANGE) ? 0 : __ldg(expert_rank + e[j]);
+        if ((unsigned)rk[j] >= (unsigned)R) f |= COACT_EFLAG_ID_RANGE;
+    }
+    src = src_rank ? __ldg(src_rank + t) : (int)((t * R) / N);
+    if ((unsigned)src >= (unsigned)R) f |= COACT_EFLAG_SRC_RANK;
+    return f;
+}
+
+// rank -> node table and node -> rank-set table in shared memory.  A node id outside
+// [0, n_nodes) raises COACT_EFLAG_ID_RANGE and is read as node 0.
+__device__ __forceinline__ void load_nodes(const int32_t *__restrict__ rank_node, int R,
+                                           int n_nodes, int *s_node, unsigned long long *s_node_ranks,
+                                           int32_t *err) {
+    const int tid = threadIdx.x;
+    if (tid < 64) {
+        int nd = 0;
+        if (tid < R && rank_node) {
+            nd = __ldg(rank_node + tid);
+            if ((unsigned)nd >= (unsigned)n_nodes) {
+                raise_flag(err, COACT_EFLAG_ID_RANGE);
+                nd = 0;
+            }
+        }
+        s_node[tid] = nd;
+        s_node_ranks[tid] = 0;
+    }
+    __syncthreads();
+    if (tid < R) atomicOr(&s_node_ranks[s_node[tid]], 1ull << tid);
+    __syncthreads();
+}
+
+// Warp-uniform OR of a 64-bit mask.
+__device__ __forceinline__ unsigned long long warp_or64(unsigned long long m) {
+    const unsigned lo = __reduce_or_sync(0xffffffffu, (unsigned)m);
+    const unsigned hi = __reduce_or_sync(0xffffffffu, (unsigned)(m >> 32));
+    return ((unsigned long long)hi << 32) | lo;
+}
+
+template <int K>
+__global__ void __launch_bounds__(kTile)
+    k_plan_tiles(const int32_t *__restrict__ ids, int64_t N, int E,
+                 const int32_t *__restrict__ expert_rank, int R,
+                 const int32_t *__restrict__ rank_node, int n_nodes,
+                 const int32_t *__restrict__ src_rank, int n_tiles, Workspace ws,
+                 int32_t *__restrict__ err) {
+    __shared__ int s_node[64];
+    __shared__ unsigned long long s_node_ranks[64];
+    __shared__ int s_wrows[kTileWarps][64];
+    __shared__ int s_wasg[kTileWarps][64];
+    __shared__ long long s_stat[kTileWarps][kStatSlots];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    load_nodes(rank_node, R, n_nodes, s_node, s_node_ranks, err);
+    for (int i = tid; i < kTileWarps * 64; i += kTile) {
+        (&s_wrows[0][0])[i] = 0;
+        (&s_wasg[0][0])[i] = 0;
+    }
+    __syncthreads();
+
+    const int64_t t = (int64_t)blockIdx.x * kTile + tid;
+    int rk[K];
+    int src = 0;
+    bool ok = false;
+    int flags = 0;
+    if (t < N) {
+        flags = load_token<K>(ids, expert_rank, src_rank, t, N, E, R, rk, src);
+        ok = flags == 0;
+    }
+    unsigned long long mask = 0;
+    int st[kStatSlots] = {0, 0, 0, 0, 0, 0};
+    if (ok) {
+        const int nsrc = s_node[src];
+        unsigned long long nmask = 0;
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+            mask |= 1ull << rk[j];
+            const int nd = s_node[rk[j]];
+            nmask |= 1ull << nd;
+            st[TS_LOCAL_ASG] += rk[j] == src;
+            st[TS_XNODE_ASG] += nd != nsrc;
+        }
+        st[TS_REMOTE_ROWS] = __popcll(mask & ~(1ull << src));
+        st[TS_XNODE_ROWS] = __popcll(mask & ~s_node_ranks[nsrc]);
+        st[TS_NODE_ROWS] = __popcll(nmask & ~(1ull << nsrc));
+        st[TS_VALID_ASG] = K;
+    }
+    // per-rank counts of this warp: rows = lanes holding the rank, asg = slots on it
+    unsigned long long wmask = warp_or64(mask);
+    while (wmask) {
+        const int r = __ffsll(wmask) - 1;
+        wmask &= wmask - 1;
+        int c = 0;
+#pragma unroll
+        for (int j = 0; j < K; ++j) c += ok && rk[j] == r;
+        const unsigned b = __ballot_sync(0xffffffffu, c > 0);
+        const int a = __reduce_add_sync(0xffffffffu, c);
+        if (lane == 0) {
+            s_wrows[warp][r] = __popc(b);
+            s_wasg[warp][r] = a;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < kStatSlots; ++i) {
+        const int v = __reduce_add_sync(0xffffffffu, st[i]);
+        if (lane == 0) s_stat[warp][i] = v;
+    }
+    raise_flag_warp(err, flags);
+    __syncthreads();
+    if (tid < R) {
+        int rows = 0, asg = 0;
+#pragma unroll
+        for (int w = 0; w < kTileWarps; ++w) {
+            rows += s_wrows[w][tid];
+            asg += s_wasg[w][tid];
+        }
+        ws.tile_rows[(int64_t)tid * n_tiles + blockIdx.x] = rows;
+        ws.tile_asg[(int64_t)tid * n_tiles + blockIdx.x] = asg;
+    }
+    if (tid < kStatSlots) {
+        long long v = 0;
+#pragma unroll
+        for (int w = 0; w < kTileWarps; ++w) v += s_stat[w][tid];
+        ws.tile_stats[(int64_t)blockIdx.x * kStatSlots + tid] = v;
+    }
+}
+
+// Exclusive scan of one int per thread over the block; returns the prefix and sets
+// *total.  All threads must call.
+__device__ __forceinline__ int block_excl_scan(int v, int *s_warp, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += u;
+    }
+    if (lane == 31) s_warp[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nw ? s_warp[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += u;
+        }
+        if (lane < nw) s_warp[lane] = wi - w;     // exclusive per-warp base
+        if (lane == 31) s_warp[32] = wi;          // block total
+    }
+    __syncthreads();
+    const int out = s_warp[warp] + inc - v;
+    *total = s_warp[32];
+    __syncthreads();
+    return out;
+}
+
+__global__ void __launch_bounds__(kScanThreads)
+    k_plan_scan(int64_t N, int K, int R, int n_tiles, Workspace ws, int64_t *__restrict__ stats,
+                int32_t *__restrict__ src_dst) {
+    __shared__ int s_warp[33];
+    __shared__ long long s_red[kStatSlots][32];
+    if ((int)blockIdx.x < R) {
+        const int r = blockIdx.x;
+        for (int which = 0; which < 2; ++which) {
+            int32_t *row = (which == 0 ? ws.tile_rows : ws.tile_asg) + (int64_t)r * n_tiles;
+            int carry = 0;
+            for (int c0 = 0; c0 < n_tiles; c0 += kScanThreads) {
+                const int i = c0 + threadIdx.x;
+                const int v = i < n_tiles ? row[i] : 0;
+                int tot;
+                const int ex = block_excl_scan(v, s_warp, &tot);
+                if (i < n_tiles) row[i] = carry + ex;
+                carry += tot;
+            }
+            if (threadIdx.x == 0) ws.tot[which * R + r] = carry;
+        }
+        return;
+    }
+    // statistics block
+    long long acc[kStatSlots] = {0, 0, 0, 0, 0, 0};
+    for (int i = threadIdx.x; i < n_tiles; i += kScanThreads)
+#pragma unroll
+        for (int s = 0; s < kStatSlots; ++s) acc[s] += ws.tile_stats[(int64_t)i * kStatSlots + s];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int s = 0; s < kStatSlots; ++s) {
+        long long v = acc[s];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) s_red[s][warp] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < kStatSlots) {
+        long long v = 0;
+        for (int w = 0; w < kScanThreads / 32; ++w) v += s_red[threadIdx.x][w];
+        s_red[threadIdx.x][0] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        stats[COACT_STAT_NAIVE_ROWS] = N * K;
+        stats[COACT_STAT_REMOTE_ROWS] = s_red[TS_REMOTE_ROWS][0];
+        stats[COACT_STAT_CROSSNODE_ROWS] = s_red[TS_XNODE_ROWS][0];
+        stats[COACT_STAT_NODE_DEDUP_ROWS] = s_red[TS_NODE_ROWS][0];
+        stats[COACT_STAT_LOCAL_ASG] = s_red[TS_LOCAL_ASG][0];
+        stats[COACT_STAT_REMOTE_ASG] = s_red[TS_VALID_ASG][0] - s_red[TS_LOCAL_ASG][0];
+        stats[COACT_STAT_CROSSNODE_ASG] = s_red[TS_XNODE_ASG][0];
+    }
+    if (src_dst)
+        for (int i = threadIdx.x; i < R * R; i += kScanThreads) src_dst[i] = 0;
+}
+
+template <int K>
+__global__ void __launch_bounds__(kTile)
+    k_plan_scatter(const int32_t *__restrict__ ids, int64_t N, int E,
+                   const int32_t *__restrict__ expert_rank, int R,
+                   const int32_t *__restrict__ src_rank, int n_tiles, Workspace ws,
+                   int32_t *__restrict__ rank_counts, int32_t *__restrict__ rank_offsets,
+                   int32_t *__restrict__ asg_offsets, unsigned long long *__restrict__ rank_mask,
+                   int32_t *__restrict__ row_token, uint8_t *__restrict__ row_kmask, int64_t cap,
+                   int32_t *__restrict__ send_row, int32_t *__restrict__ comb_row,
+                   int64_t *__restrict__ stats, int32_t *__restrict__ src_dst,
+                   int32_t *__restrict__ err) {
+    __shared__ int s_rbase[64], s_abase[64];
+    __shared__ int s_wrows[kTileWarps][64];
+    __shared__ int s_wasg[kTileWarps][64];
+    extern __shared__ int s_sd[];  // [R*R] when src_dst != NULL
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tile = blockIdx.x;
+    if (warp == 0) {
+        // rank offsets = exclusive scan of the per-rank totals (R <= 64: two per lane)
+        const int r0 = lane, r1 = lane + 32;
+        for (int which = 0; which < 2; ++which) {
+            const int32_t *tot = ws.tot + which * R;
+            const int v0 = r0 < R ? tot[r0] : 0, v1 = r1 < R ? tot[r1] : 0;
+            int i0 = v0, i1 = v1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u0 = __shfl_up_sync(0xffffffffu, i0, o);
+                const int u1 = __shfl_up_sync(0xffffffffu, i1, o);
+                if (lane >= o) {
+                    i0 += u0;
+                    i1 += u1;
+                }
+            }
+            const int total0 = __shfl_sync(0xffffffffu, i0, 31);
+            const int total = total0 + __shfl_sync(0xffffffffu, i1, 31);
+            const int e0 = i0 - v0, e1 = total0 + i1 - v1;
+            int *sbase = which == 0 ? s_rbase : s_abase;
+            const int32_t *tb = which == 0 ? ws.tile_rows : ws.tile_asg;
+            if (r0 < R) sbase[r0] = e0 + (tile < n_tiles ? tb[(int64_t)r0 * n_tiles + tile] : 0);
+            if (r1 < R) sbase[r1] = e1 + (tile < n_tiles ? tb[(int64_t)r1 * n_tiles + tile] : 0);
+            if (tile == 0) {
+                int32_t *offs = which == 0 ? rank_offsets : asg_offsets;
+                if (r0 < R) offs[r0] = e0;
+                if (r1 < R) offs[r1] = e1;
+                if (lane == 0) offs[R] = total;
+                if (which == 0) {
+                    if (r0 < R) rank_counts[r0] = v0;
+                    if (r1 < R) rank_counts[r1] = v1;
+                    if (lane == 0) stats[COACT_STAT_DEDUP_ROWS] = total;
+                }
+            }
+        }
+    }
+    for (int i = tid; i < kTileWarps * 64; i += kTile) {
+        (&s_wrows[0][0])[i] = 0;
+        (&s_wasg[0][0])[i] = 0;
+    }
+    if (src_dst)
+        for (int i = tid; i < R * R; i += kTile) s_sd[i] = 0;
+    __syncthreads();
+
+    const int64_t t = (int64_t)tile * kTile + tid;
+    int rk[K];
+    int src = 0;
+    bool ok = false;
+    int flags = 0;
+    if (t < N) ok = load_token<K>(ids, expert_rank, src_rank, t, N, E, R, rk, src) == 0;
+    unsigned long long mask = 0;
+    if (ok) {
+#pragma unroll
+        for (int j = 0; j < K; ++j) mask |= 1ull << rk[j];
+    }
+    // lanes with the same home rank, for the src x dst split counts
+    const unsigned same_src = __match_any_sync(0xffffffffu, ok ? src : -1);
+    const bool src_leader = ok && lane == __ffs(same_src) - 1;
+
+    int pre_row[K], pre_asg[K];
+#pragma unroll
+    for (int j = 0; j < K; ++j) pre_row[j] = pre_asg[j] = 0;
+    const unsigned lt = lanemask_lt();
+    unsigned long long wmask = warp_or64(mask);
+    while (wmask) {
+        const int r = __ffsll(wmask) - 1;
+        wmask &= wmask - 1;
+        int c = 0;
+#pragma unroll
+        for (int j = 0; j < K; ++j) c += ok && rk[j] == r;
+        const unsigned b = __ballot_sync(0xffffffffu, c > 0);
+        // exclusive prefix of c (0..K <= 8, four bits) over the lanes via bit ballots
+        int ap = 0, at = 0;
+#pragma unroll
+        for (int bit = 0; bit < 4; ++bit) {
+            if ((K >> bit) == 0) break;
+            const unsigned bb = __ballot_sync(0xffffffffu, (c >> bit) & 1);
+            ap += __popc(bb & lt) << bit;
+            at += __popc(bb) << bit;
+        }
+        const int rp = __popc(b & lt);
+#pragma unroll
+        for (int j = 0; j < K; ++j)
+            if (ok && rk[j] == r) {
+                pre_row[j] = rp;
+                pre_asg[j] = ap;
+            }
+        if (lane == 0) {
+            s_wrows[warp][r] = __popc(b);
+            s_wasg[warp][r] = at;
+        }
+        if (src_dst && src_leader) {
+            const int n = __popc(b & same_src);
+            if (n) atomicAdd(&s_sd[src * R + r], n);
+        }
+    }
+    __syncthreads();
+    if (tid < R) {
+        int run_r = 0, run_a = 0;
+#pragma unroll
+        for (int w = 0; w < kTileWarps; ++w) {
+            const int vr = s_wrows[w][tid], va = s_wasg[w][tid];
+            s_wrows[w][tid] = run_r;
+            s_wasg[w][tid] = run_a;
+            run_r += vr;
+            run_a += va;
+        }
+    }
+    __syncthreads();
+
+    if (t < N) {
+        if (!ok) {
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                send_row[t * K + j] = -1;
+                comb_row[t * K + j] = -1;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                const int r = rk[j];
+                unsigned km = 0;
+#pragma unroll
+                for (int jj = 0; jj < K; ++jj) km |= (unsigned)(rk[jj] == r) << jj;
+                const unsigned below = km & ((1u << j) - 1);
+                comb_row[t * K + j] = s_abase[r] + s_wasg[warp][r] + pre_asg[j] + __popc(below);
+                int sr = -1;
+                if (below == 0) {
+                    const int64_t row = (int64_t)s_rbase[r] + s_wrows[warp][r] + pre_row[j];
+                    if (row < cap) {
+                        row_token[row] = (int32_t)t;
+                        row_kmask[row] = (uint8_t)km;
+                        sr = (int)row;
+                    } else {
+                        flags |= COACT_EFLAG_CAPACITY;
+                    }
+                }
+                send_row[t * K + j] = sr;
+            }
+        }
+        if (rank_mask) rank_mask[t] = mask;
+    }
+    raise_flag_warp(err, flags);
+    if (src_dst) {
+        __syncthreads();
+        for (int i = tid; i < R * R; i += kTile) {
+            const int v = s_sd[i];
+            if (v) atomicAdd(src_dst + i, v);
+        }
+    }
+}
+
+template <int K>
+int launch_plan(const int32_t *ids, int64_t N, int E, const int32_t *expert_rank, int R,
+                const int32_t *rank_node, int n_nodes, const int32_t *src_rank,
+                int32_t *rank_counts, int32_t *rank_offsets, int32_t *asg_offsets,
+                uint64_t *rank_mask, int32_t *row_token, uint8_t *row_kmask, int64_t cap,
+                int32_t *send_row, int32_t *comb_row, int64_t *stats, int32_t *src_dst,
+                const Workspace &ws, int32_t *err, cudaStream_t st) {
+    const int n_tiles = (int)ceil_div(N, kTile);
+    if (n_tiles > 0)
+        k_plan_tiles<K><<<n_tiles, kTile, 0, st>>>(ids, N, E, expert_rank, R, rank_node, n_nodes,
+                                                   src_rank, n_tiles, ws, err);
+    k_plan_scan<<<R + 1, kScanThreads, 0, st>>>(N, K, R, n_tiles, ws, stats, src_dst);
+    const size_t smem = src_dst ? sizeof(int) * R * R : 0;
+    k_plan_scatter<K><<<std::max(n_tiles, 1), kTile, smem, st>>>(
+        ids, N, E, expert_rank, R, src_rank, n_tiles, ws, rank_counts, rank_offsets, asg_offsets,
+        reinterpret_cast<unsigned long long *>(rank_mask), row_token, row_kmask, cap, send_row,
+        comb_row, stats, src_dst, err);
+    return launch_status();
+}
+
+}  // namespace
+}  // namespace coact
+
+using namespace coact;
+
+extern "C" size_t plan_dispatch_workspace_bytes(int64_t N, int k, int E, int R) {
+    (void)k;
+    (void)E;
+    if (N < 0 || R < 1 || R > COACT_MAX_R) return 0;
+    return workspace_layout(N, R, nullptr, nullptr);
+}
+
+extern "C" int plan_dispatch(const int32_t *ids, int64_t N, int k, int E, const int32_t *expert_rank,
+                             int R, const int32_t *rank_node, int n_nodes, const int32_t *src_rank,
+                             int32_t *rank_counts, int32_t *rank_offsets, int32_t *asg_offsets,
+                             uint64_t *rank_mask, int32_t *row_token, uint8_t *row_kmask,
+                             int64_t row_capacity, int32_t *send_row, int32_t *comb_row,
+                             int64_t *stats, int32_t *src_dst, void *workspace,
+                             size_t workspace_bytes, int32_t *err_flag, coact_stream_t stream) {
+    if (N < 0 || row_capacity < 0) return COACT_ERR_INVALID;
+    if (k < 1 || k > COACT_MAX_K || E < 2 || E > COACT_MAX_E || R < 1 || R > COACT_MAX_R)
+        return COACT_ERR_UNSUPPORTED;
+    if (rank_node && (n_nodes < 1 || n_nodes > 64)) return COACT_ERR_UNSUPPORTED;
+    if (!rank_node) n_nodes = 1;
+    if (N > (int64_t)INT32_MAX / k || row_capacity > (int64_t)INT32_MAX) return COACT_ERR_UNSUPPORTED;
+    if (!expert_rank || !rank_counts || !rank_offsets || !asg_offsets || !stats)
+        return COACT_ERR_INVALID;
+    if (N > 0 && (!ids || !send_row || !comb_row)) return COACT_ERR_INVALID;
+    if (row_capacity > 0 && (!row_token || !row_kmask)) return COACT_ERR_INVALID;
+    const size_t need = workspace_layout(N, R, nullptr, nullptr);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return COACT_ERR_WORKSPACE;
+    Workspace ws;
+    workspace_layout(N, R, &ws, workspace);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+#define COACT_PLAN_CASE(KK)                                                                        \
+    case KK:                                                                                       \
+        return launch_plan<KK>(ids, N, E, expert_rank, R, rank_node, n_nodes, src_rank,            \
+                               rank_counts, rank_offsets, asg_offsets, rank_mask, row_token,       \
+                               row_kmask, row_capacity, send_row, comb_row, stats, src_dst, ws,    \
+                               err_flag, st);
+    switch (k) {
+        COACT_PLAN_CASE(1)
+        COACT_PLAN_CASE(2)
+        COACT_PLAN_CASE(3)
+        COACT_PLAN_CASE(4)
+        COACT_PLAN_CASE(5)
+        COACT_PLAN_CASE(6)
+        COACT_PLAN_CASE(7)
+        COACT_PLAN_CASE(8)
+    }
+#undef COACT_PLAN_CASE
+    return COACT_ERR_UNSUPPORTED;
+}

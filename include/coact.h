@@ -1,0 +1,222 @@
+/*
+ * coact.h -- C ABI of the B200 (sm_100a) co-activation dispatch/combine library.
+ *
+ * The library implements the data-parallel hot path that two pages share:
+ *   Cobalt, "efficient distributed MoE training using expert co-activation"
+ *     (arxivdaily 2609.36959), English abstract;
+ *   Zyphra correlated expert placement and token shuffling
+ *     (arxivdaily 2610.09372), English abstract.
+ * Under expert parallelism (EP) tokens travel to the ranks that hold their experts and
+ * the expert outputs come back to be combined.  The library counts which experts are
+ * co-activated, plans a dispatch that sends each token to each destination rank once,
+ * gathers the hidden rows into per-rank send buffers and combines expert outputs back
+ * in token order.  Logical ranks are partitions of one GPU's memory.
+ *
+ * Conventions for every entry point:
+ *  - Array pointers are DEVICE pointers owned by the caller (e.g. torch tensors).  The
+ *    library never allocates, frees or synchronises; all work is enqueued on `stream`
+ *    (a cudaStream_t; NULL = the legacy default stream).  Calls are asynchronous.
+ *  - Return value: COACT_OK (0) or a negative coact_status.  A negative status is
+ *    decided on the host before anything is enqueued (except COACT_ERR_CUDA, which
+ *    reports a failed launch).
+ *  - Data errors that only the device can see (an expert id out of range, a repeated
+ *    id within a token, a row index out of range, a full send buffer) set bits of
+ *    coact_eflag in *err_flag with an atomic OR.  err_flag is an int32 DEVICE pointer
+ *    and may be NULL; the caller zeroes it and reads it after the stream syncs.  When a
+ *    bit is set, the outputs that depend on the offending tokens are unspecified, but
+ *    no kernel ever reads or writes outside the buffers it was given, traps or hangs.
+ *  - Row data are bf16, passed as uint16_t bit patterns, row-major, rows of H elements.
+ *    Row buffers must be 16-byte aligned and H a multiple of 8 (16-byte rows).
+ *  - Limits: 1 <= k <= 8 experts per token, 2 <= E <= 1024 experts, 1 <= R <= 64
+ *    ranks, 1 <= n_nodes <= 64, N*k < 2^31, row_capacity < 2^31.
+ */
+#ifndef COACT_H
+#define COACT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *coact_stream_t;
+
+enum coact_status {
+    COACT_OK = 0,
+    COACT_ERR_INVALID = -1,      /* NULL required pointer, negative size, bad alignment */
+    COACT_ERR_UNSUPPORTED = -2,  /* argument outside the documented limits */
+    COACT_ERR_CUDA = -3,         /* a CUDA launch or attribute call failed */
+    COACT_ERR_WORKSPACE = -4,    /* workspace NULL or smaller than the query says */
+    COACT_ERR_TIMEOUT = -5       /* reserved: a bounded device wait gave up */
+};
+
+enum coact_eflag {
+    COACT_EFLAG_ID_RANGE = 1,    /* expert id (or its rank) outside its range; token skipped */
+    COACT_EFLAG_DUP_ID = 2,      /* the same expert twice in one token; token skipped */
+    COACT_EFLAG_CAPACITY = 4,    /* a send row fell at or beyond row_capacity; not written */
+    COACT_EFLAG_SRC_RANK = 8,    /* src_rank[t] outside [0, R); token skipped */
+    COACT_EFLAG_ROW_RANGE = 16,  /* send_row / comb_row entry outside the row buffer; skipped */
+    COACT_EFLAG_TIMEOUT = 32     /* a bounded wait on an mbarrier gave up; outputs unspecified */
+};
+
+#define COACT_MAX_K 8
+#define COACT_MAX_E 1024
+#define COACT_MAX_R 64
+#define COACT_NUM_STATS 8
+
+/* Indices into the stats[8] array written by plan_dispatch. */
+enum coact_stat {
+    COACT_STAT_NAIVE_ROWS = 0,          /* N*k: one row per token-expert assignment */
+    COACT_STAT_DEDUP_ROWS = 1,          /* D: one row per (token, destination rank) */
+    COACT_STAT_REMOTE_ROWS = 2,         /* rows whose rank is not the token's home rank */
+    COACT_STAT_CROSSNODE_ROWS = 3,      /* rows whose rank sits on another node */
+    COACT_STAT_NODE_DEDUP_ROWS = 4,     /* (token, remote node) pairs: rows if sent once per node */
+    COACT_STAT_LOCAL_ASG = 5,           /* assignments whose expert is on the home rank */
+    COACT_STAT_REMOTE_ASG = 6,          /* assignments whose expert is elsewhere */
+    COACT_STAT_CROSSNODE_ASG = 7        /* assignments whose expert is on another node */
+};
+
+/* Static text for a coact_status value. */
+const char *coact_strerror(int status);
+
+/* ABI version of this header (bumped on any signature change). */
+int coact_abi_version(void);
+#define COACT_ABI_VERSION 1
+
+/*
+ * coact_count -- expert co-activation pair counts and per-expert loads.
+ * Cobalt, English abstract: many pairs of experts are co-activated by single tokens,
+ * and per-expert workload statistics drive the layout planner; Zyphra, English
+ * abstract: a small share of expert pairs is selected together by a large share of
+ * tokens, and the experts a token picks at one layer predict those at the next.
+ *
+ * Co-activation mode (ids2 == NULL):
+ *   pair[a*E+b] += #{t : a and b are both among ids[t, 0..k-1], a != b}
+ *   The increment is symmetric with a zero diagonal; its strict upper triangle sums
+ *   to N*k*(k-1)/2.
+ * Cross-layer mode (ids2 != NULL, same N):
+ *   pair[a*E2+b] += #{(t, j, j2) : ids[t,j] == a, ids2[t,j2] == b}   (E x E2, not symmetric)
+ * loads[e] += #{(t, j) : ids[t,j] == e}   (loads may be NULL).
+ *
+ * ids: int32 [N, k] row-major; ids2: int32 [N, k2] or NULL (then k2, E2 are ignored).
+ * pair: int64 [E*E] (or [E*E2]), loads: int64 [E]; both ACCUMULATE (+=), so zero them
+ * for fresh counts.  A token with an id outside [0, E) (or [0, E2)) or a repeated id
+ * is not counted and sets COACT_EFLAG_ID_RANGE / COACT_EFLAG_DUP_ID.
+ */
+int coact_count(const int32_t *ids, int64_t N, int k, int E,
+                const int32_t *ids2, int k2, int E2,
+                int64_t *pair, int64_t *loads,
+                int32_t *err_flag, coact_stream_t stream);
+
+/* Bytes of device workspace plan_dispatch needs for these sizes (0 if N == 0). */
+size_t plan_dispatch_workspace_bytes(int64_t N, int k, int E, int R);
+
+/*
+ * plan_dispatch -- the deduplicated dispatch layout.
+ * Zyphra, English abstract: a dispatcher that sends each token to each GPU once;
+ * Cobalt, English abstract: routing tokens to fewer remote nodes under the current
+ * expert layout (node-level statistics).
+ *
+ * Inputs (device): ids int32 [N,k]; expert_rank int32 [E] (expert -> rank in [0,R));
+ * rank_node int32 [R] (rank -> node in [0,n_nodes)) or NULL (one node); src_rank int32
+ * [N] (the token's home rank) or NULL (contiguous shards: floor(t*R/N)).
+ * With rank(j) = expert_rank[ids[t,j]]:
+ *   rank_mask[t]   = OR_j 1 << rank(j)                         (uint64 [N], may be NULL)
+ *   kmask(t, r)    = OR_{j : rank(j) == r} 1 << j              (mask over the k slots)
+ *   rank_counts[r] = #{t : r in rank_mask[t]}                  (int32 [R])
+ *   rank_offsets   = exclusive prefix sum of rank_counts; rank_offsets[R] = D (int32 [R+1])
+ *   asg_offsets    = exclusive prefix sum over r of sum_t popcount(kmask(t,r));
+ *                    asg_offsets[R] = number of valid assignments (int32 [R+1])
+ * Rows of rank r occupy [rank_offsets[r], rank_offsets[r+1]) in ascending token order:
+ *   row_token[d] = t, row_kmask[d] = kmask(t, r)   (int32 / uint8 [row_capacity])
+ *   send_row[t,j] = the row of (t, rank(j)) if j is the smallest slot on rank(j),
+ *                   else -1                                     (int32 [N,k])
+ *   comb_row[t,j] = the row of assignment (t, j) in "expanded receive order": rank
+ *                   segments starting at asg_offsets[r], rows in order, one row per set
+ *                   slot in ascending j                         (int32 [N,k])
+ * Rows at or beyond row_capacity are not written (their send_row is -1) and set
+ * COACT_EFLAG_CAPACITY; row_capacity >= N*min(k,R) can never overflow.  Rows of
+ * [D, row_capacity) are left untouched.
+ * stats int64 [8] (see coact_stat), src_dst int32 [R*R] or NULL:
+ *   src_dst[s*R + r] = #{t : src[t] == s, r in rank_mask[t]} (the all-to-all split sizes).
+ * workspace: device memory of at least plan_dispatch_workspace_bytes(N,k,E,R) bytes,
+ * 16-byte aligned; its contents need no initialisation and are scratch afterwards.
+ * Tokens with invalid ids, an expert_rank entry outside [0,R) or a src_rank outside
+ * [0,R) contribute no rows, get send_row = comb_row = -1, and set their flag.
+ * Deterministic: no result depends on scheduling.
+ */
+int plan_dispatch(const int32_t *ids, int64_t N, int k, int E,
+                  const int32_t *expert_rank, int R,
+                  const int32_t *rank_node, int n_nodes,
+                  const int32_t *src_rank,
+                  int32_t *rank_counts, int32_t *rank_offsets, int32_t *asg_offsets,
+                  uint64_t *rank_mask,
+                  int32_t *row_token, uint8_t *row_kmask, int64_t row_capacity,
+                  int32_t *send_row, int32_t *comb_row,
+                  int64_t *stats, int32_t *src_dst,
+                  void *workspace, size_t workspace_bytes,
+                  int32_t *err_flag, coact_stream_t stream);
+
+/*
+ * dispatch_gather -- fill the per-rank send buffers.
+ * Cobalt / Zyphra, English abstracts: tokens are exchanged through all-to-all so that
+ * each reaches the ranks holding its experts, each rank once.
+ *   send[send_row[t,j]] = x[t]   for every (t, j) with send_row[t,j] >= 0
+ * i.e. send[d] = x[row_token[d]] for d < D.  Each x row is read once and written to
+ * every distinct destination row.
+ * x: bf16 [N, H]; send_row: int32 [N, k] (from plan_dispatch); send: bf16
+ * [row_capacity, H].  Entries >= row_capacity set COACT_EFLAG_ROW_RANGE and are skipped;
+ * rows not named by send_row are left untouched.  Copies are bit-exact.
+ */
+int dispatch_gather(const uint16_t *x, int64_t N, int64_t H,
+                    const int32_t *send_row, int k,
+                    uint16_t *send, int64_t row_capacity,
+                    int32_t *err_flag, coact_stream_t stream);
+
+/*
+ * combine_scatter -- the weighted combine back to token order.
+ * Zyphra, English abstract: tokens are dispatched to their experts "and then" the
+ * results are combined; neither method changes the routing decisions.
+ *   out[t] = sum_{j=0..k-1} gates[t,j] * y[comb_row[t,j]]
+ * computed per element in fp32 as acc = +0.0f; acc = fmaf(gates[t,j], y, acc) for
+ * j = 0, 1, ..., k-1 in that order (one rounding per step), then stored as fp32 or
+ * rounded to bf16 nearest-even.
+ * y: bf16 [n_rows, H] expert outputs in expanded receive order (n_rows = N*k for a full
+ * plan); gates: fp32 [N, k]; comb_row: int32 [N, k]; out: [N, H] of bf16 (out_dtype 0)
+ * or fp32 (out_dtype 1).  A comb_row entry outside [0, n_rows) is skipped: -1 silently
+ * (a slot of an invalid token), any other value with COACT_EFLAG_ROW_RANGE.
+ */
+int combine_scatter(const uint16_t *y, int64_t n_rows, const float *gates,
+                    const int32_t *comb_row, int64_t N, int k, int64_t H,
+                    void *out, int out_dtype,
+                    int32_t *err_flag, coact_stream_t stream);
+
+/* Bytes of device workspace predict_home needs (E1*R int64 scores). */
+size_t predict_home_workspace_bytes(int E1, int R);
+
+/*
+ * predict_home -- token shuffling's home-rank prediction.
+ * Zyphra, English abstract: when sequence parallelism shards tokens across the EP
+ * group, each token is moved to the GPU predicted to hold its next-layer experts.
+ * Prediction from cross-layer counts C12 (coact_count in cross mode over a calibration
+ * batch):
+ *   score(t, r) = sum_j sum_{b : expert_rank2[b] == r} C12[ids1[t,j] * E2 + b]
+ *   home[t]     = argmax_r score(t, r), ties to the lowest r
+ * ids1: int32 [N, k1] (layer-1 ids); C12: int64 [E1*E2]; expert_rank2: int32 [E2];
+ * home: int32 [N] (then usable as plan_dispatch's src_rank).  workspace: at least
+ * predict_home_workspace_bytes(E1, R) bytes.  Tokens with invalid ids get home = -1
+ * and set their flag; layer-2 experts with a rank outside [0, R) set
+ * COACT_EFLAG_ID_RANGE and are ignored.
+ */
+int predict_home(const int32_t *ids1, int64_t N, int k1, int E1,
+                 const int64_t *C12, int E2, const int32_t *expert_rank2, int R,
+                 int32_t *home, void *workspace, size_t workspace_bytes,
+                 int32_t *err_flag, coact_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* COACT_H */

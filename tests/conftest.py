@@ -17,3 +17,16 @@ def pages_figures():
     import json
     with open(os.path.join(ROOT, "tests", "golden", "pages_figures.json")) as f:
         return json.load(f)
+
+
+def pytest_sessionstart(session):
+    # The CUDA library is built in-tree (nvcc is part of the image on every box); this
+    # only compiles when a source is newer than libcoact.so or the library is missing.
+    build_library()
+
+
+def build_library() -> str:
+    """Runs co_activation_b200/build.py by path (importing the package needs the library)."""
+    import runpy
+    mod = runpy.run_path(os.path.join(ROOT, "co_activation_b200", "build.py"))
+    return mod["build"]()

@@ -1,0 +1,131 @@
+"""The C-ABI library without a GPU: it loads, exports every function include/coact.h
+declares, and rejects bad arguments on the host (nothing enqueued, no CUDA call)."""
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "coact.h")
+
+
+def _ensure_built():
+    from conftest import build_library
+    return build_library()
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = _ensure_built()
+    return ctypes.CDLL(path)
+
+
+def header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_path():
+    fns = header_functions()
+    for f in ("coact_count", "plan_dispatch", "dispatch_gather", "combine_scatter",
+              "predict_home", "plan_dispatch_workspace_bytes", "coact_strerror"):
+        assert f in fns
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [f for f in header_functions() if not hasattr(lib, f)]
+    assert not missing, missing
+    out = subprocess.run(["nm", "-D", "--defined-only", lib._name], capture_output=True, text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert set(header_functions()) <= exported
+
+
+def test_binding_names_match_header():
+    import co_activation_b200 as coact
+    assert set(coact.ABI_SYMBOLS) == set(header_functions())
+    for f in ("coact_count", "plan_dispatch", "dispatch_gather", "combine_scatter", "predict_home"):
+        assert callable(getattr(coact, f))
+
+
+def test_strerror_and_version(lib):
+    lib.coact_strerror.restype = ctypes.c_char_p
+    assert lib.coact_strerror(0) == b"ok"
+    assert b"workspace" in lib.coact_strerror(-4)
+    assert lib.coact_abi_version() == 1
+
+
+P = ctypes.c_void_p
+FAKE = P(256)   # a non-NULL, 16-byte aligned address the library never dereferences on host
+
+
+def test_count_rejects_bad_arguments(lib):
+    f = lib.coact_count
+    f.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, ctypes.c_int, ctypes.c_int,
+                  P, P, P, P]
+    assert f(FAKE, -1, 2, 8, None, 0, 0, FAKE, None, None, None) == -1      # N < 0
+    assert f(FAKE, 10, 2, 8, None, 0, 0, None, None, None, None) == -1      # pair NULL
+    assert f(FAKE, 10, 9, 8, None, 0, 0, FAKE, None, None, None) == -2      # k > 8
+    assert f(FAKE, 10, 2, 1, None, 0, 0, FAKE, None, None, None) == -2      # E < 2
+    assert f(FAKE, 10, 2, 2000, None, 0, 0, FAKE, None, None, None) == -2   # E > 1024
+    assert f(FAKE, 10, 2, 8, FAKE, 0, 8, FAKE, None, None, None) == -2      # bad k2
+    assert f(None, 0, 2, 8, None, 0, 0, FAKE, None, None, None) == 0        # N == 0: no-op
+
+
+def test_plan_rejects_bad_arguments(lib):
+    f = lib.plan_dispatch
+    f.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int,
+                  P, P, P, P, P, P, P, ctypes.c_int64, P, P, P, P, P, ctypes.c_size_t, P, P]
+    lib.plan_dispatch_workspace_bytes.restype = ctypes.c_size_t
+    lib.plan_dispatch_workspace_bytes.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    need = lib.plan_dispatch_workspace_bytes(4096, 2, 8, 4)
+    assert need > 0
+
+    def call(N=4096, k=2, E=8, R=4, ws=need, wsp=FAKE, cap=8192, n_nodes=1, rank_node=None):
+        return f(FAKE, N, k, E, FAKE, R, rank_node, n_nodes, None, FAKE, FAKE, FAKE, None, FAKE,
+                 FAKE, cap, FAKE, FAKE, FAKE, None, wsp, ws, None, None)
+
+    assert call(R=65) == -2
+    assert call(R=0) == -2
+    assert call(k=0) == -2
+    assert call(N=-5) == -1
+    assert call(cap=-1) == -1
+    assert call(ws=need - 1) == -4
+    assert call(wsp=None) == -4
+    assert call(wsp=P(264)) == -4                                  # misaligned workspace
+    assert call(rank_node=FAKE, n_nodes=65) == -2
+
+
+def test_gather_combine_reject_bad_arguments(lib):
+    g = lib.dispatch_gather
+    g.argtypes = [P, ctypes.c_int64, ctypes.c_int64, P, ctypes.c_int, P, ctypes.c_int64, P, P]
+    assert g(FAKE, 10, 12, FAKE, 2, FAKE, 20, None, None) == -2    # H % 8 != 0
+    assert g(P(258), 10, 16, FAKE, 2, FAKE, 20, None, None) == -1  # misaligned x
+    assert g(FAKE, 10, 16, FAKE, 9, FAKE, 20, None, None) == -2    # k > 8
+    assert g(None, 0, 16, None, 2, None, 0, None, None) == 0       # empty
+    c = lib.combine_scatter
+    c.argtypes = [P, ctypes.c_int64, P, P, ctypes.c_int64, ctypes.c_int, ctypes.c_int64, P,
+                  ctypes.c_int, P, P]
+    assert c(FAKE, 20, FAKE, FAKE, 10, 2, 16, FAKE, 2, None, None) == -2   # out dtype
+    assert c(FAKE, 20, None, FAKE, 10, 2, 16, FAKE, 0, None, None) == -1   # gates NULL
+    assert c(FAKE, 20, FAKE, FAKE, 10, 2, 16, P(260), 0, None, None) == -1  # misaligned out
+    assert c(None, 0, None, None, 0, 2, 16, None, 0, None, None) == 0      # empty
+
+
+def test_predict_rejects_bad_arguments(lib):
+    p = lib.predict_home
+    p.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int,
+                  P, P, ctypes.c_size_t, P, P]
+    assert p(FAKE, 10, 2, 8, FAKE, 8, FAKE, 65, FAKE, FAKE, 4096, None, None) == -2
+    assert p(FAKE, 10, 2, 8, FAKE, 8, FAKE, 4, FAKE, FAKE, 8, None, None) == -4
+
+
+def test_binding_fails_loudly_without_library():
+    env = dict(os.environ, COACT_LIB="/nonexistent/libcoact.so")
+    r = subprocess.run([sys.executable, "-c", "import co_activation_b200"], cwd=ROOT, env=env,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "libcoact.so not found" in r.stderr

@@ -1,0 +1,410 @@
+"""GPU parity: the CUDA library (through the C ABI) against the CPU oracle on the same
+seeded inputs.  Integers, masks, offsets, positions and gathered rows must be
+bit-exact; the combine must match the float64 reference within the stated tolerance
+and the fixed-order fp32 chain bit for bit.  Full-size workloads are checked in full
+where the oracle is fast (counts, plans) and on sampled rows otherwise (gathered rows,
+combined rows), with the same launch configuration the benchmark times."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workload
+from _gpu_util import (DEV, X_STREAM, Y_STREAM, assert_plan_equal, check_combine, cuda,
+                       host_bits, plan_to_host, run_plan)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def coact():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import co_activation_b200 as c
+    return c
+
+
+def zero_flag():
+    return torch.zeros(1, dtype=torch.int32, device=DEV)
+
+
+def oracle_plan_for(r, **kw):
+    cfg = r.cfg
+    args = dict(E=cfg.E, expert_rank=r.expert_rank, R=cfg.R, rank_node=r.rank_node,
+                n_nodes=cfg.n_nodes, src_rank=None)
+    args.update(kw)
+    return oracle.plan(r.ids, args["E"], args["expert_rank"], args["R"],
+                       rank_node=args["rank_node"], n_nodes=args["n_nodes"],
+                       src_rank=args["src_rank"], row_capacity=args.get("row_capacity"))
+
+
+# ----------------------------------------------------------------------------- counting
+
+
+@pytest.mark.parametrize("cfg", [0, 1, 2, 3])
+def test_count_full_size(coact, cfg):
+    r = workload.make_routing(cfg)
+    E = r.cfg.E
+    pair = torch.zeros((E, E), dtype=torch.int64, device=DEV)
+    loads = torch.zeros(E, dtype=torch.int64, device=DEV)
+    err = zero_flag()
+    ids = cuda(r.ids)
+    coact.coact_count(ids, E, pair, loads, err_flag=err)
+    op, ol, f = oracle.count(r.ids, E)
+    assert f == 0 and err.item() == 0
+    assert np.array_equal(pair.cpu().numpy(), op)
+    assert np.array_equal(loads.cpu().numpy(), ol)
+    coact.coact_count(ids, E, pair, loads)                 # accumulates
+    assert np.array_equal(pair.cpu().numpy(), 2 * op)
+    assert np.array_equal(loads.cpu().numpy(), 2 * ol)
+
+
+@pytest.mark.parametrize("N,E,k", [(1, 8, 2), (37, 8, 3), (5000, 1024, 4), (3000, 300, 8),
+                                   (70000, 32, 5), (2049, 256, 1)])
+def test_count_shapes(coact, N, E, k):
+    rng = np.random.default_rng(N + E + k)
+    ids = np.argsort(rng.random((N, E)), axis=1)[:, :k].astype(np.int32)
+    pair = torch.zeros((E, E), dtype=torch.int64, device=DEV)
+    loads = torch.zeros(E, dtype=torch.int64, device=DEV)
+    coact.coact_count(cuda(ids), E, pair, loads)
+    op, ol, _ = oracle.count(ids, E)
+    assert np.array_equal(pair.cpu().numpy(), op) and np.array_equal(loads.cpu().numpy(), ol)
+
+
+def test_count_flags_and_skips(coact):
+    r = workload.make_routing(0)
+    ids = r.ids.copy()
+    ids[10, 0] = 8           # out of range
+    ids[20, 1] = ids[20, 0]  # repeated
+    ids[30, 0] = -1
+    pair = torch.zeros((8, 8), dtype=torch.int64, device=DEV)
+    loads = torch.zeros(8, dtype=torch.int64, device=DEV)
+    err = zero_flag()
+    coact.coact_count(cuda(ids), 8, pair, loads, err_flag=err)
+    op, ol, f = oracle.count(ids, 8)
+    assert err.item() == f == (coact.EFLAG_ID_RANGE | coact.EFLAG_DUP_ID)
+    assert np.array_equal(pair.cpu().numpy(), op) and np.array_equal(loads.cpu().numpy(), ol)
+
+
+def test_count_cross_full_size(coact):
+    tl = workload.make_two_layer(4)
+    E = tl.layer1.cfg.E
+    C = torch.zeros((E, E), dtype=torch.int64, device=DEV)
+    l1 = torch.zeros(E, dtype=torch.int64, device=DEV)
+    coact.coact_count(cuda(tl.calib1), E, C, l1, ids2=cuda(tl.calib2), E2=E)
+    oc, ol, f = oracle.count_cross(tl.calib1, E, tl.calib2, E)
+    assert f == 0
+    assert np.array_equal(C.cpu().numpy(), oc) and np.array_equal(l1.cpu().numpy(), ol)
+
+
+def test_count_deterministic(coact):
+    r = workload.make_routing(3)
+    outs = []
+    for _ in range(3):
+        pair = torch.zeros((256, 256), dtype=torch.int64, device=DEV)
+        coact.coact_count(cuda(r.ids), 256, pair)
+        outs.append(pair.cpu().numpy())
+    assert all(np.array_equal(outs[0], o) for o in outs[1:])
+
+
+# ----------------------------------------------------------------------------- plans
+
+
+@pytest.mark.parametrize("cfg", [0, 1, 2, 3])
+def test_plan_full_size(coact, cfg):
+    r = workload.make_routing(cfg)
+    plan, err = run_plan(coact, r)
+    o = oracle_plan_for(r)
+    assert err.item() == 0 and o["flags"] == 0
+    assert_plan_equal(plan_to_host(plan), o)
+
+
+@pytest.mark.parametrize("variant", ["identity", "one_rank", "roundrobin3", "random_src2",
+                                     "two_nodes1", "ragged"])
+def test_plan_variants(coact, variant):
+    if variant == "identity":            # every expert alone on its rank: D == N*k
+        r = workload.make_routing(0)
+        kw = dict(E=8, expert_rank=np.arange(8, dtype=np.int32), R=8,
+                  rank_node=np.zeros(8, np.int32), n_nodes=1)
+    elif variant == "one_rank":          # one rank: nothing remote, D == N
+        r = workload.make_routing(1)
+        kw = dict(expert_rank=np.zeros(64, np.int32), R=1, rank_node=np.zeros(1, np.int32))
+    elif variant == "roundrobin3":
+        r = workload.make_routing(3, placement_kind="roundrobin")
+        kw = {}
+    elif variant == "random_src2":
+        r = workload.make_routing(2)
+        kw = dict(src_rank=np.random.default_rng(5).integers(0, 32, r.N).astype(np.int32))
+    elif variant == "two_nodes1":
+        r = workload.make_routing(1)
+        kw = dict(rank_node=(np.arange(8) // 4).astype(np.int32), n_nodes=2)
+    else:                                # token counts that leave partial warps and tiles
+        r = workload.make_routing(2, N=65536 - 4093)
+        kw = {}
+    o = oracle_plan_for(r, **kw)
+    plan, err = run_plan(coact, r, E=kw.get("E"), expert_rank=kw.get("expert_rank"),
+                         R=kw.get("R"), rank_node=kw.get("rank_node"),
+                         n_nodes=kw.get("n_nodes"), src_rank=kw.get("src_rank"))
+    assert err.item() == 0
+    g = plan_to_host(plan)
+    assert_plan_equal(g, o)
+    if variant == "identity":
+        assert g["rank_offsets"][-1] == r.N * r.k
+    if variant == "one_rank":
+        assert g["rank_offsets"][-1] == r.N and g["stats"][2] == 0
+
+
+@pytest.mark.parametrize("N,E,k,R,nodes", [(1, 8, 2, 4, 1), (31, 16, 3, 4, 2), (257, 64, 8, 64, 8),
+                                           (1000, 128, 6, 16, 4), (4096, 1024, 8, 64, 8),
+                                           (513, 12, 1, 3, 1)])
+def test_plan_shapes(coact, N, E, k, R, nodes):
+    rng = np.random.default_rng(N * 7 + k)
+    cfg = workload.CONFIGS[0].with_(N=N, E=E, k=k, R=R, n_nodes=nodes)
+    ids = np.argsort(rng.random((N, E)), axis=1)[:, :k].astype(np.int32)
+    er = (rng.permutation(E) % R).astype(np.int32)
+    rn = (np.arange(R) * nodes // R).astype(np.int32)
+    src = rng.integers(0, R, N).astype(np.int32)
+    r = workload.Routing(cfg=cfg, ids=ids, gates=np.full((N, k), 1.0 / k, np.float32),
+                         expert_rank=er, rank_node=rn, src_rank=src,
+                         groups=np.zeros((0, 2), np.int32), planted=np.zeros(N, bool), seed=0)
+    o = oracle.plan(ids, E, er, R, rank_node=rn, n_nodes=nodes, src_rank=src)
+    plan, err = run_plan(coact, r, src_rank=src)
+    assert err.item() == 0
+    assert_plan_equal(plan_to_host(plan), o)
+
+
+def test_plan_empty(coact):
+    cfg = workload.CONFIGS[0].with_(N=0)
+    r = workload.Routing(cfg=cfg, ids=np.zeros((0, 2), np.int32), gates=np.zeros((0, 2), np.float32),
+                         expert_rank=np.arange(8, dtype=np.int32) // 2,
+                         rank_node=np.zeros(4, np.int32), src_rank=np.zeros(0, np.int32),
+                         groups=np.zeros((0, 2), np.int32), planted=np.zeros(0, bool), seed=0)
+    plan, err = run_plan(coact, r, sentinel=False)
+    assert err.item() == 0
+    assert plan.rank_offsets.cpu().tolist() == [0] * 5
+    assert plan.stats.cpu().tolist() == [0] * 8
+
+
+def test_plan_capacity_overflow(coact):
+    r = workload.make_routing(1)
+    full = oracle_plan_for(r)
+    cap = full["D"] - 1000
+    o = oracle_plan_for(r, row_capacity=cap)
+    plan, err = run_plan(coact, r, row_capacity=cap)
+    assert err.item() == coact.EFLAG_CAPACITY and o["flags"] == oracle.FLAG_CAPACITY
+    assert_plan_equal(plan_to_host(plan), o, sentinel=False)
+
+
+def test_plan_invalid_tokens(coact):
+    r = workload.make_routing(0)
+    ids = r.ids.copy()
+    ids[5, 1] = 99
+    ids[6, 1] = ids[6, 0]
+    src = r.src_rank.copy()
+    src[7] = 4
+    r2 = workload.Routing(**{**r.__dict__, "ids": ids})
+    o = oracle_plan_for(r2, src_rank=src)
+    plan, err = run_plan(coact, r2, src_rank=src)
+    assert err.item() == o["flags"] == (oracle.FLAG_ID_RANGE | oracle.FLAG_DUP_ID | oracle.FLAG_SRC_RANK)
+    assert_plan_equal(plan_to_host(plan), o)
+
+
+def test_plan_deterministic(coact):
+    r = workload.make_routing(3)
+    a = plan_to_host(run_plan(coact, r)[0])
+    b = plan_to_host(run_plan(coact, r)[0])
+    for key in a:
+        assert np.array_equal(a[key], b[key]), key
+
+
+# ----------------------------------------------------------------------------- gather
+
+
+def _gather(coact, r, H, plan, sentinel_rows=True):
+    x = workload.fill_bf16(r.N, H, r.seed, X_STREAM, device=DEV)
+    send = torch.empty((plan.row_capacity, H), dtype=torch.bfloat16, device=DEV)
+    if sentinel_rows:
+        send.view(torch.int16).fill_(-1)
+    err = zero_flag()
+    coact.dispatch_gather(x, plan.send_row, send, err_flag=err)
+    torch.cuda.synchronize()
+    return x, send, err
+
+
+@pytest.mark.parametrize("cfg", [0, 1])
+def test_gather_full(coact, cfg):
+    r = workload.make_routing(cfg)
+    H = r.cfg.H
+    plan, _ = run_plan(coact, r)
+    o = oracle_plan_for(r)
+    x, send, err = _gather(coact, r, H, plan)
+    assert err.item() == 0
+    xh = host_bits(workload.fill_bf16(r.N, H, r.seed, X_STREAM))
+    want = oracle.gather(xh, o["row_token"], o["D"])
+    got = host_bits(send)
+    assert np.array_equal(got[:o["D"]], want)
+    assert (got[o["D"]:] == 0xFFFF).all()                   # rows past D untouched
+
+
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_gather_full_size_sampled(coact, cfg):
+    r = workload.make_routing(cfg)
+    H = r.cfg.H
+    plan, _ = run_plan(coact, r)
+    o = oracle_plan_for(r)
+    x, send, err = _gather(coact, r, H, plan)
+    assert err.item() == 0
+    D, cap = o["D"], plan.row_capacity
+    rng = np.random.default_rng(cfg)
+    rows = np.unique(np.concatenate([rng.integers(0, D, 1500), [0, D - 1]]))
+    want = host_bits(workload.fill_bf16(len(rows), H, r.seed, X_STREAM,
+                                        row_ids=o["row_token"][rows]))
+    got = host_bits(send[torch.as_tensor(rows, device=DEV)])
+    assert np.array_equal(got, want)
+    if D < cap:
+        tail = np.unique(rng.integers(D, cap, 64))
+        assert (host_bits(send[torch.as_tensor(tail, device=DEV)]) == 0xFFFF).all()
+
+
+@pytest.mark.parametrize("H", [8, 256, 520, 2048, 7168, 16400])
+def test_gather_row_sizes(coact, H):
+    # covers the vector path (short, odd-length and very long rows) and the bulk path
+    r = workload.make_routing(2, N=3001)
+    plan, _ = run_plan(coact, r)
+    o = oracle_plan_for(r)
+    x, send, err = _gather(coact, r, H, plan)
+    assert err.item() == 0
+    want = oracle.gather(host_bits(x), o["row_token"], o["D"])
+    got = host_bits(send)
+    assert np.array_equal(got[:o["D"]], want)
+    assert (got[o["D"]:] == 0xFFFF).all()
+
+
+def test_gather_row_range_flag(coact):
+    N, H, k = 100, 64, 2
+    x = workload.fill_bf16(N, H, 0, 1, device=DEV)
+    send_row = torch.full((N, k), -1, dtype=torch.int32, device=DEV)
+    send_row[:, 0] = torch.arange(N, dtype=torch.int32, device=DEV)
+    send_row[3, 1] = 100                                     # == capacity: out of range
+    send = torch.zeros((N, H), dtype=torch.bfloat16, device=DEV)
+    err = zero_flag()
+    coact.dispatch_gather(x, send_row, send, err_flag=err)
+    assert err.item() == coact.EFLAG_ROW_RANGE
+    assert torch.equal(send, x)
+
+
+# ----------------------------------------------------------------------------- combine
+
+
+@pytest.mark.parametrize("cfg", [0, 1])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_combine_full(coact, cfg, out_dtype):
+    r = workload.make_routing(cfg)
+    H, nk = r.cfg.H, r.N * r.k
+    plan, _ = run_plan(coact, r)
+    o = oracle_plan_for(r)
+    y = workload.fill_bf16(nk, H, r.seed, Y_STREAM, device=DEV)
+    out = torch.empty((r.N, H), dtype=out_dtype, device=DEV)
+    err = zero_flag()
+    coact.combine_scatter(y, cuda(r.gates), plan.comb_row, out, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    yh = host_bits(workload.fill_bf16(nk, H, r.seed, Y_STREAM))
+    check_combine(out, yh, r.gates, o["comb_row"])
+
+
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_combine_full_size_sampled(coact, cfg):
+    r = workload.make_routing(cfg)
+    H, nk = r.cfg.H, r.N * r.k
+    plan, _ = run_plan(coact, r)
+    o = oracle_plan_for(r)
+    y = workload.fill_bf16(nk, H, r.seed, Y_STREAM, device=DEV)
+    out = torch.empty((r.N, H), dtype=torch.bfloat16, device=DEV)
+    coact.combine_scatter(y, cuda(r.gates), plan.comb_row, out)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(10 + cfg)
+    toks = np.unique(np.concatenate([rng.integers(0, r.N, 300), [0, r.N - 1]]))
+    rows = o["comb_row"][toks]                               # oracle's rows for these tokens
+    yh = host_bits(workload.fill_bf16(rows.size, H, r.seed, Y_STREAM, row_ids=rows.ravel()))
+    local = np.arange(rows.size, dtype=np.int32).reshape(rows.shape)
+    check_combine(out, yh, r.gates[toks], local, tokens=toks)
+    del y, out
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("H", [8, 1000])
+def test_combine_k_and_h(coact, k, H):
+    rng = np.random.default_rng(k * 100 + H)
+    N = 777
+    gates = rng.random((N, k)).astype(np.float32)
+    comb = rng.permutation(N * k).reshape(N, k).astype(np.int32)
+    y = workload.fill_bf16(N * k, H, k, 3, device=DEV)
+    for dt in (torch.bfloat16, torch.float32):
+        out = torch.empty((N, H), dtype=dt, device=DEV)
+        coact.combine_scatter(y, cuda(gates), cuda(comb), out)
+        check_combine(out, host_bits(y), gates, comb)
+
+
+def test_combine_invalid_rows(coact):
+    N, k, H = 64, 3, 16
+    rng = np.random.default_rng(1)
+    gates = rng.random((N, k)).astype(np.float32)
+    comb = rng.permutation(N * k).reshape(N, k).astype(np.int32)
+    comb[4, 1] = -1                       # an invalid token's slot: skipped silently
+    comb[9, 2] = N * k + 5                # out of range: skipped and flagged
+    y = workload.fill_bf16(N * k, H, 0, 4, device=DEV)
+    out = torch.empty((N, H), dtype=torch.float32, device=DEV)
+    err = zero_flag()
+    coact.combine_scatter(y, cuda(gates), cuda(comb), out, err_flag=err)
+    assert err.item() == coact.EFLAG_ROW_RANGE
+    check_combine(out, host_bits(y), gates, comb)
+
+
+# ----------------------------------------------------------------------------- the whole path
+
+
+@pytest.mark.parametrize("cfg", [0, 1, 2])
+def test_identity_experts_end_to_end(coact, cfg):
+    """plan -> gather -> identity experts -> combine reproduces the naive (one row per
+    token-expert pair) combine bit for bit: deduplication leaves the result unchanged."""
+    r = workload.make_routing(cfg, N=min(workload.CONFIGS[cfg].N, 16384))
+    H = min(r.cfg.H, 1024)
+    plan, _ = run_plan(coact, r)
+    x, send, _ = _gather(coact, r, H, plan, sentinel_rows=False)
+    D = int(plan.rank_offsets[-1].item())
+    reps = torch.bitwise_count(plan.row_kmask[:D].to(torch.int32)) if hasattr(torch, "bitwise_count") \
+        else torch.tensor([bin(int(v)).count("1") for v in plan.row_kmask[:D].cpu()], device=DEV)
+    y = send[:D].repeat_interleave(reps.to(torch.int64), dim=0)     # identity experts
+    assert y.shape[0] == r.N * r.k
+    out = torch.empty((r.N, H), dtype=torch.float32, device=DEV)
+    coact.combine_scatter(y, cuda(r.gates), plan.comb_row, out)
+    want = oracle.naive_combine_identity_f32(host_bits(x), r.gates)
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), want.view(np.uint32))
+
+
+def test_token_shuffle_two_layers(coact):
+    """Config 4: cross-layer counts on a calibration batch -> predicted home rank ->
+    layer-2 plan with the tokens pre-sharded to it; every step against the oracle."""
+    tl = workload.make_two_layer(4)
+    cfg = tl.layer1.cfg
+    E, R = cfg.E, cfg.R
+    C = torch.zeros((E, E), dtype=torch.int64, device=DEV)
+    coact.coact_count(cuda(tl.calib1), E, C, ids2=cuda(tl.calib2), E2=E)
+    oc, _, _ = oracle.count_cross(tl.calib1, E, tl.calib2, E)
+    assert np.array_equal(C.cpu().numpy(), oc)
+    er2 = tl.layer2.expert_rank
+    home = torch.empty(tl.layer1.N, dtype=torch.int32, device=DEV)
+    err = zero_flag()
+    coact.predict_home(cuda(tl.layer1.ids), E, C, cuda(er2), R, home, err_flag=err)
+    oh, f = oracle.predict_home(tl.layer1.ids, E, oc, er2, R)
+    assert err.item() == 0 and f == 0
+    assert np.array_equal(home.cpu().numpy(), oh)
+    plan, err = run_plan(coact, tl.layer2, src_rank=oh)
+    o = oracle_plan_for(tl.layer2, src_rank=oh)
+    assert err.item() == 0
+    assert_plan_equal(plan_to_host(plan), o)
+    base = oracle_plan_for(tl.layer2)
+    nk = tl.layer2.N * tl.layer2.k
+    shuffled, baseline = o["stats"][5] / nk, base["stats"][5] / nk
+    assert abs(baseline - 1.0 / R) < 0.01       # contiguous shards: 1/R served locally
+    assert shuffled > 2 * baseline              # prediction keeps far more assignments local
