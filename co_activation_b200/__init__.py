@@ -51,12 +51,14 @@ _lib.combine_scatter.argtypes = [_P, _I64, _P, _P, _I64, _I32, _I64, _P, _I32, _
 _lib.predict_home_workspace_bytes.argtypes = [_I32, _I32]
 _lib.predict_home_workspace_bytes.restype = _SZ
 _lib.predict_home.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _SZ, _P, _P]
-for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "combine_scatter", "predict_home"):
+_lib.coact_place_correlated.argtypes = [_P, _I32, _I32, _P]
+for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "combine_scatter", "predict_home",
+           "coact_place_correlated"):
     getattr(_lib, _f).restype = _I32
 
 ABI_SYMBOLS = ("coact_strerror", "coact_abi_version", "coact_count", "plan_dispatch_workspace_bytes",
                "plan_dispatch", "dispatch_gather", "combine_scatter",
-               "predict_home_workspace_bytes", "predict_home")
+               "predict_home_workspace_bytes", "predict_home", "coact_place_correlated")
 
 
 class CoactError(RuntimeError):
@@ -272,3 +274,16 @@ def predict_home(ids1: torch.Tensor, E1: int, C12: torch.Tensor, expert_rank2: t
                              _ptr(home), _ptr(workspace), workspace.numel(), _ptr(err_flag),
                              _stream(stream)), "predict_home")
     return home
+
+
+def coact_place_correlated(pair, R: int):
+    """Correlated expert placement from co-activation counts (host computation in the
+    library).  `pair`: int64 [E, E] counts (any device; copied to host).  Returns an
+    int32 CPU tensor expert -> rank with E/R experts per rank."""
+    p = pair.detach().to("cpu", torch.int64).contiguous()
+    E = p.shape[0]
+    if tuple(p.shape) != (E, E):
+        raise ValueError("pair must be [E, E]")
+    out = torch.empty(E, dtype=torch.int32)
+    _check(_lib.coact_place_correlated(_ptr(p), E, R, _ptr(out)), "coact_place_correlated")
+    return out

@@ -1,0 +1,74 @@
+// coact_place_correlated: correlated expert placement from co-activation counts.
+//
+// Zyphra (arxivdaily 2610.09372), English abstract: correlated expert placement puts
+// experts that are often selected together on the same GPU; together with the
+// once-per-GPU dispatcher it removes dispatched rows.  Cobalt (arxivdaily 2609.36959),
+// English abstract: frequently co-activated experts are co-located to cut cross-node
+// traffic.  The pages give no algorithm; this is the plain greedy reading:
+//   1. weight(a, b) = pair[a][b] + pair[b][a] for every a < b with weight > 0;
+//   2. visit pairs by weight descending, ties by (a, b) ascending;
+//   3. both experts unplaced -> the lowest rank with two free slots;
+//      one placed and its rank has a free slot -> the other joins it;
+//   4. experts still unplaced, ascending id -> the lowest rank with a free slot.
+// Every rank ends with exactly E / R experts.  Host code: reads a host copy of the
+// counts, writes a host array.
+#include <algorithm>
+#include <vector>
+
+#include "coact.h"
+
+extern "C" int coact_place_correlated(const int64_t *pair, int E, int R, int32_t *expert_rank) {
+    if (!pair || !expert_rank) return COACT_ERR_INVALID;
+    if (E < 2 || E > COACT_MAX_E || R < 1 || R > COACT_MAX_R || E % R != 0)
+        return COACT_ERR_UNSUPPORTED;
+    const int slots = E / R;
+    struct Edge {
+        int64_t w;
+        int a, b;
+    };
+    std::vector<Edge> edges;
+    edges.reserve((size_t)E * (E - 1) / 2);
+    for (int a = 0; a < E; ++a)
+        for (int b = a + 1; b < E; ++b) {
+            const int64_t w = pair[(int64_t)a * E + b] + pair[(int64_t)b * E + a];
+            if (w > 0) edges.push_back({w, a, b});
+        }
+    std::sort(edges.begin(), edges.end(), [](const Edge &x, const Edge &y) {
+        if (x.w != y.w) return x.w > y.w;
+        if (x.a != y.a) return x.a < y.a;
+        return x.b < y.b;
+    });
+    std::vector<int> rank_of(E, -1), free_slots(R, slots);
+    for (const Edge &ed : edges) {
+        const int ra = rank_of[ed.a], rb = rank_of[ed.b];
+        if (ra < 0 && rb < 0) {
+            for (int r = 0; r < R; ++r)
+                if (free_slots[r] >= 2) {
+                    rank_of[ed.a] = rank_of[ed.b] = r;
+                    free_slots[r] -= 2;
+                    break;
+                }
+        } else if (ra >= 0 && rb < 0) {
+            if (free_slots[ra] > 0) {
+                rank_of[ed.b] = ra;
+                free_slots[ra] -= 1;
+            }
+        } else if (rb >= 0 && ra < 0) {
+            if (free_slots[rb] > 0) {
+                rank_of[ed.a] = rb;
+                free_slots[rb] -= 1;
+            }
+        }
+    }
+    for (int e = 0; e < E; ++e) {
+        if (rank_of[e] >= 0) continue;
+        for (int r = 0; r < R; ++r)
+            if (free_slots[r] > 0) {
+                rank_of[e] = r;
+                free_slots[r] -= 1;
+                break;
+            }
+    }
+    for (int e = 0; e < E; ++e) expert_rank[e] = rank_of[e];
+    return COACT_OK;
+}

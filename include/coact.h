@@ -215,6 +215,22 @@ int predict_home(const int32_t *ids1, int64_t N, int k1, int E1,
                  int32_t *home, void *workspace, size_t workspace_bytes,
                  int32_t *err_flag, coact_stream_t stream);
 
+/*
+ * coact_place_correlated -- correlated expert placement (HOST function).
+ * Zyphra, English abstract: experts that are often selected together go on the same
+ * GPU, which with the once-per-GPU dispatcher removes dispatched rows; Cobalt, English
+ * abstract: co-activated experts are co-located to cut cross-node traffic.  The pages
+ * give no algorithm; this is a plain greedy over the pair counts:
+ *   weight(a,b) = pair[a*E+b] + pair[b*E+a] for a < b, pairs with weight > 0 visited by
+ *   weight descending (ties: a, then b ascending); two unplaced experts go together to
+ *   the lowest rank with two free slots, an unplaced expert joins its placed partner if
+ *   that rank has a free slot; remaining experts, ascending id, fill the lowest rank
+ *   with a free slot.  Every rank receives exactly E/R experts.
+ * pair: HOST int64 [E*E] (e.g. a copy of coact_count's output); expert_rank: HOST
+ * int32 [E] output.  Requires E % R == 0.  Synchronous; no CUDA call.
+ */
+int coact_place_correlated(const int64_t *pair, int E, int R, int32_t *expert_rank);
+
 #ifdef __cplusplus
 }
 #endif

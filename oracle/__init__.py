@@ -64,6 +64,7 @@ def _get():
             _lib.oracle_naive_combine_identity_f32.argtypes = [P, P, I64, I32, I64, P]
             _lib.oracle_naive_combine_identity_f32.restype = None
             _lib.oracle_predict_home.argtypes = [P, I64, I32, I32, P, I32, P, I32, P]
+            _lib.oracle_place_correlated.argtypes = [P, I32, I32, P]
         return _lib
 
 
@@ -225,3 +226,13 @@ def predict_home(ids1, E1: int, C12, expert_rank2, R: int):
     home = np.zeros(N, np.int32)
     f = _get().oracle_predict_home(_p(ids1), N, k1, E1, _p(C), E2, _p(er2), R, _p(home))
     return home, f
+
+
+def place_correlated(pair, R: int) -> np.ndarray:
+    """Greedy correlated placement from pair counts (int32 expert -> rank, [E])."""
+    pr = _c(pair, np.int64)
+    E = pr.shape[0]
+    out = np.zeros(E, np.int32)
+    if _get().oracle_place_correlated(_p(pr), E, R, _p(out)) != 0:
+        raise ValueError("E must be a multiple of R")
+    return out

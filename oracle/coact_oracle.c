@@ -387,3 +387,70 @@ int oracle_predict_home(const int32_t *ids1, int64_t N, int k1, int E1, const in
     }
     return flags;
 }
+
+/*
+ * Correlated expert placement.  [Zyphra] experts that are often selected together are
+ * put on the same GPU; [Cobalt] frequently co-activated experts are co-located.  The
+ * pages give no algorithm; the reading is a greedy over pair weights
+ * w(a,b) = pair[a][b] + pair[b][a] (a < b, w > 0), heaviest first (ties: smaller a, then
+ * smaller b): two unplaced experts take the lowest rank with two free slots; an unplaced
+ * expert joins its placed partner's rank if a slot is free; then every unplaced expert,
+ * in ascending id, takes the lowest rank with a free slot.  E/R slots per rank.
+ */
+typedef struct { int64_t w; int a, b; } oracle_edge;
+
+static int edge_order(const void *p, const void *q) {
+    const oracle_edge *x = (const oracle_edge *)p, *y = (const oracle_edge *)q;
+    if (x->w != y->w) return x->w > y->w ? -1 : 1;
+    if (x->a != y->a) return x->a < y->a ? -1 : 1;
+    if (x->b != y->b) return x->b < y->b ? -1 : 1;
+    return 0;
+}
+
+int oracle_place_correlated(const int64_t *pair, int E, int R, int32_t *expert_rank) {
+    if (E % R != 0) return -1;
+    int per_rank = E / R;
+    oracle_edge *edges = (oracle_edge *)malloc(sizeof(oracle_edge) * (size_t)E * (size_t)E);
+    int *free_slots = (int *)malloc(sizeof(int) * (size_t)R);
+    int64_t n = 0;
+    for (int a = 0; a < E; ++a)
+        for (int b = a + 1; b < E; ++b) {
+            int64_t w = pair[(int64_t)a * E + b] + pair[(int64_t)b * E + a];
+            if (w > 0) { edges[n].w = w; edges[n].a = a; edges[n].b = b; ++n; }
+        }
+    qsort(edges, (size_t)n, sizeof(oracle_edge), edge_order);
+    for (int e = 0; e < E; ++e) expert_rank[e] = -1;
+    for (int r = 0; r < R; ++r) free_slots[r] = per_rank;
+    for (int64_t i = 0; i < n; ++i) {
+        int a = edges[i].a, b = edges[i].b;
+        if (expert_rank[a] < 0 && expert_rank[b] < 0) {
+            for (int r = 0; r < R; ++r)
+                if (free_slots[r] >= 2) {
+                    expert_rank[a] = r;
+                    expert_rank[b] = r;
+                    free_slots[r] -= 2;
+                    break;
+                }
+        } else if (expert_rank[a] < 0 || expert_rank[b] < 0) {
+            int placed = expert_rank[a] >= 0 ? a : b;
+            int other = placed == a ? b : a;
+            int r = expert_rank[placed];
+            if (free_slots[r] > 0) {
+                expert_rank[other] = r;
+                free_slots[r] -= 1;
+            }
+        }
+    }
+    for (int e = 0; e < E; ++e) {
+        if (expert_rank[e] >= 0) continue;
+        for (int r = 0; r < R; ++r)
+            if (free_slots[r] > 0) {
+                expert_rank[e] = r;
+                free_slots[r] -= 1;
+                break;
+            }
+    }
+    free(edges);
+    free(free_slots);
+    return 0;
+}

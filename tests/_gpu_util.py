@@ -14,10 +14,9 @@ X_STREAM, Y_STREAM = 1, 2       # fill_bf16 streams of the hidden rows and exper
 
 
 def cuda(a, dtype=None):
-    t = torch.from_numpy(np.ascontiguousarray(a))
-    if dtype is not None:
-        t = t.to(dtype)
-    return t.to(DEV)
+    """numpy array -> device tensor (dtype: an optional numpy dtype to convert to first)."""
+    a = np.asarray(a) if dtype is None else np.asarray(a, dtype=dtype)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
 
 
 def host_bits(t: torch.Tensor) -> np.ndarray:
@@ -96,7 +95,7 @@ def check_combine(out_gpu: torch.Tensor, y_bits: np.ndarray, gates: np.ndarray,
     yf = workload.bf16_bits_to_float(y_bits).astype(np.float64)
     mag = np.zeros_like(ref64)
     for j in range(gates.shape[1]):
-        valid = comb_row[:, j] >= 0
+        valid = (comb_row[:, j] >= 0) & (comb_row[:, j] < y_bits.shape[0])
         mag[valid] += np.abs(gates[valid, j, None].astype(np.float64) * yf[comb_row[valid, j]])
     got = out_gpu if tokens is None else out_gpu[torch.as_tensor(tokens, device=out_gpu.device)]
     if got.dtype == torch.float32:

@@ -408,3 +408,23 @@ def test_token_shuffle_two_layers(coact):
     shuffled, baseline = o["stats"][5] / nk, base["stats"][5] / nk
     assert abs(baseline - 1.0 / R) < 0.01       # contiguous shards: 1/R served locally
     assert shuffled > 2 * baseline              # prediction keeps far more assignments local
+
+
+def test_correlated_placement_chain_config3(coact):
+    """Config 3's co-activation-grouped placement: GPU pair counts -> the library's
+    correlated placement -> GPU plan, against oracle counts -> oracle placement ->
+    oracle plan; compared with round-robin placement."""
+    r = workload.make_routing(3, placement_kind="roundrobin")
+    E, R = r.cfg.E, r.cfg.R
+    pair = torch.zeros((E, E), dtype=torch.int64, device=DEV)
+    coact.coact_count(cuda(r.ids), E, pair)
+    placed = coact.coact_place_correlated(pair, R).numpy()
+    op, _, _ = oracle.count(r.ids, E)
+    oplaced = oracle.place_correlated(op, R)
+    assert np.array_equal(placed, oplaced)
+    plan, err = run_plan(coact, r, expert_rank=placed)
+    o = oracle_plan_for(r, expert_rank=oplaced)
+    assert err.item() == 0
+    assert_plan_equal(plan_to_host(plan), o)
+    rr = oracle_plan_for(r)
+    assert o["D"] < rr["D"] and o["stats"][4] < rr["stats"][4]   # fewer rows, fewer remote nodes
