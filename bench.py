@@ -124,6 +124,7 @@ def dist_env():
 
 
 def reduce_max(v: float, world: int, device) -> float:
+    """Max over ranks (timing: the slowest rank sets the job's time)."""
     if world == 1:
         return v
     import torch.distributed as dist
@@ -133,12 +134,25 @@ def reduce_max(v: float, world: int, device) -> float:
 
 
 def reduce_sum(v: float, world: int, device) -> float:
+    """Sum over ranks (work: every rank processes its own batch)."""
     if world == 1:
         return v
     import torch.distributed as dist
     t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own batch (weak scaling: independent problems per GPU)."""
+    return base_seed + rank
+
+
+def aggregate(tokens_per_rank: float, seconds_per_rank: float, world: int, device) -> dict:
+    """Whole-job throughput: all ranks' tokens over the slowest rank's device time."""
+    total_s = reduce_max(seconds_per_rank, world, device)
+    tokens = reduce_sum(tokens_per_rank, world, device)
+    return {"tokens": tokens, "seconds": total_s, "tokens_per_s": tokens / total_s}
 
 
 def barrier(world: int):
@@ -237,11 +251,24 @@ def run_gpu(args):
     import co_activation_b200 as coact
 
     cfg = workload.CONFIGS[args.config]
-    r = workload.make_routing(cfg, seed=args.seed + rank)   # each rank: its own batch
+    r = workload.make_routing(cfg, seed=rank_seed(args.seed, rank))
     S = GpuStep(coact, r, device)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    flush = torch.empty(max(2 * l2, 64 << 20), dtype=torch.uint8, device=device)
-    stream = torch.cuda.current_stream()
+    flush_w = torch.empty(max(2 * l2, 64 << 20), dtype=torch.uint8, device=device)
+    flush_r = torch.zeros(max(2 * l2, 64 << 20) // 8, dtype=torch.int64, device=device)
+    flush_sink = torch.empty((), dtype=torch.int64, device=device)
+
+    class _Flush:
+        """L2 flush between steps: write a buffer twice the L2 size, then read another
+        one as large, so the step starts with a cold AND clean L2 (the dirty lines of the
+        write are written back here, not inside the next timed kernel)."""
+
+        @staticmethod
+        def zero_():
+            flush_w.zero_()
+            torch.sum(flush_r, dim=0, out=flush_sink)
+
+    flush = _Flush()
 
     # warm-up (also does every lazy one-time attribute setup before graph capture)
     for _ in range(args.warmup):
@@ -256,16 +283,25 @@ def run_gpu(args):
     evs = [[torch.cuda.Event(enable_timing=True, external=args.graph) for _ in range(5)]
            for _ in range(K)]
     graph = None
+    timing = "one CUDA graph of K steps; CUDA events per step and per phase"
     if args.graph:
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            for i in range(K):
-                flush.zero_()
-                S.step(evs[i])
-        torch.cuda.synchronize()
-        # one untimed replay uploads the graph; its events are overwritten below
-        graph.replay()
-        torch.cuda.synchronize()
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):          # captured on torch's side stream
+                for i in range(K):
+                    flush.zero_()
+                    S.step(evs[i])
+            torch.cuda.synchronize()
+            # one untimed replay uploads the graph; its events are overwritten below
+            graph.replay()
+            torch.cuda.synchronize()
+        except RuntimeError as e:                  # capture refused: time the eager launches
+            graph = None
+            torch.cuda.synchronize()
+            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+            timing = f"eager launches (graph capture failed: {str(e)[:80]})"
+    if not args.graph:
+        timing = "eager launches; CUDA events per step and per phase"
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -293,9 +329,8 @@ def run_gpu(args):
     phase_ms = {name: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)]
                 for j, name in enumerate(["coact_count", "plan_dispatch", "dispatch_gather",
                                           "combine_scatter"])}
-    total_s = reduce_max(sum(step_ms) / 1e3, world, device)
-    tokens = reduce_sum(cfg.N * K, world, device)
-    value = tokens / total_s
+    agg = aggregate(cfg.N * K, sum(step_ms) / 1e3, world, device)
+    total_s, value = agg["seconds"], agg["tokens_per_s"]
     gather_ms = statistics.mean(phase_ms["dispatch_gather"])
     combine_ms = statistics.mean(phase_ms["combine_scatter"])
     dc_tokens_s = cfg.N / ((gather_ms + combine_ms) / 1e3)
@@ -322,8 +357,9 @@ def run_gpu(args):
                    "k": cfg.k, "H": cfg.H, "R": cfg.R, "n_nodes": cfg.n_nodes,
                    "placement": cfg.placement, "step": "coact_count + plan_dispatch + "
                    "dispatch_gather + combine_scatter (bf16 out)",
-                   "l2": "flushed between timed steps (write of 2x L2), outside the step events",
-                   "timing": "one CUDA graph of K steps; CUDA events per step and per phase",
+                   "l2": "flushed between timed steps (write of 2x L2, then a read of another 2x L2 "
+                         "buffer so no dirty line is left), outside the step events",
+                   "timing": timing,
                    "parallelism": f"{world} GPU(s), one independent batch per GPU"},
         "dispatch_combine_tokens_per_s": dc_tokens_s,
         "dedup_rows_over_naive": D / (cfg.N * cfg.k),
@@ -384,9 +420,8 @@ def run_e2e(coact, S: GpuStep, args, world, device):
     b.record()
     torch.cuda.synchronize()
     barrier(world)
-    total_s = reduce_max(a.elapsed_time(b) / 1e3, world, device)
-    tokens = reduce_sum(cfg.N * K, world, device)
-    return {"value": tokens / total_s, "unit": UNIT, "h2d_bytes_per_step": h2d,
+    agg = aggregate(cfg.N * K, a.elapsed_time(b) / 1e3, world, device)
+    return {"value": agg["tokens_per_s"], "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h}
 
 
