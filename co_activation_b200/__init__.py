@@ -52,13 +52,17 @@ _lib.predict_home_workspace_bytes.argtypes = [_I32, _I32]
 _lib.predict_home_workspace_bytes.restype = _SZ
 _lib.predict_home.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _SZ, _P, _P]
 _lib.coact_place_correlated.argtypes = [_P, _I32, _I32, _P]
+_lib.plan_dispatch_noalloc.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _P, _P,
+                                       _P, _P, _P, _I64, _P, _P, _P, _P, _P, _P]
 for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "combine_scatter", "predict_home",
-           "coact_place_correlated"):
+           "coact_place_correlated", "plan_dispatch_noalloc"):
     getattr(_lib, _f).restype = _I32
 
 ABI_SYMBOLS = ("coact_strerror", "coact_abi_version", "coact_count", "plan_dispatch_workspace_bytes",
                "plan_dispatch", "dispatch_gather", "combine_scatter",
-               "predict_home_workspace_bytes", "predict_home", "coact_place_correlated")
+               "predict_home_workspace_bytes", "predict_home", "coact_place_correlated",
+               "plan_dispatch_noalloc")
+NOALLOC_MAX_TOKENS = 262144
 
 
 class CoactError(RuntimeError):
@@ -287,3 +291,42 @@ def coact_place_correlated(pair, R: int):
     out = torch.empty(E, dtype=torch.int32)
     _check(_lib.coact_place_correlated(_ptr(p), E, R, _ptr(out)), "coact_place_correlated")
     return out
+
+
+def plan_dispatch_noalloc(ids: torch.Tensor, E: int, expert_rank: torch.Tensor, R: int, plan: Plan,
+                          rank_node: Optional[torch.Tensor] = None, n_nodes: int = 1,
+                          src_rank: Optional[torch.Tensor] = None,
+                          err_flag: Optional[torch.Tensor] = None, stream=None) -> Plan:
+    """plan_dispatch for callers that cannot allocate device memory (a runtime that owns
+    all device memory through its own pool or fixed memory plan, or a caller that cannot
+    afford cudaMalloc's device-wide synchronisation): the library's own file-scope device
+    scratch replaces the workspace (plan.workspace is not used).  Batches of at most
+    NOALLOC_MAX_TOKENS tokens; calls that overlap on the GPU share that scratch and race,
+    so keep them on one stream.  The first call on a device must come before any stream
+    capture (it looks up the scratch address)."""
+    N, k = ids.shape
+    if N > NOALLOC_MAX_TOKENS:
+        raise ValueError(f"plan_dispatch_noalloc handles at most {NOALLOC_MAX_TOKENS} tokens "
+                         f"(got {N}); use plan_dispatch with a workspace")
+    _need(ids, "ids", torch.int32)
+    _need(expert_rank, "expert_rank", torch.int32, (E,))
+    _need(rank_node, "rank_node", torch.int32, (R,), optional=True)
+    _need(src_rank, "src_rank", torch.int32, (N,), optional=True)
+    _need(plan.rank_counts, "rank_counts", torch.int32, (R,))
+    _need(plan.rank_offsets, "rank_offsets", torch.int32, (R + 1,))
+    _need(plan.asg_offsets, "asg_offsets", torch.int32, (R + 1,))
+    _need(plan.rank_mask, "rank_mask", torch.int64, (N,), optional=True)
+    _need(plan.row_token, "row_token", torch.int32)
+    _need(plan.row_kmask, "row_kmask", torch.uint8, (plan.row_token.shape[0],))
+    _need(plan.send_row, "send_row", torch.int32, (N, k))
+    _need(plan.comb_row, "comb_row", torch.int32, (N, k))
+    _need(plan.stats, "stats", torch.int64, (NUM_STATS,))
+    _need(plan.src_dst, "src_dst", torch.int32, (R, R), optional=True)
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.plan_dispatch_noalloc(
+        _ptr(ids), N, k, E, _ptr(expert_rank), R, _ptr(rank_node), n_nodes, _ptr(src_rank),
+        _ptr(plan.rank_counts), _ptr(plan.rank_offsets), _ptr(plan.asg_offsets),
+        _ptr(plan.rank_mask), _ptr(plan.row_token), _ptr(plan.row_kmask), plan.row_capacity,
+        _ptr(plan.send_row), _ptr(plan.comb_row), _ptr(plan.stats), _ptr(plan.src_dst),
+        _ptr(err_flag), _stream(stream)), "plan_dispatch_noalloc")
+    return plan

@@ -518,3 +518,89 @@ extern "C" int plan_dispatch(const int32_t *ids, int64_t N, int k, int E, const 
 #undef COACT_PLAN_CASE
     return COACT_ERR_UNSUPPORTED;
 }
+
+// ------------------------------------------------------------------ no-allocation variant
+//
+// plan_dispatch_noalloc: plan_dispatch for callers that cannot allocate device memory
+// -- code running inside a runtime that owns every byte of device memory through its
+// own pool or a fixed memory plan and forbids stray allocations, or a latency-critical
+// caller that cannot afford cudaMalloc's implicit device-wide synchronisation.  Its
+// scratch is a file-scope device array sized for COACT_NOALLOC_MAX_TOKENS tokens and
+// COACT_MAX_R ranks, which every GPU that loads this library holds until exit.
+
+namespace coact {
+namespace {
+
+constexpr size_t align256c(size_t b) { return (b + 255) & ~size_t(255); }
+constexpr int64_t kNoallocTiles = (COACT_NOALLOC_MAX_TOKENS + kTile - 1) / kTile;
+constexpr size_t kNoallocScratchBytes =
+    2 * align256c(sizeof(int32_t) * (size_t)COACT_MAX_R * kNoallocTiles) +
+    align256c(sizeof(int64_t) * kStatSlots * (size_t)kNoallocTiles) +
+    align256c(sizeof(int32_t) * 2 * (size_t)COACT_MAX_R);
+
+// In host code this name is only a host-side stand-in, never a device address: the
+// address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_plan_scratch[kNoallocScratchBytes];
+
+std::atomic<void *> g_plan_scratch_addr[kMaxDevices];
+
+// Device address of g_plan_scratch on the current device, looked up once per device.
+int noalloc_scratch(const DeviceInfo &di, void **out) {
+    void *p = g_plan_scratch_addr[di.device].load(std::memory_order_acquire);
+    if (!p) {
+        if (cudaGetSymbolAddress(&p, g_plan_scratch) != cudaSuccess || !p) return COACT_ERR_CUDA;
+        g_plan_scratch_addr[di.device].store(p, std::memory_order_release);
+    }
+    *out = p;
+    return COACT_OK;
+}
+
+}  // namespace
+}  // namespace coact
+
+extern "C" int plan_dispatch_noalloc(const int32_t *ids, int64_t N, int k, int E,
+                                     const int32_t *expert_rank, int R, const int32_t *rank_node,
+                                     int n_nodes, const int32_t *src_rank, int32_t *rank_counts,
+                                     int32_t *rank_offsets, int32_t *asg_offsets,
+                                     uint64_t *rank_mask, int32_t *row_token, uint8_t *row_kmask,
+                                     int64_t row_capacity, int32_t *send_row, int32_t *comb_row,
+                                     int64_t *stats, int32_t *src_dst, int32_t *err_flag,
+                                     coact_stream_t stream) {
+    if (N < 0 || row_capacity < 0) return COACT_ERR_INVALID;
+    if (N > COACT_NOALLOC_MAX_TOKENS) return COACT_ERR_UNSUPPORTED;
+    if (k < 1 || k > COACT_MAX_K || E < 2 || E > COACT_MAX_E || R < 1 || R > COACT_MAX_R)
+        return COACT_ERR_UNSUPPORTED;
+    if (rank_node && (n_nodes < 1 || n_nodes > 64)) return COACT_ERR_UNSUPPORTED;
+    if (!rank_node) n_nodes = 1;
+    if (N > (int64_t)INT32_MAX / k || row_capacity > (int64_t)INT32_MAX) return COACT_ERR_UNSUPPORTED;
+    if (!expert_rank || !rank_counts || !rank_offsets || !asg_offsets || !stats)
+        return COACT_ERR_INVALID;
+    if (N > 0 && (!ids || !send_row || !comb_row)) return COACT_ERR_INVALID;
+    if (row_capacity > 0 && (!row_token || !row_kmask)) return COACT_ERR_INVALID;
+    DeviceInfo di;
+    if (int s = device_info(&di)) return s;
+    void *scratch = nullptr;
+    if (int s = noalloc_scratch(di, &scratch)) return s;
+    if (workspace_layout(N, R, nullptr, nullptr) > kNoallocScratchBytes) return COACT_ERR_UNSUPPORTED;
+    Workspace ws;
+    workspace_layout(N, R, &ws, scratch);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+#define COACT_PLAN_NOALLOC_CASE(KK)                                                                \
+    case KK:                                                                                       \
+        return launch_plan<KK>(ids, N, E, expert_rank, R, rank_node, n_nodes, src_rank,            \
+                               rank_counts, rank_offsets, asg_offsets, rank_mask, row_token,       \
+                               row_kmask, row_capacity, send_row, comb_row, stats, src_dst, ws,    \
+                               err_flag, st);
+    switch (k) {
+        COACT_PLAN_NOALLOC_CASE(1)
+        COACT_PLAN_NOALLOC_CASE(2)
+        COACT_PLAN_NOALLOC_CASE(3)
+        COACT_PLAN_NOALLOC_CASE(4)
+        COACT_PLAN_NOALLOC_CASE(5)
+        COACT_PLAN_NOALLOC_CASE(6)
+        COACT_PLAN_NOALLOC_CASE(7)
+        COACT_PLAN_NOALLOC_CASE(8)
+    }
+#undef COACT_PLAN_NOALLOC_CASE
+    return COACT_ERR_UNSUPPORTED;
+}

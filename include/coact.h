@@ -193,6 +193,38 @@ int combine_scatter(const uint16_t *y, int64_t n_rows, const float *gates,
                     void *out, int out_dtype,
                     int32_t *err_flag, coact_stream_t stream);
 
+/*
+ * plan_dispatch_noalloc -- plan_dispatch without a caller-provided workspace.
+ * No counterpart in the papers: it exists for callers that cannot allocate device
+ * memory, such as code running inside a runtime that owns all device memory through its
+ * own pool or a fixed memory plan and forbids stray allocations, or a latency-critical
+ * caller that cannot afford cudaMalloc's implicit device-wide synchronisation.  It
+ * computes exactly what plan_dispatch computes (same arguments and outputs, minus
+ * workspace / workspace_bytes) and allocates nothing: its scratch is a file-scope
+ * device array of the library, sized for N <= COACT_NOALLOC_MAX_TOKENS and R <= 64
+ * (about 560 KB), which every GPU that loads the library holds until the process exits.
+ *  - N > COACT_NOALLOC_MAX_TOKENS returns COACT_ERR_UNSUPPORTED before anything is
+ *    enqueued; use plan_dispatch with a workspace for larger batches.
+ *  - The first call on each device looks up the scratch array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call before any
+ *    stream capture.
+ *  - All calls on a device share the one scratch array, and it keeps the last call's
+ *    contents.  Nothing in it needs clearing (every entry a call reads is written
+ *    earlier in the same call), but calls that overlap on the GPU -- e.g. two streams at
+ *    once -- race on it: order such calls on one stream.
+ */
+#define COACT_NOALLOC_MAX_TOKENS 262144
+int plan_dispatch_noalloc(const int32_t *ids, int64_t N, int k, int E,
+                          const int32_t *expert_rank, int R,
+                          const int32_t *rank_node, int n_nodes,
+                          const int32_t *src_rank,
+                          int32_t *rank_counts, int32_t *rank_offsets, int32_t *asg_offsets,
+                          uint64_t *rank_mask,
+                          int32_t *row_token, uint8_t *row_kmask, int64_t row_capacity,
+                          int32_t *send_row, int32_t *comb_row,
+                          int64_t *stats, int32_t *src_dst,
+                          int32_t *err_flag, coact_stream_t stream);
+
 /* Bytes of device workspace predict_home needs (E1*R int64 scores). */
 size_t predict_home_workspace_bytes(int E1, int R);
 
