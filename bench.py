@@ -184,6 +184,7 @@ class GpuStep:
         self.send = torch.empty((self.plan.row_capacity, H), dtype=torch.bfloat16, device=device)
         self.out = torch.empty((N, H), dtype=torch.bfloat16, device=device)
         self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.side = torch.cuda.Stream(device=device)
 
     def count(self):
         self.coact.coact_count(self.ids, self.cfg.E, self.pair, self.loads, err_flag=self.err)
@@ -201,15 +202,22 @@ class GpuStep:
                                    err_flag=self.err)
 
     def step(self, ev=None):
-        """ev: optional list of 5 events recorded at phase boundaries."""
+        """One pass of the path.  coact_count depends on nothing the other three calls
+        produce, so it runs on a side stream, overlapped with plan_dispatch; the step
+        ends when both streams have finished.  ev: optional list of 5 events for the
+        phase boundaries (the count phase is then measured on the side stream)."""
+        main = torch.cuda.current_stream()
+        self.side.wait_stream(main)
         if ev: ev[0].record()
-        self.count()
-        if ev: ev[1].record()
+        with torch.cuda.stream(self.side):
+            self.count()
+            if ev: ev[1].record()
         self.plan_()
         if ev: ev[2].record()
         self.gather()
         if ev: ev[3].record()
         self.combine()
+        main.wait_stream(self.side)
         if ev: ev[4].record()
 
     def bytes_gather(self, D):
@@ -280,55 +288,76 @@ def run_gpu(args):
     assert S.err.item() == 0, f"device error flags {S.err.item()}"
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True, external=args.graph) for _ in range(5)]
-           for _ in range(K)]
-    graph = None
-    timing = "one CUDA graph of K steps; CUDA events per step and per phase"
-    if args.graph:
-        try:
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph):          # captured on torch's side stream
-                for i in range(K):
-                    flush.zero_()
-                    S.step(evs[i])
-            torch.cuda.synchronize()
-            # one untimed replay uploads the graph; its events are overwritten below
-            graph.replay()
-            torch.cuda.synchronize()
-        except RuntimeError as e:                  # capture refused: time the eager launches
-            graph = None
-            torch.cuda.synchronize()
-            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
-            timing = f"eager launches (graph capture failed: {str(e)[:80]})"
-    if not args.graph:
-        timing = "eager launches; CUDA events per step and per phase"
+
+    def capture(with_phases: bool):
+        """K steps (each preceded by the L2 flush) as one CUDA graph.  Events at the step
+        boundaries always; at the phase boundaries only in the breakdown pass, because
+        every event node inside a graph serialises the stream (about 3 us each)."""
+        ev = [[torch.cuda.Event(enable_timing=True, external=args.graph) for _ in range(5)]
+              for _ in range(K)]
+
+        def body():
+            for i in range(K):
+                flush.zero_()
+                if with_phases:
+                    S.step(ev[i])
+                else:
+                    ev[i][0].record()
+                    S.step()
+                    ev[i][4].record()
+
+        if not args.graph:
+            return None, ev, body
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):          # captured on torch's side stream
+            body()
+        torch.cuda.synchronize()
+        g.replay()                         # upload; these events are overwritten later
+        torch.cuda.synchronize()
+        return g, ev, body
+
+    timing = "one CUDA graph of K steps per pass; CUDA events per step"
+    try:
+        g_main, evs, body_main = capture(False)
+        g_phase, evs_phase, body_phase = capture(True)
+    except RuntimeError as e:              # capture refused: time eager launches instead
+        torch.cuda.synchronize()
+        args.graph = False
+        g_main, evs, body_main = capture(False)
+        g_phase, evs_phase, body_phase = capture(True)
+        timing = f"eager launches (graph capture failed: {str(e)[:80]})"
+    if not args.graph and "failed" not in timing:
+        timing = "eager launches; CUDA events per step"
+    run = lambda g, body: g.replay() if g is not None else body()
 
     clocks = ClockSampler(local)
     clocks.start()
     # keep the GPU busy for a moment so the sampler sees the clocks under this load
     t_end = time.time() + args.clock_warm_s
     while time.time() < t_end:
-        if graph is not None:
-            graph.replay()
-        else:
-            S.step()
+        run(g_main, body_main)
         torch.cuda.synchronize()
+    # timed region: K steps, events per step (headline)
     barrier(world)
     torch.cuda.synchronize()
-    if graph is not None:
-        graph.replay()
-    else:
-        for i in range(K):
-            flush.zero_()
-            S.step(evs[i])
+    run(g_main, body_main)
+    torch.cuda.synchronize()
+    barrier(world)
+    # second timed pass: the same K steps with events at every phase boundary
+    # (per-kernel durations for the breakdown and the roofline; slightly inflated by
+    # the event nodes themselves, so the roofline fraction is a lower bound)
+    run(g_phase, body_phase)
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
 
     step_ms = [evs[i][0].elapsed_time(evs[i][4]) for i in range(K)]
-    phase_ms = {name: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)]
-                for j, name in enumerate(["coact_count", "plan_dispatch", "dispatch_gather",
-                                          "combine_scatter"])}
+    # count runs on the side stream (ev0 -> ev1); the main stream runs plan (ev0 -> ev2),
+    # gather (ev2 -> ev3) and combine (ev3 -> ev4)
+    spans = {"coact_count": (0, 1), "plan_dispatch": (0, 2), "dispatch_gather": (2, 3),
+             "combine_scatter": (3, 4)}
+    phase_ms = {name: [evs_phase[i][a].elapsed_time(evs_phase[i][b]) for i in range(K)]
+                for name, (a, b) in spans.items()}
     agg = aggregate(cfg.N * K, sum(step_ms) / 1e3, world, device)
     total_s, value = agg["seconds"], agg["tokens_per_s"]
     gather_ms = statistics.mean(phase_ms["dispatch_gather"])
@@ -355,8 +384,8 @@ def run_gpu(args):
         "data": "synthetic (seeded routing shaped after the pages' statistics; no router traces)",
         "config": {"workload": f"config {cfg.index}: {cfg.desc}", "N": cfg.N, "E": cfg.E,
                    "k": cfg.k, "H": cfg.H, "R": cfg.R, "n_nodes": cfg.n_nodes,
-                   "placement": cfg.placement, "step": "coact_count + plan_dispatch + "
-                   "dispatch_gather + combine_scatter (bf16 out)",
+                   "placement": cfg.placement, "step": "coact_count (side stream, overlapped "
+                   "with plan) + plan_dispatch + dispatch_gather + combine_scatter (bf16 out)",
                    "l2": "flushed between timed steps (write of 2x L2, then a read of another 2x L2 "
                          "buffer so no dirty line is left), outside the step events",
                    "timing": timing,
@@ -365,6 +394,8 @@ def run_gpu(args):
         "dedup_rows_over_naive": D / (cfg.N * cfg.k),
         "stats": dict(zip(coact.STAT_NAMES, stats)),
         "phase_us": {k_: statistics.mean(v) * 1e3 for k_, v in phase_ms.items()},
+        "phase_pass_step_us": statistics.mean(
+            evs_phase[i][0].elapsed_time(evs_phase[i][4]) for i in range(K)) * 1e3,
         "hbm_gbs": {"dispatch_gather": gb_g, "combine_scatter": gb_c, "gather+combine": gb_dc,
                     "pct_of_8tbs_gather+combine": 100 * gb_dc / 8000.0,
                     f"pct_of_{peak_kind}_{peak:.0f}": 100 * gb_dc / peak},
@@ -381,7 +412,7 @@ def run_gpu(args):
         result["cpu_baseline"] = cpu_baseline(S, args.cpu_seconds)
     if world > 1:
         import torch.distributed as dist
-        del graph
+        del g_main, g_phase
         torch.cuda.synchronize()
         dist.barrier()
         dist.destroy_process_group()

@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(256)
     k_combine_v16(const uint4 *__restrict__ y, int64_t n_rows, const float *__restrict__ gates,
                   const int32_t *__restrict__ comb_row, int64_t N, int64_t H16,
                   void *__restrict__ out, int32_t *__restrict__ err) {
+    pdl_trigger();
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t gwarp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -101,9 +103,8 @@ int launch(const uint16_t *y, int64_t n_rows, const float *gates, const int32_t 
     const int64_t H16 = H / 8;
     const int blocks = (int)std::max<int64_t>(
         1, std::min<int64_t>(ceil_div(N, 8), (int64_t)di.sm_count * 8));
-    k_combine_v16<K, U, F32><<<blocks, 256, 0, st>>>(reinterpret_cast<const uint4 *>(y), n_rows,
-                                                     gates, comb_row, N, H16, out, err);
-    return launch_status();
+    return launch_pdl(k_combine_v16<K, U, F32>, blocks, 256, 0, st,
+                      reinterpret_cast<const uint4 *>(y), n_rows, gates, comb_row, N, H16, out, err);
 }
 
 }  // namespace

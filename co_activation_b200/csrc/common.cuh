@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <utility>
 
 #include "coact.h"
 
@@ -63,10 +64,33 @@ __device__ __forceinline__ int load_ids(const int32_t *__restrict__ ids, int64_t
     return f;
 }
 
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 // OR of `bits` over the warp, raised once by lane 0 (all lanes must call).
 __device__ __forceinline__ void raise_flag_warp(int32_t *err, int bits) {
     const unsigned all = __reduce_or_sync(0xffffffffu, (unsigned)bits);
     if (all && (threadIdx.x & 31) == 0 && err) atomicOr(err, (int)all);
+}
+
+// Programmatic dependent launch.  Every library kernel is launched with programmatic
+// stream serialisation: it may start while the previous kernel on the stream drains,
+// runs only shared-memory set-up before pdl_wait(), and reads no global input until the
+// previous grid has completed and its writes are visible.  pdl_trigger() lets the next
+// kernel's blocks launch early; they too wait before touching our outputs.
+__device__ __forceinline__ void pdl_wait() {
+#if !defined(COACT_NO_PDL)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
+}
+
+__device__ __forceinline__ void pdl_trigger() {
+#if !defined(COACT_NO_PDL)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
 }
 
 // ------------------------------------------------------------------ host helpers
@@ -114,6 +138,29 @@ inline int blocks_per_sm(int threads, size_t smem, const DeviceInfo &di) {
 
 inline int launch_status() {
     return cudaGetLastError() == cudaSuccess ? COACT_OK : COACT_ERR_CUDA;
+}
+
+// Launches `kernel` on `stream` with programmatic stream serialisation (see pdl_wait).
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+               Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+#if defined(COACT_NO_PDL)
+    cfg.numAttrs = 0;
+#else
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+#endif
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess
+               ? COACT_OK
+               : COACT_ERR_CUDA;
 }
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -8,11 +8,12 @@
 // Two kernels:
 //  * k_count_smem -- each block privatises the strict upper triangle of the E x E count
 //    matrix (E*(E-1)/2 u32 bins, 130 KB at E = 256) plus E load bins in shared memory,
-//    adds its tokens' pairs with warp-aggregated shared atomics (lanes holding the same
-//    bin in the same slot pair are merged with __match_any_sync and add once), then
-//    flushes every non-zero bin to both halves of the int64 matrix with one global
-//    atomic each.  Used when the triangle fits and each block sees enough pairs to
-//    amortise its zero/flush pass.
+//    adds its tokens' pairs with shared atomics, then flushes every non-zero bin to both
+//    halves of the int64 matrix with one global atomic each.  Used when the triangle
+//    fits and each block sees enough pairs to amortise its zero/flush pass.  (A
+//    warp-aggregated variant -- lanes with the same bin merged by __match_any_sync --
+//    exists as AGG = true; on B200 it measured 1.4-3x slower than plain shared atomics
+//    even on the Zipf-skewed configurations, so it is off.)
 //  * k_count_global -- one global 64-bit atomic per ordered pair, for E too large for
 //    shared memory or inputs too small to amortise a private histogram.
 // Cross mode (ids2 != NULL) counts ids x ids2 into an E x E2 matrix, privatised in
@@ -43,6 +44,8 @@ __global__ void __launch_bounds__(kCountThreads)
     uint32_t *tri = sh;
     uint32_t *sload = sh + nbins;
     for (int i = threadIdx.x; i < nbins + E; i += blockDim.x) sh[i] = 0;
+    pdl_trigger();
+    pdl_wait();
     __syncthreads();
 
     const int lane = threadIdx.x & 31;
@@ -99,6 +102,8 @@ template <int K>
 __global__ void __launch_bounds__(256)
     k_count_global(const int32_t *__restrict__ ids, int64_t N, int E, ull *__restrict__ pair,
                    ull *__restrict__ loads, int32_t *__restrict__ err) {
+    pdl_trigger();
+    pdl_wait();
     int flags = 0;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < N; t += stride) {
@@ -126,10 +131,11 @@ __global__ void __launch_bounds__(512)
                   int32_t *__restrict__ err) {
     extern __shared__ uint32_t sh[];
     const int nb = SMEM ? E * E2 : 0;
-    if (SMEM) {
+    if (SMEM)
         for (int i = threadIdx.x; i < nb + E; i += blockDim.x) sh[i] = 0;
-        __syncthreads();
-    }
+    pdl_trigger();
+    pdl_wait();
+    if (SMEM) __syncthreads();
     int flags = 0;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < N; t += stride) {
@@ -180,9 +186,16 @@ __global__ void __launch_bounds__(512)
 
 // Blocks for a privatised histogram: enough pairs per block to amortise the zero and
 // flush passes over `bins` bins, capped by what fits on the GPU at once.
+#ifndef COACT_COUNT_MIN_PER_BLOCK
+#define COACT_COUNT_MIN_PER_BLOCK 2048
+#endif
+#ifndef COACT_COUNT_BINS_FACTOR
+#define COACT_COUNT_BINS_FACTOR 1
+#endif
 int hist_blocks(int64_t N, int64_t pairs_per_token, int64_t bins, int resident) {
     const int64_t total = N * pairs_per_token;
-    const int64_t per_block = std::max<int64_t>(4 * bins, 16384);
+    const int64_t per_block =
+        std::max<int64_t>(COACT_COUNT_BINS_FACTOR * bins, COACT_COUNT_MIN_PER_BLOCK);
     const int64_t want = std::max<int64_t>(1, ceil_div(total, per_block));
     return (int)std::min<int64_t>(want, resident);
 }
@@ -194,23 +207,25 @@ int count_self(const int32_t *ids, int64_t N, int E, ull *pair, ull *loads, int3
     const size_t smem = (size_t)(nbins + E) * sizeof(uint32_t);
     const int64_t ppt = (int64_t)K * (K - 1) / 2;
     bool use_smem = K > 1 && smem <= (size_t)di.smem_optin;
-#if defined(COACT_COUNT_PATH)
-    use_smem = use_smem && COACT_COUNT_PATH != 0;  // experiment builds only
-#endif
     // tiny inputs: a private histogram would cost more to clear than to fill
     if (N * ppt < 2 * nbins) use_smem = false;
+#if defined(COACT_COUNT_PATH)
+    use_smem = K > 1 && smem <= (size_t)di.smem_optin && COACT_COUNT_PATH != 0;  // experiments
+#endif
+#ifndef COACT_COUNT_AGG
+#define COACT_COUNT_AGG false  // measured on B200: match_any costs more than it saves
+#endif
     if (use_smem) {
-        auto kern = k_count_smem<K, true>;
+        auto kern = k_count_smem<K, COACT_COUNT_AGG>;
         static SmemOptIn opt;
         if (int s = ensure_smem(kern, smem, opt, di)) return s;
         const int per_sm = blocks_per_sm(kCountThreads, smem, di);
         const int blocks = hist_blocks(N, ppt, nbins, per_sm * di.sm_count);
-        kern<<<blocks, kCountThreads, smem, st>>>(ids, N, E, pair, loads, err);
+        return launch_pdl(kern, blocks, kCountThreads, smem, st, ids, N, E, pair, loads, err);
     } else {
         const int blocks = (int)std::min<int64_t>(ceil_div(N, 256), (int64_t)di.sm_count * 8);
-        k_count_global<K><<<blocks, 256, 0, st>>>(ids, N, E, pair, loads, err);
+        return launch_pdl(k_count_global<K>, blocks, 256, 0, st, ids, N, E, pair, loads, err);
     }
-    return launch_status();
 }
 
 template <int K>
@@ -225,12 +240,12 @@ int count_cross(const int32_t *ids, const int32_t *ids2, int k2, int64_t N, int 
         if (int s = ensure_smem(kern, smem, opt, di)) return s;
         const int per_sm = blocks_per_sm(512, smem, di);
         const int blocks = hist_blocks(N, (int64_t)K * k2, nb, per_sm * di.sm_count);
-        kern<<<blocks, 512, smem, st>>>(ids, ids2, k2, N, E, E2, C, loads, err);
+        return launch_pdl(kern, blocks, 512, smem, st, ids, ids2, k2, N, E, E2, C, loads, err);
     } else {
         const int blocks = (int)std::min<int64_t>(ceil_div(N, 512), (int64_t)di.sm_count * 4);
-        k_count_cross<K, false><<<blocks, 512, 0, st>>>(ids, ids2, k2, N, E, E2, C, loads, err);
+        return launch_pdl(k_count_cross<K, false>, blocks, 512, 0, st, ids, ids2, k2, N, E, E2, C,
+                          loads, err);
     }
-    return launch_status();
 }
 
 }  // namespace

@@ -7,15 +7,15 @@
 //
 // Each x row is read from HBM once and written to every distinct destination row, so
 // the algorithmic traffic is (N + D) * H * 2 bytes (+ N*k*4 for send_row).
-//  * k_gather_bulk -- TMA bulk copies.  One warp per CTA; lane 0 streams rows into a
-//    ring of shared-memory stages with cp.async.bulk (global -> shared, completion on
-//    an mbarrier), then lanes j < k each issue the cp.async.bulk store of the staged
-//    row to destination j.  The hardware copy engine moves whole 0.5-14 KB rows with a
-//    handful of instructions; many small CTAs per SM keep enough bytes in flight.
-//    No multicast: every load reads this GPU's own memory once.
-//  * k_gather_v16 -- one warp per token, 16-byte vector loads into registers and
-//    streaming 16-byte stores to each destination.  Used for unaligned rows and short
-//    rows where staging does not pay.
+//  * k_gather_v16 (default) -- one warp per token, 16-byte vector loads of the x row
+//    into registers (up to 8 per lane in flight) and streaming 16-byte stores to each
+//    destination; 8 CTAs of 8 warps per SM.
+//  * k_gather_bulk (builds with -DCOACT_GATHER_PATH=1) -- TMA bulk copies.  One warp
+//    per CTA; lane 0 streams rows into a ring of shared-memory stages with
+//    cp.async.bulk (global -> shared, completion on an mbarrier), then lanes j < k each
+//    issue the cp.async.bulk store of the staged row to destination j.  No multicast:
+//    every load reads this GPU's own memory once.  Measured on B200 it tied the vector
+//    path on 4 KB rows and lost 4-5% on 8-14 KB rows, so it is not the default.
 // All mbarrier waits are bounded by a wall-clock limit; on expiry the kernel raises
 // COACT_EFLAG_TIMEOUT, drains its own copies and returns.
 #include <algorithm>
@@ -32,6 +32,8 @@ __global__ void __launch_bounds__(256)
     k_gather_v16(const uint4 *__restrict__ x, int64_t N, int64_t H16,
                  const int32_t *__restrict__ send_row, int k, uint4 *__restrict__ send,
                  int64_t cap, int32_t *__restrict__ err) {
+    pdl_trigger();
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t gwarp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -99,12 +101,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
 // Waits for phase `parity` of the mbarrier; gives up after `limit_ns` of wall clock.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -115,19 +111,43 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
+#if defined(COACT_GATHER_EVICT_FIRST)
+// L2 policy for data touched exactly once (x rows, send rows): evict first.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+#endif
+
 __device__ __forceinline__ void bulk_load(uint32_t dst_smem, const void *src, uint32_t bytes,
                                           uint32_t bar) {
+#if defined(COACT_GATHER_EVICT_FIRST)
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1], %2, [%3], %4;" ::"r"(dst_smem),
+        "l"(src), "r"(bytes), "r"(bar), "l"(policy_evict_first())
+        : "memory");
+#else
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
             dst_smem),
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
+#endif
 }
 
 __device__ __forceinline__ void bulk_store(void *dst, uint32_t src_smem, uint32_t bytes) {
+#if defined(COACT_GATHER_EVICT_FIRST)
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(
+                     dst),
+                 "r"(src_smem), "r"(bytes), "l"(policy_evict_first())
+                 : "memory");
+#else
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
                  "r"(src_smem), "r"(bytes)
                  : "memory");
+#endif
 }
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
@@ -167,6 +187,10 @@ __global__ void __launch_bounds__(32)
 #pragma unroll
         for (int s = 0; s < S; ++s) mbar_init(bars + 8 * s, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    pdl_trigger();
+    pdl_wait();
+    if (lane == 0) {
         for (int64_t i = 0; i < n_mine && i < S; ++i) {
             const uint32_t bar = bars + 8 * (uint32_t)i;
             mbar_expect_tx(bar, row_bytes);
@@ -238,8 +262,7 @@ int launch_bulk(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row
     // at least S tokens per CTA so the ring fills, but every SM busy
     const int64_t want = std::max<int64_t>(1, ceil_div(N, 2 * S));
     const int blocks = (int)std::min<int64_t>(want, (int64_t)per_sm * di.sm_count);
-    kern<<<blocks, 32, smem, st>>>(x, N, row_bytes, send_row, k, send, cap, err);
-    return launch_status();
+    return launch_pdl(kern, blocks, 32, smem, st, x, N, row_bytes, send_row, k, send, cap, err);
 }
 
 int launch_v16(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row, int k,
@@ -250,13 +273,9 @@ int launch_v16(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row,
         1, std::min<int64_t>(ceil_div(warps_needed, 8), (int64_t)di.sm_count * 8));
     const uint4 *xv = reinterpret_cast<const uint4 *>(x);
     uint4 *sv = reinterpret_cast<uint4 *>(send);
-    if (H16 <= 32)
-        k_gather_v16<1><<<blocks, 256, 0, st>>>(xv, N, H16, send_row, k, sv, cap, err);
-    else if (H16 <= 128)
-        k_gather_v16<4><<<blocks, 256, 0, st>>>(xv, N, H16, send_row, k, sv, cap, err);
-    else
-        k_gather_v16<8><<<blocks, 256, 0, st>>>(xv, N, H16, send_row, k, sv, cap, err);
-    return launch_status();
+    if (H16 <= 32) return launch_pdl(k_gather_v16<1>, blocks, 256, 0, st, xv, N, H16, send_row, k, sv, cap, err);
+    if (H16 <= 128) return launch_pdl(k_gather_v16<4>, blocks, 256, 0, st, xv, N, H16, send_row, k, sv, cap, err);
+    return launch_pdl(k_gather_v16<8>, blocks, 256, 0, st, xv, N, H16, send_row, k, sv, cap, err);
 }
 
 }  // namespace
@@ -278,13 +297,25 @@ extern "C" int dispatch_gather(const uint16_t *x, int64_t N, int64_t H, const in
     if (int s = device_info(&di)) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int64_t row_bytes = H * 2;
-    bool bulk = row_bytes >= 1024 && row_bytes <= 32768;
+    // Default: the vector path.  On B200 it matched the bulk (TMA) path on 4 KB rows and
+    // beat it by 4-5% on 8 and 14 KB rows (5.99 vs 5.73 TB/s); the bulk path stays
+    // available to builds with -DCOACT_GATHER_PATH=1.
+    bool bulk = false;
 #if defined(COACT_GATHER_PATH)
-    bulk = bulk && COACT_GATHER_PATH != 0;  // experiment builds only
+    bulk = row_bytes >= 1024 && row_bytes <= 32768 && COACT_GATHER_PATH != 0;
+#endif
+#ifndef COACT_GATHER_STAGES_SMALL
+#define COACT_GATHER_STAGES_SMALL 8
+#endif
+#ifndef COACT_GATHER_STAGES_LARGE
+#define COACT_GATHER_STAGES_LARGE 4
 #endif
     if (bulk) {
-        if (row_bytes <= 4096) return launch_bulk<8>(x, N, H, send_row, k, send, row_capacity, err_flag, st, di);
-        return launch_bulk<4>(x, N, H, send_row, k, send, row_capacity, err_flag, st, di);
+        if (row_bytes <= 4096)
+            return launch_bulk<COACT_GATHER_STAGES_SMALL>(x, N, H, send_row, k, send, row_capacity,
+                                                          err_flag, st, di);
+        return launch_bulk<COACT_GATHER_STAGES_LARGE>(x, N, H, send_row, k, send, row_capacity,
+                                                      err_flag, st, di);
     }
     return launch_v16(x, N, H, send_row, k, send, row_capacity, err_flag, st, di);
 }

@@ -5,7 +5,9 @@
 // (token, expert).  Cobalt (arxivdaily 2609.36959), English abstract: routing tokens to
 // fewer remote nodes -- node-level statistics of the same plan.
 //
-// Three launches, none of which waits on another block:
+// Launches, none of which waits on another block (a cooperative single-launch variant
+// with two bounded grid barriers was measured on B200: slower on N = 16K tokens, 6 us
+// faster on 64-128K, so it was dropped):
 //  1. k_plan_tiles   one thread per token, 256-token tiles: per-token rank mask, per-tile
 //                    per-rank row and assignment counts (warp ballots / redux, no
 //                    atomics) and per-tile statistics partials.
@@ -116,6 +118,8 @@ __global__ void __launch_bounds__(kTile)
     __shared__ long long s_stat[kTileWarps][kStatSlots];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_trigger();
+    pdl_wait();
     load_nodes(rank_node, R, n_nodes, s_node, s_node_ranks, err);
     for (int i = tid; i < kTileWarps * 64; i += kTile) {
         (&s_wrows[0][0])[i] = 0;
@@ -225,6 +229,8 @@ __global__ void __launch_bounds__(kScanThreads)
                 int32_t *__restrict__ src_dst) {
     __shared__ int s_warp[33];
     __shared__ long long s_red[kStatSlots][32];
+    pdl_trigger();
+    pdl_wait();
     if ((int)blockIdx.x < R) {
         const int r = blockIdx.x;
         for (int which = 0; which < 2; ++which) {
@@ -293,6 +299,8 @@ __global__ void __launch_bounds__(kTile)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tile = blockIdx.x;
+    pdl_trigger();
+    pdl_wait();
     if (warp == 0) {
         // rank offsets = exclusive scan of the per-rank totals (R <= 64: two per lane)
         const int r0 = lane, r1 = lane + 32;
@@ -451,18 +459,22 @@ int launch_plan(const int32_t *ids, int64_t N, int E, const int32_t *expert_rank
                 int32_t *rank_counts, int32_t *rank_offsets, int32_t *asg_offsets,
                 uint64_t *rank_mask, int32_t *row_token, uint8_t *row_kmask, int64_t cap,
                 int32_t *send_row, int32_t *comb_row, int64_t *stats, int32_t *src_dst,
-                const Workspace &ws, int32_t *err, cudaStream_t st) {
+                const Workspace &ws, int32_t *err, cudaStream_t st, const DeviceInfo &di) {
+    (void)di;
     const int n_tiles = (int)ceil_div(N, kTile);
+    const size_t sd_smem = src_dst ? sizeof(int) * R * R : 0;
+
     if (n_tiles > 0)
-        k_plan_tiles<K><<<n_tiles, kTile, 0, st>>>(ids, N, E, expert_rank, R, rank_node, n_nodes,
-                                                   src_rank, n_tiles, ws, err);
-    k_plan_scan<<<R + 1, kScanThreads, 0, st>>>(N, K, R, n_tiles, ws, stats, src_dst);
-    const size_t smem = src_dst ? sizeof(int) * R * R : 0;
-    k_plan_scatter<K><<<std::max(n_tiles, 1), kTile, smem, st>>>(
-        ids, N, E, expert_rank, R, src_rank, n_tiles, ws, rank_counts, rank_offsets, asg_offsets,
-        reinterpret_cast<unsigned long long *>(rank_mask), row_token, row_kmask, cap, send_row,
-        comb_row, stats, src_dst, err);
-    return launch_status();
+        if (int s = launch_pdl(k_plan_tiles<K>, n_tiles, kTile, 0, st, ids, N, E, expert_rank, R,
+                               rank_node, n_nodes, src_rank, n_tiles, ws, err))
+            return s;
+    if (int s = launch_pdl(k_plan_scan, R + 1, kScanThreads, 0, st, N, K, R, n_tiles, ws, stats,
+                           src_dst))
+        return s;
+    return launch_pdl(k_plan_scatter<K>, std::max(n_tiles, 1), kTile, sd_smem, st, ids, N, E,
+                      expert_rank, R, src_rank, n_tiles, ws, rank_counts, rank_offsets,
+                      asg_offsets, reinterpret_cast<unsigned long long *>(rank_mask), row_token,
+                      row_kmask, cap, send_row, comb_row, stats, src_dst, err);
 }
 
 }  // namespace
@@ -498,13 +510,15 @@ extern "C" int plan_dispatch(const int32_t *ids, int64_t N, int k, int E, const 
     if (!workspace || workspace_bytes < need || !aligned16(workspace)) return COACT_ERR_WORKSPACE;
     Workspace ws;
     workspace_layout(N, R, &ws, workspace);
+    DeviceInfo di;
+    if (int s = device_info(&di)) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 #define COACT_PLAN_CASE(KK)                                                                        \
     case KK:                                                                                       \
         return launch_plan<KK>(ids, N, E, expert_rank, R, rank_node, n_nodes, src_rank,            \
                                rank_counts, rank_offsets, asg_offsets, rank_mask, row_token,       \
                                row_kmask, row_capacity, send_row, comb_row, stats, src_dst, ws,    \
-                               err_flag, st);
+                               err_flag, st, di);
     switch (k) {
         COACT_PLAN_CASE(1)
         COACT_PLAN_CASE(2)
@@ -590,7 +604,7 @@ extern "C" int plan_dispatch_noalloc(const int32_t *ids, int64_t N, int k, int E
         return launch_plan<KK>(ids, N, E, expert_rank, R, rank_node, n_nodes, src_rank,            \
                                rank_counts, rank_offsets, asg_offsets, rank_mask, row_token,       \
                                row_kmask, row_capacity, send_row, comb_row, stats, src_dst, ws,    \
-                               err_flag, st);
+                               err_flag, st, di);
     switch (k) {
         COACT_PLAN_NOALLOC_CASE(1)
         COACT_PLAN_NOALLOC_CASE(2)

@@ -18,6 +18,8 @@ __global__ void __launch_bounds__(256)
     k_rank_scores(const int64_t *__restrict__ C12, int E1, int E2,
                   const int32_t *__restrict__ expert_rank2, int R, int64_t *__restrict__ S,
                   int32_t *__restrict__ err) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= (int64_t)E1 * R) return;
     const int a = (int)(i / R), r = (int)(i - (int64_t)a * R);
@@ -37,6 +39,8 @@ __global__ void __launch_bounds__(256)
     k_predict_home(const int32_t *__restrict__ ids1, int64_t N, int E1,
                    const int64_t *__restrict__ S, int R, int32_t *__restrict__ home,
                    int32_t *__restrict__ err) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     int flags = 0;
     if (t < N) {
@@ -85,13 +89,15 @@ extern "C" int predict_home(const int32_t *ids1, int64_t N, int k1, int E1, cons
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     int64_t *S = static_cast<int64_t *>(workspace);
     const int64_t cells = (int64_t)E1 * R;
-    k_rank_scores<<<(int)ceil_div(cells, 256), 256, 0, st>>>(C12, E1, E2, expert_rank2, R, S, err_flag);
-    if (N == 0) return launch_status();
+    if (int s = launch_pdl(k_rank_scores, (int)ceil_div(cells, 256), 256, 0, st, C12, E1, E2,
+                           expert_rank2, R, S, err_flag))
+        return s;
+    if (N == 0) return COACT_OK;
     const int blocks = (int)ceil_div(N, 256);
 #define COACT_PREDICT_CASE(KK)                                                                   \
     case KK:                                                                                     \
-        k_predict_home<KK><<<blocks, 256, 0, st>>>(ids1, N, E1, S, R, home, err_flag);            \
-        break;
+        return launch_pdl(k_predict_home<KK>, blocks, 256, 0, st, ids1, N, E1, S, R, home,        \
+                          err_flag);
     switch (k1) {
         COACT_PREDICT_CASE(1)
         COACT_PREDICT_CASE(2)
@@ -103,5 +109,5 @@ extern "C" int predict_home(const int32_t *ids1, int64_t N, int k1, int E1, cons
         COACT_PREDICT_CASE(8)
     }
 #undef COACT_PREDICT_CASE
-    return launch_status();
+    return COACT_ERR_UNSUPPORTED;
 }

@@ -119,7 +119,7 @@ def test_plan_full_size(coact, cfg):
 
 
 @pytest.mark.parametrize("variant", ["identity", "one_rank", "roundrobin3", "random_src2",
-                                     "two_nodes1", "ragged"])
+                                     "two_nodes1", "ragged", "beyond_one_wave"])
 def test_plan_variants(coact, variant):
     if variant == "identity":            # every expert alone on its rank: D == N*k
         r = workload.make_routing(0)
@@ -137,8 +137,11 @@ def test_plan_variants(coact, variant):
     elif variant == "two_nodes1":
         r = workload.make_routing(1)
         kw = dict(rank_node=(np.arange(8) // 4).astype(np.int32), n_nodes=2)
-    else:                                # token counts that leave partial warps and tiles
+    elif variant == "ragged":            # token counts that leave partial warps and tiles
         r = workload.make_routing(2, N=65536 - 4093)
+        kw = {}
+    else:                                # more tiles than fit on the GPU at once: the
+        r = workload.make_routing(3, N=200003)   # planner's multi-launch path
         kw = {}
     o = oracle_plan_for(r, **kw)
     plan, err = run_plan(coact, r, E=kw.get("E"), expert_rank=kw.get("expert_rank"),
