@@ -27,8 +27,8 @@ __global__ void __launch_bounds__(256)
     k_combine_v16(const uint4 *__restrict__ y, int64_t n_rows, const float *__restrict__ gates,
                   const int32_t *__restrict__ comb_row, int64_t N, int64_t H16,
                   void *__restrict__ out, int32_t *__restrict__ err) {
-    pdl_trigger();
     pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int64_t gwarp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;

@@ -78,9 +78,11 @@ __device__ __forceinline__ void raise_flag_warp(int32_t *err, int bits) {
 
 // Programmatic dependent launch.  Every library kernel is launched with programmatic
 // stream serialisation: it may start while the previous kernel on the stream drains,
-// runs only shared-memory set-up before pdl_wait(), and reads no global input until the
-// previous grid has completed and its writes are visible.  pdl_trigger() lets the next
-// kernel's blocks launch early; they too wait before touching our outputs.
+// and it reads no global input written by that kernel until pdl_wait() returns (the
+// previous grid has completed and its writes are visible).  Every library kernel calls
+// pdl_trigger() only AFTER its own pdl_wait(), so when a library kernel starts, every
+// kernel before its immediate predecessor has completed: a kernel whose predecessor is
+// another library kernel of the same call may read the call's inputs before waiting.
 __device__ __forceinline__ void pdl_wait() {
 #if !defined(COACT_NO_PDL)
     asm volatile("griddepcontrol.wait;" ::: "memory");

@@ -44,8 +44,8 @@ __global__ void __launch_bounds__(kCountThreads)
     uint32_t *tri = sh;
     uint32_t *sload = sh + nbins;
     for (int i = threadIdx.x; i < nbins + E; i += blockDim.x) sh[i] = 0;
-    pdl_trigger();
     pdl_wait();
+    pdl_trigger();
     __syncthreads();
 
     const int lane = threadIdx.x & 31;
@@ -102,8 +102,8 @@ template <int K>
 __global__ void __launch_bounds__(256)
     k_count_global(const int32_t *__restrict__ ids, int64_t N, int E, ull *__restrict__ pair,
                    ull *__restrict__ loads, int32_t *__restrict__ err) {
-    pdl_trigger();
     pdl_wait();
+    pdl_trigger();
     int flags = 0;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < N; t += stride) {
@@ -133,8 +133,8 @@ __global__ void __launch_bounds__(512)
     const int nb = SMEM ? E * E2 : 0;
     if (SMEM)
         for (int i = threadIdx.x; i < nb + E; i += blockDim.x) sh[i] = 0;
-    pdl_trigger();
     pdl_wait();
+    pdl_trigger();
     if (SMEM) __syncthreads();
     int flags = 0;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;

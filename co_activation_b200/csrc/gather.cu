@@ -32,8 +32,8 @@ __global__ void __launch_bounds__(256)
     k_gather_v16(const uint4 *__restrict__ x, int64_t N, int64_t H16,
                  const int32_t *__restrict__ send_row, int k, uint4 *__restrict__ send,
                  int64_t cap, int32_t *__restrict__ err) {
-    pdl_trigger();
     pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int64_t gwarp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -188,8 +188,8 @@ __global__ void __launch_bounds__(32)
         for (int s = 0; s < S; ++s) mbar_init(bars + 8 * s, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    pdl_trigger();
     pdl_wait();
+    pdl_trigger();
     if (lane == 0) {
         for (int64_t i = 0; i < n_mine && i < S; ++i) {
             const uint32_t bar = bars + 8 * (uint32_t)i;

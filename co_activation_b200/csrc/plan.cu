@@ -14,6 +14,8 @@
 //  2. k_plan_scan    R + 1 blocks: block r turns rank r's per-tile counts into exclusive
 //                    per-tile bases (in place) and a total; the last block reduces the
 //                    statistics partials and clears src_dst.
+//     (skipped when R * n_tiles <= COACT_PLAN_SMALL_MAX: k_plan_scatter<SMALL> then sums
+//     the per-tile counts itself, which costs less than a launch at these sizes)
 //  3. k_plan_scatter one thread per token again: rank offsets from the totals, stable
 //                    in-tile positions from per-rank ballots (rows) and 4-bit ballot
 //                    prefix sums (assignments), then row_token / row_kmask / send_row /
@@ -110,7 +112,7 @@ __global__ void __launch_bounds__(kTile)
                  const int32_t *__restrict__ expert_rank, int R,
                  const int32_t *__restrict__ rank_node, int n_nodes,
                  const int32_t *__restrict__ src_rank, int n_tiles, Workspace ws,
-                 int32_t *__restrict__ err) {
+                 int32_t *__restrict__ src_dst, int32_t *__restrict__ err) {
     __shared__ int s_node[64];
     __shared__ unsigned long long s_node_ranks[64];
     __shared__ int s_wrows[kTileWarps][64];
@@ -118,8 +120,10 @@ __global__ void __launch_bounds__(kTile)
     __shared__ long long s_stat[kTileWarps][kStatSlots];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    pdl_trigger();
     pdl_wait();
+    pdl_trigger();
+    if (src_dst && blockIdx.x == 0)   // cleared here; the scatter kernel accumulates into it
+        for (int i = tid; i < R * R; i += kTile) src_dst[i] = 0;
     load_nodes(rank_node, R, n_nodes, s_node, s_node_ranks, err);
     for (int i = tid; i < kTileWarps * 64; i += kTile) {
         (&s_wrows[0][0])[i] = 0;
@@ -229,8 +233,8 @@ __global__ void __launch_bounds__(kScanThreads)
                 int32_t *__restrict__ src_dst) {
     __shared__ int s_warp[33];
     __shared__ long long s_red[kStatSlots][32];
-    pdl_trigger();
     pdl_wait();
+    pdl_trigger();
     if ((int)blockIdx.x < R) {
         const int r = blockIdx.x;
         for (int which = 0; which < 2; ++which) {
@@ -277,11 +281,61 @@ __global__ void __launch_bounds__(kScanThreads)
         stats[COACT_STAT_REMOTE_ASG] = s_red[TS_VALID_ASG][0] - s_red[TS_LOCAL_ASG][0];
         stats[COACT_STAT_CROSSNODE_ASG] = s_red[TS_XNODE_ASG][0];
     }
-    if (src_dst)
+    if (src_dst)   // only when no tiles ran (N == 0); otherwise k_plan_tiles cleared it
         for (int i = threadIdx.x; i < R * R; i += kScanThreads) src_dst[i] = 0;
 }
 
-template <int K>
+// Rank offsets from per-rank totals (R <= 64: two ranks per lane of warp 0), then this
+// tile's base per rank.  tot_row/tot_asg and before_row/before_asg give, per rank, the
+// totals over all tiles and the sums over the tiles before this one.  Block 0 also
+// writes the offset outputs.
+__device__ __forceinline__ void rank_bases(int R, int tile, const int *tot_row,
+                                           const int *tot_asg, const int *before_row,
+                                           const int *before_asg, int *s_rbase, int *s_abase,
+                                           int32_t *rank_counts, int32_t *rank_offsets,
+                                           int32_t *asg_offsets, int64_t *stats) {
+    const int lane = threadIdx.x & 31;
+    const int r0 = lane, r1 = lane + 32;
+    for (int which = 0; which < 2; ++which) {
+        const int *tot = which == 0 ? tot_row : tot_asg;
+        const int *before = which == 0 ? before_row : before_asg;
+        const int v0 = r0 < R ? tot[r0] : 0, v1 = r1 < R ? tot[r1] : 0;
+        int i0 = v0, i1 = v1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u0 = __shfl_up_sync(0xffffffffu, i0, o);
+            const int u1 = __shfl_up_sync(0xffffffffu, i1, o);
+            if (lane >= o) {
+                i0 += u0;
+                i1 += u1;
+            }
+        }
+        const int total0 = __shfl_sync(0xffffffffu, i0, 31);
+        const int total = total0 + __shfl_sync(0xffffffffu, i1, 31);
+        const int e0 = i0 - v0, e1 = total0 + i1 - v1;
+        int *sbase = which == 0 ? s_rbase : s_abase;
+        if (r0 < R) sbase[r0] = e0 + before[r0];
+        if (r1 < R) sbase[r1] = e1 + before[r1];
+        if (tile == 0) {
+            int32_t *offs = which == 0 ? rank_offsets : asg_offsets;
+            if (r0 < R) offs[r0] = e0;
+            if (r1 < R) offs[r1] = e1;
+            if (lane == 0) offs[R] = total;
+            if (which == 0) {
+                if (r0 < R) rank_counts[r0] = v0;
+                if (r1 < R) rank_counts[r1] = v1;
+                if (lane == 0) stats[COACT_STAT_DEDUP_ROWS] = total;
+            }
+        }
+    }
+}
+
+// SMALL: the scan kernel is skipped (R * n_tiles small); every block sums the raw
+// per-tile counts itself and block 0 reduces the statistics.  Otherwise the per-tile
+// counts have been scanned in place by k_plan_scan and ws.tot holds the totals.
+// Everything before pdl_wait() reads only this call's inputs (safe: the predecessor is
+// this call's own k_plan_tiles or k_plan_scan, see pdl_wait).
+template <int K, bool SMALL>
 __global__ void __launch_bounds__(kTile)
     k_plan_scatter(const int32_t *__restrict__ ids, int64_t N, int E,
                    const int32_t *__restrict__ expert_rank, int R,
@@ -295,48 +349,12 @@ __global__ void __launch_bounds__(kTile)
     __shared__ int s_rbase[64], s_abase[64];
     __shared__ int s_wrows[kTileWarps][64];
     __shared__ int s_wasg[kTileWarps][64];
+    __shared__ int s_tot[2][64], s_before[2][64];
+    __shared__ long long s_stat[kTileWarps][kStatSlots];
     extern __shared__ int s_sd[];  // [R*R] when src_dst != NULL
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tile = blockIdx.x;
-    pdl_trigger();
-    pdl_wait();
-    if (warp == 0) {
-        // rank offsets = exclusive scan of the per-rank totals (R <= 64: two per lane)
-        const int r0 = lane, r1 = lane + 32;
-        for (int which = 0; which < 2; ++which) {
-            const int32_t *tot = ws.tot + which * R;
-            const int v0 = r0 < R ? tot[r0] : 0, v1 = r1 < R ? tot[r1] : 0;
-            int i0 = v0, i1 = v1;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int u0 = __shfl_up_sync(0xffffffffu, i0, o);
-                const int u1 = __shfl_up_sync(0xffffffffu, i1, o);
-                if (lane >= o) {
-                    i0 += u0;
-                    i1 += u1;
-                }
-            }
-            const int total0 = __shfl_sync(0xffffffffu, i0, 31);
-            const int total = total0 + __shfl_sync(0xffffffffu, i1, 31);
-            const int e0 = i0 - v0, e1 = total0 + i1 - v1;
-            int *sbase = which == 0 ? s_rbase : s_abase;
-            const int32_t *tb = which == 0 ? ws.tile_rows : ws.tile_asg;
-            if (r0 < R) sbase[r0] = e0 + (tile < n_tiles ? tb[(int64_t)r0 * n_tiles + tile] : 0);
-            if (r1 < R) sbase[r1] = e1 + (tile < n_tiles ? tb[(int64_t)r1 * n_tiles + tile] : 0);
-            if (tile == 0) {
-                int32_t *offs = which == 0 ? rank_offsets : asg_offsets;
-                if (r0 < R) offs[r0] = e0;
-                if (r1 < R) offs[r1] = e1;
-                if (lane == 0) offs[R] = total;
-                if (which == 0) {
-                    if (r0 < R) rank_counts[r0] = v0;
-                    if (r1 < R) rank_counts[r1] = v1;
-                    if (lane == 0) stats[COACT_STAT_DEDUP_ROWS] = total;
-                }
-            }
-        }
-    }
     for (int i = tid; i < kTileWarps * 64; i += kTile) {
         (&s_wrows[0][0])[i] = 0;
         (&s_wasg[0][0])[i] = 0;
@@ -345,6 +363,7 @@ __global__ void __launch_bounds__(kTile)
         for (int i = tid; i < R * R; i += kTile) s_sd[i] = 0;
     __syncthreads();
 
+    // ---- in-tile work: reads only the call's inputs
     const int64_t t = (int64_t)tile * kTile + tid;
     int rk[K];
     int src = 0;
@@ -360,9 +379,10 @@ __global__ void __launch_bounds__(kTile)
     const unsigned same_src = __match_any_sync(0xffffffffu, ok ? src : -1);
     const bool src_leader = ok && lane == __ffs(same_src) - 1;
 
-    int pre_row[K], pre_asg[K];
+    // per slot: in-warp row prefix (< 32) | in-warp assignment prefix (< 256) << 8
+    int pre[K];
 #pragma unroll
-    for (int j = 0; j < K; ++j) pre_row[j] = pre_asg[j] = 0;
+    for (int j = 0; j < K; ++j) pre[j] = 0;
     const unsigned lt = lanemask_lt();
     unsigned long long wmask = warp_or64(mask);
     while (wmask) {
@@ -381,13 +401,10 @@ __global__ void __launch_bounds__(kTile)
             ap += __popc(bb & lt) << bit;
             at += __popc(bb) << bit;
         }
-        const int rp = __popc(b & lt);
+        const int packed = __popc(b & lt) | (ap << 8);
 #pragma unroll
         for (int j = 0; j < K; ++j)
-            if (ok && rk[j] == r) {
-                pre_row[j] = rp;
-                pre_asg[j] = ap;
-            }
+            if (ok && rk[j] == r) pre[j] = packed;
         if (lane == 0) {
             s_wrows[warp][r] = __popc(b);
             s_wasg[warp][r] = at;
@@ -409,6 +426,64 @@ __global__ void __launch_bounds__(kTile)
             run_a += va;
         }
     }
+
+    // ---- cross-tile bases: need the predecessor's results
+    pdl_wait();
+    pdl_trigger();
+    if (SMALL) {
+        for (int r = warp; r < R; r += kTileWarps)
+            for (int which = 0; which < 2; ++which) {
+                const int32_t *cnt = (which == 0 ? ws.tile_rows : ws.tile_asg) + (int64_t)r * n_tiles;
+                int tot = 0, before = 0;
+                for (int i = lane; i < n_tiles; i += 32) {
+                    const int v = cnt[i];
+                    tot += v;
+                    before += i < tile ? v : 0;
+                }
+                tot = __reduce_add_sync(0xffffffffu, tot);
+                before = __reduce_add_sync(0xffffffffu, before);
+                if (lane == 0) {
+                    s_tot[which][r] = tot;
+                    s_before[which][r] = before;
+                }
+            }
+        if (tile == 0) {
+            long long acc[kStatSlots] = {0, 0, 0, 0, 0, 0};
+            for (int i = tid; i < n_tiles; i += kTile)
+#pragma unroll
+                for (int q = 0; q < kStatSlots; ++q) acc[q] += ws.tile_stats[(int64_t)i * kStatSlots + q];
+#pragma unroll
+            for (int q = 0; q < kStatSlots; ++q) {
+                long long v = acc[q];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (lane == 0) s_stat[warp][q] = v;
+            }
+        }
+    } else if (warp == 0) {
+        for (int r = lane; r < R; r += 32) {
+            s_tot[0][r] = ws.tot[r];
+            s_tot[1][r] = ws.tot[R + r];
+            s_before[0][r] = tile < n_tiles ? ws.tile_rows[(int64_t)r * n_tiles + tile] : 0;
+            s_before[1][r] = tile < n_tiles ? ws.tile_asg[(int64_t)r * n_tiles + tile] : 0;
+        }
+    }
+    __syncthreads();
+    if (warp == 0)
+        rank_bases(R, tile, s_tot[0], s_tot[1], s_before[0], s_before[1], s_rbase, s_abase,
+                   rank_counts, rank_offsets, asg_offsets, stats);
+    if (SMALL && tile == 0 && tid == 0) {
+        long long tot[kStatSlots] = {0, 0, 0, 0, 0, 0};
+        for (int w = 0; w < kTileWarps; ++w)
+            for (int q = 0; q < kStatSlots; ++q) tot[q] += s_stat[w][q];
+        stats[COACT_STAT_NAIVE_ROWS] = N * K;
+        stats[COACT_STAT_REMOTE_ROWS] = tot[TS_REMOTE_ROWS];
+        stats[COACT_STAT_CROSSNODE_ROWS] = tot[TS_XNODE_ROWS];
+        stats[COACT_STAT_NODE_DEDUP_ROWS] = tot[TS_NODE_ROWS];
+        stats[COACT_STAT_LOCAL_ASG] = tot[TS_LOCAL_ASG];
+        stats[COACT_STAT_REMOTE_ASG] = tot[TS_VALID_ASG] - tot[TS_LOCAL_ASG];
+        stats[COACT_STAT_CROSSNODE_ASG] = tot[TS_XNODE_ASG];
+    }
     __syncthreads();
 
     if (t < N) {
@@ -426,10 +501,10 @@ __global__ void __launch_bounds__(kTile)
 #pragma unroll
                 for (int jj = 0; jj < K; ++jj) km |= (unsigned)(rk[jj] == r) << jj;
                 const unsigned below = km & ((1u << j) - 1);
-                comb_row[t * K + j] = s_abase[r] + s_wasg[warp][r] + pre_asg[j] + __popc(below);
+                comb_row[t * K + j] = s_abase[r] + s_wasg[warp][r] + (pre[j] >> 8) + __popc(below);
                 int sr = -1;
                 if (below == 0) {
-                    const int64_t row = (int64_t)s_rbase[r] + s_wrows[warp][r] + pre_row[j];
+                    const int64_t row = (int64_t)s_rbase[r] + s_wrows[warp][r] + (pre[j] & 0xff);
                     if (row < cap) {
                         row_token[row] = (int32_t)t;
                         row_kmask[row] = (uint8_t)km;
@@ -445,13 +520,16 @@ __global__ void __launch_bounds__(kTile)
     }
     raise_flag_warp(err, flags);
     if (src_dst) {
-        __syncthreads();
         for (int i = tid; i < R * R; i += kTile) {
             const int v = s_sd[i];
             if (v) atomicAdd(src_dst + i, v);
         }
     }
 }
+
+#ifndef COACT_PLAN_SMALL_MAX
+#define COACT_PLAN_SMALL_MAX 4096  // R * n_tiles up to which the scan kernel is skipped
+#endif
 
 template <int K>
 int launch_plan(const int32_t *ids, int64_t N, int E, const int32_t *expert_rank, int R,
@@ -463,18 +541,27 @@ int launch_plan(const int32_t *ids, int64_t N, int E, const int32_t *expert_rank
     (void)di;
     const int n_tiles = (int)ceil_div(N, kTile);
     const size_t sd_smem = src_dst ? sizeof(int) * R * R : 0;
-
+    auto *rm = reinterpret_cast<unsigned long long *>(rank_mask);
+    if (n_tiles > 0 && (int64_t)R * n_tiles <= COACT_PLAN_SMALL_MAX) {
+        if (int s = launch_pdl(k_plan_tiles<K>, n_tiles, kTile, 0, st, ids, N, E, expert_rank, R,
+                               rank_node, n_nodes, src_rank, n_tiles, ws, src_dst, err))
+            return s;
+        return launch_pdl(k_plan_scatter<K, true>, n_tiles, kTile, sd_smem, st, ids, N, E,
+                          expert_rank, R, src_rank, n_tiles, ws, rank_counts, rank_offsets,
+                          asg_offsets, rm, row_token, row_kmask, cap, send_row, comb_row, stats,
+                          src_dst, err);
+    }
     if (n_tiles > 0)
         if (int s = launch_pdl(k_plan_tiles<K>, n_tiles, kTile, 0, st, ids, N, E, expert_rank, R,
-                               rank_node, n_nodes, src_rank, n_tiles, ws, err))
+                               rank_node, n_nodes, src_rank, n_tiles, ws, src_dst, err))
             return s;
     if (int s = launch_pdl(k_plan_scan, R + 1, kScanThreads, 0, st, N, K, R, n_tiles, ws, stats,
-                           src_dst))
+                           n_tiles > 0 ? nullptr : src_dst))
         return s;
-    return launch_pdl(k_plan_scatter<K>, std::max(n_tiles, 1), kTile, sd_smem, st, ids, N, E,
-                      expert_rank, R, src_rank, n_tiles, ws, rank_counts, rank_offsets,
-                      asg_offsets, reinterpret_cast<unsigned long long *>(rank_mask), row_token,
-                      row_kmask, cap, send_row, comb_row, stats, src_dst, err);
+    return launch_pdl(k_plan_scatter<K, false>, std::max(n_tiles, 1), kTile, sd_smem, st, ids, N,
+                      E, expert_rank, R, src_rank, n_tiles, ws, rank_counts, rank_offsets,
+                      asg_offsets, rm, row_token, row_kmask, cap, send_row, comb_row, stats,
+                      src_dst, err);
 }
 
 }  // namespace

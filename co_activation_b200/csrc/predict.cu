@@ -18,8 +18,8 @@ __global__ void __launch_bounds__(256)
     k_rank_scores(const int64_t *__restrict__ C12, int E1, int E2,
                   const int32_t *__restrict__ expert_rank2, int R, int64_t *__restrict__ S,
                   int32_t *__restrict__ err) {
-    pdl_trigger();
     pdl_wait();
+    pdl_trigger();
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= (int64_t)E1 * R) return;
     const int a = (int)(i / R), r = (int)(i - (int64_t)a * R);
@@ -39,8 +39,8 @@ __global__ void __launch_bounds__(256)
     k_predict_home(const int32_t *__restrict__ ids1, int64_t N, int E1,
                    const int64_t *__restrict__ S, int R, int32_t *__restrict__ home,
                    int32_t *__restrict__ err) {
-    pdl_trigger();
     pdl_wait();
+    pdl_trigger();
     const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     int flags = 0;
     if (t < N) {
