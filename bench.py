@@ -1,20 +1,21 @@
 """Benchmark of the co-activation dispatch/combine hot path on B200.
 
 One step = one pass of the whole path over one batch of N tokens:
-  coact_count (pair counts + loads) -> plan_dispatch (3 kernels) -> dispatch_gather
+  coact_count (pair counts + loads) -> plan_dispatch -> dispatch_gather
   -> combine_scatter (bf16 out)
 with inputs already resident in HBM.  Default workload: config 1 (N=16384, E=64,
 top-2, H=2048 bf16, 8 logical ranks of 8 experts, 16 planted pairs co-selected by 42%
-of tokens, random placement), seeded synthetic routing.
+of tokens, random placement), seeded synthetic routing.  Config 3 runs with the
+correlated placement the library builds from the batch's own pair counts; config 4 is
+two consecutive layers with token shuffling (cross-layer counts, predicted home ranks).
 
 Timing: W untimed warm-up steps, then EXACTLY K steps captured in one CUDA graph, each
-step bracketed by CUDA events on the launching stream, with an L2 flush (a write of a
-buffer twice the L2 size) between steps outside the events.  A barrier and
-torch.cuda.synchronize() bracket the timed region; multi-GPU runs (torchrun, one rank
-per GPU, each rank its own batch: weak scaling, no data-path collective) report the
-max over ranks.  `e2e` times the same step through the public API from pinned host
-buffers (H2D of the step's inputs and D2H of its outputs inside the timed region).
-`--impl reference` times the CPU oracle instead (rank 0 only).
+step bracketed by CUDA events on the launching stream, with an L2 flush between steps
+outside the events.  A barrier and torch.cuda.synchronize() bracket the timed region;
+multi-GPU runs (torchrun, one rank per GPU, each rank its own batch: weak scaling, no
+data-path collective) report the max over ranks.  `e2e` times the same step through the
+public API from pinned host buffers.  `--impl reference` times the CPU oracle instead
+(rank 0 only).
 
 Prints ONE JSON line (rank 0).
 """
@@ -39,9 +40,7 @@ import workload  # noqa: E402
 
 METRIC = "dispatch+combine tokens/s and HBM GB/s (% of ~8 TB/s); dedup rows/naive rows"
 UNIT = "tokens/s"
-X_STREAM, Y_STREAM = 1, 2
-KERNELS_PER_STEP = {"coact_count": 1, "plan_dispatch": 3, "dispatch_gather": 1,
-                    "combine_scatter": 1}
+X_STREAM, Y_STREAM, Y2_STREAM = 1, 2, 3
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -161,26 +160,32 @@ def barrier(world: int):
         dist.barrier()
 
 
-# ----------------------------------------------------------------------------- the GPU path
+# ----------------------------------------------------------------------------- one layer
 
 
-class GpuStep:
-    """Device buffers and the four library calls of one step."""
+class LayerBuffers:
+    """Device buffers and the four library calls of one MoE layer."""
 
-    def __init__(self, coact, r: workload.Routing, device, fill: bool = True):
+    def __init__(self, coact, r: workload.Routing, device, fill: bool = True,
+                 y_stream: int = Y_STREAM, x=None):
         cfg = r.cfg
         self.coact, self.r, self.cfg, self.dev = coact, r, cfg, device
         N, k, E, R, H = cfg.N, cfg.k, cfg.E, cfg.R, cfg.H
-        to = lambda a, dt=None: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
         self.ids = to(r.ids)
         self.gates = to(r.gates)
         self.expert_rank = to(r.expert_rank.astype(np.int32))
         self.rank_node = to(r.rank_node.astype(np.int32))
-        if fill:
+        self.src_rank = None
+        if x is not None:
+            self.x = x                                     # fed by an earlier layer
+        elif fill:
             self.x = workload.fill_bf16(N, H, r.seed, X_STREAM, device=device)
-            self.y = workload.fill_bf16(N * k, H, r.seed, Y_STREAM, device=device)
-        else:   # contents arrive by copy (end-to-end measurement)
+        else:                                              # contents arrive by copy
             self.x = torch.empty((N, H), dtype=torch.bfloat16, device=device)
+        if fill:
+            self.y = workload.fill_bf16(N * k, H, r.seed, y_stream, device=device)
+        else:
             self.y = torch.empty((N * k, H), dtype=torch.bfloat16, device=device)
         self.pair = torch.zeros((E, E), dtype=torch.int64, device=device)
         self.loads = torch.zeros(E, dtype=torch.int64, device=device)
@@ -188,7 +193,6 @@ class GpuStep:
         self.send = torch.empty((self.plan.row_capacity, H), dtype=torch.bfloat16, device=device)
         self.out = torch.empty((N, H), dtype=torch.bfloat16, device=device)
         self.err = torch.zeros(1, dtype=torch.int32, device=device)
-        self.side = torch.cuda.Stream(device=device)
 
     def count(self):
         self.coact.coact_count(self.ids, self.cfg.E, self.pair, self.loads, err_flag=self.err)
@@ -196,7 +200,7 @@ class GpuStep:
     def plan_(self):
         self.coact.plan_dispatch(self.ids, self.cfg.E, self.expert_rank, self.cfg.R, self.plan,
                                  rank_node=self.rank_node, n_nodes=self.cfg.n_nodes,
-                                 err_flag=self.err)
+                                 src_rank=self.src_rank, err_flag=self.err)
 
     def gather(self):
         self.coact.dispatch_gather(self.x, self.plan.send_row, self.send, err_flag=self.err)
@@ -205,24 +209,8 @@ class GpuStep:
         self.coact.combine_scatter(self.y, self.gates, self.plan.comb_row, self.out,
                                    err_flag=self.err)
 
-    def step(self, ev=None):
-        """One pass of the path.  coact_count depends on nothing the other three calls
-        produce, so it runs on a side stream, overlapped with plan_dispatch; the step
-        ends when both streams have finished.  ev: optional list of 5 events for the
-        phase boundaries (the count phase is then measured on the side stream)."""
-        main = torch.cuda.current_stream()
-        self.side.wait_stream(main)
-        if ev: ev[0].record()
-        with torch.cuda.stream(self.side):
-            self.count()
-            if ev: ev[1].record()
-        self.plan_()
-        if ev: ev[2].record()
-        self.gather()
-        if ev: ev[3].record()
-        self.combine()
-        main.wait_stream(self.side)
-        if ev: ev[4].record()
+    def D(self) -> int:
+        return int(self.plan.rank_offsets[-1].item())
 
     def bytes_gather(self, D):
         c = self.cfg
@@ -231,6 +219,183 @@ class GpuStep:
     def bytes_combine(self):
         c = self.cfg
         return c.N * c.k * c.H * 2 + c.N * c.H * 2 + c.N * c.k * 8
+
+
+def plan_launches(R: int, N: int) -> int:
+    """Kernels plan_dispatch launches: 2 when R x tiles <= 4096 (scan folded), else 3."""
+    return 2 if R * (-(-N // 256)) <= 4096 else 3
+
+
+class OneLayerStep:
+    """count (side stream, overlapped with the plan: it depends on nothing the other
+    calls produce) -> plan -> gather -> combine."""
+    n_events = 5
+    phases = {"coact_count": (0, 1), "plan_dispatch": (0, 2), "dispatch_gather": (2, 3),
+              "combine_scatter": (3, 4)}
+    host_inputs = ("ids", "gates", "expert_rank", "rank_node", "x", "y")
+
+    def __init__(self, coact, r: workload.Routing, device, fill: bool = True):
+        self.L = LayerBuffers(coact, r, device, fill)
+        self.cfg, self.N = r.cfg, r.cfg.N
+        self.side = torch.cuda.Stream(device=device)
+        self.kernels_per_step = 1 + plan_launches(r.cfg.R, self.N) + 1 + 1
+
+    def inputs(self):
+        return {n: getattr(self.L, n) for n in self.host_inputs}
+
+    def outputs(self):
+        return [self.L.out, self.L.plan.stats]
+
+    def clone_for_copy(self, coact, device):
+        c = OneLayerStep(coact, self.L.r, device, fill=False)
+        return c
+
+    def step(self, ev=None):
+        main = torch.cuda.current_stream()
+        self.side.wait_stream(main)
+        if ev: ev[0].record()
+        with torch.cuda.stream(self.side):
+            self.L.count()
+            if ev: ev[1].record()
+        self.L.plan_()
+        if ev: ev[2].record()
+        self.L.gather()
+        if ev: ev[3].record()
+        self.L.combine()
+        main.wait_stream(self.side)
+        if ev: ev[4].record()
+
+    def roofline_parts(self):
+        """(phase, kernel, algorithmic bytes) for the HBM-bound kernels."""
+        D = self.L.D()
+        return [("dispatch_gather", "k_gather_v16", self.L.bytes_gather(D)),
+                ("combine_scatter", "k_combine_v16", self.L.bytes_combine())]
+
+    def summary(self):
+        L = self.L
+        return {"dedup_rows_over_naive": L.D() / (self.N * self.cfg.k),
+                "stats": dict(zip(L.coact.STAT_NAMES, L.plan.stats.cpu().tolist())),
+                "err_flag": int(L.err.item())}
+
+
+class TwoLayerStep:
+    """Config 4: two consecutive MoE layers.  Layer 1 as above with contiguous home
+    ranks; then cross-layer counts (layer-1 x layer-2 picks, accumulated for the next
+    prediction), home-rank prediction from the calibration counts, and layer 2 with its
+    tokens pre-sharded to the predicted rank; layer 2's input rows are layer 1's output."""
+    n_events = 10
+    phases = {"layer1_plan": (0, 1), "layer1_gather": (1, 2), "layer1_combine": (2, 3),
+              "predict_home": (3, 4), "layer2_plan": (4, 5), "layer2_gather": (5, 6),
+              "layer2_combine": (6, 7), "side_counts": (0, 8)}   # ev8 on the side stream
+
+    def __init__(self, coact, tl: workload.TwoLayer, device, fill: bool = True, C12=None):
+        self.coact, self.tl = coact, tl
+        self.cfg = tl.layer1.cfg
+        self.N = self.cfg.N
+        E, R = self.cfg.E, self.cfg.R
+        self.L1 = LayerBuffers(coact, tl.layer1, device, fill, Y_STREAM)
+        self.L2 = LayerBuffers(coact, tl.layer2, device, fill, Y2_STREAM, x=self.L1.out)
+        self.home = torch.empty(self.N, dtype=torch.int32, device=device)
+        self.L2.src_rank = self.home
+        self.pws = torch.empty(max(coact.predict_workspace_bytes(E, R), 16), dtype=torch.uint8,
+                               device=device)
+        self.C12_live = torch.zeros((E, E), dtype=torch.int64, device=device)
+        if C12 is None:        # calibration batch (seed + 1) counted by the library
+            C12 = torch.zeros((E, E), dtype=torch.int64, device=device)
+            to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+            coact.coact_count(to(tl.calib1), E, C12, ids2=to(tl.calib2), E2=E)
+        self.C12 = C12
+        self.side = torch.cuda.Stream(device=device)
+        # counts: 2 per layer-set + 1 cross; two plans; 2 gathers; 2 combines; predict 2
+        self.kernels_per_step = 3 + 2 * plan_launches(R, self.N) + 2 + 2 + 2
+
+    def inputs(self):
+        return {"ids1": self.L1.ids, "gates1": self.L1.gates, "er1": self.L1.expert_rank,
+                "rn1": self.L1.rank_node, "x1": self.L1.x, "y1": self.L1.y,
+                "ids2": self.L2.ids, "gates2": self.L2.gates, "er2": self.L2.expert_rank,
+                "y2": self.L2.y, "C12": self.C12}
+
+    def outputs(self):
+        return [self.L2.out, self.L2.plan.stats]
+
+    def clone_for_copy(self, coact, device):
+        return TwoLayerStep(coact, self.tl, device, fill=False, C12=torch.empty_like(self.C12))
+
+    def step(self, ev=None):
+        c, E, R = self.coact, self.cfg.E, self.cfg.R
+        main = torch.cuda.current_stream()
+        self.side.wait_stream(main)
+        if ev: ev[0].record()
+        with torch.cuda.stream(self.side):
+            self.L1.count()
+            c.coact_count(self.L1.ids, E, self.C12_live, ids2=self.L2.ids, E2=E,
+                          err_flag=self.L1.err)
+            self.L2.count()
+            if ev: ev[8].record()
+        self.L1.plan_()
+        if ev: ev[1].record()
+        self.L1.gather()
+        if ev: ev[2].record()
+        self.L1.combine()
+        if ev: ev[3].record()
+        c.predict_home(self.L1.ids, E, self.C12, self.L2.expert_rank, R, self.home,
+                       workspace=self.pws, err_flag=self.L1.err)
+        if ev: ev[4].record()
+        self.L2.plan_()
+        if ev: ev[5].record()
+        self.L2.gather()
+        if ev: ev[6].record()
+        self.L2.combine()
+        if ev: ev[7].record()
+        main.wait_stream(self.side)
+        if ev: ev[9].record()
+
+    def roofline_parts(self):
+        D1, D2 = self.L1.D(), self.L2.D()
+        return [("layer1_gather", "k_gather_v16", self.L1.bytes_gather(D1)),
+                ("layer1_combine", "k_combine_v16", self.L1.bytes_combine()),
+                ("layer2_gather", "k_gather_v16", self.L2.bytes_gather(D2)),
+                ("layer2_combine", "k_combine_v16", self.L2.bytes_combine())]
+
+    def summary(self):
+        nk = self.N * self.cfg.k
+        st2 = self.L2.plan.stats.cpu().tolist()
+        # the same layer-2 batch with contiguous home ranks, for comparison
+        base = self.coact.alloc_plan(self.N, self.cfg.k, self.cfg.E, self.cfg.R, self.L2.dev)
+        self.coact.plan_dispatch(self.L2.ids, self.cfg.E, self.L2.expert_rank, self.cfg.R, base,
+                                 rank_node=self.L2.rank_node, n_nodes=self.cfg.n_nodes)
+        stb = base.stats.cpu().tolist()
+        return {"dedup_rows_over_naive": self.L2.D() / nk,
+                "layer1_dedup_rows_over_naive": self.L1.D() / nk,
+                "local_served_share_predicted_home": st2[5] / nk,
+                "local_served_share_contiguous_home": stb[5] / nk,
+                "crossnode_asg_share_predicted_home": st2[7] / nk,
+                "crossnode_asg_share_contiguous_home": stb[7] / nk,
+                "stats": dict(zip(self.coact.STAT_NAMES, st2)),
+                "err_flag": int(self.L1.err.item()) | int(self.L2.err.item())}
+
+
+def make_step(coact, cfg_index: int, seed: int, device):
+    """The step object for a configuration, plus a description of its placement."""
+    cfg = workload.CONFIGS[cfg_index]
+    if cfg.two_layer:
+        return TwoLayerStep(coact, workload.make_two_layer(cfg, seed=seed), device), \
+            "contiguous; layer 2 pre-sharded to the predicted home rank"
+    r = workload.make_routing(cfg, seed=seed)
+    S = OneLayerStep(coact, r, device)
+    placement = cfg.placement
+    if cfg_index == 3:
+        # co-activation-grouped placement: the library's greedy over this batch's counts
+        S.L.count()
+        placed = coact.coact_place_correlated(S.L.pair, cfg.R)
+        S.L.plan_()
+        S.rr_dedup = S.L.D() / (cfg.N * cfg.k)
+        S.L.expert_rank.copy_(placed.to(device))
+        S.L.r.expert_rank = placed.numpy()
+        S.L.pair.zero_()
+        S.L.loads.zero_()
+        placement = "correlated (coact_place_correlated over this batch's pair counts)"
+    return S, placement
 
 
 def read_traffic(kernel: str, workload_name: str):
@@ -251,6 +416,9 @@ def read_traffic(kernel: str, workload_name: str):
     return None
 
 
+# ----------------------------------------------------------------------------- GPU run
+
+
 def run_gpu(args):
     rank, world, local = dist_env()
     device = torch.device("cuda", local)
@@ -263,52 +431,45 @@ def run_gpu(args):
     import co_activation_b200 as coact
 
     cfg = workload.CONFIGS[args.config]
-    r = workload.make_routing(cfg, seed=rank_seed(args.seed, rank))
-    S = GpuStep(coact, r, device)
+    S, placement = make_step(coact, args.config, rank_seed(args.seed, rank), device)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     flush_w = torch.empty(max(2 * l2, 64 << 20), dtype=torch.uint8, device=device)
     flush_r = torch.zeros(max(2 * l2, 64 << 20) // 8, dtype=torch.int64, device=device)
     flush_sink = torch.empty((), dtype=torch.int64, device=device)
 
-    class _Flush:
+    def flush():
         """L2 flush between steps: write a buffer twice the L2 size, then read another
         one as large, so the step starts with a cold AND clean L2 (the dirty lines of the
         write are written back here, not inside the next timed kernel)."""
-
-        @staticmethod
-        def zero_():
-            flush_w.zero_()
-            torch.sum(flush_r, dim=0, out=flush_sink)
-
-    flush = _Flush()
+        flush_w.zero_()
+        torch.sum(flush_r, dim=0, out=flush_sink)
 
     # warm-up (also does every lazy one-time attribute setup before graph capture)
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         S.step()
     torch.cuda.synchronize()
-    D = int(S.plan.rank_offsets[-1].item())
-    stats = S.plan.stats.cpu().tolist()
-    assert S.err.item() == 0, f"device error flags {S.err.item()}"
+    summ = S.summary()
+    assert summ["err_flag"] == 0, f"device error flags {summ['err_flag']}"
 
-    K = args.steps
+    K, NE = args.steps, S.n_events
 
     def capture(with_phases: bool):
         """K steps (each preceded by the L2 flush) as one CUDA graph.  Events at the step
         boundaries always; at the phase boundaries only in the breakdown pass, because
         every event node inside a graph serialises the stream (about 3 us each)."""
-        ev = [[torch.cuda.Event(enable_timing=True, external=args.graph) for _ in range(5)]
+        ev = [[torch.cuda.Event(enable_timing=True, external=args.graph) for _ in range(NE)]
               for _ in range(K)]
 
         def body():
             for i in range(K):
-                flush.zero_()
+                flush()
                 if with_phases:
                     S.step(ev[i])
                 else:
                     ev[i][0].record()
                     S.step()
-                    ev[i][4].record()
+                    ev[i][NE - 1].record()
 
         if not args.graph:
             return None, ev, body
@@ -355,29 +516,19 @@ def run_gpu(args):
     barrier(world)
     clk = clocks.stop()
 
-    step_ms = [evs[i][0].elapsed_time(evs[i][4]) for i in range(K)]
-    # count runs on the side stream (ev0 -> ev1); the main stream runs plan (ev0 -> ev2),
-    # gather (ev2 -> ev3) and combine (ev3 -> ev4)
-    spans = {"coact_count": (0, 1), "plan_dispatch": (0, 2), "dispatch_gather": (2, 3),
-             "combine_scatter": (3, 4)}
-    phase_ms = {name: [evs_phase[i][a].elapsed_time(evs_phase[i][b]) for i in range(K)]
-                for name, (a, b) in spans.items()}
+    step_ms = [evs[i][0].elapsed_time(evs[i][NE - 1]) for i in range(K)]
+    phase_ms = {name: statistics.mean(evs_phase[i][a].elapsed_time(evs_phase[i][b])
+                                      for i in range(K))
+                for name, (a, b) in S.phases.items()}
     agg = aggregate(cfg.N * K, sum(step_ms) / 1e3, world, device)
     total_s, value = agg["seconds"], agg["tokens_per_s"]
-    gather_ms = statistics.mean(phase_ms["dispatch_gather"])
-    combine_ms = statistics.mean(phase_ms["combine_scatter"])
-    dc_tokens_s = cfg.N / ((gather_ms + combine_ms) / 1e3)
     peak, peak_kind = peaks()
-    gb_g = S.bytes_gather(D) / (gather_ms / 1e3) / 1e9
-    gb_c = S.bytes_combine() / (combine_ms / 1e3) / 1e9
-    gb_dc = (S.bytes_gather(D) + S.bytes_combine()) / ((gather_ms + combine_ms) / 1e3) / 1e9
-    dom = "combine_scatter" if combine_ms >= gather_ms else "dispatch_gather"
-    dom_bytes = S.bytes_combine() if dom == "combine_scatter" else S.bytes_gather(D)
-    dom_ms = combine_ms if dom == "combine_scatter" else gather_ms
-    kernel_name = "k_combine_v16" if dom == "combine_scatter" else "k_gather_v16"
-    wl_name = f"config{cfg.index}"
-    traffic = read_traffic(kernel_name, wl_name)
-
+    parts = [(ph, kern, byt, phase_ms[ph]) for ph, kern, byt in S.roofline_parts()]
+    dc_ms = sum(p[3] for p in parts)
+    dc_bytes = sum(p[2] for p in parts)
+    gb_dc = dc_bytes / (dc_ms / 1e3) / 1e9
+    dom = max(parts, key=lambda p: p[3])
+    dom_gbs = dom[2] / (dom[3] / 1e3) / 1e9
     e2e = run_e2e(coact, S, args, world, device)
 
     result = {
@@ -387,30 +538,35 @@ def run_gpu(args):
         "data": "synthetic (seeded routing shaped after the pages' statistics; no router traces)",
         "config": {"workload": f"config {cfg.index}: {cfg.desc}", "N": cfg.N, "E": cfg.E,
                    "k": cfg.k, "H": cfg.H, "R": cfg.R, "n_nodes": cfg.n_nodes,
-                   "placement": cfg.placement, "step": "coact_count (side stream, overlapped "
-                   "with plan) + plan_dispatch + dispatch_gather + combine_scatter (bf16 out)",
+                   "placement": placement,
+                   "step": ("two layers: counts + cross-layer counts (side stream); plan, gather, "
+                            "combine of layer 1; predict_home; plan, gather, combine of layer 2"
+                            if cfg.two_layer else
+                            "coact_count (side stream, overlapped with plan) + plan_dispatch + "
+                            "dispatch_gather + combine_scatter (bf16 out)"),
                    "l2": "flushed between timed steps (write of 2x L2, then a read of another 2x L2 "
                          "buffer so no dirty line is left), outside the step events",
                    "timing": timing,
                    "parallelism": f"{world} GPU(s), one independent batch per GPU"},
-        "dispatch_combine_tokens_per_s": dc_tokens_s,
-        "dedup_rows_over_naive": D / (cfg.N * cfg.k),
-        "stats": dict(zip(coact.STAT_NAMES, stats)),
-        "phase_us": {k_: statistics.mean(v) * 1e3 for k_, v in phase_ms.items()},
+        "dispatch_combine_tokens_per_s": cfg.N / (dc_ms / 1e3),
+        **{k_: v for k_, v in summ.items() if k_ != "err_flag"},
+        "phase_us": {k_: v * 1e3 for k_, v in phase_ms.items()},
         "phase_pass_step_us": statistics.mean(
-            evs_phase[i][0].elapsed_time(evs_phase[i][4]) for i in range(K)) * 1e3,
-        "hbm_gbs": {"dispatch_gather": gb_g, "combine_scatter": gb_c, "gather+combine": gb_dc,
+            evs_phase[i][0].elapsed_time(evs_phase[i][NE - 1]) for i in range(K)) * 1e3,
+        "hbm_gbs": {**{p[0]: p[2] / (p[3] / 1e3) / 1e9 for p in parts},
+                    "gather+combine": gb_dc,
                     "pct_of_8tbs_gather+combine": 100 * gb_dc / 8000.0,
                     f"pct_of_{peak_kind}_{peak:.0f}": 100 * gb_dc / peak},
-        "roofline": {"kernel": kernel_name, "bound": "hbm", "achieved": dom_bytes / (dom_ms / 1e3) / 1e9,
-                     "peak": peak, "unit": "GB/s",
-                     "frac": dom_bytes / (dom_ms / 1e3) / 1e9 / peak,
-                     "peak_kind": f"of {peak_kind}", "algorithmic_bytes": dom_bytes,
-                     "traffic": traffic},
+        "roofline": {"kernel": dom[1], "phase": dom[0], "bound": "hbm", "achieved": dom_gbs,
+                     "peak": peak, "unit": "GB/s", "frac": dom_gbs / peak,
+                     "peak_kind": f"of {peak_kind}", "algorithmic_bytes": dom[2],
+                     "traffic": read_traffic(dom[1], f"config{cfg.index}")},
         "clocks": clk,
-        "gpu_launches": K * sum(KERNELS_PER_STEP.values()),
+        "gpu_launches": K * S.kernels_per_step,
         "e2e": e2e,
     }
+    if hasattr(S, "rr_dedup"):
+        result["dedup_rows_over_naive_roundrobin"] = S.rr_dedup
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(S, args.cpu_seconds)
     if world > 1:
@@ -423,20 +579,18 @@ def run_gpu(args):
         print(json.dumps(result))
 
 
-def run_e2e(coact, S: GpuStep, args, world, device):
+def run_e2e(coact, S, args, world, device):
     """The step through the public API from pinned host buffers: every step copies its
-    inputs (ids, gates, placement, x and the expert outputs y) host -> device, runs the
-    four calls and copies its outputs (combined rows and statistics) device -> host.
-    Two device buffer sets let step i+1's input copy overlap step i's compute and
-    output copy (copy engines in both directions run concurrently with the SMs)."""
+    inputs host -> device, runs the library calls and copies its outputs (combined rows
+    and statistics) device -> host.  Two device buffer sets let step i+1's input copy
+    overlap step i's compute and output copy (copy engines in both directions run
+    concurrently with the SMs)."""
     cfg = S.cfg
-    names = ("ids", "gates", "expert_rank", "rank_node", "x", "y")
-    host = {n: getattr(S, n).cpu().pin_memory() for n in names}
-    bufs = [S, GpuStep(coact, S.r, device, fill=False)]
-    out_h = [torch.empty(S.out.shape, dtype=S.out.dtype).pin_memory() for _ in range(2)]
-    stats_h = [torch.empty(8, dtype=torch.int64).pin_memory() for _ in range(2)]
+    host = {n: t.cpu().pin_memory() for n, t in S.inputs().items()}
+    bufs = [S, S.clone_for_copy(coact, device)]
+    outs_h = [[t.cpu().pin_memory() for t in S.outputs()] for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_h[0].numel() * out_h[0].element_size() + 8 * 8
+    d2h = sum(t.numel() * t.element_size() for t in outs_h[0])
     comp = torch.cuda.current_stream()
     s_in, s_out = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
 
@@ -444,12 +598,14 @@ def run_e2e(coact, S: GpuStep, args, world, device):
         free = [None, None]
         for i in range(n_steps):
             b, slot = bufs[i % 2], i % 2
+            dst = b.inputs()
             with torch.cuda.stream(s_in):
-                s_in.wait_stream(comp) if i == 0 else None
+                if i == 0:
+                    s_in.wait_stream(comp)
                 if free[slot] is not None:
                     s_in.wait_event(free[slot])
                 for n, t in host.items():
-                    getattr(b, n).copy_(t, non_blocking=True)
+                    dst[n].copy_(t, non_blocking=True)
                 ready = torch.cuda.Event()
                 ready.record(s_in)
             comp.wait_event(ready)
@@ -458,8 +614,8 @@ def run_e2e(coact, S: GpuStep, args, world, device):
             done.record(comp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(done)
-                out_h[slot].copy_(b.out, non_blocking=True)
-                stats_h[slot].copy_(b.plan.stats, non_blocking=True)
+                for h, d in zip(outs_h[slot], b.outputs()):
+                    h.copy_(d, non_blocking=True)
                 fr = torch.cuda.Event()
                 fr.record(s_out)
             free[slot] = fr
@@ -488,29 +644,50 @@ def run_e2e(coact, S: GpuStep, args, world, device):
 # ----------------------------------------------------------------------------- the oracle
 
 
-def _oracle_step(o, ids, gates, er, rn, n_nodes, E, R, xb, yb):
+def _oracle_layer(o, ids, gates, er, rn, n_nodes, E, R, xb, yb, src=None):
     o.count(ids, E)
-    p = o.plan(ids, E, er, R, rank_node=rn, n_nodes=n_nodes)
+    p = o.plan(ids, E, er, R, rank_node=rn, n_nodes=n_nodes, src_rank=src)
     o.gather(xb, p["row_token"], p["D"])
-    o.combine_f64(yb, gates, p["comb_row"])
+    return o.combine_f64(yb, gates, p["comb_row"])
 
 
-def cpu_baseline(S: GpuStep, seconds: float):
+def _oracle_step_fn(S):
+    """A closure running the oracle over the same workload as step S (host arrays)."""
+    import oracle as o
+    cfg = S.cfg
+    if isinstance(S, TwoLayerStep):
+        tl = S.tl
+        x1, y1, y2 = o._bits(S.L1.x), o._bits(S.L1.y), o._bits(S.L2.y)
+        C12 = S.C12.cpu().numpy()
+
+        def fn():
+            out1 = _oracle_layer(o, tl.layer1.ids, tl.layer1.gates, tl.layer1.expert_rank,
+                                 tl.layer1.rank_node, cfg.n_nodes, cfg.E, cfg.R, x1, y1)
+            o.count_cross(tl.layer1.ids, cfg.E, tl.layer2.ids, cfg.E)
+            home, _ = o.predict_home(tl.layer1.ids, cfg.E, C12, tl.layer2.expert_rank, cfg.R)
+            x2 = o.bf16_rne(out1.astype(np.float32))
+            _oracle_layer(o, tl.layer2.ids, tl.layer2.gates, tl.layer2.expert_rank,
+                          tl.layer2.rank_node, cfg.n_nodes, cfg.E, cfg.R, x2, y2, src=home)
+        return fn
+    L = S.L
+    xb, yb = o._bits(L.x), o._bits(L.y)
+    return lambda: _oracle_layer(o, L.r.ids, L.r.gates, L.r.expert_rank, L.r.rank_node,
+                                 cfg.n_nodes, cfg.E, cfg.R, xb, yb)
+
+
+def cpu_baseline(S, seconds: float):
     """The oracle, as it stands, on this host: whole batches of the same workload
     repeated for about `seconds` (at least one)."""
-    import oracle as o
-    from oracle import _bits
-    r, cfg = S.r, S.cfg
-    xb, yb = _bits(S.x), _bits(S.y)
+    fn = _oracle_step_fn(S)
     n, t0 = 0, time.perf_counter()
     while True:
-        _oracle_step(o, r.ids, r.gates, r.expert_rank, r.rank_node, cfg.n_nodes, cfg.E, cfg.R, xb, yb)
+        fn()
         n += 1
         if time.perf_counter() - t0 >= seconds:
             break
     dt = time.perf_counter() - t0
-    return {"value": cfg.N * n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{n} whole batches of config {cfg.index} (N={cfg.N}) through the "
+    return {"value": S.N * n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n} whole batch(es) of config {S.cfg.index} (N={S.N}) through the "
                       "single-threaded C oracle: count, plan, gather, float64 combine",
             "host_cpu": _cpu_model(), "host_nproc": os.cpu_count()}
 
@@ -532,22 +709,21 @@ def run_reference(args):
     import oracle as o
     cfg = workload.CONFIGS[args.config]
     r = workload.make_routing(cfg, seed=args.seed)
-    xb = o._bits(workload.fill_bf16(cfg.N, cfg.H, r.seed, X_STREAM))
-    yb = o._bits(workload.fill_bf16(cfg.N * cfg.k, cfg.H, r.seed, Y_STREAM))
     # each step: a bounded sample of the workload (the first n tokens' routing, whole
-    # plan/gather/combine over them) sized so K + W steps end within a few minutes
+    # count/plan/gather/combine over them) sized so K + W steps end within a few minutes
     step_tokens = min(cfg.N, max(256, int(args.ref_tokens)))
     ids, gates = r.ids[:step_tokens], r.gates[:step_tokens]
-    xs, ys = xb[:step_tokens], yb[:step_tokens * cfg.k]
+    xs = o._bits(workload.fill_bf16(step_tokens, cfg.H, r.seed, X_STREAM))
+    ys = o._bits(workload.fill_bf16(step_tokens * cfg.k, cfg.H, r.seed, Y_STREAM))
     for _ in range(args.warmup):
-        _oracle_step(o, ids, gates, r.expert_rank, r.rank_node, cfg.n_nodes, cfg.E, cfg.R, xs, ys)
+        _oracle_layer(o, ids, gates, r.expert_rank, r.rank_node, cfg.n_nodes, cfg.E, cfg.R, xs, ys)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        _oracle_step(o, ids, gates, r.expert_rank, r.rank_node, cfg.n_nodes, cfg.E, cfg.R, xs, ys)
+        _oracle_layer(o, ids, gates, r.expert_rank, r.rank_node, cfg.n_nodes, cfg.E, cfg.R, xs, ys)
     dt = time.perf_counter() - t0
     value = step_tokens * args.steps / dt
     sample = (f"first {step_tokens} tokens of config {cfg.index} per step (count, plan, gather, "
-              "float64 combine), single-threaded C oracle")
+              "float64 combine of one layer), single-threaded C oracle")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,

@@ -118,7 +118,7 @@ def test_plan_full_size(coact, cfg):
     assert_plan_equal(plan_to_host(plan), o)
 
 
-@pytest.mark.parametrize("variant", ["identity", "one_rank", "roundrobin3", "random_src2",
+@pytest.mark.parametrize("variant", ["identity", "one_rank", "planted3", "random_src2",
                                      "two_nodes1", "ragged", "beyond_one_wave"])
 def test_plan_variants(coact, variant):
     if variant == "identity":            # every expert alone on its rank: D == N*k
@@ -128,8 +128,8 @@ def test_plan_variants(coact, variant):
     elif variant == "one_rank":          # one rank: nothing remote, D == N
         r = workload.make_routing(1)
         kw = dict(expert_rank=np.zeros(64, np.int32), R=1, rank_node=np.zeros(1, np.int32))
-    elif variant == "roundrobin3":
-        r = workload.make_routing(3, placement_kind="roundrobin")
+    elif variant == "planted3":
+        r = workload.make_routing(3, placement_kind="planted")
         kw = {}
     elif variant == "random_src2":
         r = workload.make_routing(2)

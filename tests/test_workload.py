@@ -36,9 +36,9 @@ def test_routing_deterministic():
     assert not np.array_equal(a.ids, c.ids)
 
 
-def test_grouped_and_roundrobin_placement():
+def test_planted_and_roundrobin_placement():
     cfg = workload.CONFIGS[3]
-    r = workload.make_routing(cfg.with_(N=256))
+    r = workload.make_routing(cfg.with_(N=256), placement_kind="planted")
     er = r.expert_rank
     for g in r.groups:                                      # every planted pair co-located
         assert er[g[0]] == er[g[1]]

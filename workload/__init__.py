@@ -61,7 +61,7 @@ class Config:
     fixed_groups: Optional[tuple]    # explicit groups (config 0), else drawn
     bias: float                      # logit bias added to a planted token's group
     plant_prob: float                # probability that a token is planted
-    placement: str                   # contiguous | random | grouped | roundrobin
+    placement: str                   # contiguous | random | planted | roundrobin
     two_layer: bool = False
     desc: str = ""
 
@@ -101,9 +101,10 @@ CONFIGS = {
                    "8 planted groups of 4 (+2.5, 30%)"),
     3: Config(3, N=131072, E=256, k=8, H=7168, R=64, n_nodes=8, zipf_s=1.2,
               group_size=2, n_groups=32, fixed_groups=None, bias=3.0,
-              plant_prob=0.35, placement="grouped",
+              plant_prob=0.35, placement="roundrobin",
               desc="N=131072 E=256 top-8 H=7168; 64 ranks x4 experts in 8 nodes; Zipf(1.2); "
-                   "32 planted pairs (+3, 35%); grouped placement (round-robin variant)"),
+                   "32 planted pairs (+3, 35%); round-robin placement, and the correlated "
+                   "placement built from the batch's pair counts"),
     4: Config(4, N=65536, E=128, k=2, H=4096, R=16, n_nodes=2, zipf_s=None,
               group_size=2, n_groups=0, fixed_groups=None, bias=0.0,
               plant_prob=0.0, placement="contiguous", two_layer=True,
@@ -181,11 +182,11 @@ def placement(cfg: Config, kind: str, groups: Optional[np.ndarray] = None,
     contiguous : expert e -> rank e // epr
     random     : a seeded permutation perm; expert perm[i] -> rank i // epr
     roundrobin : expert e -> rank e mod R
-    grouped    : co-locates the planted co-activation groups: groups in order go to
+    planted    : co-locates the planted co-activation groups: groups in order go to
                  the lowest-index rank with room for the whole group, then the other
-                 experts, ascending id, to the lowest rank with a free slot.  The
-                 fixture stands in for a placement planner (it uses the generator's
-                 ground-truth groups, not measured counts).
+                 experts, ascending id, to the lowest rank with a free slot (uses the
+                 generator's ground-truth groups; the placement built from *measured*
+                 counts is the library's coact_place_correlated).
     identity   : E == R, expert e -> rank e (every expert alone on its rank)
     """
     E, R, epr = cfg.E, cfg.R, cfg.epr
@@ -202,9 +203,9 @@ def placement(cfg: Config, kind: str, groups: Optional[np.ndarray] = None,
         out = np.empty(E, dtype=np.int32)
         out[perm] = np.arange(E) // epr
         return out
-    if kind == "grouped":
+    if kind == "planted":
         if groups is None:
-            raise ValueError("grouped placement needs the planted groups")
+            raise ValueError("planted placement needs the planted groups")
         out = np.full(E, -1, dtype=np.int32)
         free = np.full(R, epr, dtype=np.int64)
         for g in groups:
