@@ -375,9 +375,80 @@ class TwoLayerStep:
                 "err_flag": int(self.L1.err.item()) | int(self.L2.err.item())}
 
 
-def make_step(coact, cfg_index: int, seed: int, device):
+class TwoHopStep(OneLayerStep):
+    """One layer with the two-hop dispatch (Cobalt: fewer remote nodes): count (side
+    stream) -> node-level plan + rank-level plan + forward map -> hop-1 gather into node
+    segments -> hop-2 forward into rank segments -> combine."""
+    n_events = 6
+    phases = {"coact_count": (0, 1), "plan_two_hop": (0, 2), "gather_hop1": (2, 3),
+              "forward_hop2": (3, 4), "combine_scatter": (4, 5)}
+
+    def __init__(self, coact, r: workload.Routing, device, fill: bool = True):
+        super().__init__(coact, r, device, fill)
+        c = r.cfg
+        self.th = coact.alloc_two_hop(c.N, c.k, c.E, c.R, c.n_nodes, device)
+        self.hop1 = torch.empty((self.th.node.row_capacity, c.H), dtype=torch.bfloat16,
+                                device=device)
+        # counts 1; compose 2; node plan + rank plan; forward 1; hop-1 gather; hop-2; combine
+        self.kernels_per_step = 1 + 2 + plan_launches(c.n_nodes, c.N) + plan_launches(c.R, c.N) \
+            + 1 + 1 + 1 + 1
+
+    def clone_for_copy(self, coact, device):
+        return TwoHopStep(coact, self.L.r, device, fill=False)
+
+    def step(self, ev=None):
+        L, c = self.L, self.cfg
+        main = torch.cuda.current_stream()
+        self.side.wait_stream(main)
+        if ev: ev[0].record()
+        with torch.cuda.stream(self.side):
+            L.count()
+            if ev: ev[1].record()
+        L.coact.plan_two_hop(L.ids, c.E, L.expert_rank, c.R, L.rank_node, c.n_nodes, self.th,
+                             err_flag=L.err)
+        if ev: ev[2].record()
+        L.coact.dispatch_gather(L.x, self.th.node.send_row, self.hop1, err_flag=L.err)
+        if ev: ev[3].record()
+        L.coact.forward_gather(self.hop1, self.th.fwd_src, L.send, err_flag=L.err)
+        if ev: ev[4].record()
+        L.coact.combine_scatter(L.y, L.gates, self.th.rank.comb_row, L.out, err_flag=L.err)
+        main.wait_stream(self.side)
+        if ev: ev[5].record()
+
+    def roofline_parts(self):
+        c = self.cfg
+        Dn = int(self.th.node.rank_offsets[-1].item())
+        D = int(self.th.rank.rank_offsets[-1].item())
+        return [("gather_hop1", "k_gather_v16", (c.N + Dn) * c.H * 2 + c.N * c.k * 4),
+                ("forward_hop2", "k_forward_gather", 2 * D * c.H * 2 + D * 4),
+                ("combine_scatter", "k_combine_v16", self.L.bytes_combine())]
+
+    def summary(self):
+        c, nk = self.cfg, self.N * self.cfg.k
+        sn = self.th.node.stats.cpu().tolist()
+        sr = self.th.rank.stats.cpu().tolist()
+        return {"dedup_rows_over_naive": sr[1] / nk,
+                "hop1_node_rows": sn[1], "hop1_remote_node_rows": sn[2],
+                "rank_rows": sr[1], "one_hop_crossnode_rows": sr[3],
+                "crossnode_rows_cut_by_two_hop": 1 - sn[2] / max(sr[3], 1),
+                "stats": dict(zip(self.L.coact.STAT_NAMES, sr)),
+                "err_flag": int(self.L.err.item())}
+
+
+def make_step(coact, cfg_index: int, seed: int, device, two_hop: bool = False):
     """The step object for a configuration, plus a description of its placement."""
     cfg = workload.CONFIGS[cfg_index]
+    if two_hop:
+        if cfg.two_layer or cfg.n_nodes < 2:
+            raise SystemExit("--two-hop needs a one-layer configuration with several nodes (2, 3)")
+        r = workload.make_routing(cfg, seed=seed)
+        if cfg_index == 3:   # the same correlated placement as the one-hop step
+            tmp = OneLayerStep(coact, r, device, fill=False)
+            tmp.L.count()
+            r.expert_rank = coact.coact_place_correlated(tmp.L.pair, cfg.R).numpy()
+            del tmp
+        return TwoHopStep(coact, r, device), (cfg.placement if cfg_index != 3 else
+                                              "correlated (coact_place_correlated)")
     if cfg.two_layer:
         return TwoLayerStep(coact, workload.make_two_layer(cfg, seed=seed), device), \
             "contiguous; layer 2 pre-sharded to the predicted home rank"
@@ -431,7 +502,7 @@ def run_gpu(args):
     import co_activation_b200 as coact
 
     cfg = workload.CONFIGS[args.config]
-    S, placement = make_step(coact, args.config, rank_seed(args.seed, rank), device)
+    S, placement = make_step(coact, args.config, rank_seed(args.seed, rank), device, args.two_hop)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     flush_w = torch.empty(max(2 * l2, 64 << 20), dtype=torch.uint8, device=device)
     flush_r = torch.zeros(max(2 * l2, 64 << 20) // 8, dtype=torch.int64, device=device)
@@ -542,6 +613,9 @@ def run_gpu(args):
                    "step": ("two layers: counts + cross-layer counts (side stream); plan, gather, "
                             "combine of layer 1; predict_home; plan, gather, combine of layer 2"
                             if cfg.two_layer else
+                            "coact_count (side stream) + two-hop plan (node and rank plans, "
+                            "forward map) + hop-1 gather + hop-2 forward + combine_scatter"
+                            if args.two_hop else
                             "coact_count (side stream, overlapped with plan) + plan_dispatch + "
                             "dispatch_gather + combine_scatter (bf16 out)"),
                    "l2": "flushed between timed steps (write of 2x L2, then a read of another 2x L2 "
@@ -749,6 +823,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--clock-warm-s", type=float, default=1.0)
     ap.add_argument("--ref-tokens", type=int, default=4096)
+    ap.add_argument("--two-hop", action="store_true",
+                    help="dispatch in two hops: to nodes, then inside the node to ranks")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -52,16 +52,20 @@ _lib.predict_home_workspace_bytes.argtypes = [_I32, _I32]
 _lib.predict_home_workspace_bytes.restype = _SZ
 _lib.predict_home.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _SZ, _P, _P]
 _lib.coact_place_correlated.argtypes = [_P, _I32, _I32, _P]
+_lib.coact_compose_map.argtypes = [_P, _I64, _P, _I64, _P, _P, _P]
+_lib.plan_forward.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _P, _P, _I64, _P, _P]
+_lib.forward_gather.argtypes = [_P, _I64, _I64, _P, _I64, _P, _P, _P]
 _lib.plan_dispatch_noalloc.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _P, _P,
                                        _P, _P, _P, _I64, _P, _P, _P, _P, _P, _P]
 for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "combine_scatter", "predict_home",
-           "coact_place_correlated", "plan_dispatch_noalloc"):
+           "coact_place_correlated", "plan_dispatch_noalloc", "coact_compose_map", "plan_forward",
+           "forward_gather"):
     getattr(_lib, _f).restype = _I32
 
 ABI_SYMBOLS = ("coact_strerror", "coact_abi_version", "coact_count", "plan_dispatch_workspace_bytes",
                "plan_dispatch", "dispatch_gather", "combine_scatter",
                "predict_home_workspace_bytes", "predict_home", "coact_place_correlated",
-               "plan_dispatch_noalloc")
+               "plan_dispatch_noalloc", "coact_compose_map", "plan_forward", "forward_gather")
 NOALLOC_MAX_TOKENS = 262144
 
 
@@ -330,3 +334,101 @@ def plan_dispatch_noalloc(ids: torch.Tensor, E: int, expert_rank: torch.Tensor, 
         _ptr(plan.send_row), _ptr(plan.comb_row), _ptr(plan.stats), _ptr(plan.src_dst),
         _ptr(err_flag), _stream(stream)), "plan_dispatch_noalloc")
     return plan
+
+
+# ----------------------------------------------------------------------------- two-hop dispatch
+
+
+def coact_compose_map(a: torch.Tensor, b: torch.Tensor, out: Optional[torch.Tensor] = None,
+                      err_flag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out[i] = b[a[i]] on the device (int32)."""
+    _need(a, "a", torch.int32)
+    _need(b, "b", torch.int32)
+    if out is None:
+        out = torch.empty_like(a)
+    _need(out, "out", torch.int32, tuple(a.shape))
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.coact_compose_map(_ptr(a), a.numel(), _ptr(b), b.numel(), _ptr(out),
+                                  _ptr(err_flag), _stream(stream)), "coact_compose_map")
+    return out
+
+
+def plan_forward(ids: torch.Tensor, E: int, expert_rank: torch.Tensor, R: int, rank_plan: Plan,
+                 node_plan: Plan, fwd_src: torch.Tensor, rank_node: Optional[torch.Tensor] = None,
+                 n_nodes: int = 1, err_flag: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """fwd_src[d] = the node-level (hop-1) row feeding rank-level row d; -1 past D."""
+    N, k = ids.shape
+    _need(ids, "ids", torch.int32)
+    _need(expert_rank, "expert_rank", torch.int32, (E,))
+    _need(rank_node, "rank_node", torch.int32, (R,), optional=True)
+    _need(fwd_src, "fwd_src", torch.int32, (rank_plan.row_capacity,))
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.plan_forward(_ptr(ids), N, k, E, _ptr(expert_rank), R, _ptr(rank_node), n_nodes,
+                             _ptr(rank_plan.send_row), _ptr(rank_plan.rank_offsets),
+                             _ptr(node_plan.send_row), _ptr(fwd_src), rank_plan.row_capacity,
+                             _ptr(err_flag), _stream(stream)), "plan_forward")
+    return fwd_src
+
+
+def forward_gather(src: torch.Tensor, fwd_src: torch.Tensor, dst: torch.Tensor,
+                   err_flag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """dst[d] = src[fwd_src[d]] for fwd_src[d] >= 0 (bf16 rows)."""
+    _need(_bits16(src), "src", torch.bfloat16)
+    _need(_bits16(dst), "dst", torch.bfloat16)
+    if src.shape[1] != dst.shape[1]:
+        raise ValueError("src and dst rows must have the same width")
+    _need(fwd_src, "fwd_src", torch.int32, (dst.shape[0],))
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.forward_gather(_ptr(src), src.shape[0], src.shape[1], _ptr(fwd_src), dst.shape[0],
+                               _ptr(dst), _ptr(err_flag), _stream(stream)), "forward_gather")
+    return dst
+
+
+@dataclasses.dataclass
+class TwoHopPlan:
+    """Plans of a two-hop dispatch: node level (hop 1), rank level (hop 2) and the map
+    between them.  expert_node / src_node are the device maps the node plan used;
+    node_ids (0..n_nodes-1) and contiguous_src (floor(t*R/N), the default home ranks)
+    are constant inputs made once here."""
+    node: Plan
+    rank: Plan
+    fwd_src: torch.Tensor
+    expert_node: torch.Tensor
+    src_node: torch.Tensor
+    node_ids: torch.Tensor
+    contiguous_src: torch.Tensor
+
+
+def alloc_two_hop(N: int, k: int, E: int, R: int, n_nodes: int, device="cuda") -> TwoHopPlan:
+    dev = torch.device(device)
+    rank = alloc_plan(N, k, E, R, dev)
+    t = torch.arange(N, dtype=torch.int64, device=dev)
+    return TwoHopPlan(node=alloc_plan(N, k, E, n_nodes, dev), rank=rank,
+                      fwd_src=torch.empty(rank.row_capacity, dtype=torch.int32, device=dev),
+                      expert_node=torch.empty(E, dtype=torch.int32, device=dev),
+                      src_node=torch.empty(N, dtype=torch.int32, device=dev),
+                      node_ids=torch.arange(n_nodes, dtype=torch.int32, device=dev),
+                      contiguous_src=(t * R // max(N, 1)).to(torch.int32))
+
+
+def plan_two_hop(ids: torch.Tensor, E: int, expert_rank: torch.Tensor, R: int,
+                 rank_node: torch.Tensor, n_nodes: int, th: TwoHopPlan,
+                 src_rank: Optional[torch.Tensor] = None, err_flag: Optional[torch.Tensor] = None,
+                 stream=None) -> TwoHopPlan:
+    """Both plans and the forward map, all in library kernels: expert -> node and token
+    -> home node maps (coact_compose_map), the node-level plan_dispatch, the rank-level
+    plan_dispatch and plan_forward."""
+    N = ids.shape[0]
+    coact_compose_map(expert_rank, rank_node, th.expert_node, err_flag, stream)
+    src = th.contiguous_src if src_rank is None else src_rank
+    if N:
+        coact_compose_map(src, rank_node, th.src_node, err_flag, stream)
+    plan_dispatch(ids, E, th.expert_node, n_nodes, th.node, rank_node=th.node_ids,
+                  n_nodes=n_nodes, src_rank=th.src_node if N else None, err_flag=err_flag,
+                  stream=stream)
+    plan_dispatch(ids, E, expert_rank, R, th.rank, rank_node=rank_node, n_nodes=n_nodes,
+                  src_rank=src_rank, err_flag=err_flag, stream=stream)
+    plan_forward(ids, E, expert_rank, R, th.rank, th.node, th.fwd_src, rank_node=rank_node,
+                 n_nodes=n_nodes, err_flag=err_flag, stream=stream)
+    return th

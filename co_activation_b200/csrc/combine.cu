@@ -99,7 +99,14 @@ __global__ void __launch_bounds__(256)
 template <int K, bool F32>
 int launch(const uint16_t *y, int64_t n_rows, const float *gates, const int32_t *comb_row,
            int64_t N, int64_t H, void *out, int32_t *err, cudaStream_t st, const DeviceInfo &di) {
-    constexpr int U = K <= 2 ? 4 : (K <= 4 ? 2 : 1);
+    // column chunks per lane: 8 loads in flight for k <= 2 (U = 4), U = 2 chunks for
+    // k >= 3 (6-16 loads).  Measured on B200: U = 2 made k = 6 6% faster and k = 8
+    // 0.4% faster than U = 1, while U = 8 made k = 2 1.6% slower than U = 4.
+#if defined(COACT_COMBINE_LOADS)
+    constexpr int U = K >= COACT_COMBINE_LOADS ? 1 : COACT_COMBINE_LOADS / K;  // experiments
+#else
+    constexpr int U = K <= 2 ? 4 : 2;
+#endif
     const int64_t H16 = H / 8;
     const int blocks = (int)std::max<int64_t>(
         1, std::min<int64_t>(ceil_div(N, 8), (int64_t)di.sm_count * 8));

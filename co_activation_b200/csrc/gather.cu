@@ -273,9 +273,13 @@ int launch_v16(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row,
         1, std::min<int64_t>(ceil_div(warps_needed, 8), (int64_t)di.sm_count * 8));
     const uint4 *xv = reinterpret_cast<const uint4 *>(x);
     uint4 *sv = reinterpret_cast<uint4 *>(send);
+#ifndef COACT_GATHER_UNROLL
+#define COACT_GATHER_UNROLL 8  // 16-byte loads in flight per lane on long rows
+#endif
     if (H16 <= 32) return launch_pdl(k_gather_v16<1>, blocks, 256, 0, st, xv, N, H16, send_row, k, sv, cap, err);
     if (H16 <= 128) return launch_pdl(k_gather_v16<4>, blocks, 256, 0, st, xv, N, H16, send_row, k, sv, cap, err);
-    return launch_pdl(k_gather_v16<8>, blocks, 256, 0, st, xv, N, H16, send_row, k, sv, cap, err);
+    return launch_pdl(k_gather_v16<COACT_GATHER_UNROLL>, blocks, 256, 0, st, xv, N, H16, send_row,
+                      k, sv, cap, err);
 }
 
 }  // namespace

@@ -78,20 +78,21 @@ __device__ __forceinline__ int load_token(const int32_t *__restrict__ ids,
 
 // rank -> node table and node -> rank-set table in shared memory.  A node id outside
 // [0, n_nodes) raises COACT_EFLAG_ID_RANGE and is read as node 0.
-__device__ __forceinline__ void load_nodes(const int32_t *__restrict__ rank_node, int R,
-                                           int n_nodes, int *s_node, unsigned long long *s_node_ranks,
-                                           int32_t *err) {
+__device__ __forceinline__ int fetch_node(const int32_t *__restrict__ rank_node, int R) {
+    const int tid = threadIdx.x;
+    return (tid < R && rank_node) ? __ldg(rank_node + tid) : 0;
+}
+
+// nd: this thread's fetch_node() value (issued early so its latency overlaps other loads).
+__device__ __forceinline__ void load_nodes(int nd, int R, int n_nodes, int *s_node,
+                                           unsigned long long *s_node_ranks, int32_t *err) {
     const int tid = threadIdx.x;
     if (tid < 64) {
-        int nd = 0;
-        if (tid < R && rank_node) {
-            nd = __ldg(rank_node + tid);
-            if ((unsigned)nd >= (unsigned)n_nodes) {
-                raise_flag(err, COACT_EFLAG_ID_RANGE);
-                nd = 0;
-            }
+        if (tid < R && (unsigned)nd >= (unsigned)n_nodes) {
+            raise_flag(err, COACT_EFLAG_ID_RANGE);
+            nd = 0;
         }
-        s_node[tid] = nd;
+        s_node[tid] = tid < R ? nd : 0;
         s_node_ranks[tid] = 0;
     }
     __syncthreads();
@@ -120,17 +121,16 @@ __global__ void __launch_bounds__(kTile)
     __shared__ long long s_stat[kTileWarps][kStatSlots];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    pdl_wait();
-    pdl_trigger();
-    if (src_dst && blockIdx.x == 0)   // cleared here; the scatter kernel accumulates into it
-        for (int i = tid; i < R * R; i += kTile) src_dst[i] = 0;
-    load_nodes(rank_node, R, n_nodes, s_node, s_node_ranks, err);
     for (int i = tid; i < kTileWarps * 64; i += kTile) {
         (&s_wrows[0][0])[i] = 0;
         (&s_wasg[0][0])[i] = 0;
     }
-    __syncthreads();
-
+    pdl_wait();
+    pdl_trigger();
+    if (src_dst && blockIdx.x == 0)   // cleared here; the scatter kernel accumulates into it
+        for (int i = tid; i < R * R; i += kTile) src_dst[i] = 0;
+    // the node table's load and the token's loads are in flight together
+    const int nd = fetch_node(rank_node, R);
     const int64_t t = (int64_t)blockIdx.x * kTile + tid;
     int rk[K];
     int src = 0;
@@ -140,6 +140,7 @@ __global__ void __launch_bounds__(kTile)
         flags = load_token<K>(ids, expert_rank, src_rank, t, N, E, R, rk, src);
         ok = flags == 0;
     }
+    load_nodes(nd, R, n_nodes, s_node, s_node_ranks, err);
     unsigned long long mask = 0;
     int st[kStatSlots] = {0, 0, 0, 0, 0, 0};
     if (ok) {

@@ -225,6 +225,45 @@ int plan_dispatch_noalloc(const int32_t *ids, int64_t N, int k, int E,
                           int64_t *stats, int32_t *src_dst,
                           int32_t *err_flag, coact_stream_t stream);
 
+/*
+ * Two-hop dispatch.  Cobalt, English abstract: the communication-aware task assignment
+ * "routes tokens to fewer remote nodes".  Hop 1 sends each token once to each destination
+ * NODE (an ordinary plan_dispatch at node granularity: expert -> node map, home node, R =
+ * n_nodes); hop 2 forwards each node-level row inside the node to the token's ranks there
+ * (the rank-level plan).  These three calls connect the two plans.
+ *
+ * coact_compose_map -- out[i] = b[a[i]] for i < n (device arrays; e.g. expert -> rank ->
+ * node with a = expert_rank, b = rank_node; or token home rank -> home node).  An a[i]
+ * outside [0, nb) gives out[i] = -1 and COACT_EFLAG_ID_RANGE.
+ */
+int coact_compose_map(const int32_t *a, int64_t n, const int32_t *b, int64_t nb, int32_t *out,
+                      int32_t *err_flag, coact_stream_t stream);
+
+/*
+ * plan_forward -- which hop-1 row feeds each hop-2 row.
+ *   fwd_src[d] = the node-level row of (t, node(r)) for the rank-level row d of token t on
+ *                rank r (d < D = rank_offsets[R]);  -1 for D <= d < row_capacity
+ * ids, expert_rank, rank_node, n_nodes: as given to the rank-level plan_dispatch;
+ * send_row / rank_offsets: that plan's outputs; node_send_row: the node-level plan's
+ * send_row (int32 [N,k]) for the same ids.  fwd_src: int32 [row_capacity].  Row indices
+ * at or beyond row_capacity set COACT_EFLAG_ROW_RANGE; invalid tokens are skipped.
+ */
+int plan_forward(const int32_t *ids, int64_t N, int k, int E, const int32_t *expert_rank, int R,
+                 const int32_t *rank_node, int n_nodes, const int32_t *send_row,
+                 const int32_t *rank_offsets, const int32_t *node_send_row, int32_t *fwd_src,
+                 int64_t row_capacity, int32_t *err_flag, coact_stream_t stream);
+
+/*
+ * forward_gather -- the intra-node forward of hop 2:  dst[d] = src[fwd_src[d]] for every
+ * d < n_rows with fwd_src[d] >= 0 (bf16 rows of H; other rows untouched).  src: the
+ * hop-1 send buffer [n_src_rows, H]; dst: the rank-level send buffer [n_rows, H].  An
+ * fwd_src entry at or beyond n_src_rows sets COACT_EFLAG_ROW_RANGE and is skipped.
+ * Composition: forward_gather(dispatch_gather(x, node plan), plan_forward(...)) equals
+ * dispatch_gather(x, rank plan) row for row.
+ */
+int forward_gather(const uint16_t *src, int64_t n_src_rows, int64_t H, const int32_t *fwd_src,
+                   int64_t n_rows, uint16_t *dst, int32_t *err_flag, coact_stream_t stream);
+
 /* Bytes of device workspace predict_home needs (E1*R int64 scores). */
 size_t predict_home_workspace_bytes(int E1, int R);
 

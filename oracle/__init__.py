@@ -65,6 +65,10 @@ def _get():
             _lib.oracle_naive_combine_identity_f32.restype = None
             _lib.oracle_predict_home.argtypes = [P, I64, I32, I32, P, I32, P, I32, P]
             _lib.oracle_place_correlated.argtypes = [P, I32, I32, P]
+            _lib.oracle_forward_src.argtypes = [P, P, I32, P, P, P, I32, I64, I64, P]
+            _lib.oracle_forward_src.restype = None
+            _lib.oracle_forward_gather.argtypes = [P, I64, P, I64, P]
+            _lib.oracle_forward_gather.restype = None
         return _lib
 
 
@@ -236,3 +240,52 @@ def place_correlated(pair, R: int) -> np.ndarray:
     if _get().oracle_place_correlated(_p(pr), E, R, _p(out)) != 0:
         raise ValueError("E must be a multiple of R")
     return out
+
+
+def node_maps(expert_rank, rank_node, src_rank=None, N=None, R=None):
+    """expert -> node and token -> home node maps for the node-level (hop-1) plan."""
+    er = np.asarray(expert_rank, np.int64)
+    rn = np.asarray(rank_node, np.int64)
+    expert_node = rn[er].astype(np.int32)
+    if src_rank is None:
+        src_rank = (np.arange(N, dtype=np.int64) * R) // N
+    src_node = rn[np.asarray(src_rank, np.int64)].astype(np.int32)
+    return expert_node, src_node
+
+
+def plan_two_hop(ids, E: int, expert_rank, R: int, rank_node, n_nodes: int, src_rank=None):
+    """(node-level plan, rank-level plan, fwd_src): hop 1 sends each token once per node,
+    hop 2 forwards each node-level row to the token's ranks in that node."""
+    ids = _c(ids, np.int32)
+    N = ids.shape[0]
+    en, sn = node_maps(expert_rank, rank_node, src_rank, N, R)
+    node = plan(ids, E, en, n_nodes, rank_node=np.arange(n_nodes, dtype=np.int32),
+                n_nodes=n_nodes, src_rank=sn)
+    rank = plan(ids, E, expert_rank, R, rank_node=rank_node, n_nodes=n_nodes, src_rank=src_rank)
+    fwd = forward_src(rank, rank_node, node, n_nodes)
+    return node, rank, fwd
+
+
+def forward_src(rank_plan: dict, rank_node, node_plan: dict, n_nodes: int) -> np.ndarray:
+    rt = _c(rank_plan["row_token"], np.int32)
+    ro = _c(rank_plan["rank_offsets"], np.int32)
+    R = ro.shape[0] - 1
+    rn = _c(rank_node, np.int32)
+    nrt = _c(node_plan["row_token"], np.int32)
+    no = _c(node_plan["rank_offsets"], np.int32)
+    N = rank_plan["send_row"].shape[0]
+    cap = rt.shape[0]
+    out = np.zeros(cap, np.int32)
+    _get().oracle_forward_src(_p(rt), _p(ro), R, _p(rn), _p(nrt), _p(no), n_nodes, N, cap, _p(out))
+    return out
+
+
+def forward_gather(src, fwd_src, cap=None) -> np.ndarray:
+    """dst[d] = src[fwd_src[d]] where fwd_src[d] >= 0 (zeros elsewhere)."""
+    sb = _bits(src)
+    H = sb.shape[1]
+    f = _c(fwd_src, np.int32)
+    cap = f.shape[0] if cap is None else cap
+    dst = np.zeros((cap, H), np.uint16)
+    _get().oracle_forward_gather(_p(sb), H, _p(f), cap, _p(dst))
+    return dst

@@ -454,3 +454,42 @@ int oracle_place_correlated(const int64_t *pair, int E, int R, int32_t *expert_r
     free(free_slots);
     return 0;
 }
+
+/*
+ * Two-hop dispatch (node level, then rank level).  [Cobalt] routes tokens "to fewer
+ * remote nodes": a token crosses to each destination node once (hop 1) and is then
+ * forwarded inside the node to each destination rank (hop 2).  The hop-1 plan is the
+ * ordinary plan with nodes in place of ranks (expert -> node map, home node).  For each
+ * rank-level send row d of token t on rank r, the hop-1 row that feeds it is the node-level
+ * row of (t, node(r)):
+ *   fwd_src[d] = the e with node_row_token[e] == t inside node(r)'s segment,  d < D
+ *   fwd_src[d] = -1                                                           D <= d < cap
+ * Definition by lookup: every node-level row e of node n in [node_offsets[n],
+ * node_offsets[n+1]) is indexed by (node_row_token[e], n).
+ */
+void oracle_forward_src(const int32_t *row_token, const int32_t *rank_offsets, int R,
+                        const int32_t *rank_node, const int32_t *node_row_token,
+                        const int32_t *node_offsets, int n_nodes, int64_t N, int64_t cap,
+                        int32_t *fwd_src) {
+    /* index[(t, n)] = node-level row, as a dense N x n_nodes table */
+    int32_t *index = (int32_t *)malloc(sizeof(int32_t) * (size_t)(N > 0 ? N : 1) * (size_t)n_nodes);
+    for (int64_t i = 0; i < N * n_nodes; ++i) index[i] = -1;
+    for (int n = 0; n < n_nodes; ++n)
+        for (int64_t e = node_offsets[n]; e < node_offsets[n + 1]; ++e)
+            index[(int64_t)node_row_token[e] * n_nodes + n] = (int32_t)e;
+    for (int64_t d = 0; d < cap; ++d) fwd_src[d] = -1;
+    for (int r = 0; r < R; ++r) {
+        int n = rank_node ? rank_node[r] : 0;
+        for (int64_t d = rank_offsets[r]; d < rank_offsets[r + 1] && d < cap; ++d)
+            fwd_src[d] = index[(int64_t)row_token[d] * n_nodes + n];
+    }
+    free(index);
+}
+
+/* Row gather: dst[d] = src[fwd_src[d]] for every d with fwd_src[d] >= 0 (bf16 bits). */
+void oracle_forward_gather(const uint16_t *src, int64_t H, const int32_t *fwd_src, int64_t cap,
+                           uint16_t *dst) {
+    for (int64_t d = 0; d < cap; ++d)
+        if (fwd_src[d] >= 0)
+            memcpy(dst + d * H, src + (int64_t)fwd_src[d] * H, (size_t)H * sizeof(uint16_t));
+}

@@ -431,3 +431,63 @@ def test_correlated_placement_chain_config3(coact):
     assert_plan_equal(plan_to_host(plan), o)
     rr = oracle_plan_for(r)
     assert o["D"] < rr["D"] and o["stats"][4] < rr["stats"][4]   # fewer rows, fewer remote nodes
+
+
+# ----------------------------------------------------------------------------- two-hop dispatch
+
+
+@pytest.mark.parametrize("cfg,N", [(2, None), (3, None), (2, 5000)])
+def test_two_hop_dispatch(coact, cfg, N):
+    """Hop 1 to nodes, hop 2 inside the node (Cobalt: fewer remote nodes): both plans and
+    the forward map against the oracle, and the two-hop rows against the one-hop rows."""
+    r = workload.make_routing(cfg, N=N)
+    c = r.cfg
+    src = None if N is None else np.random.default_rng(3).integers(0, c.R, r.N).astype(np.int32)
+    th = coact.alloc_two_hop(r.N, r.k, c.E, c.R, c.n_nodes, DEV)
+    err = zero_flag()
+    coact.plan_two_hop(cuda(r.ids), c.E, cuda(r.expert_rank, np.int32), c.R,
+                       cuda(r.rank_node, np.int32), c.n_nodes, th,
+                       src_rank=None if src is None else cuda(src), err_flag=err)
+    torch.cuda.synchronize()
+    node_o, rank_o, fwd_o = oracle.plan_two_hop(r.ids, c.E, r.expert_rank, c.R, r.rank_node,
+                                                c.n_nodes, src_rank=src)
+    assert err.item() == 0
+    assert_plan_equal(plan_to_host(th.node), node_o, sentinel=False)
+    assert_plan_equal(plan_to_host(th.rank), rank_o, sentinel=False)
+    assert np.array_equal(th.fwd_src.cpu().numpy(), fwd_o)
+    assert node_o["stats"][2] == rank_o["stats"][4]
+    # rows: x -> hop 1 (node segments) -> hop 2 (rank segments) == x -> rank segments
+    H = c.H if N is None else 520
+    x = workload.fill_bf16(r.N, H, r.seed, X_STREAM, device=DEV)
+    hop1 = torch.empty((th.node.row_capacity, H), dtype=torch.bfloat16, device=DEV)
+    coact.dispatch_gather(x, th.node.send_row, hop1, err_flag=err)
+    hop2 = torch.empty((th.rank.row_capacity, H), dtype=torch.bfloat16, device=DEV)
+    hop2.view(torch.int16).fill_(-1)
+    coact.forward_gather(hop1, th.fwd_src, hop2, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    D, cap = rank_o["D"], th.rank.row_capacity
+    rng = np.random.default_rng(cfg)
+    rows = np.unique(np.concatenate([rng.integers(0, D, 1200), [0, D - 1]]))
+    want = host_bits(workload.fill_bf16(len(rows), H, r.seed, X_STREAM,
+                                        row_ids=rank_o["row_token"][rows]))
+    assert np.array_equal(host_bits(hop2[torch.as_tensor(rows, device=DEV)]), want)
+    if D < cap:
+        tail = np.unique(rng.integers(D, cap, 64))
+        assert (host_bits(hop2[torch.as_tensor(tail, device=DEV)]) == 0xFFFF).all()
+
+
+def test_forward_gather_flags_and_compose_map(coact):
+    src = workload.fill_bf16(10, 16, 0, 5, device=DEV)
+    fwd = torch.tensor([3, -1, 9, 10, 0], dtype=torch.int32, device=DEV)   # 10 is out of range
+    dst = torch.zeros((5, 16), dtype=torch.bfloat16, device=DEV)
+    err = zero_flag()
+    coact.forward_gather(src, fwd, dst, err_flag=err)
+    assert err.item() == coact.EFLAG_ROW_RANGE
+    assert torch.equal(dst[0], src[3]) and torch.equal(dst[2], src[9]) and torch.equal(dst[4], src[0])
+    assert (dst[1] == 0).all() and (dst[3] == 0).all()
+    a = torch.tensor([2, 0, 5, 1], dtype=torch.int32, device=DEV)
+    b = torch.tensor([10, 11, 12], dtype=torch.int32, device=DEV)
+    err.zero_()
+    out = coact.coact_compose_map(a, b, err_flag=err)
+    assert out.cpu().tolist() == [12, 10, -1, 11] and err.item() == coact.EFLAG_ID_RANGE
