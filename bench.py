@@ -469,17 +469,28 @@ def make_step(coact, cfg_index: int, seed: int, device, two_hop: bool = False):
     return S, placement
 
 
-def read_traffic(kernel: str, workload_name: str):
-    """DRAM bytes per launch from a committed ncu summary, if its source hash matches."""
+# CUDA sources of each HBM-bound kernel: a committed DRAM-traffic figure is reported only
+# while these files are byte-identical to the ones the ncu capture was taken on.
+KERNEL_SOURCES = {"k_gather_v16": ("gather.cu", "common.cuh"),
+                  "k_combine_v16": ("combine.cu", "common.cuh"),
+                  "k_forward_gather": ("twohop.cu", "common.cuh")}
+
+
+def kernel_source_hash(kernel: str) -> str:
     import hashlib
-    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
-    if not os.path.exists(path):
-        return None
     h = hashlib.sha256()
-    for fn in sorted(os.listdir(os.path.join(ROOT, "co_activation_b200", "csrc"))):
+    for fn in KERNEL_SOURCES.get(kernel, ()):
         with open(os.path.join(ROOT, "co_activation_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
-    sha = h.hexdigest()[:16]
+    return h.hexdigest()[:16]
+
+
+def read_traffic(kernel: str, workload_name: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel's sources match."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path) or kernel not in KERNEL_SOURCES:
+        return None
+    sha = kernel_source_hash(kernel)
     for line in open(path):
         p = line.split()
         if len(p) >= 4 and not line.startswith("#") and p[0] == kernel and p[1] == workload_name:
