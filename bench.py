@@ -435,38 +435,57 @@ class TwoHopStep(OneLayerStep):
                 "err_flag": int(self.L.err.item())}
 
 
-def make_step(coact, cfg_index: int, seed: int, device, two_hop: bool = False):
+def layout(coact, r: workload.Routing, kind: str, device):
+    """Expert -> rank placement from the batch's own counts (library calls):
+    'correlated' = rank-level co-location (Zyphra), 'two-stage' = node-level co-location
+    then intra-node load rebalancing (Cobalt).  Returns (expert_rank numpy, description)."""
+    c = r.cfg
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    pair = torch.zeros((c.E, c.E), dtype=torch.int64, device=device)
+    loads = torch.zeros(c.E, dtype=torch.int64, device=device)
+    coact.coact_count(to(r.ids), c.E, pair, loads)
+    if kind == "correlated":
+        return coact.coact_place_correlated(pair, c.R).numpy(), \
+            "correlated (coact_place_correlated over this batch's pair counts)"
+    if kind == "two-stage":
+        return coact.coact_place_two_stage(pair, loads, torch.from_numpy(r.rank_node),
+                                           c.n_nodes).numpy(), \
+            "two-stage (node co-location + intra-node load rebalancing over this batch)"
+    raise SystemExit(f"unknown placement {kind}")
+
+
+def make_step(coact, cfg_index: int, seed: int, device, two_hop: bool = False,
+              placement_kind: str = "auto"):
     """The step object for a configuration, plus a description of its placement."""
     cfg = workload.CONFIGS[cfg_index]
-    if two_hop:
-        if cfg.two_layer or cfg.n_nodes < 2:
-            raise SystemExit("--two-hop needs a one-layer configuration with several nodes (2, 3)")
-        r = workload.make_routing(cfg, seed=seed)
-        if cfg_index == 3:   # the same correlated placement as the one-hop step
-            tmp = OneLayerStep(coact, r, device, fill=False)
-            tmp.L.count()
-            r.expert_rank = coact.coact_place_correlated(tmp.L.pair, cfg.R).numpy()
-            del tmp
-        return TwoHopStep(coact, r, device), (cfg.placement if cfg_index != 3 else
-                                              "correlated (coact_place_correlated)")
     if cfg.two_layer:
+        if two_hop:
+            raise SystemExit("--two-hop needs a one-layer configuration with several nodes (2, 3)")
         return TwoLayerStep(coact, workload.make_two_layer(cfg, seed=seed), device), \
             "contiguous; layer 2 pre-sharded to the predicted home rank"
     r = workload.make_routing(cfg, seed=seed)
-    S = OneLayerStep(coact, r, device)
-    placement = cfg.placement
-    if cfg_index == 3:
-        # co-activation-grouped placement: the library's greedy over this batch's counts
-        S.L.count()
-        placed = coact.coact_place_correlated(S.L.pair, cfg.R)
-        S.L.plan_()
-        S.rr_dedup = S.L.D() / (cfg.N * cfg.k)
-        S.L.expert_rank.copy_(placed.to(device))
-        S.L.r.expert_rank = placed.numpy()
-        S.L.pair.zero_()
-        S.L.loads.zero_()
-        placement = "correlated (coact_place_correlated over this batch's pair counts)"
-    return S, placement
+    kind = placement_kind if placement_kind != "auto" else (
+        "correlated" if cfg_index == 3 else "default")
+    desc = cfg.placement
+    rr_D = None
+    if kind != "default":
+        # dedup ratio under the configuration's own placement, for comparison
+        to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        base = coact.alloc_plan(cfg.N, cfg.k, cfg.E, cfg.R, device)
+        coact.plan_dispatch(to(r.ids), cfg.E, to(r.expert_rank.astype(np.int32)), cfg.R, base,
+                            rank_node=to(r.rank_node), n_nodes=cfg.n_nodes)
+        rr_D = int(base.rank_offsets[-1].item()) / (cfg.N * cfg.k)
+        del base
+        r.expert_rank, desc = layout(coact, r, kind, device)
+    if two_hop:
+        if cfg.n_nodes < 2:
+            raise SystemExit("--two-hop needs a one-layer configuration with several nodes (2, 3)")
+        S = TwoHopStep(coact, r, device)
+    else:
+        S = OneLayerStep(coact, r, device)
+    if rr_D is not None:
+        S.rr_dedup = rr_D
+    return S, desc
 
 
 # CUDA sources of each HBM-bound kernel: a committed DRAM-traffic figure is reported only
@@ -513,7 +532,8 @@ def run_gpu(args):
     import co_activation_b200 as coact
 
     cfg = workload.CONFIGS[args.config]
-    S, placement = make_step(coact, args.config, rank_seed(args.seed, rank), device, args.two_hop)
+    S, placement = make_step(coact, args.config, rank_seed(args.seed, rank), device, args.two_hop,
+                             args.placement)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     flush_w = torch.empty(max(2 * l2, 64 << 20), dtype=torch.uint8, device=device)
     flush_r = torch.zeros(max(2 * l2, 64 << 20) // 8, dtype=torch.int64, device=device)
@@ -651,7 +671,7 @@ def run_gpu(args):
         "e2e": e2e,
     }
     if hasattr(S, "rr_dedup"):
-        result["dedup_rows_over_naive_roundrobin"] = S.rr_dedup
+        result["dedup_rows_over_naive_config_placement"] = S.rr_dedup
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(S, args.cpu_seconds)
     if world > 1:
@@ -834,6 +854,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--clock-warm-s", type=float, default=1.0)
     ap.add_argument("--ref-tokens", type=int, default=4096)
+    ap.add_argument("--placement", default="auto", choices=["auto", "default", "correlated",
+                                                             "two-stage"],
+                    help="auto: the configuration's own (config 3: correlated)")
     ap.add_argument("--two-hop", action="store_true",
                     help="dispatch in two hops: to nodes, then inside the node to ranks")
     args = ap.parse_args()

@@ -52,6 +52,7 @@ _lib.predict_home_workspace_bytes.argtypes = [_I32, _I32]
 _lib.predict_home_workspace_bytes.restype = _SZ
 _lib.predict_home.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _SZ, _P, _P]
 _lib.coact_place_correlated.argtypes = [_P, _I32, _I32, _P]
+_lib.coact_rebalance_ranks.argtypes = [_P, _P, _I32, _P, _I32, _P]
 _lib.coact_compose_map.argtypes = [_P, _I64, _P, _I64, _P, _P, _P]
 _lib.plan_forward.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _P, _P, _I64, _P, _P]
 _lib.forward_gather.argtypes = [_P, _I64, _I64, _P, _I64, _P, _P, _P]
@@ -59,13 +60,14 @@ _lib.plan_dispatch_noalloc.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32,
                                        _P, _P, _P, _I64, _P, _P, _P, _P, _P, _P]
 for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "combine_scatter", "predict_home",
            "coact_place_correlated", "plan_dispatch_noalloc", "coact_compose_map", "plan_forward",
-           "forward_gather"):
+           "forward_gather", "coact_rebalance_ranks"):
     getattr(_lib, _f).restype = _I32
 
 ABI_SYMBOLS = ("coact_strerror", "coact_abi_version", "coact_count", "plan_dispatch_workspace_bytes",
                "plan_dispatch", "dispatch_gather", "combine_scatter",
                "predict_home_workspace_bytes", "predict_home", "coact_place_correlated",
-               "plan_dispatch_noalloc", "coact_compose_map", "plan_forward", "forward_gather")
+               "plan_dispatch_noalloc", "coact_compose_map", "plan_forward", "forward_gather",
+               "coact_rebalance_ranks")
 NOALLOC_MAX_TOKENS = 262144
 
 
@@ -432,3 +434,24 @@ def plan_two_hop(ids: torch.Tensor, E: int, expert_rank: torch.Tensor, R: int,
     plan_forward(ids, E, expert_rank, R, th.rank, th.node, th.fwd_src, rank_node=rank_node,
                  n_nodes=n_nodes, err_flag=err_flag, stream=stream)
     return th
+
+
+def coact_rebalance_ranks(loads, expert_node, rank_node):
+    """Cobalt's intra-node rebalancing (host computation in the library): each node's
+    experts, heaviest first, to the least-loaded rank of that node with a free slot.
+    Returns an int32 CPU tensor expert -> rank."""
+    ld = loads.detach().to("cpu", torch.int64).contiguous()
+    en = expert_node.detach().to("cpu", torch.int32).contiguous()
+    rn = rank_node.detach().to("cpu", torch.int32).contiguous()
+    out = torch.empty(ld.shape[0], dtype=torch.int32)
+    _check(_lib.coact_rebalance_ranks(_ptr(ld), _ptr(en), ld.shape[0], _ptr(rn), rn.shape[0],
+                                      _ptr(out)), "coact_rebalance_ranks")
+    return out
+
+
+def coact_place_two_stage(pair, loads, rank_node, n_nodes: int):
+    """Cobalt's two-stage layout: co-activated experts co-located per node
+    (coact_place_correlated at node granularity), then per-rank loads balanced inside
+    each node (coact_rebalance_ranks).  Returns expert -> rank (int32 CPU tensor)."""
+    expert_node = coact_place_correlated(pair, n_nodes)
+    return coact_rebalance_ranks(loads, expert_node, rank_node)

@@ -72,3 +72,49 @@ extern "C" int coact_place_correlated(const int64_t *pair, int E, int R, int32_t
     for (int e = 0; e < E; ++e) expert_rank[e] = rank_of[e];
     return COACT_OK;
 }
+
+// coact_rebalance_ranks: Cobalt's second planner stage.
+//
+// Cobalt (arxivdaily 2609.36959), English abstract: the planner periodically co-locates
+// frequently co-activated experts on the same node, then "performs per-step intra-node
+// adjustment to rebalance the workloads".  The pages give no algorithm; this is the plain
+// longest-first greedy: within each node, its experts by load descending (ties: lower id)
+// each go to the node's rank with the least load so far that still has a free slot (ties:
+// lower rank).  Every rank ends with E/R experts; no expert changes node.
+extern "C" int coact_rebalance_ranks(const int64_t *loads, const int32_t *expert_node, int E,
+                                     const int32_t *rank_node, int R, int32_t *expert_rank) {
+    if (!loads || !expert_node || !rank_node || !expert_rank) return COACT_ERR_INVALID;
+    if (E < 2 || E > COACT_MAX_E || R < 1 || R > COACT_MAX_R || E % R != 0)
+        return COACT_ERR_UNSUPPORTED;
+    const int slots = E / R;
+    int n_nodes = 0;
+    for (int r = 0; r < R; ++r) {
+        if (rank_node[r] < 0 || rank_node[r] >= 64) return COACT_ERR_INVALID;
+        n_nodes = std::max(n_nodes, rank_node[r] + 1);
+    }
+    std::vector<int> node_cap(n_nodes, 0), node_size(n_nodes, 0);
+    for (int r = 0; r < R; ++r) node_cap[rank_node[r]] += slots;
+    for (int e = 0; e < E; ++e) {
+        if (expert_node[e] < 0 || expert_node[e] >= n_nodes) return COACT_ERR_INVALID;
+        node_size[expert_node[e]] += 1;
+    }
+    for (int n = 0; n < n_nodes; ++n)
+        if (node_size[n] != node_cap[n]) return COACT_ERR_INVALID;   // the node layout must fit
+    std::vector<int> order(E);
+    for (int e = 0; e < E; ++e) order[e] = e;
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int a, int b) { return loads[a] > loads[b]; });
+    std::vector<int64_t> rank_load(R, 0);
+    std::vector<int> free_slots(R, slots);
+    for (int e : order) {
+        int best = -1;
+        for (int r = 0; r < R; ++r) {
+            if (rank_node[r] != expert_node[e] || free_slots[r] == 0) continue;
+            if (best < 0 || rank_load[r] < rank_load[best]) best = r;
+        }
+        expert_rank[e] = best;
+        rank_load[best] += loads[e];
+        free_slots[best] -= 1;
+    }
+    return COACT_OK;
+}

@@ -302,6 +302,21 @@ int predict_home(const int32_t *ids1, int64_t N, int k1, int E1,
  */
 int coact_place_correlated(const int64_t *pair, int E, int R, int32_t *expert_rank);
 
+/*
+ * coact_rebalance_ranks -- intra-node load rebalancing (HOST function).
+ * Cobalt, English abstract: a two-stage layout planner co-locates frequently co-activated
+ * experts on the same node (stage 1: coact_place_correlated with R = n_nodes gives expert ->
+ * node) and adjusts the layout inside each node to rebalance workloads (stage 2: this
+ * call).  The pages give no algorithm; this is the longest-first greedy: experts by load
+ * descending (ties: lower id), each to the least-loaded rank of its node with a free slot
+ * (ties: lower rank).  loads: HOST int64 [E] (coact_count's per-expert loads);
+ * expert_node: HOST int32 [E]; rank_node: HOST int32 [R]; expert_rank: HOST int32 [E]
+ * output.  Requires E % R == 0 and every node to hold exactly (its ranks) x E/R experts
+ * (COACT_ERR_INVALID otherwise).  Synchronous; no CUDA call.
+ */
+int coact_rebalance_ranks(const int64_t *loads, const int32_t *expert_node, int E,
+                          const int32_t *rank_node, int R, int32_t *expert_rank);
+
 #ifdef __cplusplus
 }
 #endif

@@ -65,6 +65,7 @@ def _get():
             _lib.oracle_naive_combine_identity_f32.restype = None
             _lib.oracle_predict_home.argtypes = [P, I64, I32, I32, P, I32, P, I32, P]
             _lib.oracle_place_correlated.argtypes = [P, I32, I32, P]
+            _lib.oracle_rebalance_ranks.argtypes = [P, P, I32, P, I32, P]
             _lib.oracle_forward_src.argtypes = [P, P, I32, P, P, P, I32, I64, I64, P]
             _lib.oracle_forward_src.restype = None
             _lib.oracle_forward_gather.argtypes = [P, I64, P, I64, P]
@@ -289,3 +290,21 @@ def forward_gather(src, fwd_src, cap=None) -> np.ndarray:
     dst = np.zeros((cap, H), np.uint16)
     _get().oracle_forward_gather(_p(sb), H, _p(f), cap, _p(dst))
     return dst
+
+
+def rebalance_ranks(loads, expert_node, rank_node) -> np.ndarray:
+    """Longest-first intra-node rebalancing (expert -> rank, int32 [E])."""
+    ld = _c(loads, np.int64)
+    en = _c(expert_node, np.int32)
+    rn = _c(rank_node, np.int32)
+    E, R = ld.shape[0], rn.shape[0]
+    out = np.zeros(E, np.int32)
+    if _get().oracle_rebalance_ranks(_p(ld), _p(en), E, _p(rn), R, _p(out)) != 0:
+        raise ValueError("a node's expert count does not match its slots")
+    return out
+
+
+def place_two_stage(pair, loads, rank_node, n_nodes: int) -> np.ndarray:
+    """Stage 1: correlated placement at node granularity; stage 2: rebalance in nodes."""
+    expert_node = place_correlated(pair, n_nodes)
+    return rebalance_ranks(loads, expert_node, rank_node)

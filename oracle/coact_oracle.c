@@ -493,3 +493,41 @@ void oracle_forward_gather(const uint16_t *src, int64_t H, const int32_t *fwd_sr
         if (fwd_src[d] >= 0)
             memcpy(dst + d * H, src + (int64_t)fwd_src[d] * H, (size_t)H * sizeof(uint16_t));
 }
+
+/*
+ * Intra-node load rebalancing.  [Cobalt] "per-step intra-node adjustment to rebalance the
+ * workloads".  The pages give no algorithm; the reading is the longest-first greedy: take
+ * the experts in order of load, heaviest first (equal loads: smaller id first); put each
+ * on the least-loaded rank of its own node that has a free slot (equal loads: smaller
+ * rank).  E/R slots per rank.  Returns -1 if a node's expert count does not match its
+ * slots.
+ */
+int oracle_rebalance_ranks(const int64_t *loads, const int32_t *expert_node, int E,
+                           const int32_t *rank_node, int R, int32_t *expert_rank) {
+    int per_rank = E / R;
+    int64_t *rank_load = (int64_t *)calloc((size_t)R, sizeof(int64_t));
+    int *free_slots = (int *)malloc(sizeof(int) * (size_t)R);
+    char *done = (char *)calloc((size_t)E, 1);
+    for (int r = 0; r < R; ++r) free_slots[r] = per_rank;
+    int status = 0;
+    for (int step = 0; step < E; ++step) {
+        /* the heaviest expert not yet placed (smallest id among equals) */
+        int e = -1;
+        for (int c = 0; c < E; ++c)
+            if (!done[c] && (e < 0 || loads[c] > loads[e])) e = c;
+        done[e] = 1;
+        int best = -1;
+        for (int r = 0; r < R; ++r)
+            if (rank_node[r] == expert_node[e] && free_slots[r] > 0 &&
+                (best < 0 || rank_load[r] < rank_load[best]))
+                best = r;
+        if (best < 0) { status = -1; expert_rank[e] = -1; continue; }
+        expert_rank[e] = best;
+        rank_load[best] += loads[e];
+        free_slots[best] -= 1;
+    }
+    free(rank_load);
+    free(free_slots);
+    free(done);
+    return status;
+}

@@ -80,3 +80,66 @@ def test_library_rejects_bad_sizes():
     import torch
     with pytest.raises(coact.CoactError):
         coact.coact_place_correlated(torch.zeros((6, 6), dtype=torch.int64), 4)   # 6 % 4 != 0
+
+
+# ----------------------------------------------------------------------------- two-stage planner
+
+
+def test_rebalance_hand_worked():
+    # one node, two ranks of two slots; heaviest first: e0 (10) -> r0, e2 (7) -> r1,
+    # e3 (5) -> r1 (7 < 10), r1 full, e1 (1) -> r0: loads 11 / 12
+    got = oracle.rebalance_ranks([10, 1, 7, 5], [0, 0, 0, 0], [0, 0])
+    assert got.tolist() == [0, 0, 1, 1]
+
+
+def test_rebalance_two_nodes_stays_in_node():
+    loads = [5, 9, 2, 2, 8, 1, 3, 7]
+    expert_node = [0, 1, 0, 1, 0, 1, 0, 1]
+    # node 0 (ranks 0, 1): e4 (8) r0, e0 (5) r1, e6 (3) r1, e2 (2) r0
+    # node 1 (ranks 2, 3): e1 (9) r2, e7 (7) r3, e3 (2) r3, e5 (1) r2
+    got = oracle.rebalance_ranks(loads, expert_node, [0, 0, 1, 1])
+    assert got.tolist() == [1, 2, 0, 3, 0, 2, 1, 3]
+
+
+def test_rebalance_rejects_mismatched_node_sizes():
+    with pytest.raises(ValueError):
+        oracle.rebalance_ranks([1, 2, 3, 4], [0, 0, 0, 1], [0, 1])
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_rebalance_library_matches_oracle(seed):
+    import co_activation_b200 as coact
+    import torch
+    rng = np.random.default_rng(300 + seed)
+    n_nodes = int(rng.choice([1, 2, 4]))
+    R = n_nodes * int(rng.integers(1, 5))
+    E = R * int(rng.integers(1, 5))
+    loads = rng.integers(0, 6, E).astype(np.int64)          # many equal loads
+    rank_node = (np.arange(R) // (R // n_nodes)).astype(np.int32)
+    expert_node = rng.permutation(np.repeat(np.arange(n_nodes), E // n_nodes)).astype(np.int32)
+    want = oracle.rebalance_ranks(loads, expert_node, rank_node)
+    got = coact.coact_rebalance_ranks(torch.from_numpy(loads), torch.from_numpy(expert_node),
+                                      torch.from_numpy(rank_node)).numpy()
+    assert np.array_equal(got, want)
+    assert np.bincount(got, minlength=R).tolist() == [E // R] * R
+    assert (rank_node[got] == expert_node).all()
+
+
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_two_stage_layout_on_configs(cfg):
+    """Stage 1 cuts cross-node traffic, stage 2 keeps it and evens the rank loads."""
+    import co_activation_b200 as coact
+    import torch
+    r = workload.make_routing(cfg)
+    c = r.cfg
+    pair, loads, _ = oracle.count(r.ids, c.E)
+    two = oracle.place_two_stage(pair, loads, r.rank_node, c.n_nodes)
+    got = coact.coact_place_two_stage(torch.from_numpy(pair), torch.from_numpy(loads),
+                                      torch.from_numpy(r.rank_node), c.n_nodes).numpy()
+    assert np.array_equal(got, two)
+    base = oracle.plan(r.ids, c.E, r.expert_rank, c.R, r.rank_node, c.n_nodes)
+    p2 = oracle.plan(r.ids, c.E, two, c.R, r.rank_node, c.n_nodes)
+    assert p2["stats"][4] < base["stats"][4]            # fewer (token, remote node) pairs
+    rank_load = lambda er: np.bincount(er[r.ids.ravel()], minlength=c.R)
+    corr = oracle.place_correlated(pair, c.R)
+    assert rank_load(two).max() < rank_load(corr).max()  # better balanced than rank-level co-location
