@@ -129,3 +129,33 @@ def test_binding_fails_loudly_without_library():
     r = subprocess.run([sys.executable, "-c", "import co_activation_b200"], cwd=ROOT, env=env,
                        capture_output=True, text=True)
     assert r.returncode != 0 and "libcoact.so not found" in r.stderr
+
+
+def test_two_hop_and_planner_reject_bad_arguments(lib):
+    c = lib.coact_compose_map
+    c.argtypes = [P, ctypes.c_int64, P, ctypes.c_int64, P, P, P]
+    assert c(FAKE, -1, FAKE, 4, FAKE, None, None) == -1
+    assert c(None, 5, FAKE, 4, FAKE, None, None) == -1
+    assert c(None, 0, None, 0, None, None, None) == 0
+    f = lib.plan_forward
+    f.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int,
+                  P, P, P, P, ctypes.c_int64, P, P]
+    assert f(FAKE, 10, 9, 8, FAKE, 4, None, 1, FAKE, FAKE, FAKE, FAKE, 20, None, None) == -2  # k
+    assert f(FAKE, 10, 2, 8, FAKE, 65, None, 1, FAKE, FAKE, FAKE, FAKE, 20, None, None) == -2  # R
+    assert f(FAKE, 10, 2, 8, FAKE, 4, None, 1, None, FAKE, FAKE, FAKE, 20, None, None) == -1   # send_row
+    assert f(FAKE, 10, 2, 8, FAKE, 4, None, 1, FAKE, FAKE, FAKE, None, 20, None, None) == -1   # fwd_src
+    g = lib.forward_gather
+    g.argtypes = [P, ctypes.c_int64, ctypes.c_int64, P, ctypes.c_int64, P, P, P]
+    assert g(FAKE, 10, 12, FAKE, 5, FAKE, None, None) == -2      # H % 8
+    assert g(P(264), 10, 16, FAKE, 5, FAKE, None, None) == -1    # misaligned src
+    assert g(FAKE, 10, 16, None, 5, FAKE, None, None) == -1      # fwd_src NULL
+    r = lib.coact_rebalance_ranks
+    r.argtypes = [P, P, ctypes.c_int, P, ctypes.c_int, P]
+    loads = (ctypes.c_int64 * 4)(4, 3, 2, 1)
+    en = (ctypes.c_int32 * 4)(0, 0, 1, 1)
+    rn = (ctypes.c_int32 * 2)(0, 1)
+    out = (ctypes.c_int32 * 4)()
+    assert r(loads, en, 4, rn, 2, out) == 0 and list(out) == [0, 0, 1, 1]
+    bad = (ctypes.c_int32 * 4)(0, 0, 0, 1)                        # node 0 holds 3 of 2 slots
+    assert r(loads, bad, 4, rn, 2, out) == -1
+    assert r(loads, en, 4, rn, 3, out) == -2                      # 4 % 3 != 0
