@@ -53,6 +53,9 @@ _lib.predict_home_workspace_bytes.restype = _SZ
 _lib.predict_home.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _SZ, _P, _P]
 _lib.coact_place_correlated.argtypes = [_P, _I32, _I32, _P]
 _lib.coact_rebalance_ranks.argtypes = [_P, _P, _I32, _P, _I32, _P]
+_lib.dispatch_gather_peer.argtypes = [_P, _I64, _I64, _P, _I32, _P, _I32, _P, _P, _P, _P, _P]
+_lib.combine_scatter_peer.argtypes = [_P, _P, _P, _P, _I32, _P, _P, _I64, _I32, _I64, _P, _I32,
+                                      _P, _P]
 _lib.coact_compose_map.argtypes = [_P, _I64, _P, _I64, _P, _P, _P]
 _lib.plan_forward.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _P, _P, _I64, _P, _P]
 _lib.forward_gather.argtypes = [_P, _I64, _I64, _P, _I64, _P, _P, _P]
@@ -60,14 +63,15 @@ _lib.plan_dispatch_noalloc.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32,
                                        _P, _P, _P, _I64, _P, _P, _P, _P, _P, _P]
 for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "combine_scatter", "predict_home",
            "coact_place_correlated", "plan_dispatch_noalloc", "coact_compose_map", "plan_forward",
-           "forward_gather", "coact_rebalance_ranks"):
+           "forward_gather", "coact_rebalance_ranks", "dispatch_gather_peer",
+           "combine_scatter_peer"):
     getattr(_lib, _f).restype = _I32
 
 ABI_SYMBOLS = ("coact_strerror", "coact_abi_version", "coact_count", "plan_dispatch_workspace_bytes",
                "plan_dispatch", "dispatch_gather", "combine_scatter",
                "predict_home_workspace_bytes", "predict_home", "coact_place_correlated",
                "plan_dispatch_noalloc", "coact_compose_map", "plan_forward", "forward_gather",
-               "coact_rebalance_ranks")
+               "coact_rebalance_ranks", "dispatch_gather_peer", "combine_scatter_peer")
 NOALLOC_MAX_TOKENS = 262144
 
 
@@ -455,3 +459,52 @@ def coact_place_two_stage(pair, loads, rank_node, n_nodes: int):
     each node (coact_rebalance_ranks).  Returns expert -> rank (int32 CPU tensor)."""
     expert_node = coact_place_correlated(pair, n_nodes)
     return coact_rebalance_ranks(loads, expert_node, rank_node)
+
+
+# ----------------------------------------------------------------------------- across GPUs
+
+
+def dispatch_gather_peer(x: torch.Tensor, send_row: torch.Tensor, rank_offsets: torch.Tensor,
+                         dst_bases: torch.Tensor, dst_row_offset: torch.Tensor,
+                         dst_capacity: torch.Tensor, err_flag: Optional[torch.Tensor] = None,
+                         stream=None) -> None:
+    """Rows of rank r's segment of this source's plan go straight into the destination
+    buffer dst_bases[r] (a device address, e.g. a peer GPU's symmetric buffer) at
+    dst_row_offset[r] + (row - rank_offsets[r])."""
+    N, H = x.shape
+    R = rank_offsets.shape[0] - 1
+    _need(_bits16(x), "x", torch.bfloat16)
+    _need(send_row, "send_row", torch.int32)
+    _need(rank_offsets, "rank_offsets", torch.int32)
+    _need(dst_bases, "dst_bases", torch.int64, (R,))
+    _need(dst_row_offset, "dst_row_offset", torch.int32, (R,))
+    _need(dst_capacity, "dst_capacity", torch.int32, (R,))
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.dispatch_gather_peer(_ptr(x), N, H, _ptr(send_row), send_row.shape[1],
+                                     _ptr(rank_offsets), R, _ptr(dst_bases), _ptr(dst_row_offset),
+                                     _ptr(dst_capacity), _ptr(err_flag), _stream(stream)),
+           "dispatch_gather_peer")
+
+
+def combine_scatter_peer(y_bases: torch.Tensor, y_row_offset: torch.Tensor,
+                         y_capacity: torch.Tensor, asg_offsets: torch.Tensor, gates: torch.Tensor,
+                         comb_row: torch.Tensor, out: torch.Tensor, H: int,
+                         err_flag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """combine_scatter with each expert output read from the rank that computed it."""
+    N, k = gates.shape
+    R = asg_offsets.shape[0] - 1
+    _need(y_bases, "y_bases", torch.int64, (R,))
+    _need(y_row_offset, "y_row_offset", torch.int32, (R,))
+    _need(y_capacity, "y_capacity", torch.int32, (R,))
+    _need(asg_offsets, "asg_offsets", torch.int32)
+    _need(gates, "gates", torch.float32)
+    _need(comb_row, "comb_row", torch.int32, (N, k))
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out must be bfloat16 or float32")
+    _need(out, "out", out.dtype, (N, H))
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.combine_scatter_peer(_ptr(y_bases), _ptr(y_row_offset), _ptr(y_capacity),
+                                     _ptr(asg_offsets), R, _ptr(gates), _ptr(comb_row), N, k, H,
+                                     _ptr(out), 1 if out.dtype == torch.float32 else 0,
+                                     _ptr(err_flag), _stream(stream)), "combine_scatter_peer")
+    return out

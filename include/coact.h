@@ -264,6 +264,43 @@ int plan_forward(const int32_t *ids, int64_t N, int k, int E, const int32_t *exp
 int forward_gather(const uint16_t *src, int64_t n_src_rows, int64_t H, const int32_t *fwd_src,
                    int64_t n_rows, uint16_t *dst, int32_t *err_flag, coact_stream_t stream);
 
+/*
+ * Expert parallelism across GPUs (one process per GPU; EP rank s plans its own tokens for
+ * all R destination ranks).  Cobalt / Zyphra, English abstracts: every MoE layer exchanges
+ * tokens all-to-all to the GPUs holding their experts and combines the results back.
+ * These two calls fuse that exchange into the data movement through per-rank buffer
+ * tables -- on a GPU system, the peers' NVLink-mapped buffers (e.g. symmetric memory);
+ * plain device pointers work the same way on one GPU.  With C[s][r] = rows and A[s][r] =
+ * assignments that source s sends to rank r (rank_counts / diff(asg_offsets) of s's
+ * plan), source s writes at row offsets off[r] = sum_{s'<s} C[s'][r] and reads back at
+ * sum_{s'<s} A[s'][r]; every destination buffer then holds exactly the rank-r segment the
+ * single-GPU plan of all sources' tokens would produce (sources contiguous in token
+ * order).  Ordering across GPUs (all writes done before the experts read, all expert
+ * outputs written before the combine reads) is the caller's barrier.
+ *
+ * dispatch_gather_peer -- for this source's plan (send_row [N,k], rank_offsets [R+1]):
+ *   row d of rank r's segment goes to dst_bases[r] + (dst_row_offset[r] + d - rank_offsets[r]) * H
+ * dst_bases: DEVICE array of R uint64 device addresses (bf16 [dst_capacity[r], H] each);
+ * dst_row_offset, dst_capacity: DEVICE int32 [R].  A row outside [0, dst_capacity[r]) or a
+ * NULL base sets COACT_EFLAG_ROW_RANGE and is skipped.  x: bf16 [N,H], 16-byte aligned.
+ */
+int dispatch_gather_peer(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row, int k,
+                         const int32_t *rank_offsets, int R, const uint64_t *dst_bases,
+                         const int32_t *dst_row_offset, const int32_t *dst_capacity,
+                         int32_t *err_flag, coact_stream_t stream);
+
+/*
+ * combine_scatter_peer -- combine_scatter reading the expert outputs from the ranks that
+ * computed them: assignment row a of rank r's segment (asg_offsets [R+1] of this source's
+ * plan) is read at y_bases[r] + (y_row_offset[r] + a - asg_offsets[r]) * H.  Same fp32
+ * fma chain, output types and flags as combine_scatter; y_bases / y_row_offset /
+ * y_capacity: DEVICE arrays as above.
+ */
+int combine_scatter_peer(const uint64_t *y_bases, const int32_t *y_row_offset,
+                         const int32_t *y_capacity, const int32_t *asg_offsets, int R,
+                         const float *gates, const int32_t *comb_row, int64_t N, int k, int64_t H,
+                         void *out, int out_dtype, int32_t *err_flag, coact_stream_t stream);
+
 /* Bytes of device workspace predict_home needs (E1*R int64 scores). */
 size_t predict_home_workspace_bytes(int E1, int R);
 

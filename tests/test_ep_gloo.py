@@ -1,0 +1,129 @@
+"""Expert parallelism across ranks, host logic on CPU: gloo ranks, each with its own
+contiguous block of tokens, run co_activation_b200.ep.EPLayer (transport "nccl", i.e.
+torch.distributed all-to-all) with the oracle standing in for the local kernels.  Every
+rank must receive exactly the rank-r segment of the single-process plan of all tokens,
+with the right expert ids, and get back the combined rows of its own tokens bit for bit
+(identity experts: the naive combine).  The global pair counts must be the oracle's."""
+import os
+import socket
+import sys
+import types
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+class OracleOps:
+    """The EP layer's local steps through the CPU oracle (test double)."""
+
+    def __init__(self, oracle):
+        self.o = oracle
+
+    def plan(self, ids, E, expert_rank, R, rank_node, n_nodes, src_rank):
+        p = self.o.plan(ids.numpy(), E, expert_rank.numpy(), R,
+                        rank_node=None if rank_node is None else rank_node.numpy(),
+                        n_nodes=n_nodes, src_rank=src_rank.numpy())
+        t = lambda k: torch.from_numpy(np.ascontiguousarray(p[k]))
+        return types.SimpleNamespace(row_token=t("row_token"), row_kmask=t("row_kmask"),
+                                     send_row=t("send_row"), comb_row=t("comb_row"),
+                                     rank_counts=t("rank_counts"), rank_offsets=t("rank_offsets"),
+                                     asg_offsets=t("asg_offsets"),
+                                     row_capacity=len(p["row_token"]))
+
+    def gather(self, x, plan):
+        D = int(plan.rank_offsets[-1])
+        rows = self.o.gather(self.o._bits(x), plan.row_token.numpy(), D)
+        out = torch.zeros((plan.row_capacity, x.shape[1]), dtype=torch.int16)
+        out[:D] = torch.from_numpy(rows.view(np.int16))
+        return out.view(torch.bfloat16)
+
+    def combine(self, y, gates, plan, out):
+        c = self.o.combine_f32chain(self.o._bits(y), gates.numpy(), plan.comb_row.numpy())
+        out.copy_(torch.from_numpy(c))
+        return out
+
+    def count(self, ids, E, pair, loads):
+        p, l, _ = self.o.count(ids.numpy(), E)
+        pair += torch.from_numpy(p)
+        loads += torch.from_numpy(l)
+
+
+def _worker(rank, world, port, cfg_spec, out):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        import workload
+        import co_activation_b200.ep as ep
+        N, E, k, H = cfg_spec
+        cfg = workload.CONFIGS[0].with_(N=N, E=E, k=k, H=H, R=world, n_nodes=1)
+        r = workload.make_routing(cfg)
+        lo, hi = rank * N // world, (rank + 1) * N // world
+        ids = torch.from_numpy(r.ids[lo:hi].copy())
+        gates = torch.from_numpy(r.gates[lo:hi].copy())
+        x = workload.fill_bf16(N, H, 0, 1)
+        xl = x[lo:hi].contiguous()
+        layer = ep.EPLayer(dist.group.WORLD, E, torch.from_numpy(r.expert_rank), transport="nccl",
+                           ops=OracleOps(oracle))
+        pair = torch.zeros((E, E), dtype=torch.int64)
+        loads = torch.zeros(E, dtype=torch.int64)
+        layer.count(ids, pair, loads)
+        got = layer.dispatch(ids, xl)
+        y = ep.expand_identity(got)
+        res = layer.combine(y, gates, torch.empty((hi - lo, H), dtype=torch.float32))
+        # expectations from the single-process plan of all tokens, homed by block
+        src = np.repeat(np.arange(world), np.diff([i * N // world for i in range(world + 1)]))
+        full = oracle.plan(r.ids, E, r.expert_rank, world, src_rank=src.astype(np.int32))
+        seg = slice(full["rank_offsets"][rank], full["rank_offsets"][rank + 1])
+        tok = full["row_token"][seg]
+        xb = oracle._bits(x)
+        want_rows = xb[tok]
+        km = full["row_kmask"][seg]
+        want_exp = np.where((km[:, None] >> np.arange(k)) & 1, r.ids[tok], -1)
+        want_out = oracle.naive_combine_identity_f32(xb[lo:hi], r.gates[lo:hi])
+        op, ol, _ = oracle.count(r.ids, E)
+        out[rank] = (
+            np.array_equal(oracle._bits(got.rows), want_rows),
+            np.array_equal(got.kmask.numpy(), km),
+            np.array_equal(got.experts.numpy(), want_exp),
+            np.array_equal(res.numpy().view(np.uint32), want_out.view(np.uint32)),
+            np.array_equal(pair.numpy(), op) and np.array_equal(loads.numpy(), ol),
+            int(got.rows.shape[0]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,spec", [(2, (4096, 8, 2, 64)), (3, (1000, 12, 3, 32))])
+def test_ep_exchange_matches_single_process_plan(world, spec):
+    ctx = mp.get_context("spawn")
+    manager = ctx.Manager()
+    out = manager.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, spec, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    for r in range(world):
+        rows_ok, km_ok, exp_ok, out_ok, cnt_ok, n = out[r]
+        assert rows_ok and km_ok and exp_ok, f"rank {r}: received rows or metadata differ"
+        assert out_ok, f"rank {r}: combined rows differ"
+        assert cnt_ok, f"rank {r}: global counts differ"
+        assert n > 0

@@ -491,3 +491,79 @@ def test_forward_gather_flags_and_compose_map(coact):
     err.zero_()
     out = coact.coact_compose_map(a, b, err_flag=err)
     assert out.cpu().tolist() == [12, 10, -1, 11] and err.item() == coact.EFLAG_ID_RANGE
+
+
+# ----------------------------------------------------------------------------- across GPUs (emulated)
+
+
+@pytest.mark.parametrize("cfg", [0, 1, 2])
+def test_peer_dispatch_combine_emulated(coact, cfg):
+    """Expert parallelism with the exchange fused into the data movement, on one GPU: each
+    of S = R source ranks plans its own contiguous block of tokens and writes its rows
+    straight into R per-rank buffers (dispatch_gather_peer), then combines reading the
+    expert outputs from the R per-rank buffers (combine_scatter_peer).  The sources run
+    one after another -- nothing waits on anything.  Every destination buffer must equal
+    the rank-r segment of the single-GPU plan of all tokens, and every source's combined
+    rows the single-GPU combine of its tokens, bit for bit."""
+    import co_activation_b200.ep as ep
+    r = workload.make_routing(cfg)
+    c = r.cfg
+    N, k, E, R, H = r.N, r.k, c.E, c.R, min(c.H, 1024)
+    S = R
+    blocks = [(s * N // S, (s + 1) * N // S) for s in range(S)]
+    x = workload.fill_bf16(N, H, r.seed, X_STREAM, device=DEV)
+    er = cuda(r.expert_rank, np.int32)
+    plans = []
+    for s, (lo, hi) in enumerate(blocks):
+        p = coact.alloc_plan(hi - lo, k, E, R, DEV)
+        coact.plan_dispatch(cuda(r.ids[lo:hi]), E, er, R, p,
+                            src_rank=torch.full((hi - lo,), s, dtype=torch.int32, device=DEV))
+        plans.append(p)
+    C = torch.stack([p.rank_counts.to(torch.int64) for p in plans]).cpu()
+    A = torch.stack([(p.asg_offsets[1:] - p.asg_offsets[:-1]).to(torch.int64) for p in plans]).cpu()
+    recv = [torch.full((int(C[:, q].sum()), H), -1, dtype=torch.int16, device=DEV).view(torch.bfloat16)
+            for q in range(R)]
+    bases = torch.tensor([t.data_ptr() for t in recv], dtype=torch.int64, device=DEV)
+    caps = torch.tensor([t.shape[0] for t in recv], dtype=torch.int32, device=DEV)
+    offC, offA = ep.exclusive_offsets(C), ep.exclusive_offsets(A)
+    err = zero_flag()
+    for s, (lo, hi) in enumerate(blocks):
+        coact.dispatch_gather_peer(x[lo:hi], plans[s].send_row, plans[s].rank_offsets, bases,
+                                   offC[s].to(torch.int32).to(DEV), caps, err_flag=err)
+    torch.cuda.synchronize()
+    src = np.concatenate([np.full(hi - lo, s, np.int32) for s, (lo, hi) in enumerate(blocks)])
+    full = oracle.plan(r.ids, E, r.expert_rank, R, src_rank=src)
+    xb = host_bits(x)
+    for q in range(R):
+        seg = full["row_token"][full["rank_offsets"][q]:full["rank_offsets"][q + 1]]
+        assert np.array_equal(host_bits(recv[q]), xb[seg]), f"rank {q}"
+    # expert outputs in the single-GPU expanded order, split into per-rank buffers
+    y = workload.fill_bf16(N * k, H, r.seed, Y_STREAM, device=DEV)
+    ybuf = [y[full["asg_offsets"][q]:full["asg_offsets"][q + 1]].clone() for q in range(R)]
+    ybases = torch.tensor([t.data_ptr() for t in ybuf], dtype=torch.int64, device=DEV)
+    ycaps = torch.tensor([t.shape[0] for t in ybuf], dtype=torch.int32, device=DEV)
+    want = oracle.combine_f32chain(host_bits(y), r.gates, full["comb_row"])
+    for s, (lo, hi) in enumerate(blocks):
+        out = torch.empty((hi - lo, H), dtype=torch.float32, device=DEV)
+        coact.combine_scatter_peer(ybases, offA[s].to(torch.int32).to(DEV), ycaps,
+                                   plans[s].asg_offsets, cuda(r.gates[lo:hi]), plans[s].comb_row,
+                                   out, H, err_flag=err)
+        torch.cuda.synchronize()
+        assert np.array_equal(out.cpu().numpy().view(np.uint32), want[lo:hi].view(np.uint32)), s
+    assert err.item() == 0
+
+
+def test_peer_row_range_flag(coact):
+    r = workload.make_routing(0)
+    c = r.cfg
+    p = coact.alloc_plan(r.N, r.k, c.E, c.R, DEV)
+    coact.plan_dispatch(cuda(r.ids), c.E, cuda(r.expert_rank, np.int32), c.R, p)
+    x = workload.fill_bf16(r.N, 64, 0, 1, device=DEV)
+    counts = p.rank_counts.cpu()
+    bufs = [torch.zeros((max(int(n) - 5, 1), 64), dtype=torch.bfloat16, device=DEV) for n in counts]
+    bases = torch.tensor([t.data_ptr() for t in bufs], dtype=torch.int64, device=DEV)
+    caps = torch.tensor([t.shape[0] for t in bufs], dtype=torch.int32, device=DEV)
+    err = zero_flag()
+    coact.dispatch_gather_peer(x, p.send_row, p.rank_offsets, bases,
+                               torch.zeros(c.R, dtype=torch.int32, device=DEV), caps, err_flag=err)
+    assert err.item() == coact.EFLAG_ROW_RANGE        # the last 5 rows of every rank do not fit
