@@ -165,6 +165,11 @@ def barrier(world: int):
 
 class LayerBuffers:
     """Device buffers and the four library calls of one MoE layer."""
+    tma = False                 # gather through dispatch_gather_tma (--gather tma)
+
+    @classmethod
+    def gather_kernel(cls) -> str:
+        return "k_gather_bulk" if cls.tma else "k_gather_v16"
 
     def __init__(self, coact, r: workload.Routing, device, fill: bool = True,
                  y_stream: int = Y_STREAM, x=None):
@@ -203,7 +208,8 @@ class LayerBuffers:
                                  src_rank=self.src_rank, err_flag=self.err)
 
     def gather(self):
-        self.coact.dispatch_gather(self.x, self.plan.send_row, self.send, err_flag=self.err)
+        self.coact.dispatch_gather(self.x, self.plan.send_row, self.send, err_flag=self.err,
+                                   tma=self.tma)
 
     def combine(self):
         self.coact.combine_scatter(self.y, self.gates, self.plan.comb_row, self.out,
@@ -268,7 +274,7 @@ class OneLayerStep:
     def roofline_parts(self):
         """(phase, kernel, algorithmic bytes) for the HBM-bound kernels."""
         D = self.L.D()
-        return [("dispatch_gather", "k_gather_v16", self.L.bytes_gather(D)),
+        return [("dispatch_gather", LayerBuffers.gather_kernel(), self.L.bytes_gather(D)),
                 ("combine_scatter", "k_combine_v16", self.L.bytes_combine())]
 
     def summary(self):
@@ -352,9 +358,9 @@ class TwoLayerStep:
 
     def roofline_parts(self):
         D1, D2 = self.L1.D(), self.L2.D()
-        return [("layer1_gather", "k_gather_v16", self.L1.bytes_gather(D1)),
+        return [("layer1_gather", LayerBuffers.gather_kernel(), self.L1.bytes_gather(D1)),
                 ("layer1_combine", "k_combine_v16", self.L1.bytes_combine()),
-                ("layer2_gather", "k_gather_v16", self.L2.bytes_gather(D2)),
+                ("layer2_gather", LayerBuffers.gather_kernel(), self.L2.bytes_gather(D2)),
                 ("layer2_combine", "k_combine_v16", self.L2.bytes_combine())]
 
     def summary(self):
@@ -407,7 +413,8 @@ class TwoHopStep(OneLayerStep):
         L.coact.plan_two_hop(L.ids, c.E, L.expert_rank, c.R, L.rank_node, c.n_nodes, self.th,
                              err_flag=L.err)
         if ev: ev[2].record()
-        L.coact.dispatch_gather(L.x, self.th.node.send_row, self.hop1, err_flag=L.err)
+        L.coact.dispatch_gather(L.x, self.th.node.send_row, self.hop1, err_flag=L.err,
+                                tma=L.tma)
         if ev: ev[3].record()
         L.coact.forward_gather(self.hop1, self.th.fwd_src, L.send, err_flag=L.err)
         if ev: ev[4].record()
@@ -419,7 +426,8 @@ class TwoHopStep(OneLayerStep):
         c = self.cfg
         Dn = int(self.th.node.rank_offsets[-1].item())
         D = int(self.th.rank.rank_offsets[-1].item())
-        return [("gather_hop1", "k_gather_v16", (c.N + Dn) * c.H * 2 + c.N * c.k * 4),
+        return [("gather_hop1", LayerBuffers.gather_kernel(),
+                 (c.N + Dn) * c.H * 2 + c.N * c.k * 4),
                 ("forward_hop2", "k_forward_gather", 2 * D * c.H * 2 + D * 4),
                 ("combine_scatter", "k_combine_v16", self.L.bytes_combine())]
 
@@ -491,6 +499,7 @@ def make_step(coact, cfg_index: int, seed: int, device, two_hop: bool = False,
 # CUDA sources of each HBM-bound kernel: a committed DRAM-traffic figure is reported only
 # while these files are byte-identical to the ones the ncu capture was taken on.
 KERNEL_SOURCES = {"k_gather_v16": ("gather.cu", "common.cuh"),
+                  "k_gather_bulk": ("gather.cu", "common.cuh"),
                   "k_combine_v16": ("combine.cu", "common.cuh"),
                   "k_forward_gather": ("twohop.cu", "common.cuh")}
 
@@ -532,6 +541,7 @@ def run_gpu(args):
     import co_activation_b200 as coact
 
     cfg = workload.CONFIGS[args.config]
+    LayerBuffers.tma = args.gather == "tma"
     S, placement = make_step(coact, args.config, rank_seed(args.seed, rank), device, args.two_hop,
                              args.placement)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
@@ -641,6 +651,8 @@ def run_gpu(args):
         "config": {"workload": f"config {cfg.index}: {cfg.desc}", "N": cfg.N, "E": cfg.E,
                    "k": cfg.k, "H": cfg.H, "R": cfg.R, "n_nodes": cfg.n_nodes,
                    "placement": placement,
+                   "gather": ("dispatch_gather_tma (TMA bulk copies)" if LayerBuffers.tma
+                              else "dispatch_gather (16-byte vector copies)"),
                    "step": ("two layers: counts + cross-layer counts (side stream); plan, gather, "
                             "combine of layer 1; predict_home; plan, gather, combine of layer 2"
                             if cfg.two_layer else
@@ -857,6 +869,8 @@ def main():
     ap.add_argument("--placement", default="auto", choices=["auto", "default", "correlated",
                                                              "two-stage"],
                     help="auto: the configuration's own (config 3: correlated)")
+    ap.add_argument("--gather", default="vector", choices=["vector", "tma"],
+                    help="gather implementation: dispatch_gather or dispatch_gather_tma")
     ap.add_argument("--two-hop", action="store_true",
                     help="dispatch in two hops: to nodes, then inside the node to ranks")
     args = ap.parse_args()

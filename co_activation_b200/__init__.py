@@ -47,6 +47,7 @@ _lib.plan_dispatch_workspace_bytes.restype = _SZ
 _lib.plan_dispatch.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _P, _P, _P, _P,
                                _P, _I64, _P, _P, _P, _P, _P, _SZ, _P, _P]
 _lib.dispatch_gather.argtypes = [_P, _I64, _I64, _P, _I32, _P, _I64, _P, _P]
+_lib.dispatch_gather_tma.argtypes = [_P, _I64, _I64, _P, _I32, _P, _I64, _P, _P]
 _lib.combine_scatter.argtypes = [_P, _I64, _P, _P, _I64, _I32, _I64, _P, _I32, _P, _P]
 _lib.predict_home_workspace_bytes.argtypes = [_I32, _I32]
 _lib.predict_home_workspace_bytes.restype = _SZ
@@ -61,14 +62,15 @@ _lib.plan_forward.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, 
 _lib.forward_gather.argtypes = [_P, _I64, _I64, _P, _I64, _P, _P, _P]
 _lib.plan_dispatch_noalloc.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _P, _P,
                                        _P, _P, _P, _I64, _P, _P, _P, _P, _P, _P]
-for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "combine_scatter", "predict_home",
+for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "dispatch_gather_tma",
+           "combine_scatter", "predict_home",
            "coact_place_correlated", "plan_dispatch_noalloc", "coact_compose_map", "plan_forward",
            "forward_gather", "coact_rebalance_ranks", "dispatch_gather_peer",
            "combine_scatter_peer"):
     getattr(_lib, _f).restype = _I32
 
 ABI_SYMBOLS = ("coact_strerror", "coact_abi_version", "coact_count", "plan_dispatch_workspace_bytes",
-               "plan_dispatch", "dispatch_gather", "combine_scatter",
+               "plan_dispatch", "dispatch_gather", "dispatch_gather_tma", "combine_scatter",
                "predict_home_workspace_bytes", "predict_home", "coact_place_correlated",
                "plan_dispatch_noalloc", "coact_compose_map", "plan_forward", "forward_gather",
                "coact_rebalance_ranks", "dispatch_gather_peer", "combine_scatter_peer")
@@ -228,8 +230,10 @@ def plan_dispatch(ids: torch.Tensor, E: int, expert_rank: torch.Tensor, R: int, 
 
 
 def dispatch_gather(x: torch.Tensor, send_row: torch.Tensor, send: torch.Tensor,
-                    err_flag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """send[send_row[t, j]] = x[t] for every send_row entry >= 0 (bf16 rows)."""
+                    err_flag: Optional[torch.Tensor] = None, stream=None,
+                    tma: bool = False) -> torch.Tensor:
+    """send[send_row[t, j]] = x[t] for every send_row entry >= 0 (bf16 rows).
+    tma=True uses the TMA bulk-copy implementation (dispatch_gather_tma)."""
     N, H = x.shape
     _need(_bits16(x), "x", torch.bfloat16)
     _need(send_row, "send_row", torch.int32)
@@ -239,8 +243,9 @@ def dispatch_gather(x: torch.Tensor, send_row: torch.Tensor, send: torch.Tensor,
     if send.shape[1] != H:
         raise ValueError("send rows must have x's hidden size")
     _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
-    _check(_lib.dispatch_gather(_ptr(x), N, H, _ptr(send_row), send_row.shape[1], _ptr(send),
-                                send.shape[0], _ptr(err_flag), _stream(stream)), "dispatch_gather")
+    fn = _lib.dispatch_gather_tma if tma else _lib.dispatch_gather
+    _check(fn(_ptr(x), N, H, _ptr(send_row), send_row.shape[1], _ptr(send), send.shape[0],
+              _ptr(err_flag), _stream(stream)), "dispatch_gather_tma" if tma else "dispatch_gather")
     return send
 
 

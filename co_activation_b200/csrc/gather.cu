@@ -10,12 +10,13 @@
 //  * k_gather_v16 (default) -- one warp per token, 16-byte vector loads of the x row
 //    into registers (up to 8 per lane in flight) and streaming 16-byte stores to each
 //    destination; 8 CTAs of 8 warps per SM.
-//  * k_gather_bulk (builds with -DCOACT_GATHER_PATH=1) -- TMA bulk copies.  One warp
-//    per CTA; lane 0 streams rows into a ring of shared-memory stages with
-//    cp.async.bulk (global -> shared, completion on an mbarrier), then lanes j < k each
-//    issue the cp.async.bulk store of the staged row to destination j.  No multicast:
-//    every load reads this GPU's own memory once.  Measured on B200 it tied the vector
-//    path on 4 KB rows and lost 4-5% on 8-14 KB rows, so it is not the default.
+//  * k_gather_bulk (entry point dispatch_gather_tma) -- TMA bulk copies.  One warp per
+//    CTA; lane 0 streams rows into a ring of shared-memory stages with cp.async.bulk
+//    (global -> shared, completion on an mbarrier), then lanes j < k each issue the
+//    cp.async.bulk store of the staged row to destination j.  No multicast: every load
+//    reads this GPU's own memory once.  Measured on B200 it tied the vector path on 4 KB
+//    rows and lost 4-5% on 8-14 KB rows, so it is not the default; it occupies one warp
+//    and no row registers per CTA, which leaves the SMs to work running alongside.
 // All mbarrier waits are bounded by a wall-clock limit; on expiry the kernel raises
 // COACT_EFLAG_TIMEOUT, drains its own copies and returns.
 #include <algorithm>
@@ -287,39 +288,56 @@ int launch_v16(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row,
 
 using namespace coact;
 
-extern "C" int dispatch_gather(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row,
-                               int k, uint16_t *send, int64_t row_capacity, int32_t *err_flag,
-                               coact_stream_t stream) {
+namespace coact {
+namespace {
+
+int gather_args(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row, int k,
+                uint16_t *send, int64_t row_capacity) {
     if (N < 0 || H < 0 || row_capacity < 0) return COACT_ERR_INVALID;
     if (k < 1 || k > COACT_MAX_K) return COACT_ERR_UNSUPPORTED;
     if (H % 8 != 0) return COACT_ERR_UNSUPPORTED;
-    if (N == 0 || H == 0) return COACT_OK;
+    if (N == 0 || H == 0) return -100;  // nothing to do
     if (!x || !send_row || (row_capacity > 0 && !send)) return COACT_ERR_INVALID;
     if (!aligned16(x) || (send && !aligned16(send))) return COACT_ERR_INVALID;
     if (N > (int64_t)INT32_MAX / k || row_capacity > (int64_t)INT32_MAX) return COACT_ERR_UNSUPPORTED;
+    return COACT_OK;
+}
+
+}  // namespace
+}  // namespace coact
+
+extern "C" int dispatch_gather(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row,
+                               int k, uint16_t *send, int64_t row_capacity, int32_t *err_flag,
+                               coact_stream_t stream) {
+    const int a = gather_args(x, N, H, send_row, k, send, row_capacity);
+    if (a == -100) return COACT_OK;
+    if (a) return a;
     DeviceInfo di;
     if (int s = device_info(&di)) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const int64_t row_bytes = H * 2;
-    // Default: the vector path.  On B200 it matched the bulk (TMA) path on 4 KB rows and
-    // beat it by 4-5% on 8 and 14 KB rows (5.99 vs 5.73 TB/s); the bulk path stays
-    // available to builds with -DCOACT_GATHER_PATH=1.
-    bool bulk = false;
 #if defined(COACT_GATHER_PATH)
-    bulk = row_bytes >= 1024 && row_bytes <= 32768 && COACT_GATHER_PATH != 0;
-#endif
-#ifndef COACT_GATHER_STAGES_SMALL
-#define COACT_GATHER_STAGES_SMALL 8
-#endif
-#ifndef COACT_GATHER_STAGES_LARGE
-#define COACT_GATHER_STAGES_LARGE 4
-#endif
-    if (bulk) {
-        if (row_bytes <= 4096)
-            return launch_bulk<COACT_GATHER_STAGES_SMALL>(x, N, H, send_row, k, send, row_capacity,
-                                                          err_flag, st, di);
-        return launch_bulk<COACT_GATHER_STAGES_LARGE>(x, N, H, send_row, k, send, row_capacity,
-                                                      err_flag, st, di);
+    if (COACT_GATHER_PATH != 0 && H * 2 >= 1024 && H * 2 <= 32768) {  // experiment builds only
+        if (H * 2 <= 4096)
+            return launch_bulk<8>(x, N, H, send_row, k, send, row_capacity, err_flag, st, di);
+        return launch_bulk<4>(x, N, H, send_row, k, send, row_capacity, err_flag, st, di);
     }
+#endif
     return launch_v16(x, N, H, send_row, k, send, row_capacity, err_flag, st, di);
+}
+
+extern "C" int dispatch_gather_tma(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row,
+                                   int k, uint16_t *send, int64_t row_capacity, int32_t *err_flag,
+                                   coact_stream_t stream) {
+    const int a = gather_args(x, N, H, send_row, k, send, row_capacity);
+    if (a == -100) return COACT_OK;
+    if (a) return a;
+    if (H * 2 > 32768) return COACT_ERR_UNSUPPORTED;   // one row per shared-memory stage
+    DeviceInfo di;
+    if (int s = device_info(&di)) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (H * 2 <= 4096)
+        return launch_bulk<8>(x, N, H, send_row, k, send, row_capacity, err_flag, st, di);
+    if (H * 2 <= 16384)
+        return launch_bulk<4>(x, N, H, send_row, k, send, row_capacity, err_flag, st, di);
+    return launch_bulk<2>(x, N, H, send_row, k, send, row_capacity, err_flag, st, di);
 }

@@ -176,6 +176,20 @@ int dispatch_gather(const uint16_t *x, int64_t N, int64_t H,
                     int32_t *err_flag, coact_stream_t stream);
 
 /*
+ * dispatch_gather_tma -- dispatch_gather through the Tensor Memory Accelerator: rows are
+ * staged in shared memory with bulk asynchronous copies (cp.async.bulk, one issuing warp
+ * per CTA, completion tracked by mbarriers whose waits are bounded by wall clock) and
+ * written to every destination with bulk stores.  Same arguments, results and flags as
+ * dispatch_gather (plus COACT_EFLAG_TIMEOUT if a bounded wait gives up); rows up to 32 KB
+ * (H <= 16384), else COACT_ERR_UNSUPPORTED.  It holds few SM resources, for overlapping
+ * the dispatch with other kernels; dispatch_gather is faster when running alone.
+ */
+int dispatch_gather_tma(const uint16_t *x, int64_t N, int64_t H,
+                        const int32_t *send_row, int k,
+                        uint16_t *send, int64_t row_capacity,
+                        int32_t *err_flag, coact_stream_t stream);
+
+/*
  * combine_scatter -- the weighted combine back to token order.
  * Zyphra, English abstract: tokens are dispatched to their experts "and then" the
  * results are combined; neither method changes the routing decisions.

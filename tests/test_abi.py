@@ -107,6 +107,12 @@ def test_gather_combine_reject_bad_arguments(lib):
     assert g(P(258), 10, 16, FAKE, 2, FAKE, 20, None, None) == -1  # misaligned x
     assert g(FAKE, 10, 16, FAKE, 9, FAKE, 20, None, None) == -2    # k > 8
     assert g(None, 0, 16, None, 2, None, 0, None, None) == 0       # empty
+    t = lib.dispatch_gather_tma
+    t.argtypes = g.argtypes
+    assert t(FAKE, 10, 12, FAKE, 2, FAKE, 20, None, None) == -2    # H % 8 != 0
+    assert t(P(258), 10, 16, FAKE, 2, FAKE, 20, None, None) == -1  # misaligned x
+    assert t(FAKE, 10, 16392, FAKE, 2, FAKE, 20, None, None) == -2  # row above 32 KB
+    assert t(None, 0, 16, None, 2, None, 0, None, None) == 0       # empty
     c = lib.combine_scatter
     c.argtypes = [P, ctypes.c_int64, P, P, ctypes.c_int64, ctypes.c_int, ctypes.c_int64, P,
                   ctypes.c_int, P, P]

@@ -222,24 +222,24 @@ def test_plan_deterministic(coact):
 # ----------------------------------------------------------------------------- gather
 
 
-def _gather(coact, r, H, plan, sentinel_rows=True):
+def _gather(coact, r, H, plan, sentinel_rows=True, tma=False):
     x = workload.fill_bf16(r.N, H, r.seed, X_STREAM, device=DEV)
     send = torch.empty((plan.row_capacity, H), dtype=torch.bfloat16, device=DEV)
     if sentinel_rows:
         send.view(torch.int16).fill_(-1)
     err = zero_flag()
-    coact.dispatch_gather(x, plan.send_row, send, err_flag=err)
+    coact.dispatch_gather(x, plan.send_row, send, err_flag=err, tma=tma)
     torch.cuda.synchronize()
     return x, send, err
 
 
-@pytest.mark.parametrize("cfg", [0, 1])
-def test_gather_full(coact, cfg):
+@pytest.mark.parametrize("cfg,tma", [(0, False), (1, False), (1, True)])
+def test_gather_full(coact, cfg, tma):
     r = workload.make_routing(cfg)
     H = r.cfg.H
     plan, _ = run_plan(coact, r)
     o = oracle_plan_for(r)
-    x, send, err = _gather(coact, r, H, plan)
+    x, send, err = _gather(coact, r, H, plan, tma=tma)
     assert err.item() == 0
     xh = host_bits(workload.fill_bf16(r.N, H, r.seed, X_STREAM))
     want = oracle.gather(xh, o["row_token"], o["D"])
@@ -248,13 +248,13 @@ def test_gather_full(coact, cfg):
     assert (got[o["D"]:] == 0xFFFF).all()                   # rows past D untouched
 
 
-@pytest.mark.parametrize("cfg", [2, 3])
-def test_gather_full_size_sampled(coact, cfg):
+@pytest.mark.parametrize("cfg,tma", [(2, False), (3, False), (3, True)])
+def test_gather_full_size_sampled(coact, cfg, tma):
     r = workload.make_routing(cfg)
     H = r.cfg.H
     plan, _ = run_plan(coact, r)
     o = oracle_plan_for(r)
-    x, send, err = _gather(coact, r, H, plan)
+    x, send, err = _gather(coact, r, H, plan, tma=tma)
     assert err.item() == 0
     D, cap = o["D"], plan.row_capacity
     rng = np.random.default_rng(cfg)
@@ -268,13 +268,15 @@ def test_gather_full_size_sampled(coact, cfg):
         assert (host_bits(send[torch.as_tensor(tail, device=DEV)]) == 0xFFFF).all()
 
 
-@pytest.mark.parametrize("H", [8, 256, 520, 2048, 7168, 16400])
-def test_gather_row_sizes(coact, H):
-    # covers the vector path (short, odd-length and very long rows) and the bulk path
+@pytest.mark.parametrize("H,tma", [(8, False), (256, False), (520, False), (2048, False),
+                                   (7168, False), (16400, False), (8, True), (256, True),
+                                   (2048, True), (7168, True), (16384, True)])
+def test_gather_row_sizes(coact, H, tma):
+    # the vector path (short, odd-length and very long rows) and the TMA bulk path
     r = workload.make_routing(2, N=3001)
     plan, _ = run_plan(coact, r)
     o = oracle_plan_for(r)
-    x, send, err = _gather(coact, r, H, plan)
+    x, send, err = _gather(coact, r, H, plan, tma=tma)
     assert err.item() == 0
     want = oracle.gather(host_bits(x), o["row_token"], o["D"])
     got = host_bits(send)
@@ -282,7 +284,8 @@ def test_gather_row_sizes(coact, H):
     assert (got[o["D"]:] == 0xFFFF).all()
 
 
-def test_gather_row_range_flag(coact):
+@pytest.mark.parametrize("tma", [False, True])
+def test_gather_row_range_flag(coact, tma):
     N, H, k = 100, 64, 2
     x = workload.fill_bf16(N, H, 0, 1, device=DEV)
     send_row = torch.full((N, k), -1, dtype=torch.int32, device=DEV)
@@ -290,7 +293,7 @@ def test_gather_row_range_flag(coact):
     send_row[3, 1] = 100                                     # == capacity: out of range
     send = torch.zeros((N, H), dtype=torch.bfloat16, device=DEV)
     err = zero_flag()
-    coact.dispatch_gather(x, send_row, send, err_flag=err)
+    coact.dispatch_gather(x, send_row, send, err_flag=err, tma=tma)
     assert err.item() == coact.EFLAG_ROW_RANGE
     assert torch.equal(send, x)
 
