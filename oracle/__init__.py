@@ -70,6 +70,12 @@ def _get():
             _lib.oracle_forward_src.restype = None
             _lib.oracle_forward_gather.argtypes = [P, I64, P, I64, P]
             _lib.oracle_forward_gather.restype = None
+            _lib.oracle_gather_backward_f32chain.argtypes = [P, I64, P, I64, I32, I64, P]
+            _lib.oracle_gather_backward_f32chain.restype = None
+            _lib.oracle_combine_units_f32chain.argtypes = [P, I64, P, P, I32, P, P, I64, I64, P]
+            _lib.oracle_combine_units_f32chain.restype = None
+            _lib.oracle_combine_backward.argtypes = [P, I64, P, P, I32, P, P, I64, I64, P, P, P, P]
+            _lib.oracle_combine_backward.restype = None
         return _lib
 
 
@@ -308,3 +314,74 @@ def place_two_stage(pair, loads, rank_node, n_nodes: int) -> np.ndarray:
     """Stage 1: correlated placement at node granularity; stage 2: rebalance in nodes."""
     expert_node = place_correlated(pair, n_nodes)
     return rebalance_ranks(loads, expert_node, rank_node)
+
+
+# ----------------------------------------------------------------------------- backward
+
+
+def gather_backward_f32chain(g_send, send_row) -> np.ndarray:
+    """Transpose of the dispatch: grad_x[t] = sum of grad_send[send_row[t,j]] over the
+    token's send rows (ascending j, fp32 add chain from +0) ([N, H] float32)."""
+    gb = _bits(g_send)
+    sr = _c(send_row, np.int32)
+    N, k = sr.shape
+    H = gb.shape[1]
+    out = np.zeros((N, H), np.float32)
+    _get().oracle_gather_backward_f32chain(_p(gb), gb.shape[0], _p(sr), N, k, H, _p(out))
+    return out
+
+
+def _units(row_token, row_kmask, n_units, N):
+    if row_token is None:
+        return None, None, N
+    rt = _c(row_token, np.int32)
+    km = _c(row_kmask, np.uint8)
+    n = len(rt) if n_units is None else int(n_units)
+    return rt[:n].copy(), km[:n].copy(), n
+
+
+def combine_units_f32chain(y, gates, comb_row, row_token=None, row_kmask=None,
+                           n_units=None) -> np.ndarray:
+    """Combine over units: unit u is token row_token[u] restricted to the slots of
+    row_kmask[u] (or token u, all slots, without row_token) ([n_units, H] float32)."""
+    yb = _bits(y)
+    g = _c(gates, np.float32)
+    cr = _c(comb_row, np.int32)
+    N, k = g.shape
+    rt, km, n = _units(row_token, row_kmask, n_units, N)
+    H = yb.shape[1]
+    out = np.zeros((n, H), np.float32)
+    _get().oracle_combine_units_f32chain(_p(yb), yb.shape[0], _p(g), _p(cr), k, _p(rt), _p(km),
+                                         n, H, _p(out))
+    return out
+
+
+def combine_backward(y, gates, comb_row, g_out, row_token=None, row_kmask=None, n_units=None,
+                     g_y=None):
+    """Backward of the combine.  Returns (g_y bf16 bits [n_rows, H] -- rows no slot names
+    keep the contents of the g_y passed in (zeros by default) --, g_gates float64 [N, k],
+    g_gates_abs float64 [N, k]); slots no unit covers are 0 in both."""
+    yb = _bits(y)
+    g = _c(gates, np.float32)
+    cr = _c(comb_row, np.int32)
+    N, k = g.shape
+    rt, km, n = _units(row_token, row_kmask, n_units, N)
+    H = yb.shape[1]
+    gob = _bits(g_out)
+    assert gob.shape == (n, H)
+    gy = np.zeros(yb.shape, np.uint16) if g_y is None else _bits(g_y).copy()
+    gg = np.zeros((N, k), np.float64)
+    ga = np.zeros((N, k), np.float64)
+    _get().oracle_combine_backward(_p(yb), yb.shape[0], _p(g), _p(cr), k, _p(rt), _p(km), n, H,
+                                   _p(gob), _p(gy), _p(gg), _p(ga))
+    return gy, gg, ga
+
+
+def combine_prereduced(y, gates, plan_: dict):
+    """The pre-reduced reverse path over a plan: one partial row per send row (bf16), then
+    the transposed dispatch adds each token's partial rows.  Returns (pre bf16 bits [D, H],
+    out float32 [N, H] before the final rounding)."""
+    D = plan_["D"]
+    pre = bf16_rne(combine_units_f32chain(y, gates, plan_["comb_row"], plan_["row_token"],
+                                          plan_["row_kmask"], D))
+    return pre, gather_backward_f32chain(pre, plan_["send_row"])

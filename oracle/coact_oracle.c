@@ -531,3 +531,101 @@ int oracle_rebalance_ranks(const int64_t *loads, const int32_t *expert_node, int
     free(done);
     return status;
 }
+
+/* ------------------------------------------------------------------------------------
+ * Backward pass and the pre-reduced reverse path.
+ *
+ * Both forward maps are linear in the rows they move.  The dispatch copies x[t] to every
+ * send row of the token (send_row[t,j] >= 0, one per destination rank) and the combine
+ * takes a gate-weighted sum of the token's expert outputs, so their gradients are the
+ * transposed maps over the same plan.  [Zyphra] dispatch sends each token to each GPU
+ * once "and then" combines the results; the reverse direction can therefore also carry one
+ * row per (token, GPU): each GPU first sums, with the gates, the outputs of the slots it
+ * served (one row per received row), and the token's rank adds those partial rows -- the
+ * transposed dispatch again.  Reading taken: the partial rows travel as bf16 (the type of
+ * the rows on the wire), accumulated in fp32 in ascending slot order.
+ * ------------------------------------------------------------------------------------ */
+
+/*
+ * Transpose of the dispatch: grad_x[t] = sum over j ascending with send_row[t,j] >= 0 of
+ * grad_send[send_row[t,j]], an fp32 add chain from +0 (caller rounds to bf16 if wanted).
+ * Rows outside [0, n_rows) are skipped.
+ */
+void oracle_gather_backward_f32chain(const uint16_t *g_send, int64_t n_rows, const int32_t *send_row,
+                                     int64_t N, int k, int64_t H, float *g_x) {
+    for (int64_t t = 0; t < N; ++t)
+        for (int64_t h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int j = 0; j < k; ++j) {
+                int64_t row = send_row[t * k + j];
+                if (row < 0 || row >= n_rows) continue;
+                acc = acc + bf16_to_f32(g_send[row * H + h]);
+            }
+            g_x[t * H + h] = acc;
+        }
+}
+
+/*
+ * Combine driven by units.  Unit u stands for token t = row_token[u] and the slots set in
+ * row_kmask[u]; with row_token == NULL unit u is token u with all k slots.
+ *   out[u] = sum over set slots j ascending of gates[t,j] * y[comb_row[t,j]]
+ * as an fp32 fma chain from +0.  With the plan's rows as units (row_token, row_kmask) this
+ * is the partial combine of the pre-reduced reverse path: one row per send row.
+ */
+void oracle_combine_units_f32chain(const uint16_t *y, int64_t n_rows, const float *gates,
+                                   const int32_t *comb_row, int k, const int32_t *row_token,
+                                   const uint8_t *row_kmask, int64_t n_units, int64_t H,
+                                   float *out) {
+    for (int64_t u = 0; u < n_units; ++u) {
+        int64_t t = row_token ? row_token[u] : u;
+        unsigned m = row_kmask ? row_kmask[u] : 0xffu;
+        for (int64_t h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int j = 0; j < k; ++j) {
+                if (!((m >> j) & 1u)) continue;
+                int64_t row = comb_row[t * k + j];
+                if (row < 0 || row >= n_rows) continue;
+                acc = fmaf(gates[t * k + j], bf16_to_f32(y[row * H + h]), acc);
+            }
+            out[u * H + h] = acc;
+        }
+    }
+}
+
+/*
+ * Backward of the combine out[t] = sum_j gates[t,j] * y[comb_row[t,j]], over units as in
+ * oracle_combine_units_f32chain (g_out has one row per unit):
+ *   g_y[comb_row[t,j]]  = bf16_rne(gates[t,j] * g_out[u])   (fp32 product, then RNE)
+ *   g_gates[t*k+j]      = sum_h g_out[u,h] * y[comb_row[t,j],h]   in float64
+ *   g_gates_abs[t*k+j]  = sum_h |g_out[u,h] * y[comb_row[t,j],h]| (error scale)
+ * for every set slot of every unit; a slot whose comb_row is outside [0, n_rows) gets
+ * g_gates = 0 and writes no g_y row.  g_y rows no slot names are not written.
+ */
+void oracle_combine_backward(const uint16_t *y, int64_t n_rows, const float *gates,
+                             const int32_t *comb_row, int k, const int32_t *row_token,
+                             const uint8_t *row_kmask, int64_t n_units, int64_t H,
+                             const uint16_t *g_out, uint16_t *g_y, double *g_gates,
+                             double *g_gates_abs) {
+    for (int64_t u = 0; u < n_units; ++u) {
+        int64_t t = row_token ? row_token[u] : u;
+        unsigned m = row_kmask ? row_kmask[u] : 0xffu;
+        for (int j = 0; j < k; ++j) {
+            if (!((m >> j) & 1u)) continue;
+            int64_t row = comb_row[t * k + j];
+            double dot = 0.0, mag = 0.0;
+            if (row >= 0 && row < n_rows) {
+                float g = gates[t * k + j];
+                for (int64_t h = 0; h < H; ++h) {
+                    float go = bf16_to_f32(g_out[u * H + h]);
+                    float p = g * go;
+                    g_y[row * H + h] = oracle_bf16_rne(p);
+                    double term = (double)go * (double)bf16_to_f32(y[row * H + h]);
+                    dot += term;
+                    mag += fabs(term);
+                }
+            }
+            g_gates[t * k + j] = dot;
+            g_gates_abs[t * k + j] = mag;
+        }
+    }
+}
