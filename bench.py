@@ -462,11 +462,129 @@ def layout(coact, r: workload.Routing, kind: str, device):
     raise SystemExit(f"unknown placement {kind}")
 
 
+class PreReducedStep(OneLayerStep):
+    """One layer with the pre-reduced reverse path: count (side stream) -> plan -> gather
+    -> combine_rows over the send rows (one bf16 partial row per (token, rank), D rows
+    instead of N*k) -> dispatch_gather_backward adds each token's partial rows."""
+    n_events = 6
+    phases = {"coact_count": (0, 1), "plan_dispatch": (0, 2), "dispatch_gather": (2, 3),
+              "combine_rows": (3, 4), "reduce_rows": (4, 5)}
+    step_desc = ("coact_count (side stream) + plan_dispatch + dispatch_gather + combine_rows "
+                 "(partial rows per send row) + dispatch_gather_backward (sum per token, bf16 out)")
+
+    def __init__(self, coact, r: workload.Routing, device, fill: bool = True):
+        super().__init__(coact, r, device, fill)
+        self.pre = torch.empty((self.L.plan.row_capacity, r.cfg.H), dtype=torch.bfloat16,
+                               device=device)
+        self.kernels_per_step = 1 + plan_launches(r.cfg.R, self.N) + 1 + 2
+
+    def clone_for_copy(self, coact, device):
+        return PreReducedStep(coact, self.L.r, device, fill=False)
+
+    def step(self, ev=None):
+        L, c = self.L, self.L.coact
+        main = torch.cuda.current_stream()
+        self.side.wait_stream(main)
+        if ev: ev[0].record()
+        with torch.cuda.stream(self.side):
+            L.count()
+            if ev: ev[1].record()
+        L.plan_()
+        if ev: ev[2].record()
+        L.gather()
+        if ev: ev[3].record()
+        # units: the plan's send rows, as many as the device-side D = rank_offsets[R]
+        c.combine_rows(L.y, L.gates, L.plan.comb_row, L.plan.row_token, L.plan.row_kmask,
+                       self.pre, unit_count=L.plan.rank_offsets[self.cfg.R:], err_flag=L.err)
+        if ev: ev[4].record()
+        c.dispatch_gather_backward(self.pre, L.plan.send_row, L.out, err_flag=L.err)
+        main.wait_stream(self.side)
+        if ev: ev[5].record()
+
+    def roofline_parts(self):
+        c, D = self.cfg, self.L.D()
+        return [("dispatch_gather", LayerBuffers.gather_kernel(), self.L.bytes_gather(D)),
+                ("combine_rows", "k_combine_v16",
+                 c.N * c.k * c.H * 2 + D * c.H * 2 + D * 5 + c.N * c.k * 8),
+                ("reduce_rows", "k_combine_v16", D * c.H * 2 + c.N * c.H * 2 + c.N * c.k * 4)]
+
+
+class BackwardStep:
+    """The backward pass of one layer over the forward's plan (computed once, outside the
+    timed steps): combine_scatter_backward (grad_y rows for the experts, grad_gates), then
+    dispatch_gather_backward (the experts' input gradients, one row per send row, summed
+    per token into grad_x).  The experts' own backward sits between the two and is not
+    part of this path."""
+    n_events = 3
+    phases = {"combine_backward": (0, 1), "dispatch_backward": (1, 2)}
+    host_inputs = ("g_out", "y", "g_send", "gates")
+    step_desc = ("backward: combine_scatter_backward (grad_y bf16, grad_gates fp32) + "
+                 "dispatch_gather_backward (grad_x bf16) over the forward's plan")
+
+    def __init__(self, coact, r: workload.Routing, device, fill: bool = True):
+        self.coact = coact
+        self.L = LayerBuffers(coact, r, device, fill)
+        self.cfg, self.N = r.cfg, r.cfg.N
+        c = r.cfg
+        self.L.plan_()
+        self.D = self.L.D()
+        if fill:
+            self.g_out = workload.fill_bf16(c.N, c.H, r.seed, 6, device=device)
+            self.g_send = workload.fill_bf16(self.L.plan.row_capacity, c.H, r.seed, 5,
+                                             device=device)
+        else:
+            self.g_out = torch.empty((c.N, c.H), dtype=torch.bfloat16, device=device)
+            self.g_send = torch.empty((self.L.plan.row_capacity, c.H), dtype=torch.bfloat16,
+                                      device=device)
+        self.g_y = torch.empty((c.N * c.k, c.H), dtype=torch.bfloat16, device=device)
+        self.g_gates = torch.empty((c.N, c.k), dtype=torch.float32, device=device)
+        self.g_x = torch.empty((c.N, c.H), dtype=torch.bfloat16, device=device)
+        self.kernels_per_step = 2
+
+    @property
+    def y(self):
+        return self.L.y
+
+    @property
+    def gates(self):
+        return self.L.gates
+
+    def inputs(self):
+        return {n: getattr(self, n) for n in self.host_inputs}
+
+    def outputs(self):
+        return [self.g_x, self.g_gates]
+
+    def clone_for_copy(self, coact, device):
+        return BackwardStep(coact, self.L.r, device, fill=False)
+
+    def step(self, ev=None):
+        L, c = self.L, self.coact
+        if ev: ev[0].record()
+        c.combine_scatter_backward(L.y, L.gates, L.plan.comb_row, self.g_out, self.g_y,
+                                   self.g_gates, err_flag=L.err)
+        if ev: ev[1].record()
+        c.dispatch_gather_backward(self.g_send, L.plan.send_row, self.g_x, err_flag=L.err)
+        if ev: ev[2].record()
+
+    def roofline_parts(self):
+        c, D = self.cfg, self.D
+        return [("combine_backward", "k_combine_bwd",
+                 c.N * c.H * 2 + 2 * c.N * c.k * c.H * 2 + c.N * c.k * 12),
+                ("dispatch_backward", "k_combine_v16", D * c.H * 2 + c.N * c.H * 2 + c.N * c.k * 4)]
+
+    def summary(self):
+        return {"dedup_rows_over_naive": self.D / (self.N * self.cfg.k),
+                "err_flag": int(self.L.err.item())}
+
+
 def make_step(coact, cfg_index: int, seed: int, device, two_hop: bool = False,
-              placement_kind: str = "auto"):
+              placement_kind: str = "auto", mode: str = "forward"):
     """The step object for a configuration, plus a description of its placement."""
     cfg = workload.CONFIGS[cfg_index]
     if cfg.two_layer:
+        if mode != "forward":
+            raise SystemExit("--pass backward / --combine prereduced need a one-layer configuration")
         if two_hop:
             raise SystemExit("--two-hop needs a one-layer configuration with several nodes (2, 3)")
         return TwoLayerStep(coact, workload.make_two_layer(cfg, seed=seed), device), \
@@ -488,7 +606,13 @@ def make_step(coact, cfg_index: int, seed: int, device, two_hop: bool = False,
     if two_hop:
         if cfg.n_nodes < 2:
             raise SystemExit("--two-hop needs a one-layer configuration with several nodes (2, 3)")
+        if mode != "forward":
+            raise SystemExit("--two-hop runs the forward pass with the direct combine only")
         S = TwoHopStep(coact, r, device)
+    elif mode == "backward":
+        S = BackwardStep(coact, r, device)
+    elif mode == "prereduced":
+        S = PreReducedStep(coact, r, device)
     else:
         S = OneLayerStep(coact, r, device)
     if rr_D is not None:
@@ -542,8 +666,10 @@ def run_gpu(args):
 
     cfg = workload.CONFIGS[args.config]
     LayerBuffers.tma = args.gather == "tma"
+    mode = "backward" if args.pass_ == "backward" else (
+        "prereduced" if args.combine == "prereduced" else "forward")
     S, placement = make_step(coact, args.config, rank_seed(args.seed, rank), device, args.two_hop,
-                             args.placement)
+                             args.placement, mode)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     flush_w = torch.empty(max(2 * l2, 64 << 20), dtype=torch.uint8, device=device)
     flush_r = torch.zeros(max(2 * l2, 64 << 20) // 8, dtype=torch.int64, device=device)
@@ -651,9 +777,10 @@ def run_gpu(args):
         "config": {"workload": f"config {cfg.index}: {cfg.desc}", "N": cfg.N, "E": cfg.E,
                    "k": cfg.k, "H": cfg.H, "R": cfg.R, "n_nodes": cfg.n_nodes,
                    "placement": placement,
+                   "pass": mode,
                    "gather": ("dispatch_gather_tma (TMA bulk copies)" if LayerBuffers.tma
                               else "dispatch_gather (16-byte vector copies)"),
-                   "step": ("two layers: counts + cross-layer counts (side stream); plan, gather, "
+                   "step": getattr(S, "step_desc", None) or ("two layers: counts + cross-layer counts (side stream); plan, gather, "
                             "combine of layer 1; predict_home; plan, gather, combine of layer 2"
                             if cfg.two_layer else
                             "coact_count (side stream) + two-hop plan (node and rank plans, "
@@ -787,7 +914,24 @@ def _oracle_step_fn(S):
                           tl.layer2.rank_node, cfg.n_nodes, cfg.E, cfg.R, x2, y2, src=home)
         return fn
     L = S.L
+    if isinstance(S, BackwardStep):
+        yb, gob, gsb = o._bits(L.y), o._bits(S.g_out), o._bits(S.g_send)
+        p = o.plan(L.r.ids, cfg.E, L.r.expert_rank, cfg.R, rank_node=L.r.rank_node,
+                   n_nodes=cfg.n_nodes)
+
+        def fn():
+            o.combine_backward(yb, L.r.gates, p["comb_row"], gob)
+            o.gather_backward_f32chain(gsb, p["send_row"])
+        return fn
     xb, yb = o._bits(L.x), o._bits(L.y)
+    if isinstance(S, PreReducedStep):
+        def fn():
+            o.count(L.r.ids, cfg.E)
+            p = o.plan(L.r.ids, cfg.E, L.r.expert_rank, cfg.R, rank_node=L.r.rank_node,
+                       n_nodes=cfg.n_nodes)
+            o.gather(xb, p["row_token"], p["D"])
+            o.combine_prereduced(yb, L.r.gates, p)
+        return fn
     return lambda: _oracle_layer(o, L.r.ids, L.r.gates, L.r.expert_rank, L.r.rank_node,
                                  cfg.n_nodes, cfg.E, cfg.R, xb, yb)
 
@@ -805,7 +949,12 @@ def cpu_baseline(S, seconds: float):
     dt = time.perf_counter() - t0
     return {"value": S.N * n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{n} whole batch(es) of config {S.cfg.index} (N={S.N}) through the "
-                      "single-threaded C oracle: count, plan, gather, float64 combine",
+                      "single-threaded C oracle: " + (
+                          "combine backward (float64 gate gradients) and transposed dispatch"
+                          if isinstance(S, BackwardStep) else
+                          "count, plan, gather, partial rows and their sum"
+                          if isinstance(S, PreReducedStep) else
+                          "count, plan, gather, float64 combine"),
             "host_cpu": _cpu_model(), "host_nproc": os.cpu_count()}
 
 
@@ -871,6 +1020,10 @@ def main():
                     help="auto: the configuration's own (config 3: correlated)")
     ap.add_argument("--gather", default="vector", choices=["vector", "tma"],
                     help="gather implementation: dispatch_gather or dispatch_gather_tma")
+    ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward"],
+                    help="backward: combine_scatter_backward + dispatch_gather_backward")
+    ap.add_argument("--combine", default="direct", choices=["direct", "prereduced"],
+                    help="prereduced: combine_rows per send row, then the transposed dispatch")
     ap.add_argument("--two-hop", action="store_true",
                     help="dispatch in two hops: to nodes, then inside the node to ranks")
     args = ap.parse_args()

@@ -49,6 +49,11 @@ _lib.plan_dispatch.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P,
 _lib.dispatch_gather.argtypes = [_P, _I64, _I64, _P, _I32, _P, _I64, _P, _P]
 _lib.dispatch_gather_tma.argtypes = [_P, _I64, _I64, _P, _I32, _P, _I64, _P, _P]
 _lib.combine_scatter.argtypes = [_P, _I64, _P, _P, _I64, _I32, _I64, _P, _I32, _P, _P]
+_lib.combine_rows.argtypes = [_P, _I64, _P, _P, _I64, _I32, _P, _P, _I64, _P, _I64, _P, _I32, _P,
+                              _P]
+_lib.dispatch_gather_backward.argtypes = [_P, _I64, _P, _I64, _I32, _I64, _P, _I32, _P, _P]
+_lib.combine_scatter_backward.argtypes = [_P, _I64, _P, _P, _I64, _I32, _P, _P, _I64, _P, _P,
+                                          _I64, _P, _P, _P, _P]
 _lib.predict_home_workspace_bytes.argtypes = [_I32, _I32]
 _lib.predict_home_workspace_bytes.restype = _SZ
 _lib.predict_home.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _SZ, _P, _P]
@@ -63,7 +68,8 @@ _lib.forward_gather.argtypes = [_P, _I64, _I64, _P, _I64, _P, _P, _P]
 _lib.plan_dispatch_noalloc.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _P, _P,
                                        _P, _P, _P, _I64, _P, _P, _P, _P, _P, _P]
 for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "dispatch_gather_tma",
-           "combine_scatter", "predict_home",
+           "combine_scatter", "combine_rows", "dispatch_gather_backward",
+           "combine_scatter_backward", "predict_home",
            "coact_place_correlated", "plan_dispatch_noalloc", "coact_compose_map", "plan_forward",
            "forward_gather", "coact_rebalance_ranks", "dispatch_gather_peer",
            "combine_scatter_peer"):
@@ -73,7 +79,8 @@ ABI_SYMBOLS = ("coact_strerror", "coact_abi_version", "coact_count", "plan_dispa
                "plan_dispatch", "dispatch_gather", "dispatch_gather_tma", "combine_scatter",
                "predict_home_workspace_bytes", "predict_home", "coact_place_correlated",
                "plan_dispatch_noalloc", "coact_compose_map", "plan_forward", "forward_gather",
-               "coact_rebalance_ranks", "dispatch_gather_peer", "combine_scatter_peer")
+               "coact_rebalance_ranks", "dispatch_gather_peer", "combine_scatter_peer",
+               "combine_rows", "dispatch_gather_backward", "combine_scatter_backward")
 NOALLOC_MAX_TOKENS = 262144
 
 
@@ -267,6 +274,91 @@ def combine_scatter(y: torch.Tensor, gates: torch.Tensor, comb_row: torch.Tensor
                                 _ptr(out), 1 if out.dtype == torch.float32 else 0,
                                 _ptr(err_flag), _stream(stream)), "combine_scatter")
     return out
+
+
+def _out_dtype(out: torch.Tensor) -> int:
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out must be bfloat16 or float32")
+    return 1 if out.dtype == torch.float32 else 0
+
+
+def combine_rows(y: torch.Tensor, gates: torch.Tensor, comb_row: torch.Tensor,
+                 row_token: torch.Tensor, row_kmask: torch.Tensor, out: torch.Tensor,
+                 n_units: Optional[int] = None, unit_count: Optional[torch.Tensor] = None,
+                 err_flag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out[u] = sum over the slots j of row_kmask[u] (ascending) of
+    gates[t,j] * y[comb_row[t,j]], t = row_token[u] -- over the plan's send rows, the
+    partial rows of the pre-reduced reverse path.  n_units defaults to out.shape[0];
+    unit_count: optional device int32 [1] further bounding it (e.g. the plan's
+    rank_offsets[R:], i.e. D), read by the kernel."""
+    N, k = gates.shape
+    _need(_bits16(y), "y", torch.bfloat16)
+    H = y.shape[1]
+    n = out.shape[0] if n_units is None else int(n_units)
+    _need(gates, "gates", torch.float32)
+    _need(comb_row, "comb_row", torch.int32, (N, k))
+    _need(row_token, "row_token", torch.int32)
+    _need(row_kmask, "row_kmask", torch.uint8)
+    if row_token.numel() < n or row_kmask.numel() < n or out.shape[0] < n or out.shape[1] != H:
+        raise ValueError("row_token, row_kmask and out need n_units rows")
+    _need(out, "out", out.dtype)
+    _need(unit_count, "unit_count", torch.int32, (1,), optional=True)
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.combine_rows(_ptr(y), y.shape[0], _ptr(gates), _ptr(comb_row), N, k, _ptr(row_token),
+                             _ptr(row_kmask), n, _ptr(unit_count), H, _ptr(out), _out_dtype(out),
+                             _ptr(err_flag), _stream(stream)), "combine_rows")
+    return out
+
+
+def dispatch_gather_backward(grad_send: torch.Tensor, send_row: torch.Tensor, grad_x: torch.Tensor,
+                             err_flag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """grad_x[t] = sum over the token's send rows (send_row[t,j] >= 0, ascending j) of
+    grad_send[send_row[t,j]] (fp32 add chain; grad_x bf16 or fp32)."""
+    N, k = send_row.shape
+    _need(_bits16(grad_send), "grad_send", torch.bfloat16)
+    H = grad_send.shape[1]
+    _need(send_row, "send_row", torch.int32, (N, k))
+    _need(grad_x, "grad_x", grad_x.dtype, (N, H))
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.dispatch_gather_backward(_ptr(grad_send), grad_send.shape[0], _ptr(send_row), N, k, H,
+                                         _ptr(grad_x), _out_dtype(grad_x), _ptr(err_flag),
+                                         _stream(stream)), "dispatch_gather_backward")
+    return grad_x
+
+
+def combine_scatter_backward(y: torch.Tensor, gates: torch.Tensor, comb_row: torch.Tensor,
+                             grad_out: torch.Tensor, grad_y: torch.Tensor, grad_gates: torch.Tensor,
+                             row_token: Optional[torch.Tensor] = None,
+                             row_kmask: Optional[torch.Tensor] = None,
+                             unit_count: Optional[torch.Tensor] = None,
+                             err_flag: Optional[torch.Tensor] = None, stream=None):
+    """Gradients of the combine: grad_y[comb_row[t,j]] = bf16(gates[t,j] * grad_out[u]) and
+    grad_gates[t,j] = <grad_out[u], y[comb_row[t,j]]>, u = token t (row_token None) or the
+    units row_token / row_kmask with one grad_out row each (optionally bounded by the
+    device int32 [1] unit_count)."""
+    N, k = gates.shape
+    _need(_bits16(y), "y", torch.bfloat16)
+    H = y.shape[1]
+    _need(gates, "gates", torch.float32)
+    _need(comb_row, "comb_row", torch.int32, (N, k))
+    n = N
+    if row_token is not None:
+        n = grad_out.shape[0]
+        _need(row_token, "row_token", torch.int32)
+        _need(row_kmask, "row_kmask", torch.uint8)
+        if row_token.numel() < n or row_kmask.numel() < n:
+            raise ValueError("row_token and row_kmask need one entry per grad_out row")
+    _need(_bits16(grad_out), "grad_out", torch.bfloat16, (n, H))
+    _need(_bits16(grad_y), "grad_y", torch.bfloat16, tuple(y.shape))
+    _need(grad_gates, "grad_gates", torch.float32, (N, k))
+    _need(unit_count, "unit_count", torch.int32, (1,), optional=True)
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.combine_scatter_backward(_ptr(y), y.shape[0], _ptr(gates), _ptr(comb_row), N, k,
+                                         _ptr(row_token), _ptr(row_kmask), n, _ptr(unit_count),
+                                         _ptr(grad_out), H,
+                                         _ptr(grad_y), _ptr(grad_gates), _ptr(err_flag),
+                                         _stream(stream)), "combine_scatter_backward")
+    return grad_y, grad_gates
 
 
 def predict_workspace_bytes(E1: int, R: int) -> int:

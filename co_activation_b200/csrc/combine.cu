@@ -9,6 +9,14 @@
 // step, explicit __fmaf_rn so the compiler cannot reassociate), then fp32 out or bf16
 // round-to-nearest-even.
 //
+// The same kernel, over other index arrays, gives two more entry points:
+//  * combine_rows -- units instead of tokens: unit u is token row_token[u] restricted to
+//    the slots of row_kmask[u].  Over the plan's send rows this is the partial combine of
+//    the pre-reduced reverse path (one row per (token, rank), summed where the experts ran).
+//  * dispatch_gather_backward -- the transpose of the dispatch: comb_row := send_row
+//    (-1 = no row) and unit weights, grad_x[t] = sum of grad_send over the token's send
+//    rows.  fmaf(1, v, acc) rounds exactly like acc + v, so this is the fp32 add chain.
+//
 // k_combine_v16: one warp per token.  Each lane covers 8 hidden elements per 16-byte
 // column chunk and keeps U chunks x K rows of loads in flight before the FMAs.  The K
 // source rows are scattered over y (expanded receive order), the output row is written
@@ -22,6 +30,7 @@
 namespace coact {
 namespace {
 
+// Unit u = token u with all K slots.  gates == nullptr: every weight is 1.
 template <int K, int U, bool F32>
 __global__ void __launch_bounds__(256)
     k_combine_v16(const uint4 *__restrict__ y, int64_t n_rows, const float *__restrict__ gates,
@@ -39,7 +48,7 @@ __global__ void __launch_bounds__(256)
         float gl = 0.f;
         if (lane < K) {
             rl = __ldg(comb_row + t * K + lane);
-            gl = __ldg(gates + t * K + lane);
+            gl = gates ? __ldg(gates + t * K + lane) : 1.0f;
             if (rl < -1 || (int64_t)rl >= n_rows) flags |= COACT_EFLAG_ROW_RANGE;
             if (rl < 0 || (int64_t)rl >= n_rows) rl = -1;
         }
@@ -96,9 +105,122 @@ __global__ void __launch_bounds__(256)
     raise_flag_warp(err, flags);
 }
 
-template <int K, bool F32>
+// Sparse slots.  UNITS: unit u = (token row_token[u], the slots of row_kmask[u]) -- on the
+// plan's send rows usually one or two of the K slots; otherwise unit u = token u, whose
+// slots without a row (-1, e.g. send_row entries of a rank already seen) are absent.  The
+// unit's live slots are compacted in ascending slot order with a warp ballot and streamed
+// G rows at a time, U column chunks per lane (U*G loads in flight), accumulating in that
+// order: the same fma chain as k_combine_v16, without registers and issue slots for
+// absent slots.
+template <int K, int U, int G, bool F32, bool UNITS>
+__global__ void __launch_bounds__(256)
+    k_combine_units(const uint4 *__restrict__ y, int64_t n_rows, const float *__restrict__ gates,
+                    const int32_t *__restrict__ comb_row, int64_t N,
+                    const int32_t *__restrict__ row_token, const uint8_t *__restrict__ row_kmask,
+                    int64_t n_units, const int32_t *__restrict__ unit_count, int64_t H16,
+                    void *__restrict__ out, int32_t *__restrict__ err) {
+    pdl_wait();
+    pdl_trigger();
+    if (UNITS && unit_count) n_units = min(n_units, (int64_t)max(__ldg(unit_count), 0));
+    const int lane = threadIdx.x & 31;
+    const int64_t gwarp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    int flags = 0;
+    for (int64_t u = gwarp; u < n_units; u += nwarps) {
+        int rl = -1;
+        float gl = 0.f;
+        if (lane < K) {
+            int64_t tok = u;
+            bool on = true;
+            if (UNITS) {
+                tok = __ldg(row_token + u);
+                on = (__ldg(row_kmask + u) >> lane) & 1;
+                if (tok < 0 || tok >= N) {
+                    if (on) flags |= COACT_EFLAG_ROW_RANGE;
+                    on = false;
+                }
+            }
+            if (on) {
+                rl = __ldg(comb_row + tok * K + lane);
+                gl = gates ? __ldg(gates + tok * K + lane) : 1.0f;
+                if (rl < -1 || (int64_t)rl >= n_rows) flags |= COACT_EFLAG_ROW_RANGE;
+                if (rl < 0 || (int64_t)rl >= n_rows) rl = -1;
+            }
+        }
+        unsigned live = __ballot_sync(0xffffffffu, rl >= 0);   // lanes >= K hold -1
+        const int m = __popc(live);
+        int64_t row[K];
+        float g[K];
+#pragma unroll
+        for (int i = 0; i < K; ++i) {      // i-th live slot, ascending
+            const int l = live ? __ffs(live) - 1 : 0;
+            row[i] = __shfl_sync(0xffffffffu, rl, l);
+            g[i] = __shfl_sync(0xffffffffu, gl, l);
+            live &= live - 1;
+        }
+        for (int64_t c0 = 0; c0 < H16; c0 += 32 * U) {
+            float acc[U][8];
+#pragma unroll
+            for (int q = 0; q < U; ++q)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[q][e] = 0.0f;
+#pragma unroll
+            for (int i0 = 0; i0 < K; i0 += G) {
+                if (i0 >= m) break;
+                uint4 v[U][G];
+#pragma unroll
+                for (int q = 0; q < U; ++q) {
+                    const int64_t c = c0 + q * 32 + lane;
+#pragma unroll
+                    for (int gi = 0; gi < G; ++gi)
+                        if (c < H16 && i0 + gi < K && i0 + gi < m)
+                            v[q][gi] = ld_stream(y + row[i0 + gi] * H16 + c);
+                }
+#pragma unroll
+                for (int q = 0; q < U; ++q) {
+#pragma unroll
+                    for (int gi = 0; gi < G; ++gi) {
+                        if (i0 + gi >= K || i0 + gi >= m) continue;
+                        const float gg = g[i0 + gi];
+                        const uint32_t w[4] = {v[q][gi].x, v[q][gi].y, v[q][gi].z, v[q][gi].w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            acc[q][2 * e] = __fmaf_rn(gg, bf16lo(w[e]), acc[q][2 * e]);
+                            acc[q][2 * e + 1] = __fmaf_rn(gg, bf16hi(w[e]), acc[q][2 * e + 1]);
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < U; ++q) {
+                const int64_t c = c0 + q * 32 + lane;
+                if (c >= H16) continue;
+                if (F32) {
+                    float4 *o = reinterpret_cast<float4 *>(out) + (u * H16 + c) * 2;
+                    __stcs(o, make_float4(acc[q][0], acc[q][1], acc[q][2], acc[q][3]));
+                    __stcs(o + 1, make_float4(acc[q][4], acc[q][5], acc[q][6], acc[q][7]));
+                } else {
+                    uint4 p;
+                    uint32_t *pw = &p.x;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat162 h2 =
+                            __floats2bfloat162_rn(acc[q][2 * e], acc[q][2 * e + 1]);
+                        pw[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                    }
+                    st_stream(reinterpret_cast<uint4 *>(out) + u * H16 + c, p);
+                }
+            }
+        }
+    }
+    raise_flag_warp(err, flags);
+}
+
+template <int K, bool F32, bool UNITS, bool SPARSE>
 int launch(const uint16_t *y, int64_t n_rows, const float *gates, const int32_t *comb_row,
-           int64_t N, int64_t H, void *out, int32_t *err, cudaStream_t st, const DeviceInfo &di) {
+           int64_t N, const int32_t *row_token, const uint8_t *row_kmask, int64_t n_units,
+           const int32_t *unit_count, int64_t H, void *out, int32_t *err, cudaStream_t st,
+           const DeviceInfo &di) {
     // column chunks per lane: 8 loads in flight for k <= 2 (U = 4), U = 2 chunks for
     // k >= 3 (6-16 loads).  Measured on B200: U = 2 made k = 6 6% faster and k = 8
     // 0.4% faster than U = 1, while U = 8 made k = 2 1.6% slower than U = 4.
@@ -109,9 +231,45 @@ int launch(const uint16_t *y, int64_t n_rows, const float *gates, const int32_t 
 #endif
     const int64_t H16 = H / 8;
     const int blocks = (int)std::max<int64_t>(
-        1, std::min<int64_t>(ceil_div(N, 8), (int64_t)di.sm_count * 8));
+        1, std::min<int64_t>(ceil_div(n_units, 8), (int64_t)di.sm_count * 8));
+    if (UNITS)
+        return launch_pdl(k_combine_units<K, 4, 2, F32, true>, blocks, 256, 0, st,
+                          reinterpret_cast<const uint4 *>(y), n_rows, gates, comb_row, N, row_token,
+                          row_kmask, n_units, unit_count, H16, out, err);
+    if (SPARSE && K >= 3)      // token rows with absent slots (the transposed dispatch)
+        return launch_pdl(k_combine_units<K, 4, 2, F32, false>, blocks, 256, 0, st,
+                          reinterpret_cast<const uint4 *>(y), n_rows, gates, comb_row, N, nullptr,
+                          nullptr, n_units, nullptr, H16, out, err);
     return launch_pdl(k_combine_v16<K, U, F32>, blocks, 256, 0, st,
                       reinterpret_cast<const uint4 *>(y), n_rows, gates, comb_row, N, H16, out, err);
+}
+
+// k in 1..8 -> the K instantiation
+template <bool UNITS, bool SPARSE>
+int dispatch_k(const uint16_t *y, int64_t n_rows, const float *gates, const int32_t *comb_row,
+               int64_t N, int k, const int32_t *row_token, const uint8_t *row_kmask,
+               int64_t n_units, const int32_t *unit_count, int64_t H, void *out, int out_dtype,
+               int32_t *err, cudaStream_t st, const DeviceInfo &di) {
+#define COACT_COMBINE_CASE(KK)                                                                 \
+    case KK:                                                                                   \
+        return out_dtype ? launch<KK, true, UNITS, SPARSE>(y, n_rows, gates, comb_row, N, row_token,   \
+                                                   row_kmask, n_units, unit_count, H, out, err, \
+                                                   st, di)                                     \
+                         : launch<KK, false, UNITS, SPARSE>(y, n_rows, gates, comb_row, N, row_token,  \
+                                                    row_kmask, n_units, unit_count, H, out,    \
+                                                    err, st, di);
+    switch (k) {
+        COACT_COMBINE_CASE(1)
+        COACT_COMBINE_CASE(2)
+        COACT_COMBINE_CASE(3)
+        COACT_COMBINE_CASE(4)
+        COACT_COMBINE_CASE(5)
+        COACT_COMBINE_CASE(6)
+        COACT_COMBINE_CASE(7)
+        COACT_COMBINE_CASE(8)
+    }
+#undef COACT_COMBINE_CASE
+    return COACT_ERR_UNSUPPORTED;
 }
 
 }  // namespace
@@ -131,21 +289,44 @@ extern "C" int combine_scatter(const uint16_t *y, int64_t n_rows, const float *g
     if (N > (int64_t)INT32_MAX / k) return COACT_ERR_UNSUPPORTED;
     DeviceInfo di;
     if (int s = device_info(&di)) return s;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-#define COACT_COMBINE_CASE(KK)                                                                   \
-    case KK:                                                                                     \
-        return out_dtype ? launch<KK, true>(y, n_rows, gates, comb_row, N, H, out, err_flag, st, di) \
-                         : launch<KK, false>(y, n_rows, gates, comb_row, N, H, out, err_flag, st, di);
-    switch (k) {
-        COACT_COMBINE_CASE(1)
-        COACT_COMBINE_CASE(2)
-        COACT_COMBINE_CASE(3)
-        COACT_COMBINE_CASE(4)
-        COACT_COMBINE_CASE(5)
-        COACT_COMBINE_CASE(6)
-        COACT_COMBINE_CASE(7)
-        COACT_COMBINE_CASE(8)
-    }
-#undef COACT_COMBINE_CASE
-    return COACT_ERR_UNSUPPORTED;
+    return dispatch_k<false, false>(y, n_rows, gates, comb_row, N, k, nullptr, nullptr, N, nullptr, H, out,
+                             out_dtype, err_flag, reinterpret_cast<cudaStream_t>(stream), di);
+}
+
+extern "C" int combine_rows(const uint16_t *y, int64_t n_rows, const float *gates,
+                            const int32_t *comb_row, int64_t N, int k, const int32_t *row_token,
+                            const uint8_t *row_kmask, int64_t n_units, const int32_t *unit_count,
+                            int64_t H, void *out, int out_dtype, int32_t *err_flag,
+                            coact_stream_t stream) {
+    if (N < 0 || H < 0 || n_rows < 0 || n_units < 0) return COACT_ERR_INVALID;
+    if (k < 1 || k > COACT_MAX_K || (out_dtype != 0 && out_dtype != 1)) return COACT_ERR_UNSUPPORTED;
+    if (H % 8 != 0) return COACT_ERR_UNSUPPORTED;
+    if (n_units == 0 || H == 0) return COACT_OK;
+    if (!gates || !row_token || !row_kmask || !out || (N > 0 && !comb_row) || (n_rows > 0 && !y))
+        return COACT_ERR_INVALID;
+    if ((y && !aligned16(y)) || !aligned16(out)) return COACT_ERR_INVALID;
+    if (N > (int64_t)INT32_MAX / k) return COACT_ERR_UNSUPPORTED;
+    DeviceInfo di;
+    if (int s = device_info(&di)) return s;
+    return dispatch_k<true, false>(y, n_rows, gates, comb_row, N, k, row_token, row_kmask, n_units,
+                            unit_count, H, out, out_dtype, err_flag,
+                            reinterpret_cast<cudaStream_t>(stream), di);
+}
+
+extern "C" int dispatch_gather_backward(const uint16_t *grad_send, int64_t n_rows,
+                                        const int32_t *send_row, int64_t N, int k, int64_t H,
+                                        void *grad_x, int out_dtype, int32_t *err_flag,
+                                        coact_stream_t stream) {
+    if (N < 0 || H < 0 || n_rows < 0) return COACT_ERR_INVALID;
+    if (k < 1 || k > COACT_MAX_K || (out_dtype != 0 && out_dtype != 1)) return COACT_ERR_UNSUPPORTED;
+    if (H % 8 != 0) return COACT_ERR_UNSUPPORTED;
+    if (N == 0 || H == 0) return COACT_OK;
+    if (!send_row || !grad_x || (n_rows > 0 && !grad_send)) return COACT_ERR_INVALID;
+    if ((grad_send && !aligned16(grad_send)) || !aligned16(grad_x)) return COACT_ERR_INVALID;
+    if (N > (int64_t)INT32_MAX / k) return COACT_ERR_UNSUPPORTED;
+    DeviceInfo di;
+    if (int s = device_info(&di)) return s;
+    return dispatch_k<false, true>(grad_send, n_rows, nullptr, send_row, N, k, nullptr, nullptr, N, nullptr,
+                             H, grad_x, out_dtype, err_flag, reinterpret_cast<cudaStream_t>(stream),
+                             di);
 }

@@ -14,9 +14,9 @@
 //    CTA; lane 0 streams rows into a ring of shared-memory stages with cp.async.bulk
 //    (global -> shared, completion on an mbarrier), then lanes j < k each issue the
 //    cp.async.bulk store of the staged row to destination j.  No multicast: every load
-//    reads this GPU's own memory once.  Measured on B200 it tied the vector path on 4 KB
-//    rows and lost 4-5% on 8-14 KB rows, so it is not the default; it occupies one warp
-//    and no row registers per CTA, which leaves the SMs to work running alongside.
+//    reads this GPU's own memory once.  Measured on B200 it is 2-5% slower than the
+//    vector path (4-14 KB rows), also next to a concurrent GEMM: the gather is bound by
+//    HBM bandwidth, so its lighter SM footprint does not buy overlap.
 // All mbarrier waits are bounded by a wall-clock limit; on expiry the kernel raises
 // COACT_EFLAG_TIMEOUT, drains its own copies and returns.
 #include <algorithm>

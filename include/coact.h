@@ -181,8 +181,9 @@ int dispatch_gather(const uint16_t *x, int64_t N, int64_t H,
  * per CTA, completion tracked by mbarriers whose waits are bounded by wall clock) and
  * written to every destination with bulk stores.  Same arguments, results and flags as
  * dispatch_gather (plus COACT_EFLAG_TIMEOUT if a bounded wait gives up); rows up to 32 KB
- * (H <= 16384), else COACT_ERR_UNSUPPORTED.  It holds few SM resources, for overlapping
- * the dispatch with other kernels; dispatch_gather is faster when running alone.
+ * (H <= 16384), else COACT_ERR_UNSUPPORTED.  One warp per CTA and no row registers; on
+ * B200 it is 2-3% slower than dispatch_gather, alone and next to a concurrent GEMM alike
+ * (both are bound by HBM bandwidth, not by SM resources).
  */
 int dispatch_gather_tma(const uint16_t *x, int64_t N, int64_t H,
                         const int32_t *send_row, int k,
@@ -206,6 +207,75 @@ int combine_scatter(const uint16_t *y, int64_t n_rows, const float *gates,
                     const int32_t *comb_row, int64_t N, int k, int64_t H,
                     void *out, int out_dtype,
                     int32_t *err_flag, coact_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Backward pass and the pre-reduced reverse path.
+ *
+ * The dispatch copies x[t] to the token's send rows and the combine is a gate-weighted
+ * sum, both linear, so their gradients are the transposed maps over the same plan.  The
+ * reverse direction can also carry one row per (token, rank) -- as Zyphra's dispatcher
+ * sends each token to each GPU once: the rank that ran the experts first sums, with the
+ * gates, the outputs of the slots it served (combine_rows over the plan's send rows), and
+ * the token's rank adds those partial rows (dispatch_gather_backward, the transposed
+ * dispatch), so D rows travel back instead of N*k.
+ *
+ * Units: combine_rows and combine_scatter_backward take an optional unit list.  Unit u
+ * is token row_token[u] restricted to the slots set in row_kmask[u] (e.g. the plan's
+ * row_token / row_kmask over its D send rows); with row_token NULL (backward only) unit u
+ * is token u with all k slots.  A row_token entry outside [0, N) on a unit with slots set
+ * raises COACT_EFLAG_ROW_RANGE and the unit contributes nothing.  unit_count (DEVICE
+ * int32, may be NULL): when given, only units u < min(n_units, *unit_count) are processed
+ * -- e.g. &rank_offsets[R] = D, so that n_units can be the plan's row_capacity and the
+ * call needs no host synchronisation; output rows of the other units are not written.
+ * ------------------------------------------------------------------------------------ */
+
+/*
+ * combine_rows -- the combine over units:
+ *   out[u] = sum over the slots j set in row_kmask[u], ascending, of
+ *            gates[t,j] * y[comb_row[t,j]],   t = row_token[u]
+ * as the fp32 fma chain of combine_scatter (from +0.0f), stored fp32 (out_dtype 1) or
+ * rounded to bf16 nearest-even (out_dtype 0).  out: [n_units, H].  Other arguments and
+ * flags as combine_scatter.
+ */
+int combine_rows(const uint16_t *y, int64_t n_rows, const float *gates,
+                 const int32_t *comb_row, int64_t N, int k,
+                 const int32_t *row_token, const uint8_t *row_kmask, int64_t n_units,
+                 const int32_t *unit_count, int64_t H, void *out, int out_dtype,
+                 int32_t *err_flag, coact_stream_t stream);
+
+/*
+ * dispatch_gather_backward -- the transpose of dispatch_gather:
+ *   grad_x[t] = sum over j ascending with send_row[t,j] >= 0 of grad_send[send_row[t,j]]
+ * per element an fp32 add chain from +0.0f, stored fp32 (out_dtype 1) or rounded to bf16
+ * nearest-even (out_dtype 0).  grad_send: bf16 [n_rows, H] (n_rows = the plan's
+ * row_capacity, rows >= D unread); send_row: the plan's int32 [N, k]; grad_x: [N, H].
+ * It is also the second stage of the pre-reduced combine (grad_send := the partial rows).
+ * A send_row entry below -1 or >= n_rows sets COACT_EFLAG_ROW_RANGE and is skipped.
+ */
+int dispatch_gather_backward(const uint16_t *grad_send, int64_t n_rows,
+                             const int32_t *send_row, int64_t N, int k, int64_t H,
+                             void *grad_x, int out_dtype,
+                             int32_t *err_flag, coact_stream_t stream);
+
+/*
+ * combine_scatter_backward -- gradients of the combine, per unit u (token t) and set slot j:
+ *   grad_y[comb_row[t,j]]  = bf16_rne(gates[t,j] * grad_out[u])   (fp32 product, per element)
+ *   grad_gates[t*k + j]    = sum_h grad_out[u,h] * y[comb_row[t,j],h]   (fp32)
+ * grad_out: bf16 [n_units, H] (token mode: [N, H]); grad_y: bf16 [n_rows, H], rows no
+ * slot names are not written; grad_gates: fp32 [N, k], slots no unit covers are not
+ * written, a covered slot without a row (comb_row -1) gets 0.  The dot product sums, per
+ * lane of a warp, 8*ceil(H/256) products in ascending order with fma, then adds the 32
+ * lane sums by a 5-level butterfly: its error is at most (8*ceil(H/256) + 5) * 2^-24 *
+ * sum_h |grad_out * y| (first order).  n_units and unit_count are ignored when row_token
+ * is NULL.
+ */
+int combine_scatter_backward(const uint16_t *y, int64_t n_rows, const float *gates,
+                             const int32_t *comb_row, int64_t N, int k,
+                             const int32_t *row_token, const uint8_t *row_kmask,
+                             int64_t n_units, const int32_t *unit_count,
+                             const uint16_t *grad_out, int64_t H,
+                             uint16_t *grad_y, float *grad_gates,
+                             int32_t *err_flag, coact_stream_t stream);
 
 /*
  * plan_dispatch_noalloc -- plan_dispatch without a caller-provided workspace.

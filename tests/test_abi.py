@@ -122,6 +122,33 @@ def test_gather_combine_reject_bad_arguments(lib):
     assert c(None, 0, None, None, 0, 2, 16, None, 0, None, None) == 0      # empty
 
 
+def test_backward_entry_points_reject_bad_arguments(lib):
+    b = lib.dispatch_gather_backward
+    b.argtypes = [P, ctypes.c_int64, P, ctypes.c_int64, ctypes.c_int, ctypes.c_int64, P, ctypes.c_int,
+                  P, P]
+    assert b(FAKE, 20, FAKE, 10, 2, 12, FAKE, 0, None, None) == -2     # H % 8 != 0
+    assert b(FAKE, 20, FAKE, 10, 2, 16, FAKE, 2, None, None) == -2     # out dtype
+    assert b(FAKE, 20, None, 10, 2, 16, FAKE, 0, None, None) == -1     # send_row NULL
+    assert b(P(258), 20, FAKE, 10, 2, 16, FAKE, 0, None, None) == -1   # misaligned grad_send
+    assert b(None, 0, None, 0, 2, 16, None, 0, None, None) == 0        # empty
+    c = lib.combine_rows
+    c.argtypes = [P, ctypes.c_int64, P, P, ctypes.c_int64, ctypes.c_int, P, P, ctypes.c_int64, P,
+                  ctypes.c_int64, P, ctypes.c_int, P, P]
+    assert c(FAKE, 20, FAKE, FAKE, 10, 2, None, FAKE, 5, None, 16, FAKE, 0, None, None) == -1
+    assert c(FAKE, 20, FAKE, FAKE, 10, 9, FAKE, FAKE, 5, None, 16, FAKE, 0, None, None) == -2
+    assert c(FAKE, 20, FAKE, FAKE, 10, 2, FAKE, FAKE, 5, None, 16, P(260), 0, None, None) == -1
+    assert c(None, 0, None, None, 0, 2, None, None, 0, None, 16, None, 0, None, None) == 0
+    s = lib.combine_scatter_backward
+    s.argtypes = [P, ctypes.c_int64, P, P, ctypes.c_int64, ctypes.c_int, P, P, ctypes.c_int64, P, P,
+                  ctypes.c_int64, P, P, P, P]
+    assert s(FAKE, 20, FAKE, FAKE, 10, 2, None, None, 0, None, FAKE, 12, FAKE, FAKE, None, None) == -2
+    assert s(FAKE, 20, FAKE, FAKE, 10, 2, None, None, 0, None, FAKE, 16, FAKE, None, None, None) == -1
+    assert s(FAKE, 20, FAKE, FAKE, 10, 2, FAKE, None, 4, None, FAKE, 16, FAKE, FAKE, None, None) == -1
+    assert s(FAKE, 20, FAKE, FAKE, 10, 2, None, None, 0, None, P(264), 16, FAKE, FAKE, None,
+             None) == -1
+    assert s(None, 0, None, None, 0, 2, None, None, 0, None, None, 16, None, None, None, None) == 0
+
+
 def test_predict_rejects_bad_arguments(lib):
     p = lib.predict_home
     p.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int,
