@@ -624,6 +624,8 @@ def make_step(coact, cfg_index: int, seed: int, device, two_hop: bool = False,
 # while these files are byte-identical to the ones the ncu capture was taken on.
 KERNEL_SOURCES = {"k_gather_v16": ("gather.cu", "common.cuh"),
                   "k_gather_bulk": ("gather.cu", "common.cuh"),
+                  "k_combine_units": ("combine.cu", "common.cuh"),
+                  "k_combine_bwd": ("backward.cu", "common.cuh"),
                   "k_combine_v16": ("combine.cu", "common.cuh"),
                   "k_forward_gather": ("twohop.cu", "common.cuh")}
 

@@ -584,17 +584,20 @@ def dispatch_gather_peer(x: torch.Tensor, send_row: torch.Tensor, rank_offsets: 
 
 
 def combine_scatter_peer(y_bases: torch.Tensor, y_row_offset: torch.Tensor,
-                         y_capacity: torch.Tensor, asg_offsets: torch.Tensor, gates: torch.Tensor,
-                         comb_row: torch.Tensor, out: torch.Tensor, H: int,
-                         err_flag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """combine_scatter with each expert output read from the rank that computed it."""
-    N, k = gates.shape
+                         y_capacity: torch.Tensor, asg_offsets: torch.Tensor,
+                         gates: Optional[torch.Tensor], comb_row: torch.Tensor, out: torch.Tensor,
+                         H: int, err_flag: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """combine_scatter with each expert output read from the rank that computed it.  With
+    gates None (unit weights), send_row and rank_offsets: the transposed dispatch reading
+    each row from the rank that holds it."""
+    N, k = comb_row.shape
     R = asg_offsets.shape[0] - 1
     _need(y_bases, "y_bases", torch.int64, (R,))
     _need(y_row_offset, "y_row_offset", torch.int32, (R,))
     _need(y_capacity, "y_capacity", torch.int32, (R,))
     _need(asg_offsets, "asg_offsets", torch.int32)
-    _need(gates, "gates", torch.float32)
+    _need(gates, "gates", torch.float32, (N, k), optional=True)
     _need(comb_row, "comb_row", torch.int32, (N, k))
     if out.dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("out must be bfloat16 or float32")

@@ -15,7 +15,9 @@
 //  * k_gather_peer  -- dispatch_gather with the destination row mapped to
 //                      (rank r, dst_off[r] + d - rank_offsets[r]) in bases[r]
 //  * k_combine_peer -- combine_scatter with each assignment row mapped to
-//                      (rank r, src_off[r] + a - asg_offsets[r]) in bases[r]
+//                      (rank r, src_off[r] + a - asg_offsets[r]) in bases[r]; without
+//                      gates (unit weights) over send_row / rank_offsets it is the
+//                      transposed dispatch reading each row from its rank
 // Plain loads and stores through generic pointers (no TMA multicast, no waits between
 // ranks: ordering across GPUs is the caller's barrier).
 #include <algorithm>
@@ -138,7 +140,7 @@ __global__ void __launch_bounds__(256)
         float gl = 0.f;
         if (lane < K) {
             const int a = __ldg(comb_row + t * K + lane);
-            gl = __ldg(gates + t * K + lane);
+            gl = gates ? __ldg(gates + t * K + lane) : 1.0f;
             if (a >= 0) {
                 if (a >= A) {
                     flags |= COACT_EFLAG_ROW_RANGE;
@@ -252,7 +254,7 @@ extern "C" int combine_scatter_peer(const uint64_t *y_bases, const int32_t *y_ro
         return COACT_ERR_UNSUPPORTED;
     if (H % 8 != 0) return COACT_ERR_UNSUPPORTED;
     if (N == 0 || H == 0) return COACT_OK;
-    if (!y_bases || !y_row_offset || !y_capacity || !asg_offsets || !gates || !comb_row || !out)
+    if (!y_bases || !y_row_offset || !y_capacity || !asg_offsets || !comb_row || !out)
         return COACT_ERR_INVALID;
     if (!aligned16(out)) return COACT_ERR_INVALID;
     if (N > (int64_t)INT32_MAX / k) return COACT_ERR_UNSUPPORTED;

@@ -23,6 +23,21 @@ Per layer, on every rank s of the group (R = group size = number of EP ranks):
        "nccl": all_to_all_single back, combine_scatter
   counts: coact_count locally, then one all_reduce(sum) of pair and loads.
 
+Pre-reduced combine (combine(..., reduce="rows")): the rank that ran the experts first
+sums, with the gates (exchanged with the rows), the outputs of each received row's slots
+-- one bf16 partial row per received row -- and only those travel back: D rows instead of
+N*k.  The token's rank adds them (dispatch_gather_backward, or combine_scatter_peer with
+unit weights reading them in place).
+
+Backward over the same plan (the transposed maps):
+  backward_combine(grad_out): grad_out rows are dispatched like x; where the experts ran,
+      combine_scatter_backward gives grad_y (expanded receive order, for the experts'
+      backward) and one gate gradient per served slot, which travel back to the token's
+      rank (N*k floats in all).
+  backward_dispatch(grad_rows): the experts' input gradients (one row per received row)
+      travel back and are summed per token (dispatch_gather_backward, or the peer combine
+      with unit weights).
+
 Only library kernels touch rows and plans; this module moves split sizes, builds the
 small per-row expert-id metadata the experts need, and calls the collectives.  The
 local steps are an `ops` object (the library by default) so that the exchange logic can
@@ -54,6 +69,19 @@ class Dispatched:
     experts: torch.Tensor       # int32 [n_rows, k]
     counts: torch.Tensor        # int64 [R, R] rows s -> r
     asg: torch.Tensor           # int64 [R, R] assignments s -> r
+    gates: Optional[torch.Tensor] = None   # fp32 [n_rows, k]: gate of each set slot, 0 elsewhere
+
+
+def local_slots(kmask: torch.Tensor, k: int) -> torch.Tensor:
+    """Where each received row's slots sit among the rank's expert outputs (expanded
+    receive order): int32 [n_rows, k], -1 for the slots that are not on this rank."""
+    km = kmask.to(torch.int64)
+    bits = (km[:, None] >> torch.arange(k, device=km.device)) & 1
+    cnt = bits.sum(1)
+    first = torch.cumsum(cnt, 0) - cnt                  # first expanded row of each row
+    before = torch.cumsum(bits, 1) - bits               # set slots before slot j
+    return torch.where(bits.bool(), first[:, None] + before, torch.full_like(bits, -1)).to(
+        torch.int32).contiguous()
 
 
 class LibraryOps:
@@ -76,6 +104,15 @@ class LibraryOps:
 
     def combine(self, y, gates, plan, out):
         return self.c.combine_scatter(y, gates, plan.comb_row, out)
+
+    def combine_local(self, y, gates, comb, out):
+        return self.c.combine_scatter(y, gates, comb, out)
+
+    def gather_backward(self, rows, send_row, out):
+        return self.c.dispatch_gather_backward(rows, send_row, out)
+
+    def combine_backward(self, y, gates, comb, g_out, g_y, g_gates):
+        return self.c.combine_scatter_backward(y, gates, comb, g_out, g_y, g_gates)
 
     def count(self, ids, E, pair, loads):
         self.c.coact_count(ids, E, pair, loads)
@@ -102,8 +139,9 @@ class EPLayer:
             ops = LibraryOps(coact)
         self.ops = ops
         self.peer_capacity = peer_capacity
-        self._peer = None
+        self._sym = {}
         self.plan = None
+        self._d = None
 
     # ------------------------------------------------------------------ statistics
 
@@ -136,12 +174,16 @@ class EPLayer:
         bits = (km[:, None] >> torch.arange(k, device=km.device, dtype=torch.int32)) & 1
         return torch.where(bits.bool(), ids[tok], torch.full_like(ids[tok], -1))
 
-    def dispatch(self, ids: torch.Tensor, x: torch.Tensor) -> Dispatched:
-        """Plan this rank's tokens and deliver every row to its destination rank."""
+    def dispatch(self, ids: torch.Tensor, x: torch.Tensor,
+                 gates: Optional[torch.Tensor] = None) -> Dispatched:
+        """Plan this rank's tokens and deliver every row to its destination rank.  With
+        gates, each row's slot gates travel too (needed by the pre-reduced combine and the
+        backward)."""
         R, me = self.R, self.me
         src = torch.full((ids.shape[0],), me, dtype=torch.int32, device=ids.device)
         plan = self.ops.plan(ids, self.E, self.expert_rank, R, self.rank_node, self.n_nodes, src)
         self.plan = plan
+        self._ids = ids
         C, A = self._count_rows(plan)
         Cl, Al = C.cpu(), A.cpu()
         self._C, self._A = Cl, Al
@@ -149,36 +191,105 @@ class EPLayer:
         n_recv = int(Cl[:, me].sum())
         meta_send = self._row_experts(ids, plan, D)
         kmask_send = plan.row_kmask[:D].to(torch.int32)
-        send_splits = Cl[me].tolist()
-        recv_splits = Cl[:, me].tolist()
-        H = x.shape[1]
+        rows = self._send_rows(x, "recv")
+        experts = self._rows_to_dest(meta_send.to(torch.int32))
+        kmask = self._rows_to_dest(kmask_send)
+        g = None
+        if gates is not None:
+            g = self._rows_to_dest(self._row_gates(gates, plan, D))
+        self._d = Dispatched(rows=rows, kmask=kmask.to(torch.uint8), experts=experts, counts=Cl,
+                             asg=Al, gates=g)
+        return self._d
+
+    def _row_gates(self, gates, plan, D):
+        """Gate of every set slot of each send row (0 elsewhere), fp32 [D, k]."""
+        k = gates.shape[1]
+        tok = plan.row_token[:D].to(torch.int64)
+        km = plan.row_kmask[:D].to(torch.int32)
+        bits = (km[:, None] >> torch.arange(k, device=km.device, dtype=torch.int32)) & 1
+        return torch.where(bits.bool(), gates[tok], torch.zeros_like(gates[tok])).contiguous()
+
+    def _rows_to_dest(self, t: torch.Tensor) -> torch.Tensor:
+        """Per-send-row metadata (first dim D) to the destination ranks (first dim n_recv)."""
+        me, Cl = self.me, self._C
+        out = torch.empty((int(Cl[:, me].sum()),) + tuple(t.shape[1:]), dtype=t.dtype,
+                          device=t.device)
+        dist.all_to_all_single(out, t.contiguous(), Cl[:, me].tolist(), Cl[me].tolist(),
+                               group=self.group)
+        return out
+
+    def _rows_to_source(self, t: torch.Tensor) -> torch.Tensor:
+        """Per-received-row data (first dim n_recv) back to the token's rank, landing in
+        send-row order (first dim D)."""
+        me, Cl = self.me, self._C
+        out = torch.empty((int(Cl[me].sum()),) + tuple(t.shape[1:]), dtype=t.dtype,
+                          device=t.device)
+        if t.dtype == torch.bfloat16:      # raw 32-bit words: exact on any backend
+            dist.all_to_all_single(out.view(torch.int32), t.contiguous().view(torch.int32),
+                                   Cl[me].tolist(), Cl[:, me].tolist(), group=self.group)
+        else:
+            dist.all_to_all_single(out, t.contiguous(), Cl[me].tolist(), Cl[:, me].tolist(),
+                                   group=self.group)
+        return out
+
+    def _send_rows(self, x: torch.Tensor, buf: str) -> torch.Tensor:
+        """Rows of this rank's tokens (bf16 [N, H]) to every destination rank of the current
+        plan; returns the rows this rank receives (source rank, then token order)."""
+        plan, Cl, me = self.plan, self._C, self.me
+        D, n_recv, H = int(Cl[me].sum()), int(Cl[:, me].sum()), x.shape[1]
         if self.transport == "nccl":
             send = self.ops.gather(x, plan)
             rows = torch.empty((n_recv, H), dtype=x.dtype, device=x.device)
             # rows travel as raw 32-bit words (two bf16 each): exact, any backend
             dist.all_to_all_single(rows.view(torch.int32), send[:D].contiguous().view(torch.int32),
-                                   recv_splits, send_splits, group=self.group)
-        else:
-            rows = self._peer_dispatch(x, plan, Cl, Al, n_recv)
-        experts = torch.empty((n_recv, ids.shape[1]), dtype=torch.int32, device=ids.device)
-        dist.all_to_all_single(experts, meta_send.to(torch.int32).contiguous(), recv_splits,
-                               send_splits, group=self.group)
-        kmask = torch.empty((n_recv,), dtype=torch.int32, device=ids.device)
-        dist.all_to_all_single(kmask, kmask_send.contiguous(), recv_splits, send_splits,
-                               group=self.group)
-        return Dispatched(rows=rows, kmask=kmask.to(torch.uint8), experts=experts, counts=Cl,
-                          asg=Al)
+                                   Cl[:, me].tolist(), Cl[me].tolist(), group=self.group)
+            return rows
+        import co_activation_b200 as coact
+        sb = self._symmetric(buf, int(Cl.sum(dim=0).max()), H, x.dtype, x.device)
+        off = exclusive_offsets(Cl)[me].to(torch.int32).to(x.device)
+        coact.dispatch_gather_peer(x, plan.send_row, plan.rank_offsets, sb["ptrs"], off, sb["cap"])
+        sb["handle"].barrier()
+        return sb["t"][:n_recv]
+
+    def _sum_back(self, rows: torch.Tensor, buf: str, out: torch.Tensor) -> torch.Tensor:
+        """Rows held per received row (n_recv of them, bf16) back to the token's rank and
+        summed per token over its send rows: out[t] = sum of the rows of t's send rows."""
+        plan, Cl, me = self.plan, self._C, self.me
+        if self.transport == "nccl":
+            back = self._rows_to_source(rows)
+            return self.ops.gather_backward(back, plan.send_row, out)
+        import co_activation_b200 as coact
+        H = rows.shape[1]
+        sb = self._symmetric(buf, int(Cl.sum(dim=0).max()), H, rows.dtype, rows.device)
+        sb["t"][:rows.shape[0]].copy_(rows)
+        sb["handle"].barrier()
+        off = exclusive_offsets(Cl)[me].to(torch.int32).to(rows.device)
+        coact.combine_scatter_peer(sb["ptrs"], off, sb["cap"], plan.rank_offsets, None,
+                                   plan.send_row, out, H)
+        sb["handle"].barrier()
+        return out
 
     def combine(self, y_recv: torch.Tensor, gates: torch.Tensor,
-                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                out: Optional[torch.Tensor] = None, reduce: str = "expanded") -> torch.Tensor:
         """Bring the expert outputs (expanded receive order on this rank) back to their
-        source ranks and combine them in token order."""
+        source ranks and combine them in token order.  reduce="rows": pre-reduce where the
+        experts ran (one bf16 partial row per received row; needs dispatch(..., gates))."""
         me, plan = self.me, self.plan
         Al = self._A
         H = y_recv.shape[1]
         N = gates.shape[0]
         if out is None:
             out = torch.empty((N, H), dtype=y_recv.dtype, device=y_recv.device)
+        if reduce == "rows":
+            d = self._d
+            if d is None or d.gates is None:
+                raise ValueError("reduce='rows' needs dispatch(..., gates=...) first")
+            k = gates.shape[1]
+            pre = torch.empty((d.rows.shape[0], H), dtype=torch.bfloat16, device=y_recv.device)
+            self.ops.combine_local(y_recv, d.gates, local_slots(d.kmask, k), pre)
+            return self._sum_back(pre, "pre", out)
+        if reduce != "expanded":
+            raise ValueError("reduce must be 'expanded' or 'rows'")
         if self.transport == "nccl":
             back = torch.empty((int(Al[me].sum()), H), dtype=y_recv.dtype, device=y_recv.device)
             dist.all_to_all_single(back.view(torch.int32), y_recv.contiguous().view(torch.int32),
@@ -186,52 +297,71 @@ class EPLayer:
             return self.ops.combine(back, gates, plan, out)
         return self._peer_combine(y_recv, gates, out)
 
+    # ------------------------------------------------------------------ backward
+
+    def backward_combine(self, grad_out: torch.Tensor, y_recv: torch.Tensor):
+        """Gradients of combine() (either reduce mode; same function) for grad_out [N, H]
+        (bf16, this rank's tokens).  Returns (grad_y, grad_gates): grad_y bf16 in expanded
+        receive order on this rank (for the experts' backward), grad_gates fp32 [N, k] of
+        this rank's tokens.  Needs dispatch(..., gates=...) first."""
+        d, plan, me = self._d, self.plan, self.me
+        if d is None or d.gates is None:
+            raise ValueError("backward_combine needs dispatch(..., gates=...) first")
+        N, k = self._ids.shape
+        g_recv = self._send_rows(grad_out, "grad")
+        grad_y = torch.empty_like(y_recv)
+        gg = torch.zeros((d.rows.shape[0], k), dtype=torch.float32, device=y_recv.device)
+        self.ops.combine_backward(y_recv, d.gates, local_slots(d.kmask, k), g_recv, grad_y, gg)
+        back = self._rows_to_source(gg)                      # [D, k], send-row order
+        D = back.shape[0]
+        tok = plan.row_token[:D].to(torch.int64)
+        km = plan.row_kmask[:D].to(torch.int64)
+        bits = ((km[:, None] >> torch.arange(k, device=km.device)) & 1).bool()
+        grad_gates = torch.zeros((N, k), dtype=torch.float32, device=y_recv.device)
+        cols = torch.arange(k, device=km.device).expand(D, k)
+        grad_gates[tok[:, None].expand(D, k)[bits], cols[bits]] = back[bits]
+        return grad_y, grad_gates
+
+    def backward_dispatch(self, grad_rows: torch.Tensor,
+                          out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Gradient of dispatch(): grad_rows bf16 [n_recv, H] (one per received row) back to
+        the token's rank, summed per token: grad_x [N, H] (bf16 or fp32 `out`)."""
+        N = self._ids.shape[0]
+        if out is None:
+            out = torch.empty((N, grad_rows.shape[1]), dtype=grad_rows.dtype,
+                              device=grad_rows.device)
+        return self._sum_back(grad_rows, "gback", out)
+
     # ------------------------------------------------------------------ peer transport
 
-    def _peer_buffers(self, H, dtype, device, rows, outs):
-        """Symmetric receive / output buffers on every rank and their device addresses
-        (every rank asks for the same sizes: the group-wide maxima)."""
+    def _symmetric(self, name, rows, H, dtype, device):
+        """A named symmetric-memory buffer [>= rows, H] on every rank (all ranks ask for the
+        same size: the group-wide maximum) and its per-rank device addresses."""
         import torch.distributed._symmetric_memory as symm
-        if (self._peer is None or self._peer["rows"] < rows or self._peer["outs"] < outs
-                or self._peer["H"] != H):
-            cap = max(rows, self.peer_capacity or 0)
-            ocap = max(outs, 8 * (self.peer_capacity or 0))
-            recv = symm.empty((cap, H), dtype=dtype, device=device)
-            yout = symm.empty((ocap, H), dtype=dtype, device=device)
-            h_recv = symm.rendezvous(recv, self.group)
-            h_y = symm.rendezvous(yout, self.group)
-            self._peer = {"rows": cap, "outs": ocap, "H": H, "recv": recv, "y": yout,
-                          "h_recv": h_recv,
-                          "h_y": h_y,
-                          "recv_ptrs": torch.tensor(list(h_recv.buffer_ptrs), dtype=torch.int64,
-                                                    device=device),
-                          "y_ptrs": torch.tensor(list(h_y.buffer_ptrs), dtype=torch.int64,
-                                                 device=device)}
-        return self._peer
-
-    def _peer_dispatch(self, x, plan, Cl, Al, n_recv):
-        import co_activation_b200 as coact
-        cap, ocap = int(Cl.sum(dim=0).max()), int(Al.sum(dim=0).max())
-        pb = self._peer_buffers(x.shape[1], x.dtype, x.device, cap, ocap)
-        off = exclusive_offsets(Cl)[self.me].to(torch.int32).to(x.device)
-        capv = torch.full((self.R,), pb["rows"], dtype=torch.int32, device=x.device)
-        coact.dispatch_gather_peer(x, plan.send_row, plan.rank_offsets, pb["recv_ptrs"], off, capv)
-        pb["h_recv"].barrier()
-        return pb["recv"][:n_recv]
+        sb = self._sym.get(name)
+        if sb is None or sb["t"].shape[0] < rows or sb["t"].shape[1] != H or sb["t"].dtype != dtype:
+            cap = max(rows, self.peer_capacity or 0, 1)
+            t = symm.empty((cap, H), dtype=dtype, device=device)
+            h = symm.rendezvous(t, self.group)
+            sb = {"t": t, "handle": h,
+                  "ptrs": torch.tensor(list(h.buffer_ptrs), dtype=torch.int64, device=device),
+                  "cap": torch.full((self.R,), cap, dtype=torch.int32, device=device)}
+            self._sym[name] = sb
+        return sb
 
     def _peer_combine(self, y_recv, gates, out):
         import co_activation_b200 as coact
-        pb = self._peer
+        Al, me = self._A, self.me
+        H = y_recv.shape[1]
+        cap = max(int(Al.sum(dim=0).max()), 8 * (self.peer_capacity or 0))
+        sb = self._symmetric("y", cap, H, y_recv.dtype, y_recv.device)
         n = y_recv.shape[0]
-        if n > pb["y"].shape[0]:
-            raise ValueError("expert outputs exceed the symmetric output buffer")
-        pb["y"][:n].copy_(y_recv)
-        pb["h_y"].barrier()
-        off = exclusive_offsets(self._A)[self.me].to(torch.int32).to(out.device)
-        capv = torch.full((self.R,), pb["y"].shape[0], dtype=torch.int32, device=out.device)
-        coact.combine_scatter_peer(pb["y_ptrs"], off, capv, self.plan.asg_offsets, gates,
-                                   self.plan.comb_row, out, y_recv.shape[1])
-        pb["h_y"].barrier()
+        sb["t"][:n].copy_(y_recv)
+        sb["handle"].barrier()
+        off = exclusive_offsets(Al)[me].to(torch.int32).to(out.device)
+        coact.combine_scatter_peer(sb["ptrs"], off, sb["cap"], self.plan.asg_offsets, gates,
+                                   self.plan.comb_row, out, H)
+        sb["handle"].barrier()
         return out
 
 

@@ -378,7 +378,10 @@ int dispatch_gather_peer(const uint16_t *x, int64_t N, int64_t H, const int32_t 
  * computed them: assignment row a of rank r's segment (asg_offsets [R+1] of this source's
  * plan) is read at y_bases[r] + (y_row_offset[r] + a - asg_offsets[r]) * H.  Same fp32
  * fma chain, output types and flags as combine_scatter; y_bases / y_row_offset /
- * y_capacity: DEVICE arrays as above.
+ * y_capacity: DEVICE arrays as above.  gates may be NULL (every weight 1): with send_row
+ * for comb_row and rank_offsets for asg_offsets this is dispatch_gather_backward reading
+ * each row from the rank that holds it -- the way back of the pre-reduced combine (the
+ * partial rows) and of the dispatch's gradient.  A -1 entry is skipped silently.
  */
 int combine_scatter_peer(const uint64_t *y_bases, const int32_t *y_row_offset,
                          const int32_t *y_capacity, const int32_t *asg_offsets, int R,

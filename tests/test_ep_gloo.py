@@ -59,6 +59,26 @@ class OracleOps:
         pair += torch.from_numpy(p)
         loads += torch.from_numpy(l)
 
+    def _store(self, out, f32):
+        if out.dtype == torch.bfloat16:
+            out.view(torch.int16).copy_(torch.from_numpy(self.o.bf16_rne(f32).view(np.int16)))
+        else:
+            out.copy_(torch.from_numpy(f32))
+        return out
+
+    def combine_local(self, y, gates, comb, out):
+        return self._store(out, self.o.combine_f32chain(self.o._bits(y), gates.numpy(), comb.numpy()))
+
+    def gather_backward(self, rows, send_row, out):
+        return self._store(out, self.o.gather_backward_f32chain(self.o._bits(rows), send_row.numpy()))
+
+    def combine_backward(self, y, gates, comb, g_out, g_y, g_gates):
+        gy, gg, _ = self.o.combine_backward(self.o._bits(y), gates.numpy(), comb.numpy(),
+                                            self.o._bits(g_out))
+        g_y.view(torch.int16).copy_(torch.from_numpy(gy.view(np.int16)))
+        g_gates.copy_(torch.from_numpy(gg.astype(np.float32)))
+        return g_y, g_gates
+
 
 def _worker(rank, world, port, cfg_spec, out):
     sys.path.insert(0, ROOT)
@@ -127,3 +147,75 @@ def test_ep_exchange_matches_single_process_plan(world, spec):
         assert out_ok, f"rank {r}: combined rows differ"
         assert cnt_ok, f"rank {r}: global counts differ"
         assert n > 0
+
+
+def _worker_backward(rank, world, port, cfg_spec, out):
+    """Pre-reduced combine and the backward pass across gloo ranks against the oracle's
+    single-process results over all tokens."""
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        import workload
+        import co_activation_b200.ep as ep
+        N, E, k, H = cfg_spec
+        cfg = workload.CONFIGS[0].with_(N=N, E=E, k=k, H=H, R=world, n_nodes=1)
+        r = workload.make_routing(cfg)
+        lo, hi = rank * N // world, (rank + 1) * N // world
+        ids = torch.from_numpy(r.ids[lo:hi].copy())
+        gates = torch.from_numpy(r.gates[lo:hi].copy())
+        x = workload.fill_bf16(N, H, 0, 1)
+        g_out = workload.fill_bf16(N, H, 0, 6)
+        layer = ep.EPLayer(dist.group.WORLD, E, torch.from_numpy(r.expert_rank), transport="nccl",
+                           ops=OracleOps(oracle))
+        got = layer.dispatch(ids, x[lo:hi].contiguous(), gates=gates)
+        y = workload.fill_bf16(int(got.asg[:, rank].sum()), H, rank, 2)   # this rank's outputs
+        pre_out = layer.combine(y, gates, torch.empty((hi - lo, H), dtype=torch.float32),
+                                reduce="rows")
+        grad_y, grad_gates = layer.backward_combine(g_out[lo:hi].contiguous(), y)
+        src = np.repeat(np.arange(world), np.diff([i * N // world for i in range(world + 1)]))
+        full = oracle.plan(r.ids, E, r.expert_rank, world, src_rank=src.astype(np.int32))
+        ro, ao = full["rank_offsets"], full["asg_offsets"]
+        G = workload.fill_bf16(int(ro[-1]), H, 0, 7)                     # input-gradient rows
+        grad_x = layer.backward_dispatch(G[ro[rank]:ro[rank + 1]].contiguous(),
+                                         torch.empty((hi - lo, H), dtype=torch.float32))
+        # single-process expectations: every rank's outputs at its assignment segment
+        ys = [oracle._bits(workload.fill_bf16(int(ao[q + 1] - ao[q]), H, q, 2)) for q in range(world)]
+        y_full = np.concatenate(ys)
+        seg = slice(ro[rank], ro[rank + 1])
+        tok, km = full["row_token"][seg], full["row_kmask"][seg]
+        want_g = np.where((km[:, None] >> np.arange(k)) & 1, r.gates[tok], 0).astype(np.float32)
+        _, pre_want = oracle.combine_prereduced(y_full, r.gates, full)
+        gy_w, gg_w, _ = oracle.combine_backward(y_full, r.gates, full["comb_row"], oracle._bits(g_out))
+        gx_w = oracle.gather_backward_f32chain(oracle._bits(G), full["send_row"])
+        out[rank] = (
+            np.array_equal(got.gates.numpy().view(np.uint32), want_g.view(np.uint32)),
+            np.array_equal(pre_out.numpy().view(np.uint32), pre_want[lo:hi].view(np.uint32)),
+            np.array_equal(oracle._bits(grad_y), gy_w[ao[rank]:ao[rank + 1]]),
+            np.array_equal(grad_gates.numpy(), gg_w[lo:hi].astype(np.float32)),
+            np.array_equal(grad_x.numpy().view(np.uint32), gx_w[lo:hi].view(np.uint32)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,spec", [(2, (2048, 8, 2, 32)), (3, (999, 12, 4, 24))])
+def test_ep_prereduced_and_backward_match_single_process(world, spec):
+    ctx = mp.get_context("spawn")
+    manager = ctx.Manager()
+    out = manager.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_backward, args=(r, world, port, spec, out))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    names = ("exchanged gates", "pre-reduced combine", "grad_y", "grad_gates", "grad_x")
+    for r in range(world):
+        for name, ok in zip(names, out[r]):
+            assert ok, f"rank {r}: {name} differs from the single-process oracle"

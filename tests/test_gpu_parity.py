@@ -556,6 +556,57 @@ def test_peer_dispatch_combine_emulated(coact, cfg):
     assert err.item() == 0
 
 
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_peer_sum_back_emulated(coact, cfg):
+    """The way back of the pre-reduced combine and of the dispatch's gradient over peers,
+    on one GPU: rows held per received row in R per-rank buffers (the rank-r segments of the
+    single-GPU send layout) are read in place by combine_scatter_peer with unit weights over
+    each source's send_row / rank_offsets.  Every source's result must equal the
+    transposed dispatch of the single-GPU layout for its tokens, bit for bit; and with the
+    partial rows of combine_rows as the held rows, the pre-reduced combine."""
+    import co_activation_b200.ep as ep
+    r = workload.make_routing(cfg)
+    c = r.cfg
+    N, k, E, R, H = r.N, r.k, c.E, c.R, min(c.H, 1024)
+    S = R
+    blocks = [(s * N // S, (s + 1) * N // S) for s in range(S)]
+    er = cuda(r.expert_rank, np.int32)
+    plans = []
+    for s, (lo, hi) in enumerate(blocks):
+        p = coact.alloc_plan(hi - lo, k, E, R, DEV)
+        coact.plan_dispatch(cuda(r.ids[lo:hi]), E, er, R, p,
+                            src_rank=torch.full((hi - lo,), s, dtype=torch.int32, device=DEV))
+        plans.append(p)
+    C = torch.stack([p.rank_counts.to(torch.int64) for p in plans]).cpu()
+    offC = ep.exclusive_offsets(C)
+    src = np.concatenate([np.full(hi - lo, s, np.int32) for s, (lo, hi) in enumerate(blocks)])
+    full = oracle.plan(r.ids, E, r.expert_rank, R, src_rank=src)
+    ro = full["rank_offsets"]
+    # held rows: single-GPU send-layout rows, split into per-rank buffers
+    G = workload.fill_bf16(int(ro[-1]), H, r.seed, 7, device=DEV)
+    y = workload.fill_bf16(N * k, H, r.seed, Y_STREAM, device=DEV)
+    fp = coact.alloc_plan(N, k, E, R, DEV)
+    coact.plan_dispatch(cuda(r.ids), E, er, R, fp, src_rank=cuda(src))
+    pre = torch.empty((int(ro[-1]), H), dtype=torch.bfloat16, device=DEV)
+    coact.combine_rows(y, cuda(r.gates), fp.comb_row, fp.row_token, fp.row_kmask, pre)
+    torch.cuda.synchronize()
+    want_g = oracle.gather_backward_f32chain(host_bits(G), full["send_row"])
+    _, want_pre = oracle.combine_prereduced(host_bits(y), r.gates, full)
+    err = zero_flag()
+    for held, want in ((G, want_g), (pre, want_pre)):
+        bufs = [held[ro[q]:ro[q + 1]].clone() for q in range(R)]
+        bases = torch.tensor([t.data_ptr() for t in bufs], dtype=torch.int64, device=DEV)
+        caps = torch.tensor([t.shape[0] for t in bufs], dtype=torch.int32, device=DEV)
+        for s, (lo, hi) in enumerate(blocks):
+            out = torch.empty((hi - lo, H), dtype=torch.float32, device=DEV)
+            coact.combine_scatter_peer(bases, offC[s].to(torch.int32).to(DEV), caps,
+                                       plans[s].rank_offsets, None, plans[s].send_row, out, H,
+                                       err_flag=err)
+            torch.cuda.synchronize()
+            assert np.array_equal(out.cpu().numpy().view(np.uint32), want[lo:hi].view(np.uint32)), s
+    assert err.item() == 0
+
+
 def test_peer_row_range_flag(coact):
     r = workload.make_routing(0)
     c = r.cfg
