@@ -158,7 +158,12 @@ def test_plan_variants(coact, variant):
 
 @pytest.mark.parametrize("N,E,k,R,nodes", [(1, 8, 2, 4, 1), (31, 16, 3, 4, 2), (257, 64, 8, 64, 8),
                                            (1000, 128, 6, 16, 4), (4096, 1024, 8, 64, 8),
-                                           (513, 12, 1, 3, 1)])
+                                           (513, 12, 1, 3, 1),
+                                           # the one-cluster planner's edges: odd cluster
+                                           # sizes, the largest batch it takes, the first
+                                           # one it leaves to the multi-launch planner
+                                           (8193, 64, 2, 8, 1), (12289, 256, 8, 64, 8),
+                                           (32768, 64, 4, 32, 4), (32769, 64, 4, 32, 4)])
 def test_plan_shapes(coact, N, E, k, R, nodes):
     rng = np.random.default_rng(N * 7 + k)
     cfg = workload.CONFIGS[0].with_(N=N, E=E, k=k, R=R, n_nodes=nodes)
