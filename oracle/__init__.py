@@ -76,6 +76,8 @@ def _get():
             _lib.oracle_combine_units_f32chain.restype = None
             _lib.oracle_combine_backward.argtypes = [P, I64, P, P, I32, P, P, I64, I64, P, P, P, P]
             _lib.oracle_combine_backward.restype = None
+            _lib.oracle_shuffle_reduce_f32chain.argtypes = [P, I32, I64, I64, P, I64, P]
+            _lib.oracle_shuffle_reduce_f32chain.restype = None
         return _lib
 
 
@@ -385,3 +387,27 @@ def combine_prereduced(y, gates, plan_: dict):
     pre = bf16_rne(combine_units_f32chain(y, gates, plan_["comb_row"], plan_["row_token"],
                                           plan_["row_kmask"], D))
     return pre, gather_backward_f32chain(pre, plan_["send_row"])
+
+
+# ----------------------------------------------------------------------------- token shuffling
+
+
+def shuffle_order(home, R: int) -> dict:
+    """The shuffle's permutation: the dispatch plan of every token to its predicted home
+    rank alone (k = 1, identity expert -> rank map): row_token lists the tokens grouped by
+    home rank in ascending token order, rank_offsets delimits the ranks' segments."""
+    if R < 2:
+        raise ValueError("token shuffling needs at least two ranks")
+    home = _c(home, np.int32)
+    return plan(home.reshape(-1, 1), R, np.arange(R, dtype=np.int32), R)
+
+
+def shuffle_reduce_f32chain(parts, row_token) -> np.ndarray:
+    """out[i] = sum over q of parts[q][row_token[i]], fp32 add chain in rank order
+    ([n_out, H] float32); parts: bf16 bits [P, N, H]."""
+    pb = _bits(parts)
+    Pn, N, H = pb.shape
+    rt = _c(row_token, np.int32)
+    out = np.zeros((len(rt), H), np.float32)
+    _get().oracle_shuffle_reduce_f32chain(_p(pb), Pn, N, H, _p(rt), len(rt), _p(out))
+    return out

@@ -629,3 +629,31 @@ void oracle_combine_backward(const uint16_t *y, int64_t n_rows, const float *gat
         }
     }
 }
+
+/* ------------------------------------------------------------------------------------
+ * Token shuffling fused into the post-attention reduce-scatter.
+ *
+ * [Zyphra] under sequence parallelism each token is moved, during the reduce-scatter
+ * that follows attention, to the GPU predicted to hold its next-layer experts.  Reading
+ * taken: the reduce-scatter runs over the group whose P ranks each hold a partial
+ * attention output for all N tokens; rank r receives the tokens whose predicted home is
+ * r, in ascending token order (the stable grouping the dispatch plan gives with k = 1),
+ * each row the sum of the P partial rows, added in rank order q = 0..P-1 in fp32 from +0.
+ * ------------------------------------------------------------------------------------ */
+
+/*
+ * out[i] = sum over q = 0..P-1 of parts[q][row_token[i]] (fp32 add chain, caller rounds);
+ * parts: P consecutive bf16 [N, H] blocks.  A row_token outside [0, N) gives a zero row.
+ */
+void oracle_shuffle_reduce_f32chain(const uint16_t *parts, int P, int64_t N, int64_t H,
+                                    const int32_t *row_token, int64_t n_out, float *out) {
+    for (int64_t i = 0; i < n_out; ++i) {
+        int64_t t = row_token[i];
+        for (int64_t h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            if (t >= 0 && t < N)
+                for (int q = 0; q < P; ++q) acc = acc + bf16_to_f32(parts[((int64_t)q * N + t) * H + h]);
+            out[i * H + h] = acc;
+        }
+    }
+}
