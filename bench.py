@@ -578,10 +578,82 @@ class BackwardStep:
                 "err_flag": int(self.L.err.item())}
 
 
+class ShuffleStep:
+    """Config 4's token shuffling fused into the post-attention reduce-scatter: predict
+    each token's layer-2 home rank from the calibration counts C12, plan the permutation
+    (every token to its home rank alone), and reduce the R ranks' partial attention
+    outputs (synthetic, bf16 [N, H] each) into the shuffled rows -- all R emulated ranks'
+    segments in one launch on this GPU."""
+    n_events = 4
+    phases = {"predict_home": (0, 1), "shuffle_plan": (1, 2), "reduce_scatter": (2, 3)}
+    step_desc = ("token shuffle: predict_home (layer-1 picks x calibration C12) + shuffle plan "
+                 "(plan_dispatch, k = 1) + shuffle_reduce_scatter over R partial attention "
+                 "outputs (bf16 out)")
+    e2e_skip = "not measured for --shuffle: the R partial outputs are R x N x H x 2 bytes per step"
+
+    def __init__(self, coact, tl: workload.TwoLayer, device):
+        self.coact, self.tl = coact, tl
+        self.cfg = c = tl.layer1.cfg
+        self.N = c.N
+        to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        self.ids1 = to(tl.layer1.ids)
+        self.er2 = to(tl.layer2.expert_rank.astype(np.int32))
+        self.C12 = torch.zeros((c.E, c.E), dtype=torch.int64, device=device)
+        coact.coact_count(to(tl.calib1), c.E, self.C12, ids2=to(tl.calib2), E2=c.E)
+        self.home = torch.empty(c.N, dtype=torch.int32, device=device)
+        self.pws = torch.empty(max(coact.predict_workspace_bytes(c.E, c.R), 16), dtype=torch.uint8,
+                               device=device)
+        self.sp = coact.alloc_plan(c.N, 1, c.R, c.R, device, with_rank_mask=False,
+                                   with_src_dst=False)
+        self.parts = [workload.fill_bf16(c.N, c.H, tl.layer1.seed, 100 + q, device=device)
+                      for q in range(c.R)]
+        self.bases = torch.tensor([p.data_ptr() for p in self.parts], dtype=torch.int64,
+                                  device=device)
+        self.out = torch.empty((c.N, c.H), dtype=torch.bfloat16, device=device)
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.kernels_per_step = 2 + plan_launches(c.R, c.N) + 1
+
+    def step(self, ev=None):
+        c, co = self.cfg, self.coact
+        if ev: ev[0].record()
+        co.predict_home(self.ids1, c.E, self.C12, self.er2, c.R, self.home, workspace=self.pws,
+                        err_flag=self.err)
+        if ev: ev[1].record()
+        co.shuffle_plan(self.home, c.R, plan=self.sp, err_flag=self.err)
+        if ev: ev[2].record()
+        co.shuffle_reduce_scatter(self.bases, c.N, self.sp.row_token, self.out, err_flag=self.err)
+        if ev: ev[3].record()
+
+    def roofline_parts(self):
+        c = self.cfg
+        return [("reduce_scatter", "k_shuffle_reduce",
+                 c.R * c.N * c.H * 2 + c.N * c.H * 2 + c.N * 4)]
+
+    def summary(self):
+        c, co, dev = self.cfg, self.coact, self.home.device
+        nk = c.N * c.k
+        to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+        ids2, rn = to(self.tl.layer2.ids), to(self.tl.layer2.rank_node.astype(np.int32))
+        share = {}
+        for name, src in (("predicted_home", self.home), ("contiguous_home", None)):
+            p = co.alloc_plan(c.N, c.k, c.E, c.R, dev)
+            co.plan_dispatch(ids2, c.E, self.er2, c.R, p, rank_node=rn, n_nodes=c.n_nodes,
+                             src_rank=src)
+            share[f"local_served_share_{name}"] = int(p.stats[5].item()) / nk
+        counts = self.sp.rank_counts.cpu().numpy()
+        return {**share, "tokens_per_rank_max_over_mean": float(counts.max() / counts.mean()),
+                "err_flag": int(self.err.item())}
+
+
 def make_step(coact, cfg_index: int, seed: int, device, two_hop: bool = False,
               placement_kind: str = "auto", mode: str = "forward"):
     """The step object for a configuration, plus a description of its placement."""
     cfg = workload.CONFIGS[cfg_index]
+    if mode == "shuffle":
+        if not cfg.two_layer:
+            raise SystemExit("--shuffle needs the two-layer configuration (4)")
+        return ShuffleStep(coact, workload.make_two_layer(cfg, seed=seed), device), \
+            "contiguous; tokens shuffled to the predicted layer-2 home rank"
     if cfg.two_layer:
         if mode != "forward":
             raise SystemExit("--pass backward / --combine prereduced need a one-layer configuration")
@@ -623,6 +695,7 @@ def make_step(coact, cfg_index: int, seed: int, device, two_hop: bool = False,
 # CUDA sources of each HBM-bound kernel: a committed DRAM-traffic figure is reported only
 # while these files are byte-identical to the ones the ncu capture was taken on.
 KERNEL_SOURCES = {"k_gather_v16": ("gather.cu", "common.cuh"),
+                  "k_shuffle_reduce": ("shuffle.cu", "common.cuh"),
                   "k_gather_bulk": ("gather.cu", "common.cuh"),
                   "k_combine_units": ("combine.cu", "common.cuh"),
                   "k_combine_bwd": ("backward.cu", "common.cuh"),
@@ -668,7 +741,7 @@ def run_gpu(args):
 
     cfg = workload.CONFIGS[args.config]
     LayerBuffers.tma = args.gather == "tma"
-    mode = "backward" if args.pass_ == "backward" else (
+    mode = "shuffle" if args.shuffle else "backward" if args.pass_ == "backward" else (
         "prereduced" if args.combine == "prereduced" else "forward")
     S, placement = make_step(coact, args.config, rank_seed(args.seed, rank), device, args.two_hop,
                              args.placement, mode)
@@ -769,7 +842,8 @@ def run_gpu(args):
     gb_dc = dc_bytes / (dc_ms / 1e3) / 1e9
     dom = max(parts, key=lambda p: p[3])
     dom_gbs = dom[2] / (dom[3] / 1e3) / 1e9
-    e2e = run_e2e(coact, S, args, world, device)
+    e2e = {"value": None, "note": S.e2e_skip} if hasattr(S, "e2e_skip") else \
+        run_e2e(coact, S, args, world, device)
 
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -915,6 +989,20 @@ def _oracle_step_fn(S):
             _oracle_layer(o, tl.layer2.ids, tl.layer2.gates, tl.layer2.expert_rank,
                           tl.layer2.rank_node, cfg.n_nodes, cfg.E, cfg.R, x2, y2, src=home)
         return fn
+    if isinstance(S, ShuffleStep):
+        # a bounded sample: the first 4096 tokens' predicted homes and partial rows
+        tl, n = S.tl, min(S.N, 4096)
+        C12 = S.C12.cpu().numpy()
+        toks = np.arange(n)
+        parts = np.stack([o._bits(workload.fill_bf16(n, cfg.H, tl.layer1.seed, 100 + q,
+                                                    row_ids=toks)) for q in range(cfg.R)])
+
+        def fn():
+            home, _ = o.predict_home(tl.layer1.ids[:n], cfg.E, C12, tl.layer2.expert_rank, cfg.R)
+            order = o.shuffle_order(home, cfg.R)
+            o.shuffle_reduce_f32chain(parts, order["row_token"][:n])
+        fn.tokens = n
+        return fn
     L = S.L
     if isinstance(S, BackwardStep):
         yb, gob, gsb = o._bits(L.y), o._bits(S.g_out), o._bits(S.g_send)
@@ -949,6 +1037,12 @@ def cpu_baseline(S, seconds: float):
         if time.perf_counter() - t0 >= seconds:
             break
     dt = time.perf_counter() - t0
+    if hasattr(fn, "tokens"):
+        return {"value": fn.tokens * n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+                "sample": f"{n} pass(es) over the first {fn.tokens} tokens of config "
+                          f"{S.cfg.index} through the single-threaded C oracle: home prediction, "
+                          "shuffle order and the rank-order sum of the partial rows",
+                "host_cpu": _cpu_model(), "host_nproc": os.cpu_count()}
     return {"value": S.N * n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{n} whole batch(es) of config {S.cfg.index} (N={S.N}) through the "
                       "single-threaded C oracle: " + (
@@ -1026,6 +1120,8 @@ def main():
                     help="backward: combine_scatter_backward + dispatch_gather_backward")
     ap.add_argument("--combine", default="direct", choices=["direct", "prereduced"],
                     help="prereduced: combine_rows per send row, then the transposed dispatch")
+    ap.add_argument("--shuffle", action="store_true",
+                    help="config 4: token shuffling fused into the post-attention reduce-scatter")
     ap.add_argument("--two-hop", action="store_true",
                     help="dispatch in two hops: to nodes, then inside the node to ranks")
     args = ap.parse_args()

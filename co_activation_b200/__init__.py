@@ -52,6 +52,7 @@ _lib.combine_scatter.argtypes = [_P, _I64, _P, _P, _I64, _I32, _I64, _P, _I32, _
 _lib.combine_rows.argtypes = [_P, _I64, _P, _P, _I64, _I32, _P, _P, _I64, _P, _I64, _P, _I32, _P,
                               _P]
 _lib.dispatch_gather_backward.argtypes = [_P, _I64, _P, _I64, _I32, _I64, _P, _I32, _P, _P]
+_lib.shuffle_reduce_scatter.argtypes = [_P, _I32, _I64, _I64, _P, _I64, _P, _I32, _P, _P]
 _lib.combine_scatter_backward.argtypes = [_P, _I64, _P, _P, _I64, _I32, _P, _P, _I64, _P, _P,
                                           _I64, _P, _P, _P, _P]
 _lib.predict_home_workspace_bytes.argtypes = [_I32, _I32]
@@ -69,7 +70,7 @@ _lib.plan_dispatch_noalloc.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32,
                                        _P, _P, _P, _I64, _P, _P, _P, _P, _P, _P]
 for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "dispatch_gather_tma",
            "combine_scatter", "combine_rows", "dispatch_gather_backward",
-           "combine_scatter_backward", "predict_home",
+           "combine_scatter_backward", "shuffle_reduce_scatter", "predict_home",
            "coact_place_correlated", "plan_dispatch_noalloc", "coact_compose_map", "plan_forward",
            "forward_gather", "coact_rebalance_ranks", "dispatch_gather_peer",
            "combine_scatter_peer"):
@@ -80,7 +81,8 @@ ABI_SYMBOLS = ("coact_strerror", "coact_abi_version", "coact_count", "plan_dispa
                "predict_home_workspace_bytes", "predict_home", "coact_place_correlated",
                "plan_dispatch_noalloc", "coact_compose_map", "plan_forward", "forward_gather",
                "coact_rebalance_ranks", "dispatch_gather_peer", "combine_scatter_peer",
-               "combine_rows", "dispatch_gather_backward", "combine_scatter_backward")
+               "combine_rows", "dispatch_gather_backward", "combine_scatter_backward",
+               "shuffle_reduce_scatter")
 NOALLOC_MAX_TOKENS = 262144
 
 
@@ -359,6 +361,41 @@ def combine_scatter_backward(y: torch.Tensor, gates: torch.Tensor, comb_row: tor
                                          _ptr(grad_y), _ptr(grad_gates), _ptr(err_flag),
                                          _stream(stream)), "combine_scatter_backward")
     return grad_y, grad_gates
+
+
+def shuffle_plan(home: torch.Tensor, R: int, plan: Optional["Plan"] = None,
+                 err_flag: Optional[torch.Tensor] = None, stream=None) -> "Plan":
+    """The token shuffle's permutation: plan_dispatch of every token to its predicted home
+    rank alone (ids = home [N, 1], E = R, identity expert -> rank map).  plan.row_token
+    lists the tokens grouped by home rank in ascending token order; rank r's output rows
+    are [rank_offsets[r], rank_offsets[r+1])."""
+    if R < 2:
+        raise ValueError("token shuffling needs at least two ranks")
+    _need(home, "home", torch.int32)
+    N = home.shape[0]
+    if plan is None:
+        plan = alloc_plan(N, 1, R, R, home.device, with_rank_mask=False, with_src_dst=False)
+    ident = torch.arange(R, dtype=torch.int32, device=home.device)
+    return plan_dispatch(home.view(N, 1), R, ident, R, plan, err_flag=err_flag, stream=stream)
+
+
+def shuffle_reduce_scatter(part_bases: torch.Tensor, N: int, row_token: torch.Tensor,
+                           out: torch.Tensor, err_flag: Optional[torch.Tensor] = None,
+                           stream=None) -> torch.Tensor:
+    """out[i] = sum over q of part_q[row_token[i]] (fp32 adds in rank order); part_bases:
+    device int64 [P] addresses of the P bf16 [N, H] partial outputs; H = out.shape[1]."""
+    _need(part_bases, "part_bases", torch.int64)
+    P = part_bases.shape[0]
+    _need(row_token, "row_token", torch.int32)
+    n_out, H = out.shape
+    if row_token.numel() < n_out:
+        raise ValueError("row_token needs one entry per output row")
+    _need(out, "out", out.dtype)
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.shuffle_reduce_scatter(_ptr(part_bases), P, N, H, _ptr(row_token), n_out, _ptr(out),
+                                       _out_dtype(out), _ptr(err_flag), _stream(stream)),
+           "shuffle_reduce_scatter")
+    return out
 
 
 def predict_workspace_bytes(E1: int, R: int) -> int:

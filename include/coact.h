@@ -388,6 +388,27 @@ int combine_scatter_peer(const uint64_t *y_bases, const int32_t *y_row_offset,
                          const float *gates, const int32_t *comb_row, int64_t N, int k, int64_t H,
                          void *out, int out_dtype, int32_t *err_flag, coact_stream_t stream);
 
+/*
+ * shuffle_reduce_scatter -- token shuffling fused into the post-attention reduce-scatter.
+ * Zyphra, English abstract: under sequence parallelism each token moves, during the
+ * reduce-scatter that follows attention, to the GPU predicted to hold its next-layer
+ * experts.  The P ranks each hold a partial attention output for all N tokens (bf16
+ * [N, H] at part_bases[q]: DEVICE array of P uint64 device addresses -- the peers'
+ * NVLink-mapped buffers on a GPU group, local buffers on one GPU); this call writes
+ *   out[i] = sum over q = 0..P-1 of part_q[row_token[i]]   for i < n_out
+ * per element an fp32 add chain in rank order from +0.0f, stored fp32 (out_dtype 1) or
+ * rounded to bf16 nearest-even (out_dtype 0); out: [n_out, H].  row_token: the tokens of
+ * this rank's output rows -- the row_token segment [rank_offsets[r], rank_offsets[r+1])
+ * of plan_dispatch over ids = home [N, 1], E = R, expert_rank = identity, i.e. the tokens
+ * predicted to live on rank r in ascending order (home from predict_home).  A row_token
+ * outside [0, N) gives a zero row and COACT_EFLAG_ROW_RANGE; a NULL or misaligned (not
+ * 16-byte) partial base is skipped with COACT_EFLAG_ROW_RANGE.  1 <= P <= 64.  Ordering
+ * across GPUs (partials written before this call reads them) is the caller's barrier.
+ */
+int shuffle_reduce_scatter(const uint64_t *part_bases, int P, int64_t N, int64_t H,
+                           const int32_t *row_token, int64_t n_out, void *out, int out_dtype,
+                           int32_t *err_flag, coact_stream_t stream);
+
 /* Bytes of device workspace predict_home needs (E1*R int64 scores). */
 size_t predict_home_workspace_bytes(int E1, int R);
 

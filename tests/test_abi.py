@@ -149,6 +149,19 @@ def test_backward_entry_points_reject_bad_arguments(lib):
     assert s(None, 0, None, None, 0, 2, None, None, 0, None, None, 16, None, None, None, None) == 0
 
 
+def test_shuffle_rejects_bad_arguments(lib):
+    f = lib.shuffle_reduce_scatter
+    f.argtypes = [P, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, P, ctypes.c_int64, P,
+                  ctypes.c_int, P, P]
+    assert f(FAKE, 4, 100, 12, FAKE, 10, FAKE, 0, None, None) == -2     # H % 8 != 0
+    assert f(FAKE, 0, 100, 16, FAKE, 10, FAKE, 0, None, None) == -2     # P < 1
+    assert f(FAKE, 65, 100, 16, FAKE, 10, FAKE, 0, None, None) == -2    # P > 64
+    assert f(FAKE, 4, 100, 16, FAKE, 10, FAKE, 2, None, None) == -2     # out dtype
+    assert f(None, 4, 100, 16, FAKE, 10, FAKE, 0, None, None) == -1     # bases NULL
+    assert f(FAKE, 4, 100, 16, FAKE, 10, P(264), 0, None, None) == -1   # misaligned out
+    assert f(None, 4, 100, 16, None, 0, None, 0, None, None) == 0       # nothing to write
+
+
 def test_predict_rejects_bad_arguments(lib):
     p = lib.predict_home
     p.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int,
