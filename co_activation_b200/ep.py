@@ -38,6 +38,13 @@ Backward over the same plan (the transposed maps):
       travel back and are summed per token (dispatch_gather_backward, or the peer combine
       with unit weights).
 
+Token shuffling in the post-attention reduce-scatter (shuffle_reduce_scatter): every rank
+holds a partial attention output for all N tokens of the group; rank r gets the tokens
+predicted to live on it (ascending), each the sum of the P partials in rank order --
+"peer": one shuffle_reduce_scatter reading every peer's partial buffer in place; "nccl":
+the partials permuted locally (dispatch_gather over the shuffle plan), one all_to_all of
+the rank segments, then the same kernel over the P received blocks.
+
 Only library kernels touch rows and plans; this module moves split sizes, builds the
 small per-row expert-id metadata the experts need, and calls the collectives.  The
 local steps are an `ops` object (the library by default) so that the exchange logic can
@@ -116,6 +123,13 @@ class LibraryOps:
 
     def count(self, ids, E, pair, loads):
         self.c.coact_count(ids, E, pair, loads)
+
+    def shuffle_plan(self, home, R):
+        return self.c.shuffle_plan(home, R)
+
+    def shuffle_reduce(self, blocks, row_token, N, out):
+        bases = torch.tensor([b.data_ptr() for b in blocks], dtype=torch.int64, device=out.device)
+        return self.c.shuffle_reduce_scatter(bases, N, row_token, out)
 
 
 class EPLayer:
@@ -331,6 +345,41 @@ class EPLayer:
             out = torch.empty((N, grad_rows.shape[1]), dtype=grad_rows.dtype,
                               device=grad_rows.device)
         return self._sum_back(grad_rows, "gback", out)
+
+    # ------------------------------------------------------------------ token shuffling
+
+    def shuffle_reduce_scatter(self, partial: torch.Tensor, home: torch.Tensor,
+                               out: Optional[torch.Tensor] = None):
+        """partial: bf16 [N, H], this rank's partial attention output for all N tokens of
+        the group; home: int32 [N], every token's predicted home rank (the same on every
+        rank).  Returns (rows, tokens): the rows of the tokens homed on this rank in
+        ascending token order, each the sum of the R partials in rank order, and their
+        token indices."""
+        R, me = self.R, self.me
+        N, H = partial.shape
+        sp = self.ops.shuffle_plan(home, R)
+        offs = sp.rank_offsets.cpu()
+        lo, hi = int(offs[me]), int(offs[me + 1])
+        tokens = sp.row_token[lo:hi]
+        if out is None:
+            out = torch.empty((hi - lo, H), dtype=partial.dtype, device=partial.device)
+        if self.transport == "peer":
+            sb = self._symmetric("part", N, H, partial.dtype, partial.device)
+            sb["t"][:N].copy_(partial)
+            sb["handle"].barrier()
+            import co_activation_b200 as coact
+            coact.shuffle_reduce_scatter(sb["ptrs"], N, tokens, out)
+            sb["handle"].barrier()
+            return out, tokens
+        counts = (offs[1:] - offs[:-1]).tolist()
+        permuted = self.ops.gather(partial, sp)[:N]        # rank segments, ascending tokens
+        recv = torch.empty((R * (hi - lo), H), dtype=partial.dtype, device=partial.device)
+        dist.all_to_all_single(recv.view(torch.int32), permuted.contiguous().view(torch.int32),
+                               [hi - lo] * R, counts, group=self.group)
+        blocks = [recv[q * (hi - lo):(q + 1) * (hi - lo)] for q in range(R)]
+        ident = torch.arange(hi - lo, dtype=torch.int32, device=partial.device)
+        self.ops.shuffle_reduce(blocks, ident, hi - lo, out)
+        return out, tokens
 
     # ------------------------------------------------------------------ peer transport
 

@@ -72,6 +72,19 @@ class OracleOps:
     def gather_backward(self, rows, send_row, out):
         return self._store(out, self.o.gather_backward_f32chain(self.o._bits(rows), send_row.numpy()))
 
+    def shuffle_plan(self, home, R):
+        p = self.o.shuffle_order(home.numpy(), R)
+        t = lambda k: torch.from_numpy(np.ascontiguousarray(p[k]))
+        return types.SimpleNamespace(row_token=t("row_token"), row_kmask=t("row_kmask"),
+                                     send_row=t("send_row"), comb_row=t("comb_row"),
+                                     rank_counts=t("rank_counts"), rank_offsets=t("rank_offsets"),
+                                     asg_offsets=t("asg_offsets"),
+                                     row_capacity=len(p["row_token"]))
+
+    def shuffle_reduce(self, blocks, row_token, N, out):
+        parts = np.stack([self.o._bits(b) for b in blocks])
+        return self._store(out, self.o.shuffle_reduce_f32chain(parts, row_token.numpy()))
+
     def combine_backward(self, y, gates, comb, g_out, g_y, g_gates):
         gy, gg, _ = self.o.combine_backward(self.o._bits(y), gates.numpy(), comb.numpy(),
                                             self.o._bits(g_out))
@@ -219,3 +232,54 @@ def test_ep_prereduced_and_backward_match_single_process(world, spec):
     for r in range(world):
         for name, ok in zip(names, out[r]):
             assert ok, f"rank {r}: {name} differs from the single-process oracle"
+
+
+def _worker_shuffle(rank, world, port, spec, out):
+    """Token shuffling in the reduce-scatter across gloo ranks against the oracle over all
+    ranks' partials."""
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        import workload
+        import co_activation_b200.ep as ep
+        N, H = spec
+        rng = np.random.default_rng(7)
+        home = rng.integers(0, world, N).astype(np.int32)
+        home[: N // 3] = 0                         # uneven segments
+        partial = workload.fill_bf16(N, H, 0, 100 + rank)
+        layer = ep.EPLayer(dist.group.WORLD, 8, torch.zeros(8, dtype=torch.int32),
+                           transport="nccl", ops=OracleOps(oracle))
+        rows, tokens = layer.shuffle_reduce_scatter(partial, torch.from_numpy(home),
+                                                    torch.empty((int((home == rank).sum()), H),
+                                                                dtype=torch.float32))
+        parts = np.stack([oracle._bits(workload.fill_bf16(N, H, 0, 100 + q)) for q in range(world)])
+        want_tok = np.flatnonzero(home == rank).astype(np.int32)
+        want = oracle.shuffle_reduce_f32chain(parts, want_tok)
+        out[rank] = (np.array_equal(tokens.numpy(), want_tok),
+                     np.array_equal(rows.numpy().view(np.uint32), want.view(np.uint32)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,spec", [(2, (1000, 32)), (3, (777, 24))])
+def test_ep_shuffle_reduce_scatter_matches_oracle(world, spec):
+    ctx = mp.get_context("spawn")
+    manager = ctx.Manager()
+    out = manager.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_shuffle, args=(r, world, port, spec, out))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    for r in range(world):
+        tok_ok, rows_ok = out[r]
+        assert tok_ok, f"rank {r}: shuffled tokens differ"
+        assert rows_ok, f"rank {r}: reduced rows differ"
