@@ -51,6 +51,8 @@ def _get():
             _lib.oracle_count_cross.argtypes = [P, I32, I32, P, I32, I32, I64, P, P]
             _lib.oracle_plan.argtypes = [P, I64, I32, I32, P, I32, P, I32, P, P, P, P, P, P, P,
                                          I64, P, P, P, P]
+            _lib.oracle_plan_slots.argtypes = _lib.oracle_plan.argtypes
+            _lib.oracle_assign_replicas.argtypes = [P, I64, I32, I32, P, I32, P, I32, P, I32, P, P]
             _lib.oracle_gather.argtypes = [P, I64, P, I64, P]
             _lib.oracle_gather.restype = None
             _lib.oracle_combine_f64.argtypes = [P, I64, P, P, I64, I32, I64, P]
@@ -129,11 +131,13 @@ def count_cross(ids1, E1: int, ids2, E2: int, C12=None, loads1=None):
 
 
 def plan(ids, E: int, expert_rank, R: int, rank_node=None, n_nodes: int = 1, src_rank=None,
-         row_capacity: Optional[int] = None) -> dict:
-    """Deduplicated dispatch plan; returns a dict of numpy arrays plus 'flags' and 'D'."""
+         row_capacity: Optional[int] = None, slot_rank=None) -> dict:
+    """Deduplicated dispatch plan; returns a dict of numpy arrays plus 'flags' and 'D'.
+    With slot_rank (int32 [N, k]) every slot goes to its own rank and expert_rank is not
+    used (expert replicas)."""
     ids = _c(ids, np.int32)
     N, k = ids.shape
-    er = _c(expert_rank, np.int32)
+    er = _c(expert_rank if slot_rank is None else slot_rank, np.int32)
     rn = None if rank_node is None else _c(rank_node, np.int32)
     sr = None if src_rank is None else _c(src_rank, np.int32)
     cap = N * min(k, R) if row_capacity is None else int(row_capacity)
@@ -149,7 +153,8 @@ def plan(ids, E: int, expert_rank, R: int, rank_node=None, n_nodes: int = 1, src
         "stats": np.zeros(N_STATS, np.int64),
         "src_dst": np.zeros((R, R), np.int32),
     }
-    f = _get().oracle_plan(_p(ids), N, k, E, _p(er), R, _p(rn), n_nodes, _p(sr),
+    fn = _get().oracle_plan if slot_rank is None else _get().oracle_plan_slots
+    f = fn(_p(ids), N, k, E, _p(er), R, _p(rn), n_nodes, _p(sr),
                            _p(out["rank_counts"]), _p(out["rank_offsets"]),
                            _p(out["asg_offsets"]), _p(out["rank_mask"]), _p(out["row_token"]),
                            _p(out["row_kmask"]), cap, _p(out["send_row"]), _p(out["comb_row"]),
@@ -411,3 +416,22 @@ def shuffle_reduce_f32chain(parts, row_token) -> np.ndarray:
     out = np.zeros((len(rt), H), np.float32)
     _get().oracle_shuffle_reduce_f32chain(_p(pb), Pn, N, H, _p(rt), len(rt), _p(out))
     return out
+
+
+# ----------------------------------------------------------------------------- replicas
+
+
+def assign_replicas(ids, E: int, rep_rank, n_rep, R: int, rank_node=None, n_nodes: int = 1,
+                    src_rank=None):
+    """Replica choice per (token, slot) (int32 [N, k], -1 for invalid tokens) and flags;
+    rep_rank: int32 [E, max_rep], n_rep: int32 [E]."""
+    ids = _c(ids, np.int32)
+    N, k = ids.shape
+    rr = _c(rep_rank, np.int32)
+    nr = _c(n_rep, np.int32)
+    rn = None if rank_node is None else _c(rank_node, np.int32)
+    sr = None if src_rank is None else _c(src_rank, np.int32)
+    out = np.zeros((N, k), np.int32)
+    f = _get().oracle_assign_replicas(_p(ids), N, k, E, _p(rr), rr.shape[1], _p(nr), R, _p(rn),
+                                      n_nodes, _p(sr), _p(out))
+    return out, f

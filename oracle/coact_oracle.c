@@ -136,8 +136,11 @@ int oracle_count_cross(const int32_t *ids1, int k1, int E1, const int32_t *ids2,
  * rank_mask [N] (may be NULL) is written as uint64.
  * Invalid tokens (bad id, repeated id, bad expert_rank entry, bad src) contribute
  * nothing; their send_row / comb_row entries are -1.
+ * oracle_plan_slots states all of this for a rank per slot, slot_rank[t*k + j] (with
+ * expert replicas a token's slot may go to any replica of its expert); oracle_plan is
+ * the case slot_rank[t*k + j] = expert_rank[ids[t*k + j]].
  */
-int oracle_plan(const int32_t *ids, int64_t N, int k, int E, const int32_t *expert_rank, int R,
+int oracle_plan_slots(const int32_t *ids, int64_t N, int k, int E, const int32_t *slot_rank, int R,
                 const int32_t *rank_node, int n_nodes, const int32_t *src_rank,
                 int32_t *rank_counts, int32_t *rank_offsets, int32_t *asg_offsets,
                 uint64_t *rank_mask_out, int32_t *row_token, uint8_t *row_kmask,
@@ -157,7 +160,7 @@ int oracle_plan(const int32_t *ids, int64_t N, int k, int E, const int32_t *expe
         src[t] = src_rank ? src_rank[t] : (t * R) / N;
         if (!(f & OF_ID_RANGE))
             for (int j = 0; j < k; ++j) {
-                int32_t r = expert_rank[ids[t * k + j]];
+                int32_t r = slot_rank[t * k + j];
                 if (r < 0 || r >= R) f |= OF_ID_RANGE;
             }
         if (src[t] < 0 || src[t] >= R) f |= OF_SRC_RANK;
@@ -165,7 +168,7 @@ int oracle_plan(const int32_t *ids, int64_t N, int k, int E, const int32_t *expe
         valid[t] = (char)(f == 0);
         uint64_t m = 0;
         if (valid[t])
-            for (int j = 0; j < k; ++j) m |= 1ull << expert_rank[ids[t * k + j]];
+            for (int j = 0; j < k; ++j) m |= 1ull << slot_rank[t * k + j];
         if (rank_mask_out) rank_mask_out[t] = m;
     }
 
@@ -177,7 +180,7 @@ int oracle_plan(const int32_t *ids, int64_t N, int k, int E, const int32_t *expe
             if (!valid[t]) continue;
             int in = 0;
             for (int j = 0; j < k; ++j)
-                if (expert_rank[ids[t * k + j]] == r) { in = 1; asg += 1; }
+                if (slot_rank[t * k + j] == r) { in = 1; asg += 1; }
             rows += in;
         }
         rank_counts[r] = (int32_t)rows;
@@ -197,7 +200,7 @@ int oracle_plan(const int32_t *ids, int64_t N, int k, int E, const int32_t *expe
             if (!valid[t]) continue;
             uint32_t km = 0;
             for (int j = 0; j < k; ++j)
-                if (expert_rank[ids[t * k + j]] == r) km |= 1u << j;
+                if (slot_rank[t * k + j] == r) km |= 1u << j;
             if (!km) continue;
             int first = 1;
             for (int j = 0; j < k; ++j) {
@@ -228,7 +231,7 @@ int oracle_plan(const int32_t *ids, int64_t N, int k, int E, const int32_t *expe
         char rank_set[64] = {0}, node_set[64] = {0};
         int node_src = rank_node ? rank_node[src[t]] : 0;
         for (int j = 0; j < k; ++j) {
-            int32_t r = expert_rank[ids[t * k + j]];
+            int32_t r = slot_rank[t * k + j];
             int nd = rank_node ? rank_node[r] : 0;
             rank_set[r] = 1;
             node_set[nd] = 1;
@@ -247,6 +250,26 @@ int oracle_plan(const int32_t *ids, int64_t N, int k, int E, const int32_t *expe
     free(src);
     free(valid);
     return flags;
+}
+
+/*
+ * The plan with each expert on one rank: slot (t, j) goes to expert_rank[ids[t,j]]
+ * (the definitions above, through oracle_plan_slots).
+ */
+int oracle_plan(const int32_t *ids, int64_t N, int k, int E, const int32_t *expert_rank, int R,
+                const int32_t *rank_node, int n_nodes, const int32_t *src_rank,
+                int32_t *rank_counts, int32_t *rank_offsets, int32_t *asg_offsets,
+                uint64_t *rank_mask_out, int32_t *row_token, uint8_t *row_kmask,
+                int64_t row_capacity, int32_t *send_row, int32_t *comb_row, int64_t *stats,
+                int32_t *src_dst) {
+    int32_t *slot = (int32_t *)malloc((size_t)(N * k > 0 ? N * k : 1) * sizeof(int32_t));
+    for (int64_t i = 0; i < N * k; ++i)
+        slot[i] = (ids[i] >= 0 && ids[i] < E) ? expert_rank[ids[i]] : -1;
+    int f = oracle_plan_slots(ids, N, k, E, slot, R, rank_node, n_nodes, src_rank, rank_counts,
+                              rank_offsets, asg_offsets, rank_mask_out, row_token, row_kmask,
+                              row_capacity, send_row, comb_row, stats, src_dst);
+    free(slot);
+    return f;
 }
 
 /* Gathered send buffer: send[d] = x[row_token[d]] for d < D (bf16 rows copied as bits). */
@@ -656,4 +679,78 @@ void oracle_shuffle_reduce_f32chain(const uint16_t *parts, int P, int64_t N, int
             out[i * H + h] = acc;
         }
     }
+}
+
+
+/* ------------------------------------------------------------------------------------
+ * Replica choice.
+ *
+ * [Cobalt] EP distributes expert replicas across GPUs, and a communication-aware task
+ * assignment routes tokens to fewer remote nodes under the current expert layout.  The
+ * pages give no algorithm; the reading taken is a per-token greedy over the slots:
+ * expert e has n_rep[e] replicas, on ranks rep_rank[e*max_rep + i], i < n_rep[e].  For a
+ * valid token t with home rank s and home node hn:
+ *   1. slots whose expert has one replica take it;
+ *   2. the other slots, j ascending, take the first replica (ascending i) in the first
+ *      non-empty class: (a) on s; (b) on a rank the token already uses; (c) on hn;
+ *      (d) on a node the token already uses; otherwise replica (t + j) mod n_rep[e],
+ *      which spreads the tokens that must open a new node over the replicas.
+ * "Uses" = chosen before, step 1 included.  slot_rank[t*k + j] = the chosen rank; -1 for
+ * every slot of an invalid token (bad id, repeated id, bad home rank, or a replica table
+ * entry of one of its experts out of range: n_rep outside [1, max_rep] or a rank outside
+ * [0, R)).  Returns the error flags.
+ * ------------------------------------------------------------------------------------ */
+int oracle_assign_replicas(const int32_t *ids, int64_t N, int k, int E, const int32_t *rep_rank,
+                           int max_rep, const int32_t *n_rep, int R, const int32_t *rank_node,
+                           int n_nodes, const int32_t *src_rank, int32_t *slot_rank) {
+    int flags = 0;
+    (void)n_nodes;
+    for (int64_t t = 0; t < N; ++t) {
+        int f = token_flags(ids, t, k, E);
+        int64_t s = src_rank ? src_rank[t] : (t * R) / N;
+        if (s < 0 || s >= R) f |= OF_SRC_RANK;
+        if (!(f & OF_ID_RANGE))
+            for (int j = 0; j < k; ++j) {
+                int e = ids[t * k + j];
+                if (n_rep[e] < 1 || n_rep[e] > max_rep) { f |= OF_ID_RANGE; continue; }
+                for (int i = 0; i < n_rep[e]; ++i) {
+                    int r = rep_rank[e * max_rep + i];
+                    if (r < 0 || r >= R) f |= OF_ID_RANGE;
+                }
+            }
+        flags |= f;
+        for (int j = 0; j < k; ++j) slot_rank[t * k + j] = -1;
+        if (f) continue;
+        int hn = rank_node ? rank_node[s] : 0;
+        char used_rank[64] = {0}, used_node[64] = {0};
+        for (int j = 0; j < k; ++j) {                      /* step 1 */
+            int e = ids[t * k + j];
+            if (n_rep[e] == 1) {
+                int r = rep_rank[e * max_rep];
+                slot_rank[t * k + j] = r;
+                used_rank[r] = 1;
+                used_node[rank_node ? rank_node[r] : 0] = 1;
+            }
+        }
+        for (int j = 0; j < k; ++j) {                      /* step 2 */
+            if (slot_rank[t * k + j] >= 0) continue;
+            int e = ids[t * k + j];
+            const int32_t *rep = rep_rank + e * max_rep;
+            int pick = -1;
+            for (int cls = 0; cls < 4 && pick < 0; ++cls)
+                for (int i = 0; i < n_rep[e] && pick < 0; ++i) {
+                    int r = rep[i];
+                    int nd = rank_node ? rank_node[r] : 0;
+                    if ((cls == 0 && r == s) || (cls == 1 && used_rank[r]) ||
+                        (cls == 2 && nd == hn) || (cls == 3 && used_node[nd]))
+                        pick = i;
+                }
+            if (pick < 0) pick = (int)((t + j) % n_rep[e]);
+            int r = rep[pick];
+            slot_rank[t * k + j] = r;
+            used_rank[r] = 1;
+            used_node[rank_node ? rank_node[r] : 0] = 1;
+        }
+    }
+    return flags;
 }

@@ -1,0 +1,117 @@
+"""Pins for the oracle's replica choice and per-slot plan (Cobalt, arxivdaily 2609.36959,
+English abstract: EP distributes expert replicas across GPUs; a communication-aware task
+assignment routes tokens to fewer remote nodes under the current layout).  The greedy is
+the reading stated in the oracle; it is pinned by hand-worked cases for each of its
+classes, by the single-replica case reducing to the plain plan, by invariants the
+reading guarantees, and the per-slot plan by brute force (sorting)."""
+import numpy as np
+import pytest
+
+import oracle
+from test_oracle_pins import brute_plan, rand_ids
+
+NODES6 = [0, 0, 1, 1, 2, 2]          # six ranks on three nodes
+
+
+def assign(ids, rep, R=6, rank_node=NODES6, src=None):
+    E = len(rep)
+    max_rep = max(len(r) for r in rep)
+    rr = np.full((E, max_rep), -1, np.int32)
+    for e, r in enumerate(rep):
+        rr[e, :len(r)] = r
+    nr = np.array([len(r) for r in rep], np.int32)
+    return oracle.assign_replicas(np.array(ids, np.int32), E, rr, nr, R, rank_node=rank_node,
+                                  n_nodes=max(rank_node) + 1, src_rank=src)
+
+
+def test_hand_worked_each_class():
+    # experts: 0 single on rank 2 (node 1); 1 on [3, 2]; 2 on [2, 1]; 3 on [4, 3]; 4 on [4, 5];
+    # 5 on [5, 0]
+    rep = [[2], [3, 2], [2, 1], [4, 3], [4, 5], [5, 0]]
+    ids = [[1, 0],     # t0 home 0: slot 1 forced to 2; slot 0: (b) rank 2 already used -> 2
+           [2, 5],     # t1 home 0: slot 0: (c) home node 0 -> rank 1; slot 1: (a) home rank 0 -> 0
+           [0, 3],     # t2 home 0: slot 0 forced 2 (node 1); slot 1: (d) node 1 in use -> 3
+           [4, 5],     # t3 home 0: slot 0: no class -> (t + j) % 2 = 1 -> rank 5; slot 1: (a) 0
+           [4, 2]]     # t4 home 0: slot 0: no class -> (4 + 0) % 2 = 0 -> rank 4; slot 1: (c) 1
+    got, f = assign(ids, rep, src=[0, 0, 0, 0, 0])
+    assert f == 0
+    assert got.tolist() == [[2, 2], [1, 0], [2, 3], [5, 0], [4, 1]]
+
+
+def test_home_rank_beats_used_rank_and_primary():
+    rep = [[1], [1, 4]]
+    # home 4: expert 0 forced to rank 1; expert 1 has replicas on 1 (used) and 4 (home):
+    # the home rank comes first
+    got, _ = assign([[0, 1]], rep, src=[4])
+    assert got.tolist() == [[1, 4]]
+
+
+def test_single_replicas_reduce_to_the_plain_plan():
+    rng = np.random.default_rng(5)
+    N, E, k, R = 300, 16, 3, 4
+    ids = rand_ids(rng, N, E, k)
+    er = rng.integers(0, R, E).astype(np.int32)
+    rn = np.array([0, 0, 1, 1], np.int32)
+    src = rng.integers(0, R, N).astype(np.int32)
+    slot, f = oracle.assign_replicas(ids, E, er[:, None], np.ones(E, np.int32), R, rank_node=rn,
+                                     n_nodes=2, src_rank=src)
+    assert f == 0 and np.array_equal(slot, er[ids])
+    a = oracle.plan(ids, E, er, R, rank_node=rn, n_nodes=2, src_rank=src)
+    b = oracle.plan(ids, E, None, R, rank_node=rn, n_nodes=2, src_rank=src, slot_rank=slot)
+    for key in ("rank_counts", "rank_offsets", "asg_offsets", "rank_mask", "row_token",
+                "row_kmask", "send_row", "comb_row", "stats", "src_dst"):
+        assert np.array_equal(a[key], b[key]), key
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_slot_plan_brute_force(seed):
+    rng = np.random.default_rng(100 + seed)
+    N, k, R = int(rng.integers(1, 40)), int(rng.integers(1, 5)), int(rng.integers(1, 7))
+    slot = rng.integers(0, R, (N, k)).astype(np.int32)
+    rn = np.sort(rng.integers(0, 3, R)).astype(np.int32)
+    src = rng.integers(0, R, N).astype(np.int32)
+    # one pseudo-expert per slot whose rank is the slot's: the brute-force planner over it
+    pseudo = np.arange(N * k, dtype=np.int32).reshape(N, k)
+    want = brute_plan(pseudo, slot.ravel(), R, rn, src)
+    got = oracle.plan(pseudo, N * k, None, R, rank_node=rn, n_nodes=int(rn.max()) + 1,
+                      src_rank=src, slot_rank=slot)
+    assert got["flags"] == 0
+    for key in ("rank_counts", "rank_offsets", "asg_offsets", "send_row", "comb_row", "stats",
+                "src_dst"):
+        assert np.array_equal(got[key], want[key]), key
+    D = got["D"]
+    assert np.array_equal(got["row_token"][:D], want["row_token"])
+    assert np.array_equal(got["row_kmask"][:D], want["row_kmask"])
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_invariants_on_random_layouts(seed):
+    rng = np.random.default_rng(200 + seed)
+    N, E, k, R = 500, 24, 4, 6
+    ids = rand_ids(rng, N, E, k)
+    rep = [sorted(rng.choice(R, int(rng.integers(1, 4)), replace=False).tolist()) for _ in range(E)]
+    src = rng.integers(0, R, N).astype(np.int32)
+    got, f = assign(ids, rep, src=src)
+    assert f == 0
+    for t in range(N):
+        for j in range(k):
+            e, r = ids[t][j], got[t, j]
+            assert r in rep[e]                                   # a replica of its expert
+            if len(rep[e]) == 1:
+                assert r == rep[e][0]                            # forced
+            elif src[t] in rep[e]:
+                assert r == src[t]                               # served on the home rank
+
+
+def test_validation_flags():
+    rep = np.array([[0, 1], [2, -1]], np.int32)
+    ids = np.array([[0, 1], [1, 0], [0, 1]], np.int32)
+    bad_n = np.array([2, 0], np.int32)                           # expert 1: no replica
+    got, f = oracle.assign_replicas(ids, 2, rep, bad_n, 4, src_rank=[0, 1, 2])
+    assert f & 1 and (got == -1).all()
+    bad_r = np.array([[0, 7], [2, 3]], np.int32)                 # rank 7 outside [0, 4)
+    got, f = oracle.assign_replicas(ids, 2, bad_r, np.array([2, 2], np.int32), 4, src_rank=[0, 1, 2])
+    assert f & 1 and (got == -1).all()
+    got, f = oracle.assign_replicas(ids, 2, np.array([[0, 1], [2, 3]], np.int32),
+                                    np.array([2, 2], np.int32), 4, src_rank=[0, 9, 2])
+    assert f & 8 and (got[1] == -1).all() and (got[[0, 2]] >= 0).all()
