@@ -509,6 +509,78 @@ class PreReducedStep(OneLayerStep):
                 ("reduce_rows", "k_combine_v16", D * c.H * 2 + c.N * c.H * 2 + c.N * c.k * 4)]
 
 
+class ReplicaStep(OneLayerStep):
+    """One layer over an expert layout with replicas (Cobalt: EP distributes expert
+    replicas across GPUs; task assignment routes tokens to fewer remote nodes): count
+    (side stream) -> assign_replicas -> plan over the chosen per-slot ranks -> gather ->
+    combine.  The n_hot most loaded experts of the batch have a second replica on another
+    node (workload.replicate_hot)."""
+    n_events = 6
+    phases = {"coact_count": (0, 1), "assign_replicas": (0, 2), "plan_dispatch": (2, 3),
+              "dispatch_gather": (3, 4), "combine_scatter": (4, 5)}
+
+    def __init__(self, coact, r: workload.Routing, device, n_hot: int, fill: bool = True):
+        super().__init__(coact, r, device, fill)
+        c = r.cfg
+        loads = np.bincount(r.ids.ravel(), minlength=c.E)        # the batch's expert loads
+        self.rep_h, self.nrep_h = workload.replicate_hot(loads, r.expert_rank, r.rank_node, n_hot)
+        to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        self.rep, self.nrep = to(self.rep_h), to(self.nrep_h)
+        self.slot = torch.empty((c.N, c.k), dtype=torch.int32, device=device)
+        self.n_hot = n_hot
+        self.kernels_per_step = 1 + 1 + plan_launches(c.R, self.N) + 1 + 1
+        self.step_desc = (f"coact_count (side stream) + assign_replicas ({n_hot} hottest experts "
+                          "with a second replica on another node) + plan_dispatch_slots + "
+                          "dispatch_gather + combine_scatter (bf16 out)")
+
+    def clone_for_copy(self, coact, device):
+        return ReplicaStep(coact, self.L.r, device, self.n_hot, fill=False)
+
+    def step(self, ev=None):
+        L, c, cfg = self.L, self.L.coact, self.cfg
+        main = torch.cuda.current_stream()
+        self.side.wait_stream(main)
+        if ev: ev[0].record()
+        with torch.cuda.stream(self.side):
+            L.count()
+            if ev: ev[1].record()
+        c.assign_replicas(L.ids, cfg.E, self.rep, self.nrep, cfg.R, self.slot, rank_node=L.rank_node,
+                          n_nodes=cfg.n_nodes, err_flag=L.err)
+        if ev: ev[2].record()
+        c.plan_dispatch(L.ids, cfg.E, None, cfg.R, L.plan, rank_node=L.rank_node,
+                        n_nodes=cfg.n_nodes, err_flag=L.err, slot_rank=self.slot)
+        if ev: ev[3].record()
+        L.gather()
+        if ev: ev[4].record()
+        L.combine()
+        main.wait_stream(self.side)
+        if ev: ev[5].record()
+
+    def roofline_parts(self):
+        D = self.L.D()
+        return [("dispatch_gather", LayerBuffers.gather_kernel(), self.L.bytes_gather(D)),
+                ("combine_scatter", "k_combine_v16", self.L.bytes_combine())]
+
+    def summary(self):
+        L, c, cfg = self.L, self.L.coact, self.cfg
+        out = super().summary()
+        st = L.plan.stats.cpu().tolist()
+        prim = c.alloc_plan(cfg.N, cfg.k, cfg.E, cfg.R, L.dev)
+        c.plan_dispatch(L.ids, cfg.E, self.rep[:, 0].contiguous(), cfg.R, prim,
+                        rank_node=L.rank_node, n_nodes=cfg.n_nodes)
+        sp = prim.stats.cpu().tolist()
+        load = lambda sl: np.bincount(sl.ravel(), minlength=cfg.R)
+        lc = load(self.slot.cpu().numpy())
+        lp = load(self.rep_h[:, 0][L.r.ids])
+        out.update({
+            "replicated_experts": int((self.nrep_h > 1).sum()),
+            "node_remote_pairs_replica_choice": st[4], "node_remote_pairs_primary_only": sp[4],
+            "local_served_asg_replica_choice": st[5], "local_served_asg_primary_only": sp[5],
+            "rank_load_max_over_mean_replica_choice": float(lc.max() / lc.mean()),
+            "rank_load_max_over_mean_primary_only": float(lp.max() / lp.mean())})
+        return out
+
+
 class BackwardStep:
     """The backward pass of one layer over the forward's plan (computed once, outside the
     timed steps): combine_scatter_backward (grad_y rows for the experts, grad_gates), then
@@ -681,6 +753,8 @@ def make_step(coact, cfg_index: int, seed: int, device, two_hop: bool = False,
         if mode != "forward":
             raise SystemExit("--two-hop runs the forward pass with the direct combine only")
         S = TwoHopStep(coact, r, device)
+    elif mode.startswith("replicas:"):
+        S = ReplicaStep(coact, r, device, int(mode.split(":")[1]))
     elif mode == "backward":
         S = BackwardStep(coact, r, device)
     elif mode == "prereduced":
@@ -741,7 +815,8 @@ def run_gpu(args):
 
     cfg = workload.CONFIGS[args.config]
     LayerBuffers.tma = args.gather == "tma"
-    mode = "shuffle" if args.shuffle else "backward" if args.pass_ == "backward" else (
+    mode = "shuffle" if args.shuffle else f"replicas:{args.replicas}" if args.replicas else \
+        "backward" if args.pass_ == "backward" else (
         "prereduced" if args.combine == "prereduced" else "forward")
     S, placement = make_step(coact, args.config, rank_seed(args.seed, rank), device, args.two_hop,
                              args.placement, mode)
@@ -1014,6 +1089,16 @@ def _oracle_step_fn(S):
             o.gather_backward_f32chain(gsb, p["send_row"])
         return fn
     xb, yb = o._bits(L.x), o._bits(L.y)
+    if isinstance(S, ReplicaStep):
+        def fn():
+            o.count(L.r.ids, cfg.E)
+            slot, _ = o.assign_replicas(L.r.ids, cfg.E, S.rep_h, S.nrep_h, cfg.R,
+                                        rank_node=L.r.rank_node, n_nodes=cfg.n_nodes)
+            p = o.plan(L.r.ids, cfg.E, None, cfg.R, rank_node=L.r.rank_node, n_nodes=cfg.n_nodes,
+                       slot_rank=slot)
+            o.gather(xb, p["row_token"], p["D"])
+            o.combine_f64(yb, L.r.gates, p["comb_row"])
+        return fn
     if isinstance(S, PreReducedStep):
         def fn():
             o.count(L.r.ids, cfg.E)
@@ -1120,6 +1205,9 @@ def main():
                     help="backward: combine_scatter_backward + dispatch_gather_backward")
     ap.add_argument("--combine", default="direct", choices=["direct", "prereduced"],
                     help="prereduced: combine_rows per send row, then the transposed dispatch")
+    ap.add_argument("--replicas", type=int, default=0, metavar="N_HOT",
+                    help="give the N_HOT most loaded experts a second replica on another node "
+                         "and choose replicas per token (assign_replicas)")
     ap.add_argument("--shuffle", action="store_true",
                     help="config 4: token shuffling fused into the post-attention reduce-scatter")
     ap.add_argument("--two-hop", action="store_true",

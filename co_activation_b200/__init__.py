@@ -35,7 +35,7 @@ EFLAG_ID_RANGE, EFLAG_DUP_ID, EFLAG_CAPACITY, EFLAG_SRC_RANK, EFLAG_ROW_RANGE, E
 NUM_STATS = 8
 STAT_NAMES = ("naive_rows", "dedup_rows", "remote_rows", "crossnode_rows",
               "node_dedup_crossnode_rows", "local_served_asg", "remote_asg", "crossnode_asg")
-MAX_K, MAX_E, MAX_R = 8, 1024, 64
+MAX_K, MAX_E, MAX_R, MAX_REPLICAS = 8, 1024, 64, 8
 
 _P, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
 _lib.coact_strerror.argtypes = [_I32]
@@ -46,6 +46,8 @@ _lib.plan_dispatch_workspace_bytes.argtypes = [_I64, _I32, _I32, _I32]
 _lib.plan_dispatch_workspace_bytes.restype = _SZ
 _lib.plan_dispatch.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _P, _P, _P, _P,
                                _P, _I64, _P, _P, _P, _P, _P, _SZ, _P, _P]
+_lib.plan_dispatch_slots.argtypes = _lib.plan_dispatch.argtypes
+_lib.assign_replicas.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _I32, _P, _P, _P, _P]
 _lib.dispatch_gather.argtypes = [_P, _I64, _I64, _P, _I32, _P, _I64, _P, _P]
 _lib.dispatch_gather_tma.argtypes = [_P, _I64, _I64, _P, _I32, _P, _I64, _P, _P]
 _lib.combine_scatter.argtypes = [_P, _I64, _P, _P, _I64, _I32, _I64, _P, _I32, _P, _P]
@@ -70,7 +72,8 @@ _lib.plan_dispatch_noalloc.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32,
                                        _P, _P, _P, _I64, _P, _P, _P, _P, _P, _P]
 for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "dispatch_gather_tma",
            "combine_scatter", "combine_rows", "dispatch_gather_backward",
-           "combine_scatter_backward", "shuffle_reduce_scatter", "predict_home",
+           "combine_scatter_backward", "shuffle_reduce_scatter", "plan_dispatch_slots",
+           "assign_replicas", "predict_home",
            "coact_place_correlated", "plan_dispatch_noalloc", "coact_compose_map", "plan_forward",
            "forward_gather", "coact_rebalance_ranks", "dispatch_gather_peer",
            "combine_scatter_peer"):
@@ -82,7 +85,7 @@ ABI_SYMBOLS = ("coact_strerror", "coact_abi_version", "coact_count", "plan_dispa
                "plan_dispatch_noalloc", "coact_compose_map", "plan_forward", "forward_gather",
                "coact_rebalance_ranks", "dispatch_gather_peer", "combine_scatter_peer",
                "combine_rows", "dispatch_gather_backward", "combine_scatter_backward",
-               "shuffle_reduce_scatter")
+               "shuffle_reduce_scatter", "plan_dispatch_slots", "assign_replicas")
 NOALLOC_MAX_TOKENS = 262144
 
 
@@ -206,14 +209,20 @@ def alloc_plan(N: int, k: int, E: int, R: int, device="cuda", row_capacity: Opti
                 src_dst=torch.empty((R, R), **i32) if with_src_dst else None, workspace=ws)
 
 
-def plan_dispatch(ids: torch.Tensor, E: int, expert_rank: torch.Tensor, R: int, plan: Plan,
-                  rank_node: Optional[torch.Tensor] = None, n_nodes: int = 1,
+def plan_dispatch(ids: torch.Tensor, E: int, expert_rank: Optional[torch.Tensor], R: int,
+                  plan: Plan, rank_node: Optional[torch.Tensor] = None, n_nodes: int = 1,
                   src_rank: Optional[torch.Tensor] = None,
-                  err_flag: Optional[torch.Tensor] = None, stream=None) -> Plan:
-    """Deduplicated dispatch layout into `plan`'s buffers (see include/coact.h)."""
+                  err_flag: Optional[torch.Tensor] = None, stream=None,
+                  slot_rank: Optional[torch.Tensor] = None) -> Plan:
+    """Deduplicated dispatch layout into `plan`'s buffers (see include/coact.h).  With
+    slot_rank (int32 [N, k], e.g. from assign_replicas) every slot goes to its own rank
+    (plan_dispatch_slots) and expert_rank is not used."""
     N, k = ids.shape
     _need(ids, "ids", torch.int32)
-    _need(expert_rank, "expert_rank", torch.int32, (E,))
+    if slot_rank is None:
+        _need(expert_rank, "expert_rank", torch.int32, (E,))
+    else:
+        _need(slot_rank, "slot_rank", torch.int32, (N, k))
     _need(rank_node, "rank_node", torch.int32, (R,), optional=True)
     _need(src_rank, "src_rank", torch.int32, (N,), optional=True)
     _need(plan.rank_counts, "rank_counts", torch.int32, (R,))
@@ -228,14 +237,38 @@ def plan_dispatch(ids: torch.Tensor, E: int, expert_rank: torch.Tensor, R: int, 
     _need(plan.src_dst, "src_dst", torch.int32, (R, R), optional=True)
     _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
     ws = plan.workspace
-    _check(_lib.plan_dispatch(
-        _ptr(ids), N, k, E, _ptr(expert_rank), R, _ptr(rank_node), n_nodes, _ptr(src_rank),
+    fn = _lib.plan_dispatch if slot_rank is None else _lib.plan_dispatch_slots
+    _check(fn(
+        _ptr(ids), N, k, E, _ptr(expert_rank if slot_rank is None else slot_rank), R,
+        _ptr(rank_node), n_nodes, _ptr(src_rank),
         _ptr(plan.rank_counts), _ptr(plan.rank_offsets), _ptr(plan.asg_offsets),
         _ptr(plan.rank_mask), _ptr(plan.row_token), _ptr(plan.row_kmask), plan.row_capacity,
         _ptr(plan.send_row), _ptr(plan.comb_row), _ptr(plan.stats), _ptr(plan.src_dst),
         _ptr(ws), ws.numel() * ws.element_size(), _ptr(err_flag), _stream(stream)),
-        "plan_dispatch")
+        "plan_dispatch" if slot_rank is None else "plan_dispatch_slots")
     return plan
+
+
+def assign_replicas(ids: torch.Tensor, E: int, rep_rank: torch.Tensor, n_rep: torch.Tensor, R: int,
+                    slot_rank: torch.Tensor, rank_node: Optional[torch.Tensor] = None,
+                    n_nodes: int = 1, src_rank: Optional[torch.Tensor] = None,
+                    err_flag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The replica serving each (token, slot) into slot_rank (int32 [N, k]); rep_rank:
+    int32 [E, max_rep] replica ranks, n_rep: int32 [E] replicas per expert."""
+    N, k = ids.shape
+    _need(ids, "ids", torch.int32)
+    _need(rep_rank, "rep_rank", torch.int32)
+    if rep_rank.dim() != 2 or rep_rank.shape[0] != E:
+        raise ValueError("rep_rank must be [E, max_rep]")
+    _need(n_rep, "n_rep", torch.int32, (E,))
+    _need(slot_rank, "slot_rank", torch.int32, (N, k))
+    _need(rank_node, "rank_node", torch.int32, (R,), optional=True)
+    _need(src_rank, "src_rank", torch.int32, (N,), optional=True)
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.assign_replicas(_ptr(ids), N, k, E, _ptr(rep_rank), rep_rank.shape[1], _ptr(n_rep),
+                                R, _ptr(rank_node), n_nodes, _ptr(src_rank), _ptr(slot_rank),
+                                _ptr(err_flag), _stream(stream)), "assign_replicas")
+    return slot_rank
 
 
 def dispatch_gather(x: torch.Tensor, send_row: torch.Tensor, send: torch.Tensor,

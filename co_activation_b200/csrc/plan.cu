@@ -58,17 +58,23 @@ size_t workspace_layout(int64_t N, int R, Workspace *ws, void *base) {
     return 2 * b_rows + b_stats + b_tot;
 }
 
-// Token t's per-slot ranks and home rank; returns validation bits (0 = valid).
+// Token t's per-slot ranks and home rank; returns validation bits (0 = valid).  The rank
+// of slot j is slot_rank[t*K + j] when slot_rank is given (expert replicas), else
+// expert_rank[ids[t,j]].
 template <int K>
 __device__ __forceinline__ int load_token(const int32_t *__restrict__ ids,
                                           const int32_t *__restrict__ expert_rank,
+                                          const int32_t *__restrict__ slot_rank,
                                           const int32_t *__restrict__ src_rank, int64_t t,
                                           int64_t N, int E, int R, int (&rk)[K], int &src) {
     int e[K];
     int f = load_ids<K>(ids, t, E, e);
 #pragma unroll
     for (int j = 0; j < K; ++j) {
-        rk[j] = (f & COACT_EFLAG_ID_RANGE) ? 0 : __ldg(expert_rank + e[j]);
+        if (slot_rank)
+            rk[j] = __ldg(slot_rank + t * K + j);
+        else
+            rk[j] = (f & COACT_EFLAG_ID_RANGE) ? 0 : __ldg(expert_rank + e[j]);
         if ((unsigned)rk[j] >= (unsigned)R) f |= COACT_EFLAG_ID_RANGE;
     }
     src = src_rank ? __ldg(src_rank + t) : (int)((t * R) / N);
@@ -110,7 +116,8 @@ __device__ __forceinline__ unsigned long long warp_or64(unsigned long long m) {
 template <int K>
 __global__ void __launch_bounds__(kTile)
     k_plan_tiles(const int32_t *__restrict__ ids, int64_t N, int E,
-                 const int32_t *__restrict__ expert_rank, int R,
+                 const int32_t *__restrict__ expert_rank, const int32_t *__restrict__ slot_rank,
+                 int R,
                  const int32_t *__restrict__ rank_node, int n_nodes,
                  const int32_t *__restrict__ src_rank, int n_tiles, Workspace ws,
                  int32_t *__restrict__ src_dst, int32_t *__restrict__ err) {
@@ -137,7 +144,7 @@ __global__ void __launch_bounds__(kTile)
     bool ok = false;
     int flags = 0;
     if (t < N) {
-        flags = load_token<K>(ids, expert_rank, src_rank, t, N, E, R, rk, src);
+        flags = load_token<K>(ids, expert_rank, slot_rank, src_rank, t, N, E, R, rk, src);
         ok = flags == 0;
     }
     load_nodes(nd, R, n_nodes, s_node, s_node_ranks, err);
@@ -339,7 +346,8 @@ __device__ __forceinline__ void rank_bases(int R, int tile, const int *tot_row,
 template <int K, bool SMALL>
 __global__ void __launch_bounds__(kTile)
     k_plan_scatter(const int32_t *__restrict__ ids, int64_t N, int E,
-                   const int32_t *__restrict__ expert_rank, int R,
+                   const int32_t *__restrict__ expert_rank, const int32_t *__restrict__ slot_rank,
+                   int R,
                    const int32_t *__restrict__ src_rank, int n_tiles, Workspace ws,
                    int32_t *__restrict__ rank_counts, int32_t *__restrict__ rank_offsets,
                    int32_t *__restrict__ asg_offsets, unsigned long long *__restrict__ rank_mask,
@@ -370,7 +378,7 @@ __global__ void __launch_bounds__(kTile)
     int src = 0;
     bool ok = false;
     int flags = 0;
-    if (t < N) ok = load_token<K>(ids, expert_rank, src_rank, t, N, E, R, rk, src) == 0;
+    if (t < N) ok = load_token<K>(ids, expert_rank, slot_rank, src_rank, t, N, E, R, rk, src) == 0;
     unsigned long long mask = 0;
     if (ok) {
 #pragma unroll
@@ -533,7 +541,8 @@ __global__ void __launch_bounds__(kTile)
 #endif
 
 template <int K>
-int launch_plan(const int32_t *ids, int64_t N, int E, const int32_t *expert_rank, int R,
+int launch_plan(const int32_t *ids, int64_t N, int E, const int32_t *expert_rank,
+                const int32_t *slot_rank, int R,
                 const int32_t *rank_node, int n_nodes, const int32_t *src_rank,
                 int32_t *rank_counts, int32_t *rank_offsets, int32_t *asg_offsets,
                 uint64_t *rank_mask, int32_t *row_token, uint8_t *row_kmask, int64_t cap,
@@ -544,23 +553,23 @@ int launch_plan(const int32_t *ids, int64_t N, int E, const int32_t *expert_rank
     const size_t sd_smem = src_dst ? sizeof(int) * R * R : 0;
     auto *rm = reinterpret_cast<unsigned long long *>(rank_mask);
     if (n_tiles > 0 && (int64_t)R * n_tiles <= COACT_PLAN_SMALL_MAX) {
-        if (int s = launch_pdl(k_plan_tiles<K>, n_tiles, kTile, 0, st, ids, N, E, expert_rank, R,
+        if (int s = launch_pdl(k_plan_tiles<K>, n_tiles, kTile, 0, st, ids, N, E, expert_rank, slot_rank, R,
                                rank_node, n_nodes, src_rank, n_tiles, ws, src_dst, err))
             return s;
         return launch_pdl(k_plan_scatter<K, true>, n_tiles, kTile, sd_smem, st, ids, N, E,
-                          expert_rank, R, src_rank, n_tiles, ws, rank_counts, rank_offsets,
+                          expert_rank, slot_rank, R, src_rank, n_tiles, ws, rank_counts, rank_offsets,
                           asg_offsets, rm, row_token, row_kmask, cap, send_row, comb_row, stats,
                           src_dst, err);
     }
     if (n_tiles > 0)
-        if (int s = launch_pdl(k_plan_tiles<K>, n_tiles, kTile, 0, st, ids, N, E, expert_rank, R,
+        if (int s = launch_pdl(k_plan_tiles<K>, n_tiles, kTile, 0, st, ids, N, E, expert_rank, slot_rank, R,
                                rank_node, n_nodes, src_rank, n_tiles, ws, src_dst, err))
             return s;
     if (int s = launch_pdl(k_plan_scan, R + 1, kScanThreads, 0, st, N, K, R, n_tiles, ws, stats,
                            n_tiles > 0 ? nullptr : src_dst))
         return s;
     return launch_pdl(k_plan_scatter<K, false>, std::max(n_tiles, 1), kTile, sd_smem, st, ids, N,
-                      E, expert_rank, R, src_rank, n_tiles, ws, rank_counts, rank_offsets,
+                      E, expert_rank, slot_rank, R, src_rank, n_tiles, ws, rank_counts, rank_offsets,
                       asg_offsets, rm, row_token, row_kmask, cap, send_row, comb_row, stats,
                       src_dst, err);
 }
@@ -577,20 +586,25 @@ extern "C" size_t plan_dispatch_workspace_bytes(int64_t N, int k, int E, int R) 
     return workspace_layout(N, R, nullptr, nullptr);
 }
 
-extern "C" int plan_dispatch(const int32_t *ids, int64_t N, int k, int E, const int32_t *expert_rank,
-                             int R, const int32_t *rank_node, int n_nodes, const int32_t *src_rank,
-                             int32_t *rank_counts, int32_t *rank_offsets, int32_t *asg_offsets,
-                             uint64_t *rank_mask, int32_t *row_token, uint8_t *row_kmask,
-                             int64_t row_capacity, int32_t *send_row, int32_t *comb_row,
-                             int64_t *stats, int32_t *src_dst, void *workspace,
-                             size_t workspace_bytes, int32_t *err_flag, coact_stream_t stream) {
+namespace coact {
+namespace {
+
+// plan_dispatch and plan_dispatch_slots: the rank of each slot comes from expert_rank
+// (per expert) or slot_rank (per slot), exactly one of them non-NULL.
+int plan_entry(const int32_t *ids, int64_t N, int k, int E, const int32_t *expert_rank,
+               const int32_t *slot_rank, int R, const int32_t *rank_node, int n_nodes,
+               const int32_t *src_rank, int32_t *rank_counts, int32_t *rank_offsets,
+               int32_t *asg_offsets, uint64_t *rank_mask, int32_t *row_token, uint8_t *row_kmask,
+               int64_t row_capacity, int32_t *send_row, int32_t *comb_row, int64_t *stats,
+               int32_t *src_dst, void *workspace, size_t workspace_bytes, int32_t *err_flag,
+               coact_stream_t stream) {
     if (N < 0 || row_capacity < 0) return COACT_ERR_INVALID;
     if (k < 1 || k > COACT_MAX_K || E < 2 || E > COACT_MAX_E || R < 1 || R > COACT_MAX_R)
         return COACT_ERR_UNSUPPORTED;
     if (rank_node && (n_nodes < 1 || n_nodes > 64)) return COACT_ERR_UNSUPPORTED;
     if (!rank_node) n_nodes = 1;
     if (N > (int64_t)INT32_MAX / k || row_capacity > (int64_t)INT32_MAX) return COACT_ERR_UNSUPPORTED;
-    if (!expert_rank || !rank_counts || !rank_offsets || !asg_offsets || !stats)
+    if ((!expert_rank && !slot_rank) || !rank_counts || !rank_offsets || !asg_offsets || !stats)
         return COACT_ERR_INVALID;
     if (N > 0 && (!ids || !send_row || !comb_row)) return COACT_ERR_INVALID;
     if (row_capacity > 0 && (!row_token || !row_kmask)) return COACT_ERR_INVALID;
@@ -603,7 +617,7 @@ extern "C" int plan_dispatch(const int32_t *ids, int64_t N, int k, int E, const 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 #define COACT_PLAN_CASE(KK)                                                                        \
     case KK:                                                                                       \
-        return launch_plan<KK>(ids, N, E, expert_rank, R, rank_node, n_nodes, src_rank,            \
+        return launch_plan<KK>(ids, N, E, expert_rank, slot_rank, R, rank_node, n_nodes, src_rank, \
                                rank_counts, rank_offsets, asg_offsets, rank_mask, row_token,       \
                                row_kmask, row_capacity, send_row, comb_row, stats, src_dst, ws,    \
                                err_flag, st, di);
@@ -619,6 +633,39 @@ extern "C" int plan_dispatch(const int32_t *ids, int64_t N, int k, int E, const 
     }
 #undef COACT_PLAN_CASE
     return COACT_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+}  // namespace coact
+
+extern "C" int plan_dispatch(const int32_t *ids, int64_t N, int k, int E, const int32_t *expert_rank,
+                             int R, const int32_t *rank_node, int n_nodes, const int32_t *src_rank,
+                             int32_t *rank_counts, int32_t *rank_offsets, int32_t *asg_offsets,
+                             uint64_t *rank_mask, int32_t *row_token, uint8_t *row_kmask,
+                             int64_t row_capacity, int32_t *send_row, int32_t *comb_row,
+                             int64_t *stats, int32_t *src_dst, void *workspace,
+                             size_t workspace_bytes, int32_t *err_flag, coact_stream_t stream) {
+    if (!expert_rank) return COACT_ERR_INVALID;
+    return plan_entry(ids, N, k, E, expert_rank, nullptr, R, rank_node, n_nodes, src_rank,
+                      rank_counts, rank_offsets, asg_offsets, rank_mask, row_token, row_kmask,
+                      row_capacity, send_row, comb_row, stats, src_dst, workspace, workspace_bytes,
+                      err_flag, stream);
+}
+
+extern "C" int plan_dispatch_slots(const int32_t *ids, int64_t N, int k, int E,
+                                   const int32_t *slot_rank, int R, const int32_t *rank_node,
+                                   int n_nodes, const int32_t *src_rank, int32_t *rank_counts,
+                                   int32_t *rank_offsets, int32_t *asg_offsets, uint64_t *rank_mask,
+                                   int32_t *row_token, uint8_t *row_kmask, int64_t row_capacity,
+                                   int32_t *send_row, int32_t *comb_row, int64_t *stats,
+                                   int32_t *src_dst, void *workspace, size_t workspace_bytes,
+                                   int32_t *err_flag, coact_stream_t stream) {
+    if (!slot_rank && N > 0) return COACT_ERR_INVALID;
+    static const int32_t kNone = 0;   // a non-NULL marker when N == 0 (never read)
+    return plan_entry(ids, N, k, E, nullptr, slot_rank ? slot_rank : &kNone, R, rank_node, n_nodes,
+                      src_rank, rank_counts, rank_offsets, asg_offsets, rank_mask, row_token,
+                      row_kmask, row_capacity, send_row, comb_row, stats, src_dst, workspace,
+                      workspace_bytes, err_flag, stream);
 }
 
 // ------------------------------------------------------------------ no-allocation variant
@@ -689,7 +736,7 @@ extern "C" int plan_dispatch_noalloc(const int32_t *ids, int64_t N, int k, int E
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 #define COACT_PLAN_NOALLOC_CASE(KK)                                                                \
     case KK:                                                                                       \
-        return launch_plan<KK>(ids, N, E, expert_rank, R, rank_node, n_nodes, src_rank,            \
+        return launch_plan<KK>(ids, N, E, expert_rank, nullptr, R, rank_node, n_nodes, src_rank,   \
                                rank_counts, rank_offsets, asg_offsets, rank_mask, row_token,       \
                                row_kmask, row_capacity, send_row, comb_row, stats, src_dst, ws,    \
                                err_flag, st, di);

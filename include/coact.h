@@ -64,6 +64,7 @@ enum coact_eflag {
 #define COACT_MAX_K 8
 #define COACT_MAX_E 1024
 #define COACT_MAX_R 64
+#define COACT_MAX_REPLICAS 8   /* replicas per expert (assign_replicas) */
 #define COACT_NUM_STATS 8
 
 /* Indices into the stats[8] array written by plan_dispatch. */
@@ -158,6 +159,46 @@ int plan_dispatch(const int32_t *ids, int64_t N, int k, int E,
                   int64_t *stats, int32_t *src_dst,
                   void *workspace, size_t workspace_bytes,
                   int32_t *err_flag, coact_stream_t stream);
+
+/*
+ * assign_replicas -- which replica serves each (token, slot).
+ * Cobalt, English abstract: EP distributes expert replicas across GPUs, and a
+ * communication-aware task assignment routes tokens to fewer remote nodes under the
+ * current expert layout.  Expert e has n_rep[e] replicas (1 <= n_rep[e] <= max_rep <=
+ * COACT_MAX_REPLICAS) on ranks rep_rank[e*max_rep + i], i < n_rep[e] (int32 DEVICE
+ * arrays).  Per token t (home rank s = src_rank[t], or floor(t*R/N) when src_rank is
+ * NULL; home node hn): slots whose expert has one replica take it; the other slots, j
+ * ascending, take the first replica (ascending i) in the first non-empty class -- (a) on
+ * s, (b) on a rank the token already uses, (c) on hn, (d) on a node the token already
+ * uses -- otherwise replica (t + j) mod n_rep[e].  slot_rank: int32 [N, k] out, the
+ * chosen rank per slot, -1 for every slot of an invalid token (bad or repeated id, bad
+ * home rank: COACT_EFLAG_ID_RANGE / _DUP_ID / _SRC_RANK; a replica table entry out of
+ * range: COACT_EFLAG_ID_RANGE).  The pages give no algorithm; this greedy is the reading
+ * taken.  Feed the result to plan_dispatch_slots.
+ */
+int assign_replicas(const int32_t *ids, int64_t N, int k, int E,
+                    const int32_t *rep_rank, int max_rep, const int32_t *n_rep, int R,
+                    const int32_t *rank_node, int n_nodes, const int32_t *src_rank,
+                    int32_t *slot_rank, int32_t *err_flag, coact_stream_t stream);
+
+/*
+ * plan_dispatch_slots -- plan_dispatch with a rank per slot instead of a rank per expert:
+ * slot (t, j) goes to slot_rank[t*k + j] (int32 [N, k] DEVICE, e.g. from assign_replicas;
+ * a value outside [0, R) makes the token invalid, COACT_EFLAG_ID_RANGE).  ids are still
+ * validated (range, repeats) and every output, layout and flag is as in plan_dispatch
+ * with expert_rank[ids[t,j]] replaced by slot_rank[t*k + j]; same workspace size.
+ */
+int plan_dispatch_slots(const int32_t *ids, int64_t N, int k, int E,
+                        const int32_t *slot_rank, int R,
+                        const int32_t *rank_node, int n_nodes,
+                        const int32_t *src_rank,
+                        int32_t *rank_counts, int32_t *rank_offsets, int32_t *asg_offsets,
+                        uint64_t *rank_mask,
+                        int32_t *row_token, uint8_t *row_kmask, int64_t row_capacity,
+                        int32_t *send_row, int32_t *comb_row,
+                        int64_t *stats, int32_t *src_dst,
+                        void *workspace, size_t workspace_bytes,
+                        int32_t *err_flag, coact_stream_t stream);
 
 /*
  * dispatch_gather -- fill the per-rank send buffers.

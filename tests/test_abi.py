@@ -162,6 +162,26 @@ def test_shuffle_rejects_bad_arguments(lib):
     assert f(None, 4, 100, 16, None, 0, None, 0, None, None) == 0       # nothing to write
 
 
+def test_replica_entry_points_reject_bad_arguments(lib):
+    a = lib.assign_replicas
+    a.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int,
+                  P, ctypes.c_int, P, P, P, P]
+    assert a(FAKE, 10, 2, 8, FAKE, 9, FAKE, 4, None, 1, None, FAKE, None, None) == -2   # max_rep 9
+    assert a(FAKE, 10, 2, 8, FAKE, 0, FAKE, 4, None, 1, None, FAKE, None, None) == -2   # max_rep 0
+    assert a(FAKE, 10, 2, 8, None, 2, FAKE, 4, None, 1, None, FAKE, None, None) == -1   # no table
+    assert a(FAKE, 10, 2, 8, FAKE, 2, FAKE, 65, None, 1, None, FAKE, None, None) == -2  # R > 64
+    assert a(None, 0, 2, 8, None, 2, None, 4, None, 1, None, None, None, None) == 0     # empty
+    p = lib.plan_dispatch_slots
+    p.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int,
+                  P, P, P, P, P, P, P, ctypes.c_int64, P, P, P, P, P, ctypes.c_size_t, P, P]
+    args = [FAKE, 10, 2, 8, None, 4, None, 1, None, FAKE, FAKE, FAKE, None, FAKE, FAKE, 20, FAKE,
+            FAKE, FAKE, None, FAKE, 1 << 20, None, None]
+    assert p(*args) == -1                                           # slot_rank NULL
+    args[4] = FAKE
+    args[2] = 9
+    assert p(*args) == -2                                           # k > 8
+
+
 def test_predict_rejects_bad_arguments(lib):
     p = lib.predict_home
     p.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int,

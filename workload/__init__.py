@@ -429,3 +429,37 @@ def pages_stats(r: Routing) -> dict:
     load = np.bincount(ids.ravel(), minlength=cfg.E)
     return {"group_coselect_share": share,
             "load_max_over_mean": float(load.max() / max(load.mean(), 1e-9))}
+
+
+# ----------------------------------------------------------------------------- replicas
+
+
+def replicate_hot(loads, expert_rank, rank_node, n_hot: int, max_rep: int = 2):
+    """Replica layout fixture (the pages give none; Cobalt says only that EP distributes
+    expert replicas across GPUs): every expert keeps its rank as replica 0; the n_hot most
+    loaded experts (ties: lower id) each get one more replica, heaviest first, on the
+    rank with the least current load among the ranks of other nodes (ties: lower rank),
+    counting half of the expert's load as moved there.  Returns (rep_rank int32
+    [E, max_rep] with -1 padding, n_rep int32 [E])."""
+    loads = np.asarray(loads, dtype=np.int64)
+    er = np.asarray(expert_rank, dtype=np.int64)
+    rn = np.asarray(rank_node, dtype=np.int64)
+    E, R = len(loads), len(rn)
+    rep = np.full((E, max_rep), -1, np.int32)
+    rep[:, 0] = er
+    n_rep = np.ones(E, np.int32)
+    rank_load = np.zeros(R, np.float64)
+    np.add.at(rank_load, er, loads.astype(np.float64))
+    hot = sorted(range(E), key=lambda e: (-loads[e], e))[:n_hot]
+    for e in hot:
+        if max_rep < 2:
+            break
+        cand = [r for r in range(R) if rn[r] != rn[er[e]]]
+        if not cand:
+            continue
+        r = min(cand, key=lambda q: (rank_load[q], q))
+        rep[e, 1] = r
+        n_rep[e] = 2
+        rank_load[er[e]] -= loads[e] / 2
+        rank_load[r] += loads[e] / 2
+    return rep, n_rep
