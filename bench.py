@@ -384,7 +384,9 @@ class TwoLayerStep:
 class TwoHopStep(OneLayerStep):
     """One layer with the two-hop dispatch (Cobalt: fewer remote nodes): count (side
     stream) -> node-level plan + rank-level plan + forward map -> hop-1 gather into node
-    segments -> hop-2 forward into rank segments -> combine."""
+    segments -> hop-2 forward into rank segments -> combine.  The forward runs in token
+    order (forward_gather_tokens: each hop-1 row read once) unless forward = "rows"."""
+    forward = "tokens"
     n_events = 6
     phases = {"coact_count": (0, 1), "plan_two_hop": (0, 2), "gather_hop1": (2, 3),
               "forward_hop2": (3, 4), "combine_scatter": (4, 5)}
@@ -416,7 +418,11 @@ class TwoHopStep(OneLayerStep):
         L.coact.dispatch_gather(L.x, self.th.node.send_row, self.hop1, err_flag=L.err,
                                 tma=L.tma)
         if ev: ev[3].record()
-        L.coact.forward_gather(self.hop1, self.th.fwd_src, L.send, err_flag=L.err)
+        if self.forward == "rows":
+            L.coact.forward_gather(self.hop1, self.th.fwd_src, L.send, err_flag=L.err)
+        else:
+            L.coact.forward_gather_tokens(self.hop1, self.th.rank.send_row, self.th.fwd_src,
+                                          L.send, err_flag=L.err)
         if ev: ev[4].record()
         L.coact.combine_scatter(L.y, L.gates, self.th.rank.comb_row, L.out, err_flag=L.err)
         main.wait_stream(self.side)
@@ -428,7 +434,10 @@ class TwoHopStep(OneLayerStep):
         D = int(self.th.rank.rank_offsets[-1].item())
         return [("gather_hop1", LayerBuffers.gather_kernel(),
                  (c.N + Dn) * c.H * 2 + c.N * c.k * 4),
-                ("forward_hop2", "k_forward_gather", 2 * D * c.H * 2 + D * 4),
+                (("forward_hop2", "k_forward_gather", 2 * D * c.H * 2 + D * 4)
+                 if self.forward == "rows" else
+                 ("forward_hop2", "k_forward_tokens",
+                  (Dn + D) * c.H * 2 + c.N * c.k * 4 + D * 4)),
                 ("combine_scatter", "k_combine_v16", self.L.bytes_combine())]
 
     def summary(self):
@@ -774,7 +783,8 @@ KERNEL_SOURCES = {"k_gather_v16": ("gather.cu", "common.cuh"),
                   "k_combine_units": ("combine.cu", "common.cuh"),
                   "k_combine_bwd": ("backward.cu", "common.cuh"),
                   "k_combine_v16": ("combine.cu", "common.cuh"),
-                  "k_forward_gather": ("twohop.cu", "common.cuh")}
+                  "k_forward_gather": ("twohop.cu", "common.cuh"),
+                  "k_forward_tokens": ("twohop.cu", "common.cuh")}
 
 
 def kernel_source_hash(kernel: str) -> str:
@@ -815,6 +825,7 @@ def run_gpu(args):
 
     cfg = workload.CONFIGS[args.config]
     LayerBuffers.tma = args.gather == "tma"
+    TwoHopStep.forward = args.forward
     mode = "shuffle" if args.shuffle else f"replicas:{args.replicas}" if args.replicas else \
         "backward" if args.pass_ == "backward" else (
         "prereduced" if args.combine == "prereduced" else "forward")
@@ -935,7 +946,8 @@ def run_gpu(args):
                             "combine of layer 1; predict_home; plan, gather, combine of layer 2"
                             if cfg.two_layer else
                             "coact_count (side stream) + two-hop plan (node and rank plans, "
-                            "forward map) + hop-1 gather + hop-2 forward + combine_scatter"
+                            f"forward map) + hop-1 gather + hop-2 forward ({args.forward}) + "
+                            "combine_scatter"
                             if args.two_hop else
                             "coact_count (side stream, overlapped with plan) + plan_dispatch + "
                             "dispatch_gather + combine_scatter (bf16 out)"),
@@ -1210,6 +1222,9 @@ def main():
                          "and choose replicas per token (assign_replicas)")
     ap.add_argument("--shuffle", action="store_true",
                     help="config 4: token shuffling fused into the post-attention reduce-scatter")
+    ap.add_argument("--forward", default="tokens", choices=["tokens", "rows"],
+                    help="two-hop forward: token order, each hop-1 row read once "
+                         "(forward_gather_tokens), or one read per rank row (forward_gather)")
     ap.add_argument("--two-hop", action="store_true",
                     help="dispatch in two hops: to nodes, then inside the node to ranks")
     args = ap.parse_args()

@@ -68,6 +68,7 @@ _lib.combine_scatter_peer.argtypes = [_P, _P, _P, _P, _I32, _P, _P, _I64, _I32, 
 _lib.coact_compose_map.argtypes = [_P, _I64, _P, _I64, _P, _P, _P]
 _lib.plan_forward.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _P, _P, _I64, _P, _P]
 _lib.forward_gather.argtypes = [_P, _I64, _I64, _P, _I64, _P, _P, _P]
+_lib.forward_gather_tokens.argtypes = [_P, _I64, _I64, _P, _I64, _I32, _P, _I64, _P, _P, _P]
 _lib.plan_dispatch_noalloc.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _P, _P,
                                        _P, _P, _P, _I64, _P, _P, _P, _P, _P, _P]
 for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "dispatch_gather_tma",
@@ -75,7 +76,7 @@ for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "dispatch_gather_t
            "combine_scatter_backward", "shuffle_reduce_scatter", "plan_dispatch_slots",
            "assign_replicas", "predict_home",
            "coact_place_correlated", "plan_dispatch_noalloc", "coact_compose_map", "plan_forward",
-           "forward_gather", "coact_rebalance_ranks", "dispatch_gather_peer",
+           "forward_gather", "forward_gather_tokens", "coact_rebalance_ranks", "dispatch_gather_peer",
            "combine_scatter_peer"):
     getattr(_lib, _f).restype = _I32
 
@@ -85,7 +86,8 @@ ABI_SYMBOLS = ("coact_strerror", "coact_abi_version", "coact_count", "plan_dispa
                "plan_dispatch_noalloc", "coact_compose_map", "plan_forward", "forward_gather",
                "coact_rebalance_ranks", "dispatch_gather_peer", "combine_scatter_peer",
                "combine_rows", "dispatch_gather_backward", "combine_scatter_backward",
-               "shuffle_reduce_scatter", "plan_dispatch_slots", "assign_replicas")
+               "shuffle_reduce_scatter", "plan_dispatch_slots", "assign_replicas",
+               "forward_gather_tokens")
 NOALLOC_MAX_TOKENS = 262144
 
 
@@ -555,6 +557,25 @@ def forward_gather(src: torch.Tensor, fwd_src: torch.Tensor, dst: torch.Tensor,
     _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
     _check(_lib.forward_gather(_ptr(src), src.shape[0], src.shape[1], _ptr(fwd_src), dst.shape[0],
                                _ptr(dst), _ptr(err_flag), _stream(stream)), "forward_gather")
+    return dst
+
+
+def forward_gather_tokens(src: torch.Tensor, send_row: torch.Tensor, fwd_src: torch.Tensor,
+                          dst: torch.Tensor, err_flag: Optional[torch.Tensor] = None,
+                          stream=None) -> torch.Tensor:
+    """forward_gather in token order: each hop-1 row read once and written to every rank
+    row it feeds (send_row: the rank plan's [N, k])."""
+    _need(_bits16(src), "src", torch.bfloat16)
+    _need(_bits16(dst), "dst", torch.bfloat16)
+    if src.shape[1] != dst.shape[1]:
+        raise ValueError("src and dst rows must have the same width")
+    _need(send_row, "send_row", torch.int32)
+    N, k = send_row.shape
+    _need(fwd_src, "fwd_src", torch.int32, (dst.shape[0],))
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.forward_gather_tokens(_ptr(src), src.shape[0], src.shape[1], _ptr(send_row), N, k,
+                                      _ptr(fwd_src), dst.shape[0], _ptr(dst), _ptr(err_flag),
+                                      _stream(stream)), "forward_gather_tokens")
     return dst
 
 

@@ -10,6 +10,9 @@
 //  * plan_forward       fwd_src[d] = the hop-1 (node-level) row that feeds rank-level
 //                       row d, -1 past D
 //  * forward_gather     dst[d] = src[fwd_src[d]]: the intra-node forward of hop 2
+//  * forward_gather_tokens  the same rows, token-major: a token's rank rows are grouped
+//                       by their hop-1 row, each hop-1 row is read once and written to
+//                       every rank row it feeds (reads Dn rows instead of D)
 #include <algorithm>
 
 #include "common.cuh"
@@ -138,6 +141,80 @@ __global__ void __launch_bounds__(256)
     raise_flag_warp(err, flags);
 }
 
+// Token-major forward: one warp per token.  Lane j < K holds the token's rank row
+// d_j = send_row[t, j] (first slot of each rank) and its hop-1 row s_j = fwd_src[d_j];
+// lanes with the same s_j form a group (warp ballots), the group's source row is read
+// once (UNROLL 16-byte loads per lane in flight) and stored to each of its rank rows.
+template <int K, int UNROLL>
+__global__ void __launch_bounds__(256)
+    k_forward_tokens(const uint4 *__restrict__ src, int64_t n_src, int64_t H16,
+                     const int32_t *__restrict__ send_row, int64_t N,
+                     const int32_t *__restrict__ fwd_src, int64_t n_rows, uint4 *__restrict__ dst,
+                     int32_t *__restrict__ err) {
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int64_t gwarp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    int flags = 0;
+    for (int64_t t = gwarp; t < N; t += nwarps) {
+        int d = -1, sr = -1;
+        if (lane < K) {
+            d = __ldg(send_row + t * K + lane);
+            if (d >= 0) {
+                if ((int64_t)d >= n_rows) {
+                    flags |= COACT_EFLAG_ROW_RANGE;
+                    d = -1;
+                } else {
+                    sr = __ldg(fwd_src + d);
+                    if ((int64_t)sr >= n_src) {
+                        flags |= COACT_EFLAG_ROW_RANGE;
+                        sr = -1;
+                    }
+                    if (sr < 0) d = -1;
+                }
+            } else if (d < -1) {
+                flags |= COACT_EFLAG_ROW_RANGE;
+                d = -1;
+            }
+        }
+        unsigned pending = __ballot_sync(0xffffffffu, d >= 0);
+        while (pending) {
+            const int s0 = __shfl_sync(0xffffffffu, sr, __ffs(pending) - 1);
+            const unsigned grp = __ballot_sync(0xffffffffu, d >= 0 && sr == s0) & pending;
+            pending &= ~grp;
+            const int m = __popc(grp);
+            int64_t drow[K];
+            unsigned g = grp;
+#pragma unroll
+            for (int i = 0; i < K; ++i) {
+                const int l = g ? __ffs(g) - 1 : 0;
+                drow[i] = __shfl_sync(0xffffffffu, d, l);
+                g &= g - 1;
+            }
+            const uint4 *in = src + (int64_t)s0 * H16;
+            for (int64_t c0 = 0; c0 < H16; c0 += 32 * UNROLL) {
+                uint4 v[UNROLL];
+#pragma unroll
+                for (int u = 0; u < UNROLL; ++u) {
+                    const int64_t c = c0 + u * 32 + lane;
+                    if (c < H16) v[u] = ld_stream(in + c);
+                }
+#pragma unroll
+                for (int i = 0; i < K; ++i) {
+                    if (i >= m) break;
+#pragma unroll
+                    for (int u = 0; u < UNROLL; ++u) {
+                        const int64_t c = c0 + u * 32 + lane;
+                        if (c < H16) st_stream(dst + drow[i] * H16 + c, v[u]);
+                    }
+                }
+            }
+        }
+    }
+    raise_flag_warp(err, flags);
+}
+
 }  // namespace
 }  // namespace coact
 
@@ -220,4 +297,47 @@ extern "C" int forward_gather(const uint16_t *src, int64_t n_src_rows, int64_t H
                           n_rows, dv, err_flag);
     return launch_pdl(k_forward_gather<8>, blocks, 256, 0, st, sv, n_src_rows, H16, fwd_src, n_rows,
                       dv, err_flag);
+}
+
+extern "C" int forward_gather_tokens(const uint16_t *src, int64_t n_src_rows, int64_t H,
+                                     const int32_t *send_row, int64_t N, int k,
+                                     const int32_t *fwd_src, int64_t n_rows, uint16_t *dst,
+                                     int32_t *err_flag, coact_stream_t stream) {
+    if (n_src_rows < 0 || H < 0 || n_rows < 0 || N < 0) return COACT_ERR_INVALID;
+    if (k < 1 || k > COACT_MAX_K) return COACT_ERR_UNSUPPORTED;
+    if (H % 8 != 0) return COACT_ERR_UNSUPPORTED;
+    if (N > (int64_t)INT32_MAX / k) return COACT_ERR_UNSUPPORTED;
+    if (N == 0 || n_rows == 0 || H == 0) return COACT_OK;
+    if (!send_row || !fwd_src || !dst || (n_src_rows > 0 && !src)) return COACT_ERR_INVALID;
+    if ((src && !aligned16(src)) || !aligned16(dst)) return COACT_ERR_INVALID;
+    DeviceInfo di;
+    if (int s = device_info(&di)) return s;
+    const int64_t H16 = H / 8;
+    const int blocks = (int)std::max<int64_t>(
+        1, std::min<int64_t>(ceil_div(N, 8), (int64_t)di.sm_count * 8));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const uint4 *sv = reinterpret_cast<const uint4 *>(src);
+    uint4 *dv = reinterpret_cast<uint4 *>(dst);
+#define COACT_FWT_CASE(KK)                                                                        \
+    case KK:                                                                                      \
+        if (H16 <= 32)                                                                            \
+            return launch_pdl(k_forward_tokens<KK, 1>, blocks, 256, 0, st, sv, n_src_rows, H16,   \
+                              send_row, N, fwd_src, n_rows, dv, err_flag);                        \
+        if (H16 <= 128)                                                                           \
+            return launch_pdl(k_forward_tokens<KK, 4>, blocks, 256, 0, st, sv, n_src_rows, H16,   \
+                              send_row, N, fwd_src, n_rows, dv, err_flag);                        \
+        return launch_pdl(k_forward_tokens<KK, 8>, blocks, 256, 0, st, sv, n_src_rows, H16,       \
+                          send_row, N, fwd_src, n_rows, dv, err_flag);
+    switch (k) {
+        COACT_FWT_CASE(1)
+        COACT_FWT_CASE(2)
+        COACT_FWT_CASE(3)
+        COACT_FWT_CASE(4)
+        COACT_FWT_CASE(5)
+        COACT_FWT_CASE(6)
+        COACT_FWT_CASE(7)
+        COACT_FWT_CASE(8)
+    }
+#undef COACT_FWT_CASE
+    return COACT_ERR_UNSUPPORTED;
 }

@@ -390,6 +390,19 @@ int forward_gather(const uint16_t *src, int64_t n_src_rows, int64_t H, const int
                    int64_t n_rows, uint16_t *dst, int32_t *err_flag, coact_stream_t stream);
 
 /*
+ * forward_gather_tokens -- forward_gather's rows in token order: for each token t, its
+ * rank rows d = send_row[t, j] >= 0 (the rank plan's [N, k]) are grouped by their hop-1
+ * row fwd_src[d]; each hop-1 row is read once and written to every rank row it feeds, so
+ * the forward reads Dn hop-1 rows instead of D.  Results equal forward_gather's for every
+ * rank row a token reaches (all d < D); other rows untouched.  A send_row entry below -1
+ * or >= n_rows, or an fwd_src entry >= n_src_rows, sets COACT_EFLAG_ROW_RANGE and is
+ * skipped.
+ */
+int forward_gather_tokens(const uint16_t *src, int64_t n_src_rows, int64_t H,
+                          const int32_t *send_row, int64_t N, int k, const int32_t *fwd_src,
+                          int64_t n_rows, uint16_t *dst, int32_t *err_flag, coact_stream_t stream);
+
+/*
  * Expert parallelism across GPUs (one process per GPU; EP rank s plans its own tokens for
  * all R destination ranks).  Cobalt / Zyphra, English abstracts: every MoE layer exchanges
  * tokens all-to-all to the GPUs holding their experts and combines the results back.

@@ -182,6 +182,17 @@ def test_replica_entry_points_reject_bad_arguments(lib):
     assert p(*args) == -2                                           # k > 8
 
 
+def test_forward_gather_tokens_rejects_bad_arguments(lib):
+    f = lib.forward_gather_tokens
+    f.argtypes = [P, ctypes.c_int64, ctypes.c_int64, P, ctypes.c_int64, ctypes.c_int, P,
+                  ctypes.c_int64, P, P, P]
+    assert f(FAKE, 10, 12, FAKE, 5, 2, FAKE, 20, FAKE, None, None) == -2     # H % 8 != 0
+    assert f(FAKE, 10, 16, FAKE, 5, 9, FAKE, 20, FAKE, None, None) == -2     # k > 8
+    assert f(FAKE, 10, 16, None, 5, 2, FAKE, 20, FAKE, None, None) == -1     # send_row NULL
+    assert f(P(258), 10, 16, FAKE, 5, 2, FAKE, 20, FAKE, None, None) == -1   # misaligned src
+    assert f(None, 0, 16, None, 0, 2, None, 0, None, None, None) == 0        # empty
+
+
 def test_predict_rejects_bad_arguments(lib):
     p = lib.predict_home
     p.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int,

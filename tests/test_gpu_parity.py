@@ -483,6 +483,39 @@ def test_two_hop_dispatch(coact, cfg, N):
     if D < cap:
         tail = np.unique(rng.integers(D, cap, 64))
         assert (host_bits(hop2[torch.as_tensor(tail, device=DEV)]) == 0xFFFF).all()
+    # the token-major forward writes the same rows, bit for bit, and nothing past D
+    hop2t = torch.empty_like(hop2)
+    hop2t.view(torch.int16).fill_(-1)
+    coact.forward_gather_tokens(hop1, th.rank.send_row, th.fwd_src, hop2t, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    assert torch.equal(hop2t.view(torch.int16), hop2.view(torch.int16))
+
+
+def test_forward_gather_tokens_flags(coact):
+    N, k, H = 40, 3, 64
+    src = workload.fill_bf16(10, H, 0, 5, device=DEV)
+    send_row = np.full((N, k), -1, np.int32)
+    send_row[:, 0] = np.arange(N)
+    send_row[:20, 1] = np.arange(N, N + 20)
+    send_row[3, 2] = 2 * N + 5                 # beyond n_rows: skipped, flagged
+    fwd = np.full(2 * N, -1, np.int32)
+    fwd[:N] = np.arange(N) % 10
+    fwd[N:N + 20] = (np.arange(20) * 3) % 10
+    fwd[7] = 12                                # beyond the hop-1 rows: skipped, flagged
+    dst = torch.full((2 * N, H), -1, dtype=torch.int16, device=DEV).view(torch.bfloat16)
+    err = zero_flag()
+    coact.forward_gather_tokens(src, cuda(send_row), cuda(fwd), dst, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == coact.EFLAG_ROW_RANGE
+    sb, db = host_bits(src), host_bits(dst)
+    for d in range(2 * N):
+        s_ = fwd[d]
+        reached = d < N or (N <= d < N + 20)
+        if reached and 0 <= s_ < 10:
+            assert np.array_equal(db[d], sb[s_]), d
+        else:
+            assert (db[d] == 0xFFFF).all(), d
 
 
 def test_forward_gather_flags_and_compose_map(coact):
