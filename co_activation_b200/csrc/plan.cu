@@ -28,7 +28,11 @@
 namespace coact {
 namespace {
 
+#if defined(COACT_PLAN_TILE)
+constexpr int kTile = COACT_PLAN_TILE;     // experiment builds (a multiple of 32, <= 1024)
+#else
 constexpr int kTile = 256;                 // tokens per tile, one per thread
+#endif
 constexpr int kTileWarps = kTile / 32;
 constexpr int kScanThreads = 1024;
 constexpr int kStatSlots = 6;              // per-tile partials (see TileStat)
@@ -590,9 +594,9 @@ namespace coact {
 namespace {
 
 // plan_dispatch and plan_dispatch_slots: the rank of each slot comes from expert_rank
-// (per expert) or slot_rank (per slot), exactly one of them non-NULL.
+// (per expert, per_slot false) or slot_rank (per slot, per_slot true).
 int plan_entry(const int32_t *ids, int64_t N, int k, int E, const int32_t *expert_rank,
-               const int32_t *slot_rank, int R, const int32_t *rank_node, int n_nodes,
+               const int32_t *slot_rank, bool per_slot, int R, const int32_t *rank_node, int n_nodes,
                const int32_t *src_rank, int32_t *rank_counts, int32_t *rank_offsets,
                int32_t *asg_offsets, uint64_t *rank_mask, int32_t *row_token, uint8_t *row_kmask,
                int64_t row_capacity, int32_t *send_row, int32_t *comb_row, int64_t *stats,
@@ -604,8 +608,8 @@ int plan_entry(const int32_t *ids, int64_t N, int k, int E, const int32_t *exper
     if (rank_node && (n_nodes < 1 || n_nodes > 64)) return COACT_ERR_UNSUPPORTED;
     if (!rank_node) n_nodes = 1;
     if (N > (int64_t)INT32_MAX / k || row_capacity > (int64_t)INT32_MAX) return COACT_ERR_UNSUPPORTED;
-    if ((!expert_rank && !slot_rank) || !rank_counts || !rank_offsets || !asg_offsets || !stats)
-        return COACT_ERR_INVALID;
+    if (per_slot ? (N > 0 && !slot_rank) : !expert_rank) return COACT_ERR_INVALID;
+    if (!rank_counts || !rank_offsets || !asg_offsets || !stats) return COACT_ERR_INVALID;
     if (N > 0 && (!ids || !send_row || !comb_row)) return COACT_ERR_INVALID;
     if (row_capacity > 0 && (!row_token || !row_kmask)) return COACT_ERR_INVALID;
     const size_t need = workspace_layout(N, R, nullptr, nullptr);
@@ -645,8 +649,7 @@ extern "C" int plan_dispatch(const int32_t *ids, int64_t N, int k, int E, const 
                              int64_t row_capacity, int32_t *send_row, int32_t *comb_row,
                              int64_t *stats, int32_t *src_dst, void *workspace,
                              size_t workspace_bytes, int32_t *err_flag, coact_stream_t stream) {
-    if (!expert_rank) return COACT_ERR_INVALID;
-    return plan_entry(ids, N, k, E, expert_rank, nullptr, R, rank_node, n_nodes, src_rank,
+    return plan_entry(ids, N, k, E, expert_rank, nullptr, false, R, rank_node, n_nodes, src_rank,
                       rank_counts, rank_offsets, asg_offsets, rank_mask, row_token, row_kmask,
                       row_capacity, send_row, comb_row, stats, src_dst, workspace, workspace_bytes,
                       err_flag, stream);
@@ -660,9 +663,7 @@ extern "C" int plan_dispatch_slots(const int32_t *ids, int64_t N, int k, int E,
                                    int32_t *send_row, int32_t *comb_row, int64_t *stats,
                                    int32_t *src_dst, void *workspace, size_t workspace_bytes,
                                    int32_t *err_flag, coact_stream_t stream) {
-    if (!slot_rank && N > 0) return COACT_ERR_INVALID;
-    static const int32_t kNone = 0;   // a non-NULL marker when N == 0 (never read)
-    return plan_entry(ids, N, k, E, nullptr, slot_rank ? slot_rank : &kNone, R, rank_node, n_nodes,
+    return plan_entry(ids, N, k, E, nullptr, slot_rank, true, R, rank_node, n_nodes,
                       src_rank, rank_counts, rank_offsets, asg_offsets, rank_mask, row_token,
                       row_kmask, row_capacity, send_row, comb_row, stats, src_dst, workspace,
                       workspace_bytes, err_flag, stream);
