@@ -404,14 +404,15 @@ def shuffle_plan(home: torch.Tensor, R: int, plan: Optional["Plan"] = None,
     rank alone (ids = home [N, 1], E = R, identity expert -> rank map).  plan.row_token
     lists the tokens grouped by home rank in ascending token order; rank r's output rows
     are [rank_offsets[r], rank_offsets[r+1])."""
-    if R < 2:
-        raise ValueError("token shuffling needs at least two ranks")
+    if R < 1:
+        raise ValueError("token shuffling needs at least one rank")
     _need(home, "home", torch.int32)
     N = home.shape[0]
+    E = max(R, 2)                  # the planner takes E >= 2; with one rank both map to it
     if plan is None:
-        plan = alloc_plan(N, 1, R, R, home.device, with_rank_mask=False, with_src_dst=False)
-    ident = torch.arange(R, dtype=torch.int32, device=home.device)
-    return plan_dispatch(home.view(N, 1), R, ident, R, plan, err_flag=err_flag, stream=stream)
+        plan = alloc_plan(N, 1, E, R, home.device, with_rank_mask=False, with_src_dst=False)
+    ident = torch.arange(E, dtype=torch.int32, device=home.device).clamp_(max=R - 1)
+    return plan_dispatch(home.view(N, 1), E, ident, R, plan, err_flag=err_flag, stream=stream)
 
 
 def shuffle_reduce_scatter(part_bases: torch.Tensor, N: int, row_token: torch.Tensor,

@@ -401,10 +401,11 @@ def shuffle_order(home, R: int) -> dict:
     """The shuffle's permutation: the dispatch plan of every token to its predicted home
     rank alone (k = 1, identity expert -> rank map): row_token lists the tokens grouped by
     home rank in ascending token order, rank_offsets delimits the ranks' segments."""
-    if R < 2:
-        raise ValueError("token shuffling needs at least two ranks")
+    if R < 1:
+        raise ValueError("token shuffling needs at least one rank")
     home = _c(home, np.int32)
-    return plan(home.reshape(-1, 1), R, np.arange(R, dtype=np.int32), R)
+    E = max(R, 2)                  # the plan takes E >= 2; with one rank both map to it
+    return plan(home.reshape(-1, 1), E, np.minimum(np.arange(E, dtype=np.int32), R - 1), R)
 
 
 def shuffle_reduce_f32chain(parts, row_token) -> np.ndarray:

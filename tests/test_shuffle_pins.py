@@ -86,6 +86,9 @@ def test_invalid_token_gives_a_zero_row():
     assert (out[0] != 0).any()
 
 
-def test_rejects_one_rank():
+def test_one_rank_is_the_identity():
+    o = oracle.shuffle_order([0, 0, 0, 0], 1)
+    assert o["row_token"][:4].tolist() == [0, 1, 2, 3]
+    assert o["rank_offsets"].tolist() == [0, 4]
     with pytest.raises(ValueError):
-        oracle.shuffle_order([0, 0, 0], 1)
+        oracle.shuffle_order([0], 0)
