@@ -227,6 +227,16 @@ class LayerBuffers:
         return c.N * c.k * c.H * 2 + c.N * c.H * 2 + c.N * c.k * 8
 
 
+def rank_balance(plan) -> dict:
+    """Receive-side balance of a plan: the busiest rank's rows and assignments over the
+    mean (1.0 = perfectly even)."""
+    rows = plan.rank_counts.cpu().numpy().astype(np.float64)
+    ao = plan.asg_offsets.cpu().numpy().astype(np.float64)
+    asg = ao[1:] - ao[:-1]
+    ratio = lambda a: float(a.max() / a.mean()) if a.mean() > 0 else 0.0
+    return {"rank_rows_max_over_mean": ratio(rows), "rank_asg_max_over_mean": ratio(asg)}
+
+
 def plan_launches(R: int, N: int) -> int:
     """Kernels plan_dispatch launches: 2 when R x tiles <= 4096 (scan folded), else 3."""
     return 2 if R * (-(-N // 256)) <= 4096 else 3
@@ -280,6 +290,7 @@ class OneLayerStep:
     def summary(self):
         L = self.L
         return {"dedup_rows_over_naive": L.D() / (self.N * self.cfg.k),
+                **rank_balance(L.plan),
                 "stats": dict(zip(L.coact.STAT_NAMES, L.plan.stats.cpu().tolist())),
                 "err_flag": int(L.err.item())}
 

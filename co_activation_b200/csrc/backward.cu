@@ -193,6 +193,7 @@ extern "C" int combine_scatter_backward(const uint16_t *y, int64_t n_rows, const
                                         const uint16_t *grad_out, int64_t H,
                                         uint16_t *grad_y, float *grad_gates, int32_t *err_flag,
                                         coact_stream_t stream) {
+    COACT_RANGE("combine_scatter_backward");
     if (N < 0 || H < 0 || n_rows < 0 || n_units < 0) return COACT_ERR_INVALID;
     if (k < 1 || k > COACT_MAX_K) return COACT_ERR_UNSUPPORTED;
     if (H % 8 != 0) return COACT_ERR_UNSUPPORTED;

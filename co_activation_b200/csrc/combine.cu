@@ -280,6 +280,7 @@ using namespace coact;
 extern "C" int combine_scatter(const uint16_t *y, int64_t n_rows, const float *gates,
                                const int32_t *comb_row, int64_t N, int k, int64_t H, void *out,
                                int out_dtype, int32_t *err_flag, coact_stream_t stream) {
+    COACT_RANGE("combine_scatter");
     if (N < 0 || H < 0 || n_rows < 0) return COACT_ERR_INVALID;
     if (k < 1 || k > COACT_MAX_K || (out_dtype != 0 && out_dtype != 1)) return COACT_ERR_UNSUPPORTED;
     if (H % 8 != 0) return COACT_ERR_UNSUPPORTED;
@@ -298,6 +299,7 @@ extern "C" int combine_rows(const uint16_t *y, int64_t n_rows, const float *gate
                             const uint8_t *row_kmask, int64_t n_units, const int32_t *unit_count,
                             int64_t H, void *out, int out_dtype, int32_t *err_flag,
                             coact_stream_t stream) {
+    COACT_RANGE("combine_rows");
     if (N < 0 || H < 0 || n_rows < 0 || n_units < 0) return COACT_ERR_INVALID;
     if (k < 1 || k > COACT_MAX_K || (out_dtype != 0 && out_dtype != 1)) return COACT_ERR_UNSUPPORTED;
     if (H % 8 != 0) return COACT_ERR_UNSUPPORTED;
@@ -317,6 +319,7 @@ extern "C" int dispatch_gather_backward(const uint16_t *grad_send, int64_t n_row
                                         const int32_t *send_row, int64_t N, int k, int64_t H,
                                         void *grad_x, int out_dtype, int32_t *err_flag,
                                         coact_stream_t stream) {
+    COACT_RANGE("dispatch_gather_backward");
     if (N < 0 || H < 0 || n_rows < 0) return COACT_ERR_INVALID;
     if (k < 1 || k > COACT_MAX_K || (out_dtype != 0 && out_dtype != 1)) return COACT_ERR_UNSUPPORTED;
     if (H % 8 != 0) return COACT_ERR_UNSUPPORTED;

@@ -5,6 +5,10 @@
 #include <stdint.h>
 
 #include <atomic>
+
+#if defined(COACT_NVTX)
+#include <nvtx3/nvToolsExt.h>
+#endif
 #include <utility>
 
 #include "coact.h"
@@ -166,6 +170,18 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
 }
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// NVTX range around each C-ABI call, for timeline profilers (builds with -DCOACT_NVTX; the
+// NVTX v3 headers are header-only and cost nothing when no tool is attached).
+#if defined(COACT_NVTX)
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
+#define COACT_RANGE(name) ::coact::NvtxRange coact_nvtx_range_(name)
+#else
+#define COACT_RANGE(name) ((void)0)
+#endif
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 

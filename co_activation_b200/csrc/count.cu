@@ -256,6 +256,7 @@ using namespace coact;
 extern "C" int coact_count(const int32_t *ids, int64_t N, int k, int E, const int32_t *ids2, int k2,
                            int E2, int64_t *pair, int64_t *loads, int32_t *err_flag,
                            coact_stream_t stream) {
+    COACT_RANGE("coact_count");
     if (N < 0 || !pair || (N > 0 && !ids)) return COACT_ERR_INVALID;
     if (k < 1 || k > COACT_MAX_K || E < 2 || E > COACT_MAX_E) return COACT_ERR_UNSUPPORTED;
     if (ids2 && (k2 < 1 || k2 > COACT_MAX_K || E2 < 2 || E2 > COACT_MAX_E))

@@ -309,6 +309,7 @@ int gather_args(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row
 extern "C" int dispatch_gather(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row,
                                int k, uint16_t *send, int64_t row_capacity, int32_t *err_flag,
                                coact_stream_t stream) {
+    COACT_RANGE("dispatch_gather");
     const int a = gather_args(x, N, H, send_row, k, send, row_capacity);
     if (a == -100) return COACT_OK;
     if (a) return a;
@@ -328,6 +329,7 @@ extern "C" int dispatch_gather(const uint16_t *x, int64_t N, int64_t H, const in
 extern "C" int dispatch_gather_tma(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row,
                                    int k, uint16_t *send, int64_t row_capacity, int32_t *err_flag,
                                    coact_stream_t stream) {
+    COACT_RANGE("dispatch_gather_tma");
     const int a = gather_args(x, N, H, send_row, k, send, row_capacity);
     if (a == -100) return COACT_OK;
     if (a) return a;

@@ -219,6 +219,7 @@ extern "C" int dispatch_gather_peer(const uint16_t *x, int64_t N, int64_t H, con
                                     const uint64_t *dst_bases, const int32_t *dst_row_offset,
                                     const int32_t *dst_capacity, int32_t *err_flag,
                                     coact_stream_t stream) {
+    COACT_RANGE("dispatch_gather_peer");
     if (N < 0 || H < 0) return COACT_ERR_INVALID;
     if (k < 1 || k > COACT_MAX_K || R < 1 || R > COACT_MAX_R) return COACT_ERR_UNSUPPORTED;
     if (H % 8 != 0) return COACT_ERR_UNSUPPORTED;
@@ -249,6 +250,7 @@ extern "C" int combine_scatter_peer(const uint64_t *y_bases, const int32_t *y_ro
                                     const float *gates, const int32_t *comb_row, int64_t N, int k,
                                     int64_t H, void *out, int out_dtype, int32_t *err_flag,
                                     coact_stream_t stream) {
+    COACT_RANGE("combine_scatter_peer");
     if (N < 0 || H < 0) return COACT_ERR_INVALID;
     if (k < 1 || k > COACT_MAX_K || R < 1 || R > COACT_MAX_R || (out_dtype != 0 && out_dtype != 1))
         return COACT_ERR_UNSUPPORTED;

@@ -15,9 +15,10 @@
 #include <algorithm>
 #include <vector>
 
-#include "coact.h"
+#include "common.cuh"
 
 extern "C" int coact_place_correlated(const int64_t *pair, int E, int R, int32_t *expert_rank) {
+    COACT_RANGE("coact_place_correlated");
     if (!pair || !expert_rank) return COACT_ERR_INVALID;
     if (E < 2 || E > COACT_MAX_E || R < 1 || R > COACT_MAX_R || E % R != 0)
         return COACT_ERR_UNSUPPORTED;
@@ -83,6 +84,7 @@ extern "C" int coact_place_correlated(const int64_t *pair, int E, int R, int32_t
 // lower rank).  Every rank ends with E/R experts; no expert changes node.
 extern "C" int coact_rebalance_ranks(const int64_t *loads, const int32_t *expert_node, int E,
                                      const int32_t *rank_node, int R, int32_t *expert_rank) {
+    COACT_RANGE("coact_rebalance_ranks");
     if (!loads || !expert_node || !rank_node || !expert_rank) return COACT_ERR_INVALID;
     if (E < 2 || E > COACT_MAX_E || R < 1 || R > COACT_MAX_R || E % R != 0)
         return COACT_ERR_UNSUPPORTED;

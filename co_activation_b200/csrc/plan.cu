@@ -649,6 +649,7 @@ extern "C" int plan_dispatch(const int32_t *ids, int64_t N, int k, int E, const 
                              int64_t row_capacity, int32_t *send_row, int32_t *comb_row,
                              int64_t *stats, int32_t *src_dst, void *workspace,
                              size_t workspace_bytes, int32_t *err_flag, coact_stream_t stream) {
+    COACT_RANGE("plan_dispatch");
     return plan_entry(ids, N, k, E, expert_rank, nullptr, false, R, rank_node, n_nodes, src_rank,
                       rank_counts, rank_offsets, asg_offsets, rank_mask, row_token, row_kmask,
                       row_capacity, send_row, comb_row, stats, src_dst, workspace, workspace_bytes,
@@ -663,6 +664,7 @@ extern "C" int plan_dispatch_slots(const int32_t *ids, int64_t N, int k, int E,
                                    int32_t *send_row, int32_t *comb_row, int64_t *stats,
                                    int32_t *src_dst, void *workspace, size_t workspace_bytes,
                                    int32_t *err_flag, coact_stream_t stream) {
+    COACT_RANGE("plan_dispatch_slots");
     return plan_entry(ids, N, k, E, nullptr, slot_rank, true, R, rank_node, n_nodes,
                       src_rank, rank_counts, rank_offsets, asg_offsets, rank_mask, row_token,
                       row_kmask, row_capacity, send_row, comb_row, stats, src_dst, workspace,
@@ -716,6 +718,7 @@ extern "C" int plan_dispatch_noalloc(const int32_t *ids, int64_t N, int k, int E
                                      int64_t row_capacity, int32_t *send_row, int32_t *comb_row,
                                      int64_t *stats, int32_t *src_dst, int32_t *err_flag,
                                      coact_stream_t stream) {
+    COACT_RANGE("plan_dispatch_noalloc");
     if (N < 0 || row_capacity < 0) return COACT_ERR_INVALID;
     if (N > COACT_NOALLOC_MAX_TOKENS) return COACT_ERR_UNSUPPORTED;
     if (k < 1 || k > COACT_MAX_K || E < 2 || E > COACT_MAX_E || R < 1 || R > COACT_MAX_R)

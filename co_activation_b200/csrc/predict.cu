@@ -78,6 +78,7 @@ extern "C" int predict_home(const int32_t *ids1, int64_t N, int k1, int E1, cons
                             int E2, const int32_t *expert_rank2, int R, int32_t *home,
                             void *workspace, size_t workspace_bytes, int32_t *err_flag,
                             coact_stream_t stream) {
+    COACT_RANGE("predict_home");
     if (N < 0) return COACT_ERR_INVALID;
     if (k1 < 1 || k1 > COACT_MAX_K || E1 < 2 || E1 > COACT_MAX_E || E2 < 2 || E2 > COACT_MAX_E ||
         R < 1 || R > COACT_MAX_R)

@@ -117,6 +117,7 @@ extern "C" int assign_replicas(const int32_t *ids, int64_t N, int k, int E, cons
                                int max_rep, const int32_t *n_rep, int R, const int32_t *rank_node,
                                int n_nodes, const int32_t *src_rank, int32_t *slot_rank,
                                int32_t *err_flag, coact_stream_t stream) {
+    COACT_RANGE("assign_replicas");
     if (N < 0) return COACT_ERR_INVALID;
     if (k < 1 || k > COACT_MAX_K || E < 2 || E > COACT_MAX_E || R < 1 || R > COACT_MAX_R ||
         max_rep < 1 || max_rep > COACT_MAX_REPLICAS)

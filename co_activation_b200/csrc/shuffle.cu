@@ -122,6 +122,7 @@ using namespace coact;
 extern "C" int shuffle_reduce_scatter(const uint64_t *part_bases, int P, int64_t N, int64_t H,
                                       const int32_t *row_token, int64_t n_out, void *out,
                                       int out_dtype, int32_t *err_flag, coact_stream_t stream) {
+    COACT_RANGE("shuffle_reduce_scatter");
     if (N < 0 || H < 0 || n_out < 0) return COACT_ERR_INVALID;
     if (P < 1 || P > COACT_MAX_R || (out_dtype != 0 && out_dtype != 1)) return COACT_ERR_UNSUPPORTED;
     if (H % 8 != 0) return COACT_ERR_UNSUPPORTED;

@@ -222,6 +222,7 @@ using namespace coact;
 
 extern "C" int coact_compose_map(const int32_t *a, int64_t n, const int32_t *b, int64_t nb,
                                  int32_t *out, int32_t *err_flag, coact_stream_t stream) {
+    COACT_RANGE("coact_compose_map");
     if (n < 0 || nb < 0) return COACT_ERR_INVALID;
     if (n == 0) return COACT_OK;
     if (!a || !b || !out) return COACT_ERR_INVALID;
@@ -237,6 +238,7 @@ extern "C" int plan_forward(const int32_t *ids, int64_t N, int k, int E, const i
                             const int32_t *rank_offsets, const int32_t *node_send_row,
                             int32_t *fwd_src, int64_t row_capacity, int32_t *err_flag,
                             coact_stream_t stream) {
+    COACT_RANGE("plan_forward");
     if (N < 0 || row_capacity < 0) return COACT_ERR_INVALID;
     if (k < 1 || k > COACT_MAX_K || E < 2 || E > COACT_MAX_E || R < 1 || R > COACT_MAX_R)
         return COACT_ERR_UNSUPPORTED;
@@ -276,6 +278,7 @@ extern "C" int plan_forward(const int32_t *ids, int64_t N, int k, int E, const i
 extern "C" int forward_gather(const uint16_t *src, int64_t n_src_rows, int64_t H,
                               const int32_t *fwd_src, int64_t n_rows, uint16_t *dst,
                               int32_t *err_flag, coact_stream_t stream) {
+    COACT_RANGE("forward_gather");
     if (n_src_rows < 0 || H < 0 || n_rows < 0) return COACT_ERR_INVALID;
     if (H % 8 != 0) return COACT_ERR_UNSUPPORTED;
     if (n_rows == 0 || H == 0) return COACT_OK;
@@ -303,6 +306,7 @@ extern "C" int forward_gather_tokens(const uint16_t *src, int64_t n_src_rows, in
                                      const int32_t *send_row, int64_t N, int k,
                                      const int32_t *fwd_src, int64_t n_rows, uint16_t *dst,
                                      int32_t *err_flag, coact_stream_t stream) {
+    COACT_RANGE("forward_gather_tokens");
     if (n_src_rows < 0 || H < 0 || n_rows < 0 || N < 0) return COACT_ERR_INVALID;
     if (k < 1 || k > COACT_MAX_K) return COACT_ERR_UNSUPPORTED;
     if (H % 8 != 0) return COACT_ERR_UNSUPPORTED;
