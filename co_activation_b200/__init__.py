@@ -41,6 +41,7 @@ _P, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_si
 _lib.coact_strerror.argtypes = [_I32]
 _lib.coact_strerror.restype = ctypes.c_char_p
 _lib.coact_abi_version.restype = _I32
+_lib.coact_last_cuda_error.restype = _I32
 _lib.coact_count.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _I32, _P, _P, _P, _P]
 _lib.plan_dispatch_workspace_bytes.argtypes = [_I64, _I32, _I32, _I32]
 _lib.plan_dispatch_workspace_bytes.restype = _SZ
@@ -80,7 +81,7 @@ for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "dispatch_gather_t
            "combine_scatter_peer"):
     getattr(_lib, _f).restype = _I32
 
-ABI_SYMBOLS = ("coact_strerror", "coact_abi_version", "coact_count", "plan_dispatch_workspace_bytes",
+ABI_SYMBOLS = ("coact_strerror", "coact_abi_version", "coact_last_cuda_error", "coact_count", "plan_dispatch_workspace_bytes",
                "plan_dispatch", "dispatch_gather", "dispatch_gather_tma", "combine_scatter",
                "predict_home_workspace_bytes", "predict_home", "coact_place_correlated",
                "plan_dispatch_noalloc", "coact_compose_map", "plan_forward", "forward_gather",
@@ -93,7 +94,11 @@ NOALLOC_MAX_TOKENS = 262144
 
 class CoactError(RuntimeError):
     def __init__(self, status: int, where: str):
-        super().__init__(f"{where}: {_lib.coact_strerror(status).decode()} (status {status})")
+        msg = f"{where}: {_lib.coact_strerror(status).decode()} (status {status})"
+        self.cuda_error = _lib.coact_last_cuda_error() if status == ERR_CUDA else 0
+        if self.cuda_error:
+            msg += f"; cudaError_t {self.cuda_error}"
+        super().__init__(msg)
         self.status = status
 
 

@@ -4,25 +4,30 @@
 namespace coact {
 
 namespace {
+thread_local int g_last_cuda = 0;
 std::atomic<int> g_sm_count[kMaxDevices];
 std::atomic<int> g_smem_optin[kMaxDevices];
 std::atomic<int> g_smem_sm[kMaxDevices];
 }  // namespace
 
+int cuda_fail(cudaError_t e) {
+    g_last_cuda = (int)e;
+    (void)cudaGetLastError();
+    return COACT_ERR_CUDA;
+}
+
 int device_info(DeviceInfo *out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return COACT_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return COACT_ERR_CUDA;
+    if (cudaError_t e = cudaGetDevice(&dev)) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return COACT_ERR_UNSUPPORTED;
     int sms = g_sm_count[dev].load(std::memory_order_relaxed);
     int smem = g_smem_optin[dev].load(std::memory_order_relaxed);
     int smem_sm = g_smem_sm[dev].load(std::memory_order_relaxed);
     if (sms <= 0 || smem <= 0 || smem_sm <= 0) {
-        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
-                cudaSuccess ||
-            cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
-                cudaSuccess)
-            return COACT_ERR_CUDA;
+        cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (!e) e = cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (!e) e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+        if (e) return cuda_fail(e);
         g_sm_count[dev].store(sms, std::memory_order_relaxed);
         g_smem_optin[dev].store(smem, std::memory_order_relaxed);
         g_smem_sm[dev].store(smem_sm, std::memory_order_relaxed);
@@ -49,3 +54,5 @@ extern "C" const char *coact_strerror(int status) {
 }
 
 extern "C" int coact_abi_version(void) { return COACT_ABI_VERSION; }
+
+extern "C" int coact_last_cuda_error(void) { return coact::g_last_cuda; }

@@ -113,6 +113,11 @@ int device_info(DeviceInfo *out);  // returns COACT_OK or COACT_ERR_CUDA
 constexpr int kMaxDevices = 64;
 
 // Largest dynamic shared-memory size already opted in, per device, for one kernel.
+// The CUDA error behind the last COACT_ERR_CUDA of this host thread (coact_last_cuda_error).
+// A failed call is recorded here and consumed (cudaGetLastError), so it is not reported
+// again by an unrelated later check.
+int cuda_fail(cudaError_t e);
+
 struct SmemOptIn {
     std::atomic<int> bytes[kMaxDevices];
 };
@@ -125,9 +130,9 @@ int ensure_smem(F kernel, size_t bytes, SmemOptIn &cache, const DeviceInfo &di) 
     if (bytes > (size_t)di.smem_optin) return COACT_ERR_UNSUPPORTED;
     std::atomic<int> &slot = cache.bytes[di.device];
     if (slot.load(std::memory_order_relaxed) >= (int)bytes) return COACT_OK;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
-        cudaSuccess)
-        return COACT_ERR_CUDA;
+    if (cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)bytes))
+        return cuda_fail(e);
     slot.store((int)bytes, std::memory_order_relaxed);
     return COACT_OK;
 }
@@ -143,7 +148,8 @@ inline int blocks_per_sm(int threads, size_t smem, const DeviceInfo &di) {
 }
 
 inline int launch_status() {
-    return cudaGetLastError() == cudaSuccess ? COACT_OK : COACT_ERR_CUDA;
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? COACT_OK : cuda_fail(e);
 }
 
 // Launches `kernel` on `stream` with programmatic stream serialisation (see pdl_wait).
@@ -164,9 +170,8 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
     cfg.attrs = attr;
     cfg.numAttrs = 1;
 #endif
-    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess
-               ? COACT_OK
-               : COACT_ERR_CUDA;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    return e == cudaSuccess ? COACT_OK : cuda_fail(e);
 }
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -700,7 +700,8 @@ std::atomic<void *> g_plan_scratch_addr[kMaxDevices];
 int noalloc_scratch(const DeviceInfo &di, void **out) {
     void *p = g_plan_scratch_addr[di.device].load(std::memory_order_acquire);
     if (!p) {
-        if (cudaGetSymbolAddress(&p, g_plan_scratch) != cudaSuccess || !p) return COACT_ERR_CUDA;
+        if (cudaError_t e = cudaGetSymbolAddress(&p, g_plan_scratch)) return cuda_fail(e);
+        if (!p) return COACT_ERR_CUDA;
         g_plan_scratch_addr[di.device].store(p, std::memory_order_release);
     }
     *out = p;

@@ -84,6 +84,13 @@ const char *coact_strerror(int status);
 
 /* ABI version of this header (bumped on any signature change). */
 int coact_abi_version(void);
+
+/*
+ * coact_last_cuda_error -- the cudaError_t behind the last COACT_ERR_CUDA returned on the
+ * calling host thread (0 if none).  A failed CUDA call inside the library is recorded
+ * here and consumed, so no later, unrelated cudaGetLastError check reports it again.
+ */
+int coact_last_cuda_error(void);
 #define COACT_ABI_VERSION 1
 
 /*

@@ -52,6 +52,11 @@ def test_binding_names_match_header():
         assert callable(getattr(coact, f))
 
 
+def test_last_cuda_error_starts_clear(lib):
+    lib.coact_last_cuda_error.restype = ctypes.c_int
+    assert lib.coact_last_cuda_error() == 0
+
+
 def test_strerror_and_version(lib):
     lib.coact_strerror.restype = ctypes.c_char_p
     assert lib.coact_strerror(0) == b"ok"
