@@ -91,7 +91,13 @@ int coact_abi_version(void);
  * here and consumed, so no later, unrelated cudaGetLastError check reports it again.
  */
 int coact_last_cuda_error(void);
-#define COACT_ABI_VERSION 1
+
+/* ABI versions (additions only; no earlier call changed meaning):
+ *   1  count, plan, gather, combine, predict_home, placement, two-hop, peer calls, noalloc
+ *   2  dispatch_gather_tma, backward (dispatch_gather_backward, combine_scatter_backward),
+ *      combine_rows, shuffle_reduce_scatter, assign_replicas, plan_dispatch_slots,
+ *      forward_gather_tokens, coact_last_cuda_error; combine_scatter_peer takes NULL gates */
+#define COACT_ABI_VERSION 2
 
 /*
  * coact_count -- expert co-activation pair counts and per-expert loads.

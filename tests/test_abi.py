@@ -61,7 +61,7 @@ def test_strerror_and_version(lib):
     lib.coact_strerror.restype = ctypes.c_char_p
     assert lib.coact_strerror(0) == b"ok"
     assert b"workspace" in lib.coact_strerror(-4)
-    assert lib.coact_abi_version() == 1
+    assert lib.coact_abi_version() == 2
 
 
 P = ctypes.c_void_p
