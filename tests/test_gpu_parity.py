@@ -393,6 +393,41 @@ def test_identity_experts_end_to_end(coact, cfg):
     assert np.array_equal(out.cpu().numpy().view(np.uint32), want.view(np.uint32))
 
 
+@pytest.mark.parametrize("cfg,seed", [(1, 1), (1, 7), (2, 3), (3, 5)])
+def test_whole_path_other_seeds(coact, cfg, seed):
+    """The whole path on other seeded batches of the configurations (full N): counts and
+    plan bit-exact, sampled gathered rows bit-exact, sampled combined rows equal to the
+    oracle's fixed-order chain."""
+    r = workload.make_routing(cfg, seed=seed)
+    c = r.cfg
+    H = min(c.H, 2048)
+    pair = torch.zeros((c.E, c.E), dtype=torch.int64, device=DEV)
+    loads = torch.zeros(c.E, dtype=torch.int64, device=DEV)
+    coact.coact_count(cuda(r.ids), c.E, pair, loads)
+    op, ol, _ = oracle.count(r.ids, c.E)
+    assert np.array_equal(pair.cpu().numpy(), op) and np.array_equal(loads.cpu().numpy(), ol)
+    plan, err = run_plan(coact, r)
+    o = oracle_plan_for(r)
+    assert err.item() == 0
+    assert_plan_equal(plan_to_host(plan), o)
+    x = workload.fill_bf16(r.N, H, seed, X_STREAM, device=DEV)
+    send = torch.empty((plan.row_capacity, H), dtype=torch.bfloat16, device=DEV)
+    coact.dispatch_gather(x, plan.send_row, send)
+    y = workload.fill_bf16(r.N * r.k, H, seed, Y_STREAM, device=DEV)
+    out = torch.empty((r.N, H), dtype=torch.bfloat16, device=DEV)
+    coact.combine_scatter(y, cuda(r.gates), plan.comb_row, out)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([rng.integers(0, o["D"], 400), [0, o["D"] - 1]]))
+    want = host_bits(workload.fill_bf16(len(rows), H, seed, X_STREAM, row_ids=o["row_token"][rows]))
+    assert np.array_equal(host_bits(send[torch.as_tensor(rows, device=DEV)]), want)
+    toks = np.unique(np.concatenate([rng.integers(0, r.N, 200), [0, r.N - 1]]))
+    cr = o["comb_row"][toks]
+    yh = host_bits(workload.fill_bf16(cr.size, H, seed, Y_STREAM, row_ids=cr.ravel()))
+    check_combine(out, yh, r.gates[toks], np.arange(cr.size, dtype=np.int32).reshape(cr.shape),
+                  tokens=toks)
+
+
 def test_token_shuffle_two_layers(coact):
     """Config 4: cross-layer counts on a calibration batch -> predicted home rank ->
     layer-2 plan with the tokens pre-sharded to it; every step against the oracle."""
