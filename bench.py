@@ -300,10 +300,10 @@ class TwoLayerStep:
     ranks; then cross-layer counts (layer-1 x layer-2 picks, accumulated for the next
     prediction), home-rank prediction from the calibration counts, and layer 2 with its
     tokens pre-sharded to the predicted rank; layer 2's input rows are layer 1's output."""
-    n_events = 10
+    n_events = 11
     phases = {"layer1_plan": (0, 1), "layer1_gather": (1, 2), "layer1_combine": (2, 3),
-              "predict_home": (3, 4), "layer2_plan": (4, 5), "layer2_gather": (5, 6),
-              "layer2_combine": (6, 7), "side_counts": (0, 8)}   # ev8 on the side stream
+              "layer2_plan": (4, 5), "layer2_gather": (5, 6), "layer2_combine": (6, 7),
+              "side_counts": (0, 8), "side_predict_home": (8, 9)}   # ev8, ev9: side stream
 
     def __init__(self, coact, tl: workload.TwoLayer, device, fill: bool = True, C12=None):
         self.coact, self.tl = coact, tl
@@ -323,6 +323,7 @@ class TwoLayerStep:
             coact.coact_count(to(tl.calib1), E, C12, ids2=to(tl.calib2), E2=E)
         self.C12 = C12
         self.side = torch.cuda.Stream(device=device)
+        self.home_ready = torch.cuda.Event()
         # counts: 2 per layer-set + 1 cross; two plans; 2 gathers; 2 combines; predict 2
         self.kernels_per_step = 3 + 2 * plan_launches(R, self.N) + 2 + 2 + 2
 
@@ -344,19 +345,24 @@ class TwoLayerStep:
         self.side.wait_stream(main)
         if ev: ev[0].record()
         with torch.cuda.stream(self.side):
+            # statistics, and the layer-2 home prediction: it needs only layer 1's picks
+            # and the calibration counts, so it runs beside layer 1's dispatch and combine
             self.L1.count()
             c.coact_count(self.L1.ids, E, self.C12_live, ids2=self.L2.ids, E2=E,
                           err_flag=self.L1.err)
             self.L2.count()
             if ev: ev[8].record()
+            c.predict_home(self.L1.ids, E, self.C12, self.L2.expert_rank, R, self.home,
+                           workspace=self.pws, err_flag=self.L1.err)
+            if ev: ev[9].record()
+            self.home_ready.record(self.side)
         self.L1.plan_()
         if ev: ev[1].record()
         self.L1.gather()
         if ev: ev[2].record()
         self.L1.combine()
         if ev: ev[3].record()
-        c.predict_home(self.L1.ids, E, self.C12, self.L2.expert_rank, R, self.home,
-                       workspace=self.pws, err_flag=self.L1.err)
+        main.wait_event(self.home_ready)
         if ev: ev[4].record()
         self.L2.plan_()
         if ev: ev[5].record()
@@ -365,7 +371,7 @@ class TwoLayerStep:
         self.L2.combine()
         if ev: ev[7].record()
         main.wait_stream(self.side)
-        if ev: ev[9].record()
+        if ev: ev[10].record()
 
     def roofline_parts(self):
         D1, D2 = self.L1.D(), self.L2.D()
@@ -953,8 +959,9 @@ def run_gpu(args):
                    "pass": mode,
                    "gather": ("dispatch_gather_tma (TMA bulk copies)" if LayerBuffers.tma
                               else "dispatch_gather (16-byte vector copies)"),
-                   "step": getattr(S, "step_desc", None) or ("two layers: counts + cross-layer counts (side stream); plan, gather, "
-                            "combine of layer 1; predict_home; plan, gather, combine of layer 2"
+                   "step": getattr(S, "step_desc", None) or ("two layers: counts + cross-layer counts + predict_home (side stream, "
+                            "beside layer 1); plan, gather, combine of layer 1; plan, gather, "
+                            "combine of layer 2"
                             if cfg.two_layer else
                             "coact_count (side stream) + two-hop plan (node and rank plans, "
                             f"forward map) + hop-1 gather + hop-2 forward ({args.forward}) + "
