@@ -53,6 +53,7 @@ def _get():
                                          I64, P, P, P, P]
             _lib.oracle_plan_slots.argtypes = _lib.oracle_plan.argtypes
             _lib.oracle_assign_replicas.argtypes = [P, I64, I32, I32, P, I32, P, I32, P, I32, P, P]
+            _lib.oracle_place_replicas.argtypes = [P, P, P, I32, P, I32, I32, I32, P, P]
             _lib.oracle_gather.argtypes = [P, I64, P, I64, P]
             _lib.oracle_gather.restype = None
             _lib.oracle_combine_f64.argtypes = [P, I64, P, P, I64, I32, I64, P]
@@ -436,3 +437,18 @@ def assign_replicas(ids, E: int, rep_rank, n_rep, R: int, rank_node=None, n_node
     f = _get().oracle_assign_replicas(_p(ids), N, k, E, _p(rr), rr.shape[1], _p(nr), R, _p(rn),
                                       n_nodes, _p(sr), _p(out))
     return out, f
+
+
+def place_replicas(pair, loads, expert_rank, rank_node, budget: int, max_rep: int = 2):
+    """Replica layout from co-activation and load statistics: (rep_rank int32 [E, max_rep]
+    with -1 padding, n_rep int32 [E], replicas added)."""
+    pr = _c(pair, np.int64)
+    ld = _c(loads, np.int64)
+    er = _c(expert_rank, np.int32)
+    rn = _c(rank_node, np.int32)
+    E, R = len(ld), len(rn)
+    rep = np.zeros((E, max_rep), np.int32)
+    nrep = np.zeros(E, np.int32)
+    added = _get().oracle_place_replicas(_p(pr), _p(ld), _p(er), E, _p(rn), R, budget, max_rep,
+                                         _p(rep), _p(nrep))
+    return rep, nrep, added

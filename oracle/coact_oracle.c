@@ -754,3 +754,96 @@ int oracle_assign_replicas(const int32_t *ids, int64_t N, int k, int E, const in
     }
     return flags;
 }
+
+/* ------------------------------------------------------------------------------------
+ * Replica placement.
+ *
+ * [Cobalt] EP distributes expert replicas across GPUs; its planner acts on co-activation
+ * and workload statistics.  The pages give no algorithm; reading taken (integer
+ * arithmetic throughout: an expert's load is shared equally by its replicas, counted in
+ * units of 1/840 so every share is exact for up to 8 replicas):
+ *   every expert starts with its rank as replica 0; rank_load[r] = sum over the experts
+ *   with a replica on r of loads[e]*840/n_rep[e].  Then, budget times:
+ *   1. r* = the rank with the largest load (ties: lower rank);
+ *   2. e* = among r*'s experts with fewer than max_rep replicas, the one with the largest
+ *      share loads[e]*840/n_rep[e] (ties: lower id); none -> stop;
+ *   3. candidate ranks: those without a replica of e*, on a node without one if any such
+ *      rank exists; among them the node with the largest affinity
+ *      A(node) = sum over experts f != e* whose replica 0 is on the node of
+ *      pair[e*][f] + pair[f][e*] (ties: lower node), then on it the rank with the
+ *      smallest load (ties: lower rank); none -> stop;
+ *   4. add that rank as e*'s next replica and recompute the shares of e*'s replicas.
+ * Returns the number of replicas added.  rep_rank [E*max_rep] (-1 padded), n_rep [E].
+ * ------------------------------------------------------------------------------------ */
+int oracle_place_replicas(const int64_t *pair, const int64_t *loads, const int32_t *expert_rank,
+                          int E, const int32_t *rank_node, int R, int budget, int max_rep,
+                          int32_t *rep_rank, int32_t *n_rep) {
+    const int64_t L = 840;
+    int64_t *rank_load = (int64_t *)calloc((size_t)R, sizeof(int64_t));
+    int n_nodes = 1;
+    for (int r = 0; r < R; ++r)
+        if (rank_node[r] + 1 > n_nodes) n_nodes = rank_node[r] + 1;
+    int64_t *aff = (int64_t *)calloc((size_t)n_nodes, sizeof(int64_t));
+    for (int e = 0; e < E; ++e) {
+        for (int i = 0; i < max_rep; ++i) rep_rank[e * max_rep + i] = -1;
+        rep_rank[e * max_rep] = expert_rank[e];
+        n_rep[e] = 1;
+        rank_load[expert_rank[e]] += loads[e] * L;
+    }
+    int added = 0;
+    for (int b = 0; b < budget; ++b) {
+        int rs = 0;                                              /* step 1 */
+        for (int r = 1; r < R; ++r)
+            if (rank_load[r] > rank_load[rs]) rs = r;
+        int es = -1;                                             /* step 2 */
+        int64_t best_share = -1;
+        for (int e = 0; e < E; ++e) {
+            if (n_rep[e] >= max_rep) continue;
+            int on = 0;
+            for (int i = 0; i < n_rep[e]; ++i) on |= rep_rank[e * max_rep + i] == rs;
+            if (!on) continue;
+            int64_t share = loads[e] * L / n_rep[e];
+            if (share > best_share) { best_share = share; es = e; }
+        }
+        if (es < 0) break;
+        /* step 3: ranks and nodes that already hold a replica of es */
+        char *has_rank = (char *)calloc((size_t)R, 1);
+        char *has_node = (char *)calloc((size_t)n_nodes, 1);
+        for (int i = 0; i < n_rep[es]; ++i) {
+            has_rank[rep_rank[es * max_rep + i]] = 1;
+            has_node[rank_node[rep_rank[es * max_rep + i]]] = 1;
+        }
+        int fresh_node_exists = 0;
+        for (int r = 0; r < R; ++r)
+            if (!has_rank[r] && !has_node[rank_node[r]]) fresh_node_exists = 1;
+        for (int n = 0; n < n_nodes; ++n) aff[n] = 0;
+        for (int f = 0; f < E; ++f)
+            if (f != es) aff[rank_node[expert_rank[f]]] += pair[(int64_t)es * E + f] + pair[(int64_t)f * E + es];
+        int bn = -1;
+        for (int n = 0; n < n_nodes; ++n) {
+            int usable = 0;
+            for (int r = 0; r < R; ++r)
+                if (rank_node[r] == n && !has_rank[r] && (!fresh_node_exists || !has_node[n])) usable = 1;
+            if (!usable) continue;
+            if (bn < 0 || aff[n] > aff[bn]) bn = n;
+        }
+        int rt = -1;
+        if (bn >= 0)
+            for (int r = 0; r < R; ++r) {
+                if (rank_node[r] != bn || has_rank[r]) continue;
+                if (rt < 0 || rank_load[r] < rank_load[rt]) rt = r;
+            }
+        free(has_rank);
+        free(has_node);
+        if (rt < 0) break;
+        /* step 4 */
+        for (int i = 0; i < n_rep[es]; ++i) rank_load[rep_rank[es * max_rep + i]] -= loads[es] * L / n_rep[es];
+        rep_rank[es * max_rep + n_rep[es]] = rt;
+        n_rep[es] += 1;
+        for (int i = 0; i < n_rep[es]; ++i) rank_load[rep_rank[es * max_rep + i]] += loads[es] * L / n_rep[es];
+        added += 1;
+    }
+    free(rank_load);
+    free(aff);
+    return added;
+}

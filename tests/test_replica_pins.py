@@ -115,3 +115,78 @@ def test_validation_flags():
     got, f = oracle.assign_replicas(ids, 2, np.array([[0, 1], [2, 3]], np.int32),
                                     np.array([2, 2], np.int32), 4, src_rank=[0, 9, 2])
     assert f & 8 and (got[1] == -1).all() and (got[[0, 2]] >= 0).all()
+
+
+# ----------------------------------------------------------------------------- replica placement
+
+
+def sym_pairs(E, w):
+    p = np.zeros((E, E), np.int64)
+    for (a, b), v in w.items():
+        p[a, b] = p[b, a] = v
+    return p
+
+
+def rank_loads(rep, n_rep, loads, R):
+    out = np.zeros(R, np.int64)
+    for e in range(len(loads)):
+        for i in range(n_rep[e]):
+            out[rep[e, i]] += loads[e] * 840 // n_rep[e]
+    return out
+
+
+def test_placement_hand_worked_fresh_node():
+    # ranks 0,1 on node 0, ranks 2,3 on node 1; rank 0 is the heaviest (experts 0, 1) and
+    # expert 0 its heaviest share; the only node without a replica of it is node 1, whose
+    # lighter rank is 3
+    pair = sym_pairs(4, {(0, 2): 5, (0, 3): 1})
+    rep, n_rep, added = oracle.place_replicas(pair, [10, 1, 2, 3], [0, 0, 1, 2], [0, 0, 1, 1], 1)
+    assert added == 1
+    assert rep.tolist() == [[0, 3], [0, -1], [1, -1], [2, -1]] and n_rep.tolist() == [2, 1, 1, 1]
+
+
+def test_placement_hand_worked_affinity_picks_the_node():
+    # one rank per node; expert 0 (rank 0) is co-activated with expert 2 (node 2) more than
+    # with expert 1 (node 1): its replica goes to node 2
+    pair = sym_pairs(3, {(0, 1): 1, (0, 2): 4})
+    rep, n_rep, _ = oracle.place_replicas(pair, [9, 2, 2], [0, 1, 2], [0, 1, 2], 1)
+    assert rep[0].tolist() == [0, 2]
+    # without co-activation the lower node wins the tie
+    rep, _, _ = oracle.place_replicas(np.zeros((3, 3), np.int64), [9, 2, 2], [0, 1, 2], [0, 1, 2], 1)
+    assert rep[0].tolist() == [0, 1]
+
+
+def test_placement_budget_zero_and_exhaustion():
+    er, rn = [0, 1, 2, 3], [0, 0, 1, 1]
+    rep, n_rep, added = oracle.place_replicas(np.zeros((4, 4), np.int64), [5, 4, 3, 2], er, rn, 0)
+    assert added == 0 and rep[:, 0].tolist() == er and (n_rep == 1).all()
+    # max_rep 2 on 4 experts: at most 4 replicas can be added, then the loop stops
+    rep, n_rep, added = oracle.place_replicas(np.zeros((4, 4), np.int64), [5, 4, 3, 2], er, rn, 50)
+    assert added == 4 and (n_rep == 2).all()
+    for e in range(4):
+        assert len(set(rep[e].tolist())) == 2                 # distinct ranks per expert
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_placement_invariants_random(seed):
+    rng = np.random.default_rng(700 + seed)
+    R = int(rng.choice([4, 8, 16]))
+    n_nodes = int(rng.choice([1, 2, 4]))
+    E = R * int(rng.integers(1, 5))
+    rn = (np.arange(R) * n_nodes // R).astype(np.int32)
+    er = rng.permutation(np.arange(E) % R).astype(np.int32)
+    loads = rng.zipf(1.5, E).astype(np.int64) * 10
+    pair = rng.integers(0, 20, (E, E)).astype(np.int64)
+    max_rep = int(rng.integers(2, 5))
+    budget = int(rng.integers(1, E))
+    rep, n_rep, added = oracle.place_replicas(pair, loads, er, rn, budget, max_rep)
+    assert added == int((n_rep - 1).sum()) and added <= budget
+    assert (rep[:, 0] == er).all() and (n_rep <= max_rep).all()
+    for e in range(E):
+        rs = rep[e, :n_rep[e]].tolist()
+        assert len(set(rs)) == len(rs) and all(0 <= r < R for r in rs)
+        assert (rep[e, n_rep[e]:] == -1).all()
+    # replicas only ever take load off the heaviest rank
+    before = rank_loads(er[:, None], np.ones(E, np.int32), loads, R)
+    after = rank_loads(rep, n_rep, loads, R)
+    assert after.sum() <= before.sum() and after.max() <= before.max()
