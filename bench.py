@@ -545,19 +545,33 @@ class ReplicaStep(OneLayerStep):
     phases = {"coact_count": (0, 1), "assign_replicas": (0, 2), "plan_dispatch": (2, 3),
               "dispatch_gather": (3, 4), "combine_scatter": (4, 5)}
 
+    layout_kind = "hot"        # "hot": workload.replicate_hot; "planned": coact_place_replicas
+
     def __init__(self, coact, r: workload.Routing, device, n_hot: int, fill: bool = True):
         super().__init__(coact, r, device, fill)
         c = r.cfg
-        loads = np.bincount(r.ids.ravel(), minlength=c.E)        # the batch's expert loads
-        self.rep_h, self.nrep_h = workload.replicate_hot(loads, r.expert_rank, r.rank_node, n_hot)
+        if self.layout_kind == "planned":
+            # the library's planner over the batch's own counts (library calls)
+            to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+            pair = torch.zeros((c.E, c.E), dtype=torch.int64, device=device)
+            loads = torch.zeros(c.E, dtype=torch.int64, device=device)
+            coact.coact_count(to(r.ids), c.E, pair, loads)
+            rep, nrep, _ = coact.coact_place_replicas(pair, loads, torch.from_numpy(r.expert_rank),
+                                                       torch.from_numpy(r.rank_node), n_hot)
+            self.rep_h, self.nrep_h = rep.numpy(), nrep.numpy()
+        else:
+            loads = np.bincount(r.ids.ravel(), minlength=c.E)    # the batch's expert loads
+            self.rep_h, self.nrep_h = workload.replicate_hot(loads, r.expert_rank, r.rank_node,
+                                                             n_hot)
         to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
         self.rep, self.nrep = to(self.rep_h), to(self.nrep_h)
         self.slot = torch.empty((c.N, c.k), dtype=torch.int32, device=device)
         self.n_hot = n_hot
         self.kernels_per_step = 1 + 1 + plan_launches(c.R, self.N) + 1 + 1
-        self.step_desc = (f"coact_count (side stream) + assign_replicas ({n_hot} hottest experts "
-                          "with a second replica on another node) + plan_dispatch_slots + "
-                          "dispatch_gather + combine_scatter (bf16 out)")
+        layout = ("coact_place_replicas over the batch's counts" if self.layout_kind == "planned"
+                  else "the hottest experts with a second replica on another node")
+        self.step_desc = (f"coact_count (side stream) + assign_replicas ({n_hot} replicas: {layout})"
+                          " + plan_dispatch_slots + dispatch_gather + combine_scatter (bf16 out)")
 
     def clone_for_copy(self, coact, device):
         return ReplicaStep(coact, self.L.r, device, self.n_hot, fill=False)
@@ -843,6 +857,7 @@ def run_gpu(args):
     cfg = workload.CONFIGS[args.config]
     LayerBuffers.tma = args.gather == "tma"
     TwoHopStep.forward = args.forward
+    ReplicaStep.layout_kind = args.replica_layout
     mode = "shuffle" if args.shuffle else f"replicas:{args.replicas}" if args.replicas else \
         "backward" if args.pass_ == "backward" else (
         "prereduced" if args.combine == "prereduced" else "forward")
@@ -1238,6 +1253,9 @@ def main():
     ap.add_argument("--replicas", type=int, default=0, metavar="N_HOT",
                     help="give the N_HOT most loaded experts a second replica on another node "
                          "and choose replicas per token (assign_replicas)")
+    ap.add_argument("--replica-layout", default="hot", choices=["hot", "planned"],
+                    help="which experts get the replicas: the most loaded (fixture) or "
+                         "coact_place_replicas over the batch's counts")
     ap.add_argument("--shuffle", action="store_true",
                     help="config 4: token shuffling fused into the post-attention reduce-scatter")
     ap.add_argument("--forward", default="tokens", choices=["tokens", "rows"],

@@ -63,6 +63,7 @@ _lib.predict_home_workspace_bytes.restype = _SZ
 _lib.predict_home.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _SZ, _P, _P]
 _lib.coact_place_correlated.argtypes = [_P, _I32, _I32, _P]
 _lib.coact_rebalance_ranks.argtypes = [_P, _P, _I32, _P, _I32, _P]
+_lib.coact_place_replicas.argtypes = [_P, _P, _P, _I32, _P, _I32, _I32, _I32, _P, _P]
 _lib.dispatch_gather_peer.argtypes = [_P, _I64, _I64, _P, _I32, _P, _I32, _P, _P, _P, _P, _P]
 _lib.combine_scatter_peer.argtypes = [_P, _P, _P, _P, _I32, _P, _P, _I64, _I32, _I64, _P, _I32,
                                       _P, _P]
@@ -77,7 +78,8 @@ for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "dispatch_gather_t
            "combine_scatter_backward", "shuffle_reduce_scatter", "plan_dispatch_slots",
            "assign_replicas", "predict_home",
            "coact_place_correlated", "plan_dispatch_noalloc", "coact_compose_map", "plan_forward",
-           "forward_gather", "forward_gather_tokens", "coact_rebalance_ranks", "dispatch_gather_peer",
+           "forward_gather", "forward_gather_tokens", "coact_rebalance_ranks",
+           "coact_place_replicas", "dispatch_gather_peer",
            "combine_scatter_peer"):
     getattr(_lib, _f).restype = _I32
 
@@ -88,7 +90,7 @@ ABI_SYMBOLS = ("coact_strerror", "coact_abi_version", "coact_last_cuda_error", "
                "coact_rebalance_ranks", "dispatch_gather_peer", "combine_scatter_peer",
                "combine_rows", "dispatch_gather_backward", "combine_scatter_backward",
                "shuffle_reduce_scatter", "plan_dispatch_slots", "assign_replicas",
-               "forward_gather_tokens")
+               "forward_gather_tokens", "coact_place_replicas")
 NOALLOC_MAX_TOKENS = 262144
 
 
@@ -705,3 +707,24 @@ def combine_scatter_peer(y_bases: torch.Tensor, y_row_offset: torch.Tensor,
                                      _ptr(out), 1 if out.dtype == torch.float32 else 0,
                                      _ptr(err_flag), _stream(stream)), "combine_scatter_peer")
     return out
+
+
+def coact_place_replicas(pair: torch.Tensor, loads: torch.Tensor, expert_rank: torch.Tensor,
+                         rank_node: torch.Tensor, budget: int, max_rep: int = 2):
+    """Replica layout from co-activation counts and loads (host code; CPU tensors or
+    copies of device ones): (rep_rank int32 [E, max_rep] with -1 padding, n_rep int32
+    [E], replicas added)."""
+    pr = pair.detach().to("cpu", torch.int64).contiguous()
+    ld = loads.detach().to("cpu", torch.int64).contiguous()
+    er = expert_rank.detach().to("cpu", torch.int32).contiguous()
+    rn = rank_node.detach().to("cpu", torch.int32).contiguous()
+    E, R = ld.shape[0], rn.shape[0]
+    if pr.shape != (E, E) or er.shape != (E,):
+        raise ValueError("pair must be [E, E] and expert_rank [E]")
+    rep = torch.empty((E, max_rep), dtype=torch.int32)
+    nrep = torch.empty(E, dtype=torch.int32)
+    added = _lib.coact_place_replicas(pr.data_ptr(), ld.data_ptr(), er.data_ptr(), E, rn.data_ptr(),
+                                      R, budget, max_rep, rep.data_ptr(), nrep.data_ptr())
+    if added < 0:
+        raise CoactError(added, "coact_place_replicas")
+    return rep, nrep, added

@@ -529,6 +529,25 @@ int coact_place_correlated(const int64_t *pair, int E, int R, int32_t *expert_ra
 int coact_rebalance_ranks(const int64_t *loads, const int32_t *expert_node, int E,
                           const int32_t *rank_node, int R, int32_t *expert_rank);
 
+/*
+ * coact_place_replicas -- a replica layout from co-activation and workload statistics
+ * (host code).  Cobalt, English abstract: EP distributes expert replicas across GPUs; the
+ * planner follows co-activation and workload statistics.  Reading taken: an expert's load
+ * is shared equally by its replicas (units of 1/840); `budget` times, the most loaded
+ * rank holding a replicable expert (fewer than max_rep replicas, some rank without one)
+ * gives its largest such share a new replica, on a node holding no replica of that
+ * expert if such a node still has a rank,
+ * the node with the largest co-activation sum_f pair[e][f] + pair[f][e] over the experts f
+ * whose replica 0 lives there, on that node's least loaded rank (ties: lower id).  pair:
+ * HOST int64 [E, E]; loads: HOST int64 [E]; expert_rank: HOST int32 [E] (replica 0);
+ * rank_node: HOST int32 [R]; out: rep_rank HOST int32 [E, max_rep] (-1 padded), n_rep
+ * HOST int32 [E] -- the tables assign_replicas takes.  Returns the number of replicas
+ * added (>= 0), or a negative status.
+ */
+int coact_place_replicas(const int64_t *pair, const int64_t *loads, const int32_t *expert_rank,
+                         int E, const int32_t *rank_node, int R, int budget, int max_rep,
+                         int32_t *rep_rank, int32_t *n_rep);
+
 #ifdef __cplusplus
 }
 #endif

@@ -763,10 +763,12 @@ int oracle_assign_replicas(const int32_t *ids, int64_t N, int k, int E, const in
  * arithmetic throughout: an expert's load is shared equally by its replicas, counted in
  * units of 1/840 so every share is exact for up to 8 replicas):
  *   every expert starts with its rank as replica 0; rank_load[r] = sum over the experts
- *   with a replica on r of loads[e]*840/n_rep[e].  Then, budget times:
- *   1. r* = the rank with the largest load (ties: lower rank);
- *   2. e* = among r*'s experts with fewer than max_rep replicas, the one with the largest
- *      share loads[e]*840/n_rep[e] (ties: lower id); none -> stop;
+ *   with a replica on r of loads[e]*840/n_rep[e].  An expert is replicable while it has
+ *   fewer than max_rep replicas and some rank holds none of them.  Then, budget times:
+ *   1. r* = the most loaded rank holding a replica of a replicable expert (ties: lower
+ *      rank); none -> stop;
+ *   2. e* = among those experts on r*, the one with the largest share
+ *      loads[e]*840/n_rep[e] (ties: lower id);
  *   3. candidate ranks: those without a replica of e*, on a node without one if any such
  *      rank exists; among them the node with the largest affinity
  *      A(node) = sum over experts f != e* whose replica 0 is on the node of
@@ -792,19 +794,23 @@ int oracle_place_replicas(const int64_t *pair, const int64_t *loads, const int32
     }
     int added = 0;
     for (int b = 0; b < budget; ++b) {
-        int rs = 0;                                              /* step 1 */
-        for (int r = 1; r < R; ++r)
-            if (rank_load[r] > rank_load[rs]) rs = r;
-        int es = -1;                                             /* step 2 */
+        int rs = -1, es = -1;                                    /* steps 1 and 2 */
         int64_t best_share = -1;
-        for (int e = 0; e < E; ++e) {
-            if (n_rep[e] >= max_rep) continue;
-            int on = 0;
-            for (int i = 0; i < n_rep[e]; ++i) on |= rep_rank[e * max_rep + i] == rs;
-            if (!on) continue;
-            int64_t share = loads[e] * L / n_rep[e];
-            if (share > best_share) { best_share = share; es = e; }
+        for (int r = 0; r < R; ++r) {
+            if (rs >= 0 && rank_load[r] <= rank_load[rs]) continue;
+            int pick = -1;
+            int64_t pick_share = -1;
+            for (int e = 0; e < E; ++e) {
+                if (n_rep[e] >= max_rep || n_rep[e] >= R) continue;
+                int on = 0;
+                for (int i = 0; i < n_rep[e]; ++i) on |= rep_rank[e * max_rep + i] == r;
+                if (!on) continue;
+                int64_t share = loads[e] * L / n_rep[e];
+                if (share > pick_share) { pick_share = share; pick = e; }
+            }
+            if (pick >= 0) { rs = r; es = pick; best_share = pick_share; }
         }
+        (void)best_share;
         if (es < 0) break;
         /* step 3: ranks and nodes that already hold a replica of es */
         char *has_rank = (char *)calloc((size_t)R, 1);

@@ -190,3 +190,49 @@ def test_placement_invariants_random(seed):
     before = rank_loads(er[:, None], np.ones(E, np.int32), loads, R)
     after = rank_loads(rep, n_rep, loads, R)
     assert after.sum() <= before.sum() and after.max() <= before.max()
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_placement_library_matches_oracle_random(seed):
+    import co_activation_b200 as coact
+    import torch
+    rng = np.random.default_rng(800 + seed)
+    R = int(rng.choice([2, 8, 32, 64]))
+    n_nodes = int(rng.choice([1, 2, 4, 8]))
+    E = R * int(rng.integers(1, 5))
+    rn = (np.arange(R) * n_nodes // R).astype(np.int32)
+    er = rng.permutation(np.arange(E) % R).astype(np.int32)
+    loads = rng.integers(0, 6, E).astype(np.int64)                 # many ties
+    pair = rng.integers(0, 3, (E, E)).astype(np.int64)
+    max_rep = int(rng.integers(1, 9))
+    budget = int(rng.integers(0, 2 * E))
+    want = oracle.place_replicas(pair, loads, er, rn, budget, max_rep)
+    got = coact.coact_place_replicas(torch.from_numpy(pair), torch.from_numpy(loads),
+                                     torch.from_numpy(er), torch.from_numpy(rn), budget, max_rep)
+    assert np.array_equal(got[0].numpy(), want[0]) and np.array_equal(got[1].numpy(), want[1])
+    assert got[2] == want[2]
+
+
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_placement_on_config_counts(cfg):
+    """On the configurations' own counts the planned replicas (as many as the load fixture
+    places) leave fewer (token, remote node) pairs and a lighter busiest rank than serving
+    every slot on replica 0."""
+    import co_activation_b200 as coact
+    import torch
+    import workload
+    r = workload.make_routing(cfg)
+    c = r.cfg
+    pair, loads, _ = oracle.count(r.ids, c.E)
+    rep, n_rep, added = oracle.place_replicas(pair, loads, r.expert_rank, r.rank_node, c.E // 8)
+    lib = coact.coact_place_replicas(torch.from_numpy(pair), torch.from_numpy(loads),
+                                     torch.from_numpy(r.expert_rank.astype(np.int32)),
+                                     torch.from_numpy(r.rank_node.astype(np.int32)), c.E // 8)
+    assert np.array_equal(lib[0].numpy(), rep) and added == c.E // 8
+    slot, _ = oracle.assign_replicas(r.ids, c.E, rep, n_rep, c.R, rank_node=r.rank_node,
+                                     n_nodes=c.n_nodes)
+    p = oracle.plan(r.ids, c.E, None, c.R, rank_node=r.rank_node, n_nodes=c.n_nodes, slot_rank=slot)
+    prim = oracle.plan(r.ids, c.E, r.expert_rank, c.R, rank_node=r.rank_node, n_nodes=c.n_nodes)
+    assert p["stats"][4] < prim["stats"][4]
+    asg = lambda pl: np.diff(pl["asg_offsets"])
+    assert asg(p).max() < asg(prim).max()
