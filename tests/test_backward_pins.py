@@ -259,3 +259,13 @@ def test_prereduced_within_bound_of_exact(cfg):
     # and it does round: the pre-reduced result is not the direct chain everywhere
     if c.k > c.E // c.R:
         assert not np.array_equal(out, oracle.combine_f32chain(y, r.gates, p["comb_row"]))
+
+
+def test_gather_backward_slot_order_matters():
+    # one token whose three slots go to three ranks: rows 1, 2^24, -2^24 summed in slot
+    # order give 0 (1 + 2^24 rounds to 2^24), in reverse order 1
+    send_row = np.array([[0, 1, 2]], np.int32)
+    g = bf16_bits_torch(np.array([[1.0], [2.0 ** 24], [-2.0 ** 24]], np.float32))
+    assert oracle.gather_backward_f32chain(g, send_row)[0, 0] == 0.0
+    g2 = bf16_bits_torch(np.array([[-2.0 ** 24], [2.0 ** 24], [1.0]], np.float32))
+    assert oracle.gather_backward_f32chain(g2, send_row)[0, 0] == 1.0

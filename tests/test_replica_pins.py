@@ -236,3 +236,13 @@ def test_placement_on_config_counts(cfg):
     assert p["stats"][4] < prim["stats"][4]
     asg = lambda pl: np.diff(pl["asg_offsets"])
     assert asg(p).max() < asg(prim).max()
+
+
+def test_used_rank_beats_home_node_and_rotation_uses_the_slot():
+    # expert 0 single on rank 2 (node 1); expert 1 on [1, 2]: home 0 (node 0) -- rank 2 is
+    # already used by the token (class b) and comes before the home-node replica 1 (class c)
+    got, _ = assign([[0, 1]], [[2], [1, 2], [4, 5]], src=[0])
+    assert got.tolist() == [[2, 2]]
+    # token 0, slot 1 must open a node: replica (t + j) mod 2 = 1 -> rank 5, not rank 4
+    got, _ = assign([[0, 2]], [[0], [1, 2], [4, 5]], src=[0])
+    assert got.tolist() == [[0, 5]]

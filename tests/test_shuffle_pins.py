@@ -92,3 +92,11 @@ def test_one_rank_is_the_identity():
     assert o["rank_offsets"].tolist() == [0, 4]
     with pytest.raises(ValueError):
         oracle.shuffle_order([0], 0)
+
+
+def test_rank_order_matters():
+    # 1 + 2^24 rounds back to 2^24 in fp32, so the rank order decides the result:
+    # ((0 + 1) + 2^24) - 2^24 = 0, while the reverse order gives 1
+    parts = bf16_bits(np.array([[[1.0]], [[2.0 ** 24]], [[-2.0 ** 24]]], np.float32))
+    out = oracle.shuffle_reduce_f32chain(parts, np.array([0], np.int32))
+    assert out[0, 0] == 0.0
