@@ -351,3 +351,19 @@ def test_backward_empty(coact):
     coact.combine_scatter_backward(y, gates, comb, g, torch.empty_like(y), torch.empty_like(gates))
     coact.dispatch_gather_backward(g, comb, torch.empty((0, H), dtype=torch.bfloat16, device=DEV))
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("k", [3, 8])
+def test_gather_backward_slot_order_of_the_sum(coact, k):
+    """Rows 1, 2^24, -2^24 on a token's first three send rows: 0 when added in slot order,
+    1 in reverse -- the kernel (also its sparse-slot form for k >= 3) adds in slot order."""
+    H = 64
+    send_row = np.full((2, k), -1, np.int32)
+    send_row[0, :3] = [0, 1, 2]
+    send_row[1, :3] = [2, 1, 0]
+    g = torch.tensor([[1.0], [2.0 ** 24], [-(2.0 ** 24)]], dtype=torch.float32).expand(3, H)
+    g = g.contiguous().to(torch.bfloat16).to(DEV)
+    gx = torch.empty((2, H), dtype=torch.float32, device=DEV)
+    coact.dispatch_gather_backward(g, cuda(send_row), gx)
+    torch.cuda.synchronize()
+    assert (gx[0] == 0.0).all() and (gx[1] == 1.0).all()

@@ -126,3 +126,16 @@ def test_flags_invalid_tokens_and_bases(coact):
     torch.cuda.synchronize()
     assert err.item() == coact.EFLAG_ROW_RANGE
     check_rows(out, pb[[0, 3]], np.arange(N, dtype=np.int32))
+
+
+def test_rank_order_of_the_sum(coact):
+    """Partials 1, 2^24, -2^24 (and the reverse): in rank order the fp32 sum is 0 (1 + 2^24
+    rounds back to 2^24), in reverse order it is 1 -- the kernel must add in rank order."""
+    H = 8
+    vals = [1.0, 2.0 ** 24, -(2.0 ** 24)]
+    for order, want in ((vals, 0.0), (vals[::-1], 1.0)):
+        parts = [torch.full((1, H), v, dtype=torch.bfloat16, device=DEV) for v in order]
+        out = torch.empty((1, H), dtype=torch.float32, device=DEV)
+        coact.shuffle_reduce_scatter(bases_of(parts), 1, cuda(np.zeros(1, np.int32)), out)
+        torch.cuda.synchronize()
+        assert (out == want).all(), (order, out)
