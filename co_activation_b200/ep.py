@@ -192,7 +192,10 @@ class EPLayer:
                  gates: Optional[torch.Tensor] = None) -> Dispatched:
         """Plan this rank's tokens and deliver every row to its destination rank.  With
         gates, each row's slot gates travel too (needed by the pre-reduced combine and the
-        backward)."""
+        backward).  On the peer transport the returned rows are a view of this rank's
+        symmetric receive buffer: valid until the next dispatch (every rank passes the
+        combine's closing barrier, after its experts have read them, before any rank
+        writes that buffer again)."""
         R, me = self.R, self.me
         src = torch.full((ids.shape[0],), me, dtype=torch.int32, device=ids.device)
         plan = self.ops.plan(ids, self.E, self.expert_rank, R, self.rank_node, self.n_nodes, src)
