@@ -758,20 +758,23 @@ class ShuffleStep:
 
 
 def make_step(coact, cfg_index: int, seed: int, device, two_hop: bool = False,
-              placement_kind: str = "auto", mode: str = "forward"):
-    """The step object for a configuration, plus a description of its placement."""
+              placement_kind: str = "auto", mode: str = "forward", tokens: Optional[int] = None):
+    """The step object for a configuration, plus a description of its placement.  tokens:
+    a smaller batch of the same configuration (profiling captures)."""
     cfg = workload.CONFIGS[cfg_index]
+    if tokens:
+        cfg = cfg.with_(N=int(tokens))
     if mode == "shuffle":
         if not cfg.two_layer:
             raise SystemExit("--shuffle needs the two-layer configuration (4)")
-        return ShuffleStep(coact, workload.make_two_layer(cfg, seed=seed), device), \
+        return ShuffleStep(coact, workload.make_two_layer(cfg, seed=seed, N=cfg.N), device), \
             "contiguous; tokens shuffled to the predicted layer-2 home rank"
     if cfg.two_layer:
         if mode != "forward":
             raise SystemExit("--pass backward / --combine prereduced need a one-layer configuration")
         if two_hop:
             raise SystemExit("--two-hop needs a one-layer configuration with several nodes (2, 3)")
-        return TwoLayerStep(coact, workload.make_two_layer(cfg, seed=seed), device), \
+        return TwoLayerStep(coact, workload.make_two_layer(cfg, seed=seed, N=cfg.N), device), \
             "contiguous; layer 2 pre-sharded to the predicted home rank"
     r = workload.make_routing(cfg, seed=seed)
     kind = placement_kind if placement_kind != "auto" else (
@@ -855,6 +858,8 @@ def run_gpu(args):
     import co_activation_b200 as coact
 
     cfg = workload.CONFIGS[args.config]
+    if args.tokens:
+        cfg = cfg.with_(N=int(args.tokens))
     LayerBuffers.tma = args.gather == "tma"
     TwoHopStep.forward = args.forward
     ReplicaStep.layout_kind = args.replica_layout
@@ -862,7 +867,7 @@ def run_gpu(args):
         "backward" if args.pass_ == "backward" else (
         "prereduced" if args.combine == "prereduced" else "forward")
     S, placement = make_step(coact, args.config, rank_seed(args.seed, rank), device, args.two_hop,
-                             args.placement, mode)
+                             args.placement, mode, args.tokens)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     flush_w = torch.empty(max(2 * l2, 64 << 20), dtype=torch.uint8, device=device)
     flush_r = torch.zeros(max(2 * l2, 64 << 20) // 8, dtype=torch.int64, device=device)
@@ -968,7 +973,9 @@ def run_gpu(args):
         "warmup": args.warmup, "ms_per_step": total_s * 1e3 / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded routing shaped after the pages' statistics; no router traces)",
-        "config": {"workload": f"config {cfg.index}: {cfg.desc}", "N": cfg.N, "E": cfg.E,
+        "config": {"workload": f"config {cfg.index}: {cfg.desc}" + (
+                       f" -- reduced to N={cfg.N} for a profiling capture" if args.tokens else ""),
+                   "N": cfg.N, "E": cfg.E,
                    "k": cfg.k, "H": cfg.H, "R": cfg.R, "n_nodes": cfg.n_nodes,
                    "placement": placement,
                    "pass": mode,
@@ -1244,6 +1251,9 @@ def main():
     ap.add_argument("--placement", default="auto", choices=["auto", "default", "correlated",
                                                              "two-stage"],
                     help="auto: the configuration's own (config 3: correlated)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="a smaller batch of the configuration (profiling captures); the "
+                         "JSON line's config shows the N used")
     ap.add_argument("--gather", default="vector", choices=["vector", "tma"],
                     help="gather implementation: dispatch_gather or dispatch_gather_tma")
     ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward"],
