@@ -1141,6 +1141,15 @@ def _oracle_step_fn(S):
             o.gather_backward_f32chain(gsb, p["send_row"])
         return fn
     xb, yb = o._bits(L.x), o._bits(L.y)
+    if isinstance(S, TwoHopStep):
+        def fn():
+            o.count(L.r.ids, cfg.E)
+            node, rank, fwd = o.plan_two_hop(L.r.ids, cfg.E, L.r.expert_rank, cfg.R,
+                                             L.r.rank_node, cfg.n_nodes)
+            hop1 = o.gather(xb, node["row_token"], node["D"])
+            o.forward_gather(hop1, fwd)
+            o.combine_f64(yb, L.r.gates, rank["comb_row"])
+        return fn
     if isinstance(S, ReplicaStep):
         def fn():
             o.count(L.r.ids, cfg.E)
@@ -1185,6 +1194,10 @@ def cpu_baseline(S, seconds: float):
                       "single-threaded C oracle: " + (
                           "combine backward (float64 gate gradients) and transposed dispatch"
                           if isinstance(S, BackwardStep) else
+                          "count, node and rank plans, hop-1 gather, hop-2 forward, float64 combine"
+                          if isinstance(S, TwoHopStep) else
+                          "count, replica choice, plan, gather, float64 combine"
+                          if isinstance(S, ReplicaStep) else
                           "count, plan, gather, partial rows and their sum"
                           if isinstance(S, PreReducedStep) else
                           "count, plan, gather, float64 combine"),
