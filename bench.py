@@ -998,6 +998,8 @@ def run_gpu(args):
         "dispatch_combine_tokens_per_s": cfg.N / (dc_ms / 1e3),
         **{k_: v for k_, v in summ.items() if k_ != "err_flag"},
         "phase_us": {k_: v * 1e3 for k_, v in phase_ms.items()},
+        "step_us_median": statistics.median(step_ms) * 1e3,
+        "step_us_min": min(step_ms) * 1e3,
         "phase_pass_step_us": statistics.mean(
             evs_phase[i][0].elapsed_time(evs_phase[i][NE - 1]) for i in range(K)) * 1e3,
         "hbm_gbs": {**{p[0]: p[2] / (p[3] / 1e3) / 1e9 for p in parts},
