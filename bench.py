@@ -243,11 +243,10 @@ def plan_launches(R: int, N: int) -> int:
 
 
 class OneLayerStep:
-    """plan -> gather -> combine, with the count on a side stream beside the gather (it
-    depends only on the ids; beside the latency-bound plan it slowed the plan more than
-    it now takes from the gather: 73.9 -> 72.1 us per config-1 step)."""
+    """count (side stream, overlapped with the plan: it depends on nothing the other
+    calls produce) -> plan -> gather -> combine."""
     n_events = 5
-    phases = {"coact_count": (2, 1), "plan_dispatch": (0, 2), "dispatch_gather": (2, 3),
+    phases = {"coact_count": (0, 1), "plan_dispatch": (0, 2), "dispatch_gather": (2, 3),
               "combine_scatter": (3, 4)}
     host_inputs = ("ids", "gates", "expert_rank", "rank_node", "x", "y")
 
@@ -269,13 +268,13 @@ class OneLayerStep:
 
     def step(self, ev=None):
         main = torch.cuda.current_stream()
-        if ev: ev[0].record()
-        self.L.plan_()
-        if ev: ev[2].record()
         self.side.wait_stream(main)
+        if ev: ev[0].record()
         with torch.cuda.stream(self.side):
             self.L.count()
             if ev: ev[1].record()
+        self.L.plan_()
+        if ev: ev[2].record()
         self.L.gather()
         if ev: ev[3].record()
         self.L.combine()
@@ -345,9 +344,6 @@ class TwoLayerStep:
         main = torch.cuda.current_stream()
         self.side.wait_stream(main)
         if ev: ev[0].record()
-        # side work from the start: the statistics (~107 us on config 4) overlap the
-        # latency-bound layer-1 plan; started after it, they slowed layer 1's gather
-        # (1,043 -> 1,059 us per step)
         with torch.cuda.stream(self.side):
             # statistics, and the layer-2 home prediction: it needs only layer 1's picks
             # and the calibration counts, so it runs beside layer 1's dispatch and combine
@@ -409,7 +405,7 @@ class TwoHopStep(OneLayerStep):
     order (forward_gather_tokens: each hop-1 row read once) unless forward = "rows"."""
     forward = "tokens"
     n_events = 6
-    phases = {"coact_count": (2, 1), "plan_two_hop": (0, 2), "gather_hop1": (2, 3),
+    phases = {"coact_count": (0, 1), "plan_two_hop": (0, 2), "gather_hop1": (2, 3),
               "forward_hop2": (3, 4), "combine_scatter": (4, 5)}
 
     def __init__(self, coact, r: workload.Routing, device, fill: bool = True):
@@ -428,14 +424,14 @@ class TwoHopStep(OneLayerStep):
     def step(self, ev=None):
         L, c = self.L, self.cfg
         main = torch.cuda.current_stream()
-        if ev: ev[0].record()
-        L.coact.plan_two_hop(L.ids, c.E, L.expert_rank, c.R, L.rank_node, c.n_nodes, self.th,
-                             err_flag=L.err)
-        if ev: ev[2].record()
         self.side.wait_stream(main)
+        if ev: ev[0].record()
         with torch.cuda.stream(self.side):
             L.count()
             if ev: ev[1].record()
+        L.coact.plan_two_hop(L.ids, c.E, L.expert_rank, c.R, L.rank_node, c.n_nodes, self.th,
+                             err_flag=L.err)
+        if ev: ev[2].record()
         L.coact.dispatch_gather(L.x, self.th.node.send_row, self.hop1, err_flag=L.err,
                                 tma=L.tma)
         if ev: ev[3].record()
@@ -497,7 +493,7 @@ class PreReducedStep(OneLayerStep):
     -> combine_rows over the send rows (one bf16 partial row per (token, rank), D rows
     instead of N*k) -> dispatch_gather_backward adds each token's partial rows."""
     n_events = 6
-    phases = {"coact_count": (2, 1), "plan_dispatch": (0, 2), "dispatch_gather": (2, 3),
+    phases = {"coact_count": (0, 1), "plan_dispatch": (0, 2), "dispatch_gather": (2, 3),
               "combine_rows": (3, 4), "reduce_rows": (4, 5)}
     step_desc = ("coact_count (side stream) + plan_dispatch + dispatch_gather + combine_rows "
                  "(partial rows per send row) + dispatch_gather_backward (sum per token, bf16 out)")
@@ -514,13 +510,13 @@ class PreReducedStep(OneLayerStep):
     def step(self, ev=None):
         L, c = self.L, self.L.coact
         main = torch.cuda.current_stream()
-        if ev: ev[0].record()
-        L.plan_()
-        if ev: ev[2].record()
         self.side.wait_stream(main)
+        if ev: ev[0].record()
         with torch.cuda.stream(self.side):
             L.count()
             if ev: ev[1].record()
+        L.plan_()
+        if ev: ev[2].record()
         L.gather()
         if ev: ev[3].record()
         # units: the plan's send rows, as many as the device-side D = rank_offsets[R]
@@ -546,7 +542,7 @@ class ReplicaStep(OneLayerStep):
     combine.  The n_hot most loaded experts of the batch have a second replica on another
     node (workload.replicate_hot)."""
     n_events = 6
-    phases = {"coact_count": (3, 1), "assign_replicas": (0, 2), "plan_dispatch": (2, 3),
+    phases = {"coact_count": (0, 1), "assign_replicas": (0, 2), "plan_dispatch": (2, 3),
               "dispatch_gather": (3, 4), "combine_scatter": (4, 5)}
 
     layout_kind = "hot"        # "hot": workload.replicate_hot; "planned": coact_place_replicas
@@ -583,17 +579,17 @@ class ReplicaStep(OneLayerStep):
     def step(self, ev=None):
         L, c, cfg = self.L, self.L.coact, self.cfg
         main = torch.cuda.current_stream()
+        self.side.wait_stream(main)
         if ev: ev[0].record()
+        with torch.cuda.stream(self.side):
+            L.count()
+            if ev: ev[1].record()
         c.assign_replicas(L.ids, cfg.E, self.rep, self.nrep, cfg.R, self.slot, rank_node=L.rank_node,
                           n_nodes=cfg.n_nodes, err_flag=L.err)
         if ev: ev[2].record()
         c.plan_dispatch(L.ids, cfg.E, None, cfg.R, L.plan, rank_node=L.rank_node,
                         n_nodes=cfg.n_nodes, err_flag=L.err, slot_rank=self.slot)
         if ev: ev[3].record()
-        self.side.wait_stream(main)
-        with torch.cuda.stream(self.side):
-            L.count()
-            if ev: ev[1].record()
         L.gather()
         if ev: ev[4].record()
         L.combine()
@@ -993,7 +989,7 @@ def run_gpu(args):
                             f"forward map) + hop-1 gather + hop-2 forward ({args.forward}) + "
                             "combine_scatter"
                             if args.two_hop else
-                            "plan_dispatch + coact_count (side stream, beside the gather) + "
+                            "coact_count (side stream, overlapped with plan) + plan_dispatch + "
                             "dispatch_gather + combine_scatter (bf16 out)"),
                    "l2": "flushed between timed steps (write of 2x L2, then a read of another 2x L2 "
                          "buffer so no dirty line is left), outside the step events",
