@@ -230,8 +230,10 @@ int launch(const uint16_t *y, int64_t n_rows, const float *gates, const int32_t 
     constexpr int U = K <= 2 ? 4 : 2;
 #endif
     const int64_t H16 = H / 8;
-    const int blocks = (int)std::max<int64_t>(
-        1, std::min<int64_t>(ceil_div(n_units, 8), (int64_t)di.sm_count * 8));
+#ifndef COACT_COMBINE_PER_SM
+#define COACT_COMBINE_PER_SM 8  // CTAs per SM in the grid (0: one resident wave)
+#endif
+    const int blocks = grid_for(k_combine_v16<K, U, F32>, n_units, COACT_COMBINE_PER_SM, di);
     if (UNITS)
         return launch_pdl(k_combine_units<K, 4, 2, F32, true>, blocks, 256, 0, st,
                           reinterpret_cast<const uint4 *>(y), n_rows, gates, comb_row, N, row_token,

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <atomic>
 
 #if defined(COACT_NVTX)
@@ -48,6 +49,15 @@ __device__ __forceinline__ void st_stream(uint4 *p, const uint4 &v) {
                  : "memory");
 }
 
+// Asks the copy engine of the SM (TMA) to bring [p, p + bytes) of this GPU's memory into
+// L2; p 16-byte aligned, bytes a multiple of 16.  A hint with no completion: nothing is
+// returned, no mbarrier is involved and nothing needs waiting for.  L2 is where every
+// access to this GPU's memory meets, so a line fetched before its last writer finished
+// is updated there by that write, never served stale.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // Loads token t's K expert ids (row t of an int32 [N, K] array) and returns the
 // validation bits: COACT_EFLAG_ID_RANGE for an id outside [0, E), COACT_EFLAG_DUP_ID
 // for an id that repeats within the token.  0 means the token is valid.
@@ -83,10 +93,12 @@ __device__ __forceinline__ void raise_flag_warp(int32_t *err, int bits) {
 // Programmatic dependent launch.  Every library kernel is launched with programmatic
 // stream serialisation: it may start while the previous kernel on the stream drains,
 // and it reads no global input written by that kernel until pdl_wait() returns (the
-// previous grid has completed and its writes are visible).  Every library kernel calls
-// pdl_trigger() only AFTER its own pdl_wait(), so when a library kernel starts, every
-// kernel before its immediate predecessor has completed: a kernel whose predecessor is
-// another library kernel of the same call may read the call's inputs before waiting.
+// previous grid has completed and its writes are visible).  A kernel that is not the
+// last of its call calls pdl_trigger() only AFTER its own pdl_wait(), so when the next
+// kernel of the same call starts, every kernel before it has completed: such a kernel
+// may read the call's inputs before waiting.  The first kernel of a call reads no
+// global memory before pdl_wait() (it may warm L2 with prefetch_l2_bulk, which reads
+// nothing into the program), so the last kernel of a call may trigger early.
 __device__ __forceinline__ void pdl_wait() {
 #if !defined(COACT_NO_PDL)
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -137,8 +149,8 @@ int ensure_smem(F kernel, size_t bytes, SmemOptIn &cache, const DeviceInfo &di) 
     return COACT_OK;
 }
 
-// Resident blocks per SM for a kernel limited by threads and shared memory (the
-// library's kernels use few enough registers that registers never bind).
+// Resident blocks per SM for a kernel limited by threads and shared memory (for the
+// kernels sized with it, which use few enough registers that registers never bind).
 inline int blocks_per_sm(int threads, size_t smem, const DeviceInfo &di) {
     int by_threads = 2048 / threads;
     int by_smem = smem ? (int)(di.smem_per_sm / (smem + 1024)) : 32;
@@ -150,6 +162,26 @@ inline int blocks_per_sm(int threads, size_t smem, const DeviceInfo &di) {
 inline int launch_status() {
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? COACT_OK : cuda_fail(e);
+}
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Grid for a grid-stride kernel of 256-thread CTAs over `units` work items, 8 per CTA
+// (one per warp): at most `per_sm` CTAs per SM, where per_sm <= 0 means the CTAs of
+// `kernel` that fit on an SM at once (one wave, every CTA resident from the start).
+template <typename... KArgs>
+int grid_for(void (*kernel)(KArgs...), int64_t units, int per_sm, const DeviceInfo &di) {
+    if (per_sm <= 0) {
+        int occ = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, 256, 0) != cudaSuccess ||
+            occ < 1) {
+            (void)cudaGetLastError();
+            occ = 1;
+        }
+        per_sm = occ;
+    }
+    const int64_t b = std::min<int64_t>(ceil_div(units, 8), (int64_t)di.sm_count * per_sm);
+    return (int)(b > 1 ? b : 1);
 }
 
 // Launches `kernel` on `stream` with programmatic stream serialisation (see pdl_wait).
@@ -188,6 +220,5 @@ struct NvtxRange {
 #define COACT_RANGE(name) ((void)0)
 #endif
 
-inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 }  // namespace coact

@@ -9,7 +9,11 @@
 // the algorithmic traffic is (N + D) * H * 2 bytes (+ N*k*4 for send_row).
 //  * k_gather_v16 (default) -- one warp per token, 16-byte vector loads of the x row
 //    into registers (up to 8 per lane in flight) and streaming 16-byte stores to each
-//    destination; 8 CTAs of 8 warps per SM.
+//    destination; a grid of 8 CTAs of 8 warps per SM (4 resident at 60 registers: the
+//    extra waves balance the tail better than one resident wave, measured).  Before its
+//    wait on the predecessor, each warp warms L2 with the x rows it will copy first
+//    (bulk L2 prefetch): behind the latency-bound plan, whose last kernel lets this one
+//    launch at once, HBM streams x while the plan finishes.
 //  * k_gather_bulk (entry point dispatch_gather_tma) -- TMA bulk copies.  One warp per
 //    CTA; lane 0 streams rows into a ring of shared-memory stages with cp.async.bulk
 //    (global -> shared, completion on an mbarrier), then lanes j < k each issue the
@@ -28,16 +32,22 @@ namespace {
 
 // ------------------------------------------------------------------ vector path
 
+// n_prefetch: tokens [0, n_prefetch) have their x rows warmed into L2 before the wait on
+// the predecessor (each warp its own tokens, in the order it copies them), so that
+// while a latency-bound predecessor (the plan) runs, HBM already streams x.
 template <int UNROLL>
 __global__ void __launch_bounds__(256)
     k_gather_v16(const uint4 *__restrict__ x, int64_t N, int64_t H16,
                  const int32_t *__restrict__ send_row, int k, uint4 *__restrict__ send,
-                 int64_t cap, int32_t *__restrict__ err) {
-    pdl_wait();
-    pdl_trigger();
+                 int64_t cap, int64_t n_prefetch, int32_t *__restrict__ err) {
     const int lane = threadIdx.x & 31;
     const int64_t gwarp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    if (lane == 0)
+        for (int64_t t = gwarp; t < n_prefetch; t += nwarps)
+            prefetch_l2_bulk(x + t * H16, (uint32_t)(H16 * 16));
+    pdl_wait();
+    pdl_trigger();
     int flags = 0;
     for (int64_t t = gwarp; t < N; t += nwarps) {
         // destinations: lane j < k reads send_row[t, j]; broadcast by shuffles below
@@ -269,18 +279,30 @@ int launch_bulk(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row
 int launch_v16(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row, int k,
                uint16_t *send, int64_t cap, int32_t *err, cudaStream_t st, const DeviceInfo &di) {
     const int64_t H16 = H / 8;
-    const int64_t warps_needed = N;
-    const int blocks = (int)std::max<int64_t>(
-        1, std::min<int64_t>(ceil_div(warps_needed, 8), (int64_t)di.sm_count * 8));
+#ifndef COACT_GATHER_PER_SM
+#define COACT_GATHER_PER_SM 8  // CTAs per SM in the grid (0: one resident wave)
+#endif
     const uint4 *xv = reinterpret_cast<const uint4 *>(x);
     uint4 *sv = reinterpret_cast<uint4 *>(send);
 #ifndef COACT_GATHER_UNROLL
 #define COACT_GATHER_UNROLL 8  // 16-byte loads in flight per lane on long rows
 #endif
-    if (H16 <= 32) return launch_pdl(k_gather_v16<1>, blocks, 256, 0, st, xv, N, H16, send_row, k, sv, cap, err);
-    if (H16 <= 128) return launch_pdl(k_gather_v16<4>, blocks, 256, 0, st, xv, N, H16, send_row, k, sv, cap, err);
-    return launch_pdl(k_gather_v16<COACT_GATHER_UNROLL>, blocks, 256, 0, st, xv, N, H16, send_row,
-                      k, sv, cap, err);
+#ifndef COACT_GATHER_PREFETCH_BYTES
+// x bytes warmed into L2 before the wait.  Measured on B200 behind the plan of a
+// 16K-token, 4 KB-row batch: 16-32 MB took ~1% off the step; 64 MB no longer did (more
+// than the plan's ~8 us of idle HBM time covers).
+#define COACT_GATHER_PREFETCH_BYTES (32ll << 20)
+#endif
+    // the bulk prefetch takes a 32-bit size: rows beyond 16 MB are not prefetched
+    const int64_t n_pf =
+        H * 2 > (1 << 24) ? 0 : std::min<int64_t>(N, (int64_t)(COACT_GATHER_PREFETCH_BYTES) / (H * 2));
+    auto go = [&](auto kern) {
+        return launch_pdl(kern, grid_for(kern, N, COACT_GATHER_PER_SM, di), 256, 0, st, xv, N,
+                          H16, send_row, k, sv, cap, n_pf, err);
+    };
+    if (H16 <= 32) return go(k_gather_v16<1>);
+    if (H16 <= 128) return go(k_gather_v16<4>);
+    return go(k_gather_v16<COACT_GATHER_UNROLL>);
 }
 
 }  // namespace

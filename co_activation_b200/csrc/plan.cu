@@ -34,6 +34,9 @@ constexpr int kTile = COACT_PLAN_TILE;     // experiment builds (a multiple of 3
 constexpr int kTile = 256;                 // tokens per tile, one per thread
 #endif
 constexpr int kTileWarps = kTile / 32;
+#ifndef COACT_PLAN_EARLY_TRIGGER
+#define COACT_PLAN_EARLY_TRIGGER 1  // k_plan_scatter lets the next call's kernel launch at once
+#endif
 constexpr int kScanThreads = 1024;
 constexpr int kStatSlots = 6;              // per-tile partials (see TileStat)
 enum TileStat { TS_REMOTE_ROWS, TS_XNODE_ROWS, TS_NODE_ROWS, TS_LOCAL_ASG, TS_XNODE_ASG, TS_VALID_ASG };
@@ -368,6 +371,12 @@ __global__ void __launch_bounds__(kTile)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tile = blockIdx.x;
+#if COACT_PLAN_EARLY_TRIGGER
+    // The last kernel of the call: the next call's first kernel reads nothing before its
+    // own wait, so it may launch now (the dispatch gather then warms L2 with x while the
+    // plan finishes).
+    pdl_trigger();
+#endif
     for (int i = tid; i < kTileWarps * 64; i += kTile) {
         (&s_wrows[0][0])[i] = 0;
         (&s_wasg[0][0])[i] = 0;
@@ -442,7 +451,9 @@ __global__ void __launch_bounds__(kTile)
 
     // ---- cross-tile bases: need the predecessor's results
     pdl_wait();
+#if !COACT_PLAN_EARLY_TRIGGER
     pdl_trigger();
+#endif
     if (SMALL) {
         for (int r = warp; r < R; r += kTileWarps)
             for (int which = 0; which < 2; ++which) {
