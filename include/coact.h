@@ -16,6 +16,13 @@
  *  - Array pointers are DEVICE pointers owned by the caller (e.g. torch tensors).  The
  *    library never allocates, frees or synchronises; all work is enqueued on `stream`
  *    (a cudaStream_t; NULL = the legacy default stream).  Calls are asynchronous.
+ *  - Kernels are launched with programmatic stream serialisation (programmatic dependent
+ *    launch): a library kernel may start while the previous kernel on the stream drains,
+ *    and waits for it (griddepcontrol.wait) before touching its outputs.  Work that the
+ *    caller enqueues normally after a call sees all of that call's results.  A kernel
+ *    of the caller's own that is launched with programmatic stream serialisation right
+ *    after a call must likewise wait before reading that call's outputs: the last kernel
+ *    of plan_dispatch lets such a successor start while the plan is still running.
  *  - Return value: COACT_OK (0) or a negative coact_status.  A negative status is
  *    decided on the host before anything is enqueued (except COACT_ERR_CUDA, which
  *    reports a failed launch).
