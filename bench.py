@@ -917,7 +917,8 @@ def run_gpu(args):
         torch.cuda.synchronize()
         return g, ev, body
 
-    timing = "one CUDA graph of K steps per pass; CUDA events per step"
+    timing = ("one CUDA graph of K steps per pass; CUDA events per step (per-step times of "
+              "~70 us fall on levels ~2.1 us apart on B200: value and step_us_mean are means)")
     try:
         g_main, evs, body_main = capture(False)
         g_phase, evs_phase, body_phase = capture(True)
@@ -998,6 +999,7 @@ def run_gpu(args):
         "dispatch_combine_tokens_per_s": cfg.N / (dc_ms / 1e3),
         **{k_: v for k_, v in summ.items() if k_ != "err_flag"},
         "phase_us": {k_: v * 1e3 for k_, v in phase_ms.items()},
+        "step_us_mean": statistics.mean(step_ms) * 1e3,
         "step_us_median": statistics.median(step_ms) * 1e3,
         "step_us_min": min(step_ms) * 1e3,
         "phase_pass_step_us": statistics.mean(
