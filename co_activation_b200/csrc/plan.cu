@@ -455,22 +455,28 @@ __global__ void __launch_bounds__(kTile)
     pdl_trigger();
 #endif
     if (SMALL) {
-        for (int r = warp; r < R; r += kTileWarps)
+        // rank r's row and assignment counts read together (one round trip), then reduced
+        for (int r = warp; r < R; r += kTileWarps) {
+            const int32_t *cr = ws.tile_rows + (int64_t)r * n_tiles;
+            const int32_t *ca = ws.tile_asg + (int64_t)r * n_tiles;
+            int tot[2] = {0, 0}, before[2] = {0, 0};
+            for (int i = lane; i < n_tiles; i += 32) {
+                const int vr = cr[i], va = ca[i];
+                tot[0] += vr;
+                tot[1] += va;
+                before[0] += i < tile ? vr : 0;
+                before[1] += i < tile ? va : 0;
+            }
+#pragma unroll
             for (int which = 0; which < 2; ++which) {
-                const int32_t *cnt = (which == 0 ? ws.tile_rows : ws.tile_asg) + (int64_t)r * n_tiles;
-                int tot = 0, before = 0;
-                for (int i = lane; i < n_tiles; i += 32) {
-                    const int v = cnt[i];
-                    tot += v;
-                    before += i < tile ? v : 0;
-                }
-                tot = __reduce_add_sync(0xffffffffu, tot);
-                before = __reduce_add_sync(0xffffffffu, before);
+                const int t_all = __reduce_add_sync(0xffffffffu, tot[which]);
+                const int t_before = __reduce_add_sync(0xffffffffu, before[which]);
                 if (lane == 0) {
-                    s_tot[which][r] = tot;
-                    s_before[which][r] = before;
+                    s_tot[which][r] = t_all;
+                    s_before[which][r] = t_before;
                 }
             }
+        }
         if (tile == 0) {
             long long acc[kStatSlots] = {0, 0, 0, 0, 0, 0};
             for (int i = tid; i < n_tiles; i += kTile)
