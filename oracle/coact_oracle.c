@@ -527,6 +527,7 @@ void oracle_forward_gather(const uint16_t *src, int64_t H, const int32_t *fwd_sr
  */
 int oracle_rebalance_ranks(const int64_t *loads, const int32_t *expert_node, int E,
                            const int32_t *rank_node, int R, int32_t *expert_rank) {
+    if (R < 1 || E < 1) return -1;   /* no rank or no expert: nothing to balance */
     int per_rank = E / R;
     int64_t *rank_load = (int64_t *)calloc((size_t)R, sizeof(int64_t));
     int *free_slots = (int *)malloc(sizeof(int) * (size_t)R);
