@@ -45,6 +45,21 @@ def test_library_exports_every_declared_symbol(lib):
     assert set(header_functions()) <= exported
 
 
+def test_every_entry_point_is_declared():
+    """The reverse direction: no extern "C" function of the sources is missing from the
+    header (the header is the whole boundary)."""
+    csrc = os.path.join(ROOT, "co_activation_b200", "csrc")
+    defined = set()
+    for fn in os.listdir(csrc):
+        if fn.endswith((".cu", ".cuh")):
+            src = open(os.path.join(csrc, fn)).read()
+            defined |= set(re.findall(r'extern "C"\s+(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(',
+                                      src))
+    assert defined, "no entry points found"
+    assert defined == set(header_functions()), (sorted(defined - set(header_functions())),
+                                                 sorted(set(header_functions()) - defined))
+
+
 def test_binding_names_match_header():
     import co_activation_b200 as coact
     assert set(coact.ABI_SYMBOLS) == set(header_functions())
