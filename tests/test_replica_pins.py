@@ -167,6 +167,45 @@ def test_placement_budget_zero_and_exhaustion():
         assert len(set(rep[e].tolist())) == 2                 # distinct ranks per expert
 
 
+def test_placement_moves_on_when_the_heaviest_rank_is_exhausted():
+    """Budget 3, max_rep 2; ranks 0,1 on node 0, ranks 2,3 on node 1; two experts per
+    rank, loads 200,200 | 90,10 | 20,20 | 10,10 (units of 1/840 below omitted).
+    1. rank 0 (400) gives expert 0 (share 200, lower id of the tie) a replica on node 1's
+       lighter rank 3: rank 0 -> 300, rank 3 -> 120;
+    2. rank 0 (300) gives expert 1 a replica on rank 2 (40 < 120): rank 0 -> 200,
+       rank 2 -> 140;
+    3. rank 0 (200) is still the heaviest, but both its experts are at max_rep.  The
+       budget is the number of replicas to add, so the next most loaded rank that can
+       still be relieved gives one: rank 2 (140), expert 4 (share 20, lower id), on node 0
+       (the only node without it), whose lighter rank is 1 (100 < 200).
+    Stopping at step 3 instead (added = 2) would leave budget unspent although rank 2
+    could still be relieved."""
+    er = [0, 0, 1, 1, 2, 2, 3, 3]
+    rn = [0, 0, 1, 1]
+    loads = [200, 200, 90, 10, 20, 20, 10, 10]
+    rep, n_rep, added = oracle.place_replicas(np.zeros((8, 8), np.int64), loads, er, rn, 3, 2)
+    assert added == 3
+    assert rep.tolist() == [[0, 3], [0, 2], [1, -1], [1, -1], [2, 1], [2, -1], [3, -1], [3, -1]]
+    assert n_rep.tolist() == [2, 2, 1, 1, 2, 1, 1, 1]
+    assert rank_loads(rep, n_rep, loads, 4).tolist() == [200 * 840, 110 * 840, 130 * 840,
+                                                         120 * 840]
+
+
+def test_placement_skips_experts_already_on_every_rank():
+    """Two ranks on two nodes, max_rep 4 > R: replicas sit on distinct ranks, so an
+    expert with a replica on each of the R ranks cannot take another.  Loads 100 | 1:
+    1. rank 0 (100) gives expert 0 a replica on rank 1: both ranks at 50 + (1 on rank 1);
+    2. rank 1 (51) holds expert 0 (on both ranks already: not replicable) and expert 1:
+       expert 1 gets its replica on rank 0;
+    3. no expert is replicable any more: the loop ends with added = 2.
+    Taking expert 0 at step 2 (its share 50 beats 1) would find no rank for it and end
+    the loop with added = 1, the budget unspent while expert 1 could still be placed."""
+    rep, n_rep, added = oracle.place_replicas(np.zeros((2, 2), np.int64), [100, 1], [0, 1],
+                                              [0, 1], 3, 4)
+    assert added == 2
+    assert rep.tolist() == [[0, 1, -1, -1], [1, 0, -1, -1]] and n_rep.tolist() == [2, 2]
+
+
 @pytest.mark.parametrize("seed", range(6))
 def test_placement_invariants_random(seed):
     rng = np.random.default_rng(700 + seed)
