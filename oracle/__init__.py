@@ -81,6 +81,8 @@ def _get():
             _lib.oracle_combine_backward.restype = None
             _lib.oracle_shuffle_reduce_f32chain.argtypes = [P, I32, I64, I64, P, I64, P]
             _lib.oracle_shuffle_reduce_f32chain.restype = None
+            _lib.oracle_row_meta.argtypes = [P, P, I64, P, I32, P, P, P, I64, I32, P, P, P, P]
+            _lib.oracle_gather_row_slots.argtypes = [P, I64, P, P, I64, I32, P]
         return _lib
 
 
@@ -452,3 +454,39 @@ def place_replicas(pair, loads, expert_rank, rank_node, budget: int, max_rep: in
     added = _get().oracle_place_replicas(_p(pr), _p(ld), _p(er), E, _p(rn), R, budget, max_rep,
                                          _p(rep), _p(nrep))
     return rep, nrep, added
+
+
+# ----------------------------------------------------------------------------- EP row metadata
+
+
+def row_meta(plan_: dict, ids, gates, slot_base=None, n_rows=None):
+    """Per send row of a plan, one entry per slot: (expert ids int32 [n, k], gates fp32
+    [n, k], expert-output slots int32 [n, k], flags) -- -1 / 0 / -1 where the row does not
+    serve the slot; slots are comb_row + slot_base[rank of the row] (slot_base None: 0).
+    n_rows defaults to the plan's D."""
+    ids = _c(ids, np.int32)
+    g = _c(gates, np.float32)
+    N, k = ids.shape
+    n = plan_["D"] if n_rows is None else int(n_rows)
+    ro = _c(plan_["rank_offsets"], np.int32)
+    sb = None if slot_base is None else _c(slot_base, np.int32)
+    ex = np.zeros((n, k), np.int32)
+    go = np.zeros((n, k), np.float32)
+    sl = np.zeros((n, k), np.int32)
+    f = _get().oracle_row_meta(_p(_c(plan_["row_token"], np.int32)),
+                               _p(_c(plan_["row_kmask"], np.uint8)), n, _p(ro), len(ro) - 1,
+                               _p(ids), _p(g), _p(_c(plan_["comb_row"], np.int32)), N, k, _p(sb),
+                               _p(ex), _p(go), _p(sl))
+    return ex, go, sl, f
+
+
+def gather_row_slots(vals, send_row, row_kmask):
+    """out[t, j] = vals[d, j] for the send row d of token t that holds slot j (0 where none
+    does); vals fp32 [n_rows, k].  Returns (out fp32 [N, k], flags)."""
+    v = _c(vals, np.float32)
+    sr = _c(send_row, np.int32)
+    km = _c(row_kmask, np.uint8)
+    N, k = sr.shape
+    out = np.zeros((N, k), np.float32)
+    f = _get().oracle_gather_row_slots(_p(v), v.shape[0], _p(sr), _p(km), N, k, _p(out))
+    return out, f

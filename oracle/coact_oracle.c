@@ -854,3 +854,65 @@ int oracle_place_replicas(const int64_t *pair, const int64_t *loads, const int32
     free(aff);
     return added;
 }
+
+/* ------------------------------------------------------------------ EP row metadata
+ *
+ * [Cobalt], [Zyphra]: under expert parallelism every token travels to the ranks that
+ * hold its experts (each rank once), those ranks run the experts, and the results travel
+ * back to be combined.  A rank receiving a deduplicated row needs, besides the row, the
+ * expert id and the gate of each slot the row serves, and where each slot's expert
+ * output goes among the rank's outputs.  Reading taken (the pages define no format): one
+ * entry per (send row, slot), -1 / 0 / -1 for the slots the row does not serve.
+ *
+ * oracle_row_meta: for d < n_rows, t = row_token[d], r = the rank whose segment
+ * [rank_offsets[r], rank_offsets[r+1]) holds d; for j < k:
+ *   bit j of row_kmask[d] set:  experts[d,j] = ids[t,j], gates_out[d,j] = gates[t,j],
+ *                               slots[d,j] = comb_row[t,j] + slot_base[r]
+ *   else:                       -1, 0, -1
+ * (slot_base NULL: 0).  With slot_base[r] = (rows of rank r's outputs that earlier
+ * sources send it) - asg_offsets[r], slots[d,j] is where slot j's output sits in the
+ * destination's expanded receive order.  Any output pointer may be NULL (skipped);
+ * a row whose token is outside [0, N) gets -1 / 0 / -1 everywhere and returns flag 16.
+ */
+int oracle_row_meta(const int32_t *row_token, const uint8_t *row_kmask, int64_t n_rows,
+                    const int32_t *rank_offsets, int R, const int32_t *ids, const float *gates,
+                    const int32_t *comb_row, int64_t N, int k, const int32_t *slot_base,
+                    int32_t *experts, float *gates_out, int32_t *slots) {
+    int flags = 0;
+    for (int64_t d = 0; d < n_rows; ++d) {
+        int r = 0;
+        while (r + 1 < R && d >= rank_offsets[r + 1]) ++r;
+        int64_t t = row_token[d];
+        int ok = t >= 0 && t < N;
+        if (!ok) flags |= 16;
+        for (int j = 0; j < k; ++j) {
+            int on = ok && ((row_kmask[d] >> j) & 1);
+            if (experts) experts[d * k + j] = on ? ids[t * k + j] : -1;
+            if (gates_out) gates_out[d * k + j] = on ? gates[t * k + j] : 0.0f;
+            if (slots) slots[d * k + j] = on ? comb_row[t * k + j] + (slot_base ? slot_base[r] : 0) : -1;
+        }
+    }
+    return flags;
+}
+
+/* oracle_gather_row_slots: the way back of one value per (send row, slot) -- e.g. the
+ * gate gradients computed where the experts ran -- to token order:
+ *   out[t,j] = vals[d,j] for the send row d of token t whose mask holds bit j,
+ *   0 for a slot that none of the token's send rows holds.
+ * The token's send rows are the send_row[t, j0] >= 0.  A send row outside [0, n_rows)
+ * is skipped and returns flag 16. */
+int oracle_gather_row_slots(const float *vals, int64_t n_rows, const int32_t *send_row,
+                            const uint8_t *row_kmask, int64_t N, int k, float *out) {
+    int flags = 0;
+    for (int64_t t = 0; t < N; ++t) {
+        for (int j = 0; j < k; ++j) out[t * k + j] = 0.0f;
+        for (int j0 = 0; j0 < k; ++j0) {
+            int64_t d = send_row[t * k + j0];
+            if (d < 0) continue;
+            if (d >= n_rows) { flags |= 16; continue; }
+            for (int j = 0; j < k; ++j)
+                if ((row_kmask[d] >> j) & 1) out[t * k + j] = vals[d * k + j];
+        }
+    }
+    return flags;
+}
