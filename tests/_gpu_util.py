@@ -83,7 +83,16 @@ def ulp_bf16(v: np.ndarray) -> np.ndarray:
 def check_combine(out_gpu: torch.Tensor, y_bits: np.ndarray, gates: np.ndarray,
                   comb_row: np.ndarray, tokens=None):
     """out_gpu rows (all, or `tokens`) against the oracle.  y_bits holds the rows that
-    comb_row (already restricted to `tokens`) indexes.
+    comb_row (already restricted to `tokens`) indexes."""
+    got = out_gpu if tokens is None else out_gpu[torch.as_tensor(tokens, device=out_gpu.device)]
+    got = got.cpu().numpy() if got.dtype == torch.float32 else host_bits(got)
+    check_combine_host(got, y_bits, gates, comb_row)
+
+
+def check_combine_host(got: np.ndarray, y_bits: np.ndarray, gates: np.ndarray,
+                       comb_row: np.ndarray):
+    """Combined rows already on the host (float32, or uint16 bf16 bit patterns) against
+    the oracle.
 
     Tolerance (stated for floating point): fp32 output within 1e-5 of the magnitude
     sum_j |g_j y_j| of the float64 reference (fp32 accumulation error is defined relative
@@ -97,13 +106,64 @@ def check_combine(out_gpu: torch.Tensor, y_bits: np.ndarray, gates: np.ndarray,
     for j in range(gates.shape[1]):
         valid = (comb_row[:, j] >= 0) & (comb_row[:, j] < y_bits.shape[0])
         mag[valid] += np.abs(gates[valid, j, None].astype(np.float64) * yf[comb_row[valid, j]])
-    got = out_gpu if tokens is None else out_gpu[torch.as_tensor(tokens, device=out_gpu.device)]
-    if got.dtype == torch.float32:
-        g = got.cpu().numpy()
-        assert (np.abs(g.astype(np.float64) - ref64) <= 1e-5 * mag + 1e-30).all()
-        assert np.array_equal(g.view(np.uint32), chain.view(np.uint32))
+    if got.dtype == np.float32:
+        assert (np.abs(got.astype(np.float64) - ref64) <= 1e-5 * mag + 1e-30).all()
+        assert np.array_equal(got.view(np.uint32), chain.view(np.uint32))
     else:
-        gb = host_bits(got)
-        gf = workload.bf16_bits_to_float(gb).astype(np.float64)
+        gf = workload.bf16_bits_to_float(got).astype(np.float64)
         assert (np.abs(gf - ref64) <= ulp_bf16(ref64) + 1e-5 * mag).all()
-        assert np.array_equal(gb, oracle.bf16_rne(chain))
+        assert np.array_equal(got, oracle.bf16_rne(chain))
+
+
+def _first_bad_row(got: np.ndarray, want: np.ndarray) -> int:
+    return int(np.nonzero((got != want).reshape(len(got), -1).any(axis=1))[0][0])
+
+
+def check_gather_complete(send: torch.Tensor, x_bits: np.ndarray, row_token: np.ndarray,
+                          D: int, chunk: int = 1 << 15):
+    """Every one of the D gathered rows against the oracle's gather of the host copy of x,
+    streamed in chunks of rows (no sampling)."""
+    for d0 in range(0, D, chunk):
+        d1 = min(D, d0 + chunk)
+        got = host_bits(send[d0:d1])
+        want = oracle.gather(x_bits, row_token[d0:d1], d1 - d0)
+        if not np.array_equal(got, want):
+            raise AssertionError(f"gathered row {d0 + _first_bad_row(got, want)} differs")
+
+
+def check_combine_complete(out: torch.Tensor, y: torch.Tensor, gates: np.ndarray,
+                           comb_row: np.ndarray, chunk: int = 512, workers: int = 0):
+    """Every combined row against the oracle (check_combine_host), in chunks of tokens.
+
+    For each chunk the expert-output rows that the ORACLE's comb_row names are copied from
+    the device (the generated inputs, selected by the oracle's indices), and the chunk is
+    checked on a worker thread (the oracle's C calls release the GIL).  At most
+    2 x workers chunks are in flight, which bounds host memory."""
+    import concurrent.futures as cf
+    import os
+    N, k = gates.shape
+    workers = workers or max(1, min(16, os.cpu_count() or 1))
+    pending = []
+
+    def job(t0, got, yh, g, local):
+        try:
+            check_combine_host(got, yh, g, local)
+        except AssertionError as e:
+            raise AssertionError(f"combined rows of tokens [{t0}, {t0 + len(g)}): {e}") from None
+
+    with cf.ThreadPoolExecutor(workers) as ex:
+        for t0 in range(0, N, chunk):
+            t1 = min(N, t0 + chunk)
+            rows = comb_row[t0:t1]
+            valid = rows >= 0
+            sel = rows[valid].astype(np.int64)
+            yh = host_bits(y.index_select(0, torch.as_tensor(sel, device=y.device)))
+            local = np.full(rows.shape, -1, np.int32)
+            local[valid] = np.arange(sel.size, dtype=np.int32)
+            o = out[t0:t1]
+            got = o.cpu().numpy() if o.dtype == torch.float32 else host_bits(o)
+            pending.append(ex.submit(job, t0, got, yh, gates[t0:t1], local))
+            if len(pending) >= 2 * workers:
+                pending.pop(0).result()
+        for f in pending:
+            f.result()
