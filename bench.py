@@ -3,11 +3,12 @@
 One step = one pass of the whole path over one batch of N tokens:
   coact_count (pair counts + loads) -> plan_dispatch -> dispatch_gather
   -> combine_scatter (bf16 out)
-with inputs already resident in HBM.  Default workload: config 1 (N=16384, E=64,
-top-2, H=2048 bf16, 8 logical ranks of 8 experts, 16 planted pairs co-selected by 42%
-of tokens, random placement), seeded synthetic routing.  Config 3 runs with the
-correlated placement the library builds from the batch's own pair counts; config 4 is
-two consecutive layers with token shuffling (cross-layer counts, predicted home ranks).
+with inputs already resident in HBM.  Default workload: config 3, the largest
+single-GPU configuration (N=131072, E=256, top-8, H=7168 bf16, 64 logical ranks of 4
+experts in 8 nodes, Zipf(1.2) expert popularity, 32 planted pairs), with the correlated
+placement the library builds from the batch's own pair counts; seeded synthetic routing.
+`--config 1` selects the small single-node case (N=16384, E=64, top-2, H=2048); config 4
+is two consecutive layers with token shuffling (cross-layer counts, predicted home ranks).
 
 Timing: W untimed warm-up steps, then EXACTLY K steps captured in one CUDA graph, each
 step bracketed by CUDA events on the launching stream, with an L2 flush between steps
@@ -29,6 +30,7 @@ import subprocess
 import sys
 import threading
 import time
+from typing import Optional
 
 import numpy as np
 import torch
@@ -488,6 +490,60 @@ def layout(coact, r: workload.Routing, kind: str, device):
     raise SystemExit(f"unknown placement {kind}")
 
 
+class RebalanceStep(OneLayerStep):
+    """One layer with Cobalt's two-stage layout planner: stage 1 (periodic, outside the
+    step) co-locates co-activated experts on nodes from the batch's pair counts; stage 2
+    runs every step on the device -- fresh loads from coact_count, rebalance_ranks inside
+    each node, and the plan over that placement -- then gather and combine.  Nothing in the
+    step returns to the host."""
+    n_events = 6
+    phases = {"coact_count": (0, 1), "rebalance_ranks": (1, 2), "plan_dispatch": (2, 3),
+              "dispatch_gather": (3, 4), "combine_scatter": (4, 5)}
+
+    def __init__(self, coact, r: workload.Routing, device, fill: bool = True):
+        super().__init__(coact, r, device, fill)
+        c = r.cfg
+        to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        pair = torch.zeros((c.E, c.E), dtype=torch.int64, device=device)
+        coact.coact_count(to(r.ids), c.E, pair)
+        self.expert_node = to(coact.coact_place_correlated(pair, c.n_nodes).numpy())
+        self.er = torch.empty(c.E, dtype=torch.int32, device=device)
+        self.kernels_per_step = 1 + 1 + plan_launches(c.R, self.N) + 1 + 1
+        self.step_desc = ("coact_count (fresh loads) + rebalance_ranks (per-step intra-node "
+                          "rebalance on the device; node co-location from the batch's pair "
+                          "counts, outside the step) + plan_dispatch + dispatch_gather + "
+                          "combine_scatter (bf16 out)")
+
+    def clone_for_copy(self, coact, device):
+        return RebalanceStep(coact, self.L.r, device, fill=False)
+
+    def step(self, ev=None):
+        L, c, cfg = self.L, self.L.coact, self.cfg
+        if ev: ev[0].record()
+        L.pair.zero_()
+        L.loads.zero_()
+        L.count()
+        if ev: ev[1].record()
+        c.rebalance_ranks(L.loads, self.expert_node, L.rank_node, cfg.n_nodes, out=self.er,
+                          err_flag=L.err)
+        if ev: ev[2].record()
+        c.plan_dispatch(L.ids, cfg.E, self.er, cfg.R, L.plan, rank_node=L.rank_node,
+                        n_nodes=cfg.n_nodes, src_rank=L.src_rank, err_flag=L.err)
+        if ev: ev[3].record()
+        L.gather()
+        if ev: ev[4].record()
+        L.combine()
+        if ev: ev[5].record()
+
+    def summary(self):
+        out = super().summary()
+        loads = self.L.loads.cpu().numpy()
+        er = self.er.cpu().numpy()
+        rank_load = np.bincount(er, weights=loads, minlength=self.cfg.R)
+        out["rank_load_max_over_mean"] = float(rank_load.max() / rank_load.mean())
+        return out
+
+
 class PreReducedStep(OneLayerStep):
     """One layer with the pre-reduced reverse path: count (side stream) -> plan -> gather
     -> combine_rows over the send rows (one bf16 partial row per (token, rank), D rows
@@ -802,6 +858,8 @@ def make_step(coact, cfg_index: int, seed: int, device, two_hop: bool = False,
         S = BackwardStep(coact, r, device)
     elif mode == "prereduced":
         S = PreReducedStep(coact, r, device)
+    elif mode == "rebalance":
+        S = RebalanceStep(coact, r, device)
     else:
         S = OneLayerStep(coact, r, device)
     if rr_D is not None:
@@ -864,7 +922,7 @@ def run_gpu(args):
     TwoHopStep.forward = args.forward
     ReplicaStep.layout_kind = args.replica_layout
     mode = "shuffle" if args.shuffle else f"replicas:{args.replicas}" if args.replicas else \
-        "backward" if args.pass_ == "backward" else (
+        "backward" if args.pass_ == "backward" else "rebalance" if args.rebalance else (
         "prereduced" if args.combine == "prereduced" else "forward")
     S, placement = make_step(coact, args.config, rank_seed(args.seed, rank), device, args.two_hop,
                              args.placement, mode, args.tokens)
@@ -967,6 +1025,7 @@ def run_gpu(args):
     dom = max(parts, key=lambda p: p[3])
     dom_gbs = dom[2] / (dom[3] / 1e3) / 1e9
     e2e = {"value": None, "note": S.e2e_skip} if hasattr(S, "e2e_skip") else \
+        {"value": None, "note": "skipped (--no-e2e)"} if args.no_e2e else \
         run_e2e(coact, S, args, world, device)
 
     result = {
@@ -1019,7 +1078,7 @@ def run_gpu(args):
     if hasattr(S, "rr_dedup"):
         result["dedup_rows_over_naive_config_placement"] = S.rr_dedup
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(S, args.cpu_seconds)
+        result["cpu_baseline"] = cpu_baseline(S, args.cpu_seconds, args.cpu_tokens)
     if world > 1:
         import torch.distributed as dist
         del g_main, g_phase
@@ -1037,9 +1096,16 @@ def run_e2e(coact, S, args, world, device):
     overlap step i's compute and output copy (copy engines in both directions run
     concurrently with the SMs)."""
     cfg = S.cfg
-    host = {n: t.cpu().pin_memory() for n, t in S.inputs().items()}
+
+    def pinned(t, fill: bool):
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        if fill:
+            h.copy_(t)
+        return h
+
+    host = {n: pinned(t, True) for n, t in S.inputs().items()}
     bufs = [S, S.clone_for_copy(coact, device)]
-    outs_h = [[t.cpu().pin_memory() for t in S.outputs()] for _ in range(2)]
+    outs_h = [[pinned(t, False) for t in S.outputs()] for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = sum(t.numel() * t.element_size() for t in outs_h[0])
     comp = torch.cuda.current_stream()
@@ -1102,8 +1168,9 @@ def _oracle_layer(o, ids, gates, er, rn, n_nodes, E, R, xb, yb, src=None):
     return o.combine_f64(yb, gates, p["comb_row"])
 
 
-def _oracle_step_fn(S):
-    """A closure running the oracle over the same workload as step S (host arrays)."""
+def _oracle_step_fn(S, max_tokens: Optional[int] = None):
+    """A closure running the oracle over the same workload as step S (host arrays); its
+    `tokens` attribute is the number of tokens one call processes."""
     import oracle as o
     cfg = S.cfg
     if isinstance(S, TwoLayerStep):
@@ -1119,6 +1186,7 @@ def _oracle_step_fn(S):
             x2 = o.bf16_rne(out1.astype(np.float32))
             _oracle_layer(o, tl.layer2.ids, tl.layer2.gates, tl.layer2.expert_rank,
                           tl.layer2.rank_node, cfg.n_nodes, cfg.E, cfg.R, x2, y2, src=home)
+        fn.tokens = S.N
         return fn
     if isinstance(S, ShuffleStep):
         # a bounded sample: the first 4096 tokens' predicted homes and partial rows
@@ -1143,43 +1211,59 @@ def _oracle_step_fn(S):
         def fn():
             o.combine_backward(yb, L.r.gates, p["comb_row"], gob)
             o.gather_backward_f32chain(gsb, p["send_row"])
+        fn.tokens = S.N
         return fn
-    xb, yb = o._bits(L.x), o._bits(L.y)
+    # a bounded sample: the batch's first n tokens (their routing, x rows and as many
+    # expert-output rows as n tokens have), the whole path over them
+    n = S.N if not max_tokens else min(S.N, int(max_tokens))
+    ids, gates = L.r.ids[:n], L.r.gates[:n]
+    xb, yb = o._bits(L.x[:n]), o._bits(L.y[:n * cfg.k])
     if isinstance(S, TwoHopStep):
         def fn():
-            o.count(L.r.ids, cfg.E)
-            node, rank, fwd = o.plan_two_hop(L.r.ids, cfg.E, L.r.expert_rank, cfg.R,
+            o.count(ids, cfg.E)
+            node, rank, fwd = o.plan_two_hop(ids, cfg.E, L.r.expert_rank, cfg.R,
                                              L.r.rank_node, cfg.n_nodes)
             hop1 = o.gather(xb, node["row_token"], node["D"])
             o.forward_gather(hop1, fwd)
-            o.combine_f64(yb, L.r.gates, rank["comb_row"])
-        return fn
-    if isinstance(S, ReplicaStep):
+            o.combine_f64(yb, gates, rank["comb_row"])
+    elif isinstance(S, ReplicaStep):
         def fn():
-            o.count(L.r.ids, cfg.E)
-            slot, _ = o.assign_replicas(L.r.ids, cfg.E, S.rep_h, S.nrep_h, cfg.R,
+            o.count(ids, cfg.E)
+            slot, _ = o.assign_replicas(ids, cfg.E, S.rep_h, S.nrep_h, cfg.R,
                                         rank_node=L.r.rank_node, n_nodes=cfg.n_nodes)
-            p = o.plan(L.r.ids, cfg.E, None, cfg.R, rank_node=L.r.rank_node, n_nodes=cfg.n_nodes,
+            p = o.plan(ids, cfg.E, None, cfg.R, rank_node=L.r.rank_node, n_nodes=cfg.n_nodes,
                        slot_rank=slot)
             o.gather(xb, p["row_token"], p["D"])
-            o.combine_f64(yb, L.r.gates, p["comb_row"])
-        return fn
-    if isinstance(S, PreReducedStep):
+            o.combine_f64(yb, gates, p["comb_row"])
+    elif isinstance(S, RebalanceStep):
+        en = S.expert_node.cpu().numpy()
+
         def fn():
-            o.count(L.r.ids, cfg.E)
-            p = o.plan(L.r.ids, cfg.E, L.r.expert_rank, cfg.R, rank_node=L.r.rank_node,
+            _, loads, _ = o.count(ids, cfg.E)
+            er = o.rebalance_ranks(loads, en, L.r.rank_node)
+            p = o.plan(ids, cfg.E, er, cfg.R, rank_node=L.r.rank_node, n_nodes=cfg.n_nodes)
+            o.gather(xb, p["row_token"], p["D"])
+            o.combine_f64(yb, gates, p["comb_row"])
+    elif isinstance(S, PreReducedStep):
+        def fn():
+            o.count(ids, cfg.E)
+            p = o.plan(ids, cfg.E, L.r.expert_rank, cfg.R, rank_node=L.r.rank_node,
                        n_nodes=cfg.n_nodes)
             o.gather(xb, p["row_token"], p["D"])
-            o.combine_prereduced(yb, L.r.gates, p)
-        return fn
-    return lambda: _oracle_layer(o, L.r.ids, L.r.gates, L.r.expert_rank, L.r.rank_node,
-                                 cfg.n_nodes, cfg.E, cfg.R, xb, yb)
+            o.combine_prereduced(yb, gates, p)
+    else:
+        def fn():
+            _oracle_layer(o, ids, gates, L.r.expert_rank, L.r.rank_node, cfg.n_nodes, cfg.E,
+                          cfg.R, xb, yb)
+    fn.tokens = n
+    return fn
 
 
-def cpu_baseline(S, seconds: float):
-    """The oracle, as it stands, on this host: whole batches of the same workload
-    repeated for about `seconds` (at least one)."""
-    fn = _oracle_step_fn(S)
+def cpu_baseline(S, seconds: float, max_tokens: Optional[int] = None):
+    """The oracle, as it stands, on this host: passes over the same workload (whole
+    batches, or the batch's first max_tokens tokens when N is larger) repeated for about
+    `seconds` (at least one pass)."""
+    fn = _oracle_step_fn(S, max_tokens)
     n, t0 = 0, time.perf_counter()
     while True:
         fn()
@@ -1187,25 +1271,30 @@ def cpu_baseline(S, seconds: float):
         if time.perf_counter() - t0 >= seconds:
             break
     dt = time.perf_counter() - t0
-    if hasattr(fn, "tokens"):
-        return {"value": fn.tokens * n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-                "sample": f"{n} pass(es) over the first {fn.tokens} tokens of config "
-                          f"{S.cfg.index} through the single-threaded C oracle: home prediction, "
-                          "shuffle order and the rank-order sum of the partial rows",
-                "host_cpu": _cpu_model(), "host_nproc": os.cpu_count()}
-    return {"value": S.N * n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{n} whole batch(es) of config {S.cfg.index} (N={S.N}) through the "
-                      "single-threaded C oracle: " + (
-                          "combine backward (float64 gate gradients) and transposed dispatch"
-                          if isinstance(S, BackwardStep) else
-                          "count, node and rank plans, hop-1 gather, hop-2 forward, float64 combine"
-                          if isinstance(S, TwoHopStep) else
-                          "count, replica choice, plan, gather, float64 combine"
-                          if isinstance(S, ReplicaStep) else
-                          "count, plan, gather, partial rows and their sum"
-                          if isinstance(S, PreReducedStep) else
-                          "count, plan, gather, float64 combine"),
-            "host_cpu": _cpu_model(), "host_nproc": os.cpu_count()}
+    what = ("home prediction, shuffle order and the rank-order sum of the partial rows"
+            if isinstance(S, ShuffleStep) else
+            "both layers' count, plan, gather and float64 combine, cross-layer counts and the "
+            "home prediction" if isinstance(S, TwoLayerStep) else
+            "combine backward (float64 gate gradients) and transposed dispatch"
+            if isinstance(S, BackwardStep) else
+            "count, node and rank plans, hop-1 gather, hop-2 forward, float64 combine"
+            if isinstance(S, TwoHopStep) else
+            "count, replica choice, plan, gather, float64 combine"
+            if isinstance(S, ReplicaStep) else
+            "count, plan, gather, partial rows and their sum"
+            if isinstance(S, PreReducedStep) else
+            "count, intra-node rebalance, plan, gather, float64 combine"
+            if isinstance(S, RebalanceStep) else
+            "count, plan, gather, float64 combine")
+    if fn.tokens < S.N:
+        sample = (f"{n} pass(es) over the first {fn.tokens} of the {S.N} tokens of config "
+                  f"{S.cfg.index} (same placement, rows of H={S.cfg.H}) through the "
+                  f"single-threaded C oracle: {what}")
+    else:
+        sample = (f"{n} whole batch(es) of config {S.cfg.index} (N={S.N}) through the "
+                  f"single-threaded C oracle: {what}")
+    return {"value": fn.tokens * n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": sample, "host_cpu": _cpu_model(), "host_nproc": os.cpu_count()}
 
 
 def _cpu_model():
@@ -1225,6 +1314,10 @@ def run_reference(args):
     import oracle as o
     cfg = workload.CONFIGS[args.config]
     r = workload.make_routing(cfg, seed=args.seed)
+    if args.config == 3 and args.placement in ("auto", "correlated"):
+        # the timed arm's placement: correlated, from the whole batch's pair counts (built
+        # once per batch, outside the timed steps in both arms)
+        r.expert_rank = o.place_correlated(o.count(r.ids, cfg.E)[0], cfg.R)
     # each step: a bounded sample of the workload (the first n tokens' routing, whole
     # count/plan/gather/combine over them) sized so K + W steps end within a few minutes
     step_tokens = min(cfg.N, max(256, int(args.ref_tokens)))
@@ -1238,8 +1331,8 @@ def run_reference(args):
         _oracle_layer(o, ids, gates, r.expert_rank, r.rank_node, cfg.n_nodes, cfg.E, cfg.R, xs, ys)
     dt = time.perf_counter() - t0
     value = step_tokens * args.steps / dt
-    sample = (f"first {step_tokens} tokens of config {cfg.index} per step (count, plan, gather, "
-              "float64 combine of one layer), single-threaded C oracle")
+    sample = (f"first {step_tokens} of the {cfg.N} tokens of config {cfg.index} per step (count, "
+              "plan, gather, float64 combine of one layer), single-threaded C oracle")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
@@ -1257,12 +1350,17 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=1, choices=sorted(workload.CONFIGS))
+    ap.add_argument("--config", type=int, default=3, choices=sorted(workload.CONFIGS))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="coact", choices=["coact", "reference"])
     ap.add_argument("--no-graph", dest="graph", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end pass (profiling captures of the kernels)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-tokens", type=int, default=16384,
+                    help="cpu_baseline sample: the first CPU_TOKENS tokens of the batch (whole "
+                         "batches when N is smaller)")
     ap.add_argument("--clock-warm-s", type=float, default=1.0)
     ap.add_argument("--ref-tokens", type=int, default=4096)
     ap.add_argument("--placement", default="auto", choices=["auto", "default", "correlated",
@@ -1288,6 +1386,9 @@ def main():
     ap.add_argument("--forward", default="tokens", choices=["tokens", "rows"],
                     help="two-hop forward: token order, each hop-1 row read once "
                          "(forward_gather_tokens), or one read per rank row (forward_gather)")
+    ap.add_argument("--rebalance", action="store_true",
+                    help="Cobalt's per-step intra-node rebalance on the device inside the step "
+                         "(node co-location from the batch's counts, outside the step)")
     ap.add_argument("--two-hop", action="store_true",
                     help="dispatch in two hops: to nodes, then inside the node to ranks")
     args = ap.parse_args()
