@@ -423,6 +423,46 @@ def test_bf16_rne_against_torch():
     assert (nan & 0x7F80) == 0x7F80 and (nan & 0x7F) != 0
 
 
+def _nan_as_nan_equal(a: np.ndarray, b: np.ndarray) -> bool:
+    """Bitwise equality of float32 arrays where a NaN meets a NaN of any payload."""
+    na, nb = np.isnan(a), np.isnan(b)
+    return bool(np.array_equal(na, nb) and np.array_equal(a.view(np.uint32)[~na],
+                                                         b.view(np.uint32)[~nb]))
+
+
+@pytest.mark.parametrize("k", [1, 2])
+def test_combine_chain_special_values_ieee(k):
+    """The fixed-order chain on every class of bf16 value (+-0, subnormals, +-inf, NaNs,
+    the largest values) and special gates, against IEEE float32 arithmetic in numpy.
+    The gates are bf16-representable with |g| in {0} u [2^-8, 1] or infinite, so every
+    product g*y is exact in fp32 (at most 16 significant bits, no overflow, no loss in
+    the subnormal range): then fma(g1, y1, +0) is the product plus +0 (which turns -0
+    into +0) and fma(g2, y2, acc) is one rounded float32 addition.  NaN meets NaN."""
+    rng = np.random.default_rng(40 + k)
+    N, H = 3000, 64
+    y = rng.integers(0, 1 << 16, (N * k, H), dtype=np.uint32).astype(np.uint16)
+    y[:, :13] = np.array([0x0000, 0x8000, 0x7F80, 0xFF80, 0x7FC0, 0xFFC1, 0x7F81, 0x0001,
+                          0x8001, 0x007F, 0x7F7F, 0xFF7F, 0x3F80], np.uint16)
+    pool = np.array([0.0, -0.0, 1.0, -1.0, 0.5, 0.75, -0.375, 2.0 ** -8, 0.9921875,
+                     np.inf, -np.inf, np.nan], np.float32)
+    g = pool[rng.integers(0, len(pool), (N, k))]
+    comb = rng.permutation(N * k).reshape(N, k).astype(np.int32)
+    got = oracle.combine_f32chain(y, g, comb)
+    yf = workload.bf16_bits_to_float(y)
+    with np.errstate(invalid="ignore", over="ignore"):
+        want = g[:, 0, None] * yf[comb[:, 0]] + np.float32(0.0)
+        for j in range(1, k):
+            want = want + g[:, j, None] * yf[comb[:, j]]
+    assert want.dtype == np.float32
+    assert _nan_as_nan_equal(got, want)
+    assert np.isnan(got).any() and np.isinf(got).any() and (got == 0).any()
+    # and its rounding to bf16 matches torch's conversion (NaN as NaN)
+    import torch
+    b = oracle.bf16_rne(got)
+    t = torch.from_numpy(got.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert _nan_as_nan_equal(workload.bf16_bits_to_float(b), workload.bf16_bits_to_float(t))
+
+
 # ----------------------------------------------------------------------------- prediction pins
 
 
