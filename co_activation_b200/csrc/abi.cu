@@ -1,4 +1,6 @@
 // Status strings, ABI version and the per-device attribute cache.
+#include <cuda.h>  // the driver's types for cuCtxGetId, resolved at run time (no -lcuda)
+
 #include "common.cuh"
 
 namespace coact {
@@ -16,6 +18,27 @@ int cuda_fail(cudaError_t e) {
     return COACT_ERR_CUDA;
 }
 
+namespace {
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// cuCtxGetId through the runtime's driver entry-point lookup, once per process; NULL if
+// this driver does not provide it (the context id then reads 0 everywhere).
+CtxGetIdFn ctx_get_id_fn() {
+    static const CtxGetIdFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            (void)cudaGetLastError();
+            p = nullptr;
+        }
+        return reinterpret_cast<CtxGetIdFn>(p);
+    }();
+    return fn;
+}
+}  // namespace
+
 int device_info(DeviceInfo *out) {
     int dev = 0;
     if (cudaError_t e = cudaGetDevice(&dev)) return cuda_fail(e);
@@ -32,7 +55,17 @@ int device_info(DeviceInfo *out) {
         g_smem_optin[dev].store(smem, std::memory_order_relaxed);
         g_smem_sm[dev].store(smem_sm, std::memory_order_relaxed);
     }
+    unsigned long long ctx = 0;
+    if (CtxGetIdFn f = ctx_get_id_fn()) {
+        if (f(nullptr, &ctx) != CUDA_SUCCESS) {
+            // no current context (e.g. right after a device reset): make the device's
+            // primary context current, as any runtime call would, and ask again
+            if (cudaError_t e = cudaSetDevice(dev)) return cuda_fail(e);
+            if (f(nullptr, &ctx) != CUDA_SUCCESS) ctx = 0;
+        }
+    }
     out->device = dev;
+    out->ctx = ctx;
     out->sm_count = sms;
     out->smem_optin = smem;
     out->smem_per_sm = smem_sm;

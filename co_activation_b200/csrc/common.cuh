@@ -119,6 +119,11 @@ struct DeviceInfo {
     int sm_count;
     int smem_optin;   // max dynamic shared memory per block (opt-in)
     int smem_per_sm;  // shared memory per SM
+    // Id of the current CUDA context (unique for the life of the process; 0 if the driver
+    // cannot tell).  Per-context state -- a kernel's shared-memory opt-in, the device
+    // address of a __device__ array -- is cached under it, so a device reset (which ends
+    // the context and unloads the module) makes the next call set it up again.
+    unsigned long long ctx;
 };
 int device_info(DeviceInfo *out);  // returns COACT_OK or COACT_ERR_CUDA
 
@@ -132,20 +137,28 @@ int cuda_fail(cudaError_t e);
 
 struct SmemOptIn {
     std::atomic<int> bytes[kMaxDevices];
+    std::atomic<unsigned long long> ctx[kMaxDevices];
 };
 
-// Opts `kernel` in to `bytes` of dynamic shared memory on the current device once;
-// later calls only read the cache, so a stream capture sees launches alone.
+// Opts `kernel` in to `bytes` of dynamic shared memory on the current device once per
+// context; later calls only read the cache, so a stream capture sees launches alone.
+// (Two threads racing here at most repeat the idempotent attribute call.)
 template <typename F>
 int ensure_smem(F kernel, size_t bytes, SmemOptIn &cache, const DeviceInfo &di) {
     if (bytes <= 48 * 1024) return COACT_OK;
     if (bytes > (size_t)di.smem_optin) return COACT_ERR_UNSUPPORTED;
     std::atomic<int> &slot = cache.bytes[di.device];
-    if (slot.load(std::memory_order_relaxed) >= (int)bytes) return COACT_OK;
+    std::atomic<unsigned long long> &ctx = cache.ctx[di.device];
+    if (ctx.load(std::memory_order_acquire) == di.ctx &&
+        slot.load(std::memory_order_relaxed) >= (int)bytes)
+        return COACT_OK;
     if (cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)bytes))
         return cuda_fail(e);
-    slot.store((int)bytes, std::memory_order_relaxed);
+    if (ctx.load(std::memory_order_relaxed) != di.ctx) slot.store(0, std::memory_order_relaxed);
+    slot.store(std::max(slot.load(std::memory_order_relaxed), (int)bytes),
+               std::memory_order_relaxed);
+    ctx.store(di.ctx, std::memory_order_release);
     return COACT_OK;
 }
 

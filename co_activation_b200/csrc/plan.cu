@@ -23,6 +23,8 @@
 // Positions depend only on token order, so every output is deterministic.
 #include <algorithm>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace coact {
@@ -711,17 +713,27 @@ constexpr size_t kNoallocScratchBytes =
 // address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_plan_scratch[kNoallocScratchBytes];
 
-std::atomic<void *> g_plan_scratch_addr[kMaxDevices];
+struct ScratchAddr {
+    std::mutex m;
+    unsigned long long ctx = 0;  // context the address belongs to
+    void *addr = nullptr;
+};
+ScratchAddr g_plan_scratch_addr[kMaxDevices];
 
-// Device address of g_plan_scratch on the current device, looked up once per device.
+// Device address of g_plan_scratch in the current context of the current device, looked
+// up once per device and again whenever the context changes (a device reset unloads the
+// module, and the array may come back at another address).
 int noalloc_scratch(const DeviceInfo &di, void **out) {
-    void *p = g_plan_scratch_addr[di.device].load(std::memory_order_acquire);
-    if (!p) {
+    ScratchAddr &slot = g_plan_scratch_addr[di.device];
+    std::lock_guard<std::mutex> lock(slot.m);
+    if (!slot.addr || slot.ctx != di.ctx) {
+        void *p = nullptr;
         if (cudaError_t e = cudaGetSymbolAddress(&p, g_plan_scratch)) return cuda_fail(e);
         if (!p) return COACT_ERR_CUDA;
-        g_plan_scratch_addr[di.device].store(p, std::memory_order_release);
+        slot.addr = p;
+        slot.ctx = di.ctx;
     }
-    *out = p;
+    *out = slot.addr;
     return COACT_OK;
 }
 
