@@ -71,6 +71,10 @@ _lib.coact_compose_map.argtypes = [_P, _I64, _P, _I64, _P, _P, _P]
 _lib.plan_forward.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _P, _P, _I64, _P, _P]
 _lib.forward_gather.argtypes = [_P, _I64, _I64, _P, _I64, _P, _P, _P]
 _lib.forward_gather_tokens.argtypes = [_P, _I64, _I64, _P, _I64, _I32, _P, _I64, _P, _P, _P]
+_lib.plan_row_meta.argtypes = [_P, _P, _I64, _P, _I32, _P, _P, _P, _I64, _I32, _P, _P, _P, _P, _P,
+                               _P]
+_lib.gather_row_slots.argtypes = [_P, _I64, _P, _P, _I64, _I32, _P, _P, _P]
+_lib.rebalance_ranks.argtypes = [_P, _P, _I32, _P, _I32, _I32, _P, _P, _P]
 _lib.plan_dispatch_noalloc.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _I32, _P, _P, _P, _P,
                                        _P, _P, _P, _I64, _P, _P, _P, _P, _P, _P]
 for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "dispatch_gather_tma",
@@ -80,7 +84,7 @@ for _f in ("coact_count", "plan_dispatch", "dispatch_gather", "dispatch_gather_t
            "coact_place_correlated", "plan_dispatch_noalloc", "coact_compose_map", "plan_forward",
            "forward_gather", "forward_gather_tokens", "coact_rebalance_ranks",
            "coact_place_replicas", "dispatch_gather_peer",
-           "combine_scatter_peer"):
+           "combine_scatter_peer", "plan_row_meta", "gather_row_slots", "rebalance_ranks"):
     getattr(_lib, _f).restype = _I32
 
 ABI_SYMBOLS = ("coact_strerror", "coact_abi_version", "coact_last_cuda_error", "coact_count", "plan_dispatch_workspace_bytes",
@@ -90,7 +94,8 @@ ABI_SYMBOLS = ("coact_strerror", "coact_abi_version", "coact_last_cuda_error", "
                "coact_rebalance_ranks", "dispatch_gather_peer", "combine_scatter_peer",
                "combine_rows", "dispatch_gather_backward", "combine_scatter_backward",
                "shuffle_reduce_scatter", "plan_dispatch_slots", "assign_replicas",
-               "forward_gather_tokens", "coact_place_replicas")
+               "forward_gather_tokens", "coact_place_replicas", "plan_row_meta",
+               "gather_row_slots", "rebalance_ranks")
 NOALLOC_MAX_TOKENS = 262144
 
 
@@ -489,8 +494,8 @@ def plan_dispatch_noalloc(ids: torch.Tensor, E: int, expert_rank: torch.Tensor, 
     afford cudaMalloc's device-wide synchronisation): the library's own file-scope device
     scratch replaces the workspace (plan.workspace is not used).  Batches of at most
     NOALLOC_MAX_TOKENS tokens; calls that overlap on the GPU share that scratch and race,
-    so keep them on one stream.  The first call on a device must come before any stream
-    capture (it looks up the scratch address)."""
+    so keep them on one stream.  The first call on a device, and the first after a device
+    reset, must come before any stream capture (it looks up the scratch address)."""
     N, k = ids.shape
     if N > NOALLOC_MAX_TOKENS:
         raise ValueError(f"plan_dispatch_noalloc handles at most {NOALLOC_MAX_TOKENS} tokens "
@@ -517,6 +522,58 @@ def plan_dispatch_noalloc(ids: torch.Tensor, E: int, expert_rank: torch.Tensor, 
         _ptr(plan.send_row), _ptr(plan.comb_row), _ptr(plan.stats), _ptr(plan.src_dst),
         _ptr(err_flag), _stream(stream)), "plan_dispatch_noalloc")
     return plan
+
+
+# ----------------------------------------------------------------------------- EP row metadata
+
+
+def plan_row_meta(plan: "Plan", ids: Optional[torch.Tensor] = None,
+                  gates: Optional[torch.Tensor] = None, slot_base: Optional[torch.Tensor] = None,
+                  experts: bool = True, with_slots: bool = True,
+                  err_flag: Optional[torch.Tensor] = None, stream=None):
+    """Per send row of `plan` (rows < rank_offsets[R], read on the device), one entry per
+    slot: the expert id (ids given), the gate (gates given) and the expert-output position
+    comb_row + slot_base[rank of the row] (with_slots); -1 / 0 / -1 where the row does not
+    serve the slot.  Returns (row_experts int32, row_gates fp32, row_slots int32), each
+    [row_capacity, k] or None; rows past D are left uninitialised."""
+    N, k = plan.send_row.shape
+    R = plan.rank_counts.shape[0]
+    cap = plan.row_capacity
+    dev = plan.send_row.device
+    _need(ids, "ids", torch.int32, (N, k), optional=True)
+    _need(gates, "gates", torch.float32, (N, k), optional=True)
+    _need(slot_base, "slot_base", torch.int32, (R,), optional=True)
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    ex = torch.empty((cap, k), dtype=torch.int32, device=dev) if (experts and ids is not None) else None
+    gt = torch.empty((cap, k), dtype=torch.float32, device=dev) if gates is not None else None
+    sl = torch.empty((cap, k), dtype=torch.int32, device=dev) if with_slots else None
+    _check(_lib.plan_row_meta(_ptr(plan.row_token), _ptr(plan.row_kmask), cap,
+                              _ptr(plan.rank_offsets), R, _ptr(ids), _ptr(gates),
+                              _ptr(plan.comb_row), N, k, _ptr(slot_base), _ptr(ex), _ptr(gt),
+                              _ptr(sl), _ptr(err_flag), _stream(stream)), "plan_row_meta")
+    return ex, gt, sl
+
+
+def gather_row_slots(vals: torch.Tensor, send_row: torch.Tensor, row_kmask: torch.Tensor,
+                     out: Optional[torch.Tensor] = None, err_flag: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """out[t, j] = vals[d, j] for the send row d of token t that holds slot j (0 where
+    none does); vals fp32 [n_rows, k] in send-row order."""
+    N, k = send_row.shape
+    _need(vals, "vals", torch.float32)
+    if vals.dim() != 2 or vals.shape[1] != k:
+        raise ValueError("vals must be [n_rows, k]")
+    _need(send_row, "send_row", torch.int32, (N, k))
+    _need(row_kmask, "row_kmask", torch.uint8)
+    if row_kmask.numel() < vals.shape[0]:
+        raise ValueError("row_kmask needs an entry per row of vals")
+    if out is None:
+        out = torch.empty((N, k), dtype=torch.float32, device=send_row.device)
+    _need(out, "out", torch.float32, (N, k))
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.gather_row_slots(_ptr(vals), vals.shape[0], _ptr(send_row), _ptr(row_kmask), N, k,
+                                 _ptr(out), _ptr(err_flag), _stream(stream)), "gather_row_slots")
+    return out
 
 
 # ----------------------------------------------------------------------------- two-hop dispatch
@@ -646,6 +703,27 @@ def coact_rebalance_ranks(loads, expert_node, rank_node):
     out = torch.empty(ld.shape[0], dtype=torch.int32)
     _check(_lib.coact_rebalance_ranks(_ptr(ld), _ptr(en), ld.shape[0], _ptr(rn), rn.shape[0],
                                       _ptr(out)), "coact_rebalance_ranks")
+    return out
+
+
+def rebalance_ranks(loads: torch.Tensor, expert_node: torch.Tensor, rank_node: torch.Tensor,
+                    n_nodes: int, out: Optional[torch.Tensor] = None,
+                    err_flag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """coact_rebalance_ranks on the device (Cobalt's per-step intra-node adjustment): the
+    node's experts by load descending, each to the node's least loaded rank with a free
+    slot.  loads: device int64 [E]; expert_node: int32 [E]; rank_node: int32 [R].
+    Returns the int32 [E] expert -> rank map (-1 and a flag where the layout does not
+    fit)."""
+    E, R = loads.shape[0], rank_node.shape[0]
+    _need(loads, "loads", torch.int64, (E,))
+    _need(expert_node, "expert_node", torch.int32, (E,))
+    _need(rank_node, "rank_node", torch.int32, (R,))
+    if out is None:
+        out = torch.empty(E, dtype=torch.int32, device=loads.device)
+    _need(out, "out", torch.int32, (E,))
+    _need(err_flag, "err_flag", torch.int32, (1,), optional=True)
+    _check(_lib.rebalance_ranks(_ptr(loads), _ptr(expert_node), E, _ptr(rank_node), R, n_nodes,
+                                _ptr(out), _ptr(err_flag), _stream(stream)), "rebalance_ranks")
     return out
 
 

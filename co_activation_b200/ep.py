@@ -45,10 +45,13 @@ predicted to live on it (ascending), each the sum of the P partials in rank orde
 the partials permuted locally (dispatch_gather over the shuffle plan), one all_to_all of
 the rank segments, then the same kernel over the P received blocks.
 
-Only library kernels touch rows and plans; this module moves split sizes, builds the
-small per-row expert-id metadata the experts need, and calls the collectives.  The
-local steps are an `ops` object (the library by default) so that the exchange logic can
-run on CPU test doubles.
+Only library kernels touch rows, plans and their per-row metadata (plan_row_meta: each
+send row's expert ids, gates and output positions at the destination; gather_row_slots:
+per-slot values back to token order); this module moves split sizes and calls the
+collectives.  One host synchronisation per dispatch remains: NCCL's all_to_all_single
+takes its split sizes as host lists, and the received tensors' shapes depend on the
+exchanged counts.  The local steps are an `ops` object (the library by default) so that
+the exchange logic can run on CPU test doubles.
 """
 from __future__ import annotations
 
@@ -70,25 +73,15 @@ def exclusive_offsets(C: torch.Tensor) -> torch.Tensor:
 @dataclasses.dataclass
 class Dispatched:
     """What rank r receives: its rows (source rank, then token order), the slot mask of
-    each row and the expert id of every set slot (-1 elsewhere)."""
+    each row, the expert id of every set slot (-1 elsewhere) and where each set slot's
+    expert output goes in this rank's expanded receive order (-1 elsewhere)."""
     rows: torch.Tensor          # bf16 [n_rows, H]
     kmask: torch.Tensor         # uint8 [n_rows]
     experts: torch.Tensor       # int32 [n_rows, k]
+    slots: torch.Tensor         # int32 [n_rows, k]
     counts: torch.Tensor        # int64 [R, R] rows s -> r
     asg: torch.Tensor           # int64 [R, R] assignments s -> r
     gates: Optional[torch.Tensor] = None   # fp32 [n_rows, k]: gate of each set slot, 0 elsewhere
-
-
-def local_slots(kmask: torch.Tensor, k: int) -> torch.Tensor:
-    """Where each received row's slots sit among the rank's expert outputs (expanded
-    receive order): int32 [n_rows, k], -1 for the slots that are not on this rank."""
-    km = kmask.to(torch.int64)
-    bits = (km[:, None] >> torch.arange(k, device=km.device)) & 1
-    cnt = bits.sum(1)
-    first = torch.cumsum(cnt, 0) - cnt                  # first expanded row of each row
-    before = torch.cumsum(bits, 1) - bits               # set slots before slot j
-    return torch.where(bits.bool(), first[:, None] + before, torch.full_like(bits, -1)).to(
-        torch.int32).contiguous()
 
 
 class LibraryOps:
@@ -123,6 +116,14 @@ class LibraryOps:
 
     def count(self, ids, E, pair, loads):
         self.c.coact_count(ids, E, pair, loads)
+
+    def row_meta(self, plan, ids, gates, slot_base):
+        """Per send row and slot: expert id, gate (gates given) and output position."""
+        return self.c.plan_row_meta(plan, ids, gates, slot_base)
+
+    def gather_row_slots(self, vals, plan, out):
+        """Per-(send row, slot) values back to token order [N, k]."""
+        return self.c.gather_row_slots(vals, plan.send_row, plan.row_kmask, out)
 
     def shuffle_plan(self, home, R):
         return self.c.shuffle_plan(home, R)
@@ -180,14 +181,6 @@ class EPLayer:
         M = torch.stack(allrows)                  # [R sources, 2R]
         return M[:, :self.R].contiguous(), M[:, self.R:].contiguous()
 
-    def _row_experts(self, ids, plan, D):
-        """Expert id of every set slot of each send row (-1 elsewhere), int32 [D, k]."""
-        k = ids.shape[1]
-        tok = plan.row_token[:D].to(torch.int64)
-        km = plan.row_kmask[:D].to(torch.int32)
-        bits = (km[:, None] >> torch.arange(k, device=km.device, dtype=torch.int32)) & 1
-        return torch.where(bits.bool(), ids[tok], torch.full_like(ids[tok], -1))
-
     def dispatch(self, ids: torch.Tensor, x: torch.Tensor,
                  gates: Optional[torch.Tensor] = None) -> Dispatched:
         """Plan this rank's tokens and deliver every row to its destination rank.  With
@@ -202,29 +195,25 @@ class EPLayer:
         self.plan = plan
         self._ids = ids
         C, A = self._count_rows(plan)
+        # the one host synchronisation of a layer: all_to_all_single takes its split sizes
+        # as host lists, and the received tensors' shapes depend on the counts
         Cl, Al = C.cpu(), A.cpu()
         self._C, self._A = Cl, Al
         D = int(Cl[me].sum())
-        n_recv = int(Cl[:, me].sum())
-        meta_send = self._row_experts(ids, plan, D)
-        kmask_send = plan.row_kmask[:D].to(torch.int32)
+        # per send row and slot, computed by the library: the expert id, the gate and the
+        # slot's output position in the destination's expanded receive order, i.e. past
+        # the assignment rows that earlier sources send that rank
+        base = (exclusive_offsets(A)[me] - plan.asg_offsets[:R].to(torch.int64)).to(torch.int32)
+        ex, g, sl = self.ops.row_meta(plan, ids, gates, base)
         rows = self._send_rows(x, "recv")
-        experts = self._rows_to_dest(meta_send.to(torch.int32))
-        kmask = self._rows_to_dest(kmask_send)
-        g = None
-        if gates is not None:
-            g = self._rows_to_dest(self._row_gates(gates, plan, D))
-        self._d = Dispatched(rows=rows, kmask=kmask.to(torch.uint8), experts=experts, counts=Cl,
-                             asg=Al, gates=g)
+        experts = self._rows_to_dest(ex[:D])
+        slots = self._rows_to_dest(sl[:D])
+        kmask = self._rows_to_dest(plan.row_kmask[:D].to(torch.int32))
+        if g is not None:
+            g = self._rows_to_dest(g[:D])
+        self._d = Dispatched(rows=rows, kmask=kmask.to(torch.uint8), experts=experts, slots=slots,
+                             counts=Cl, asg=Al, gates=g)
         return self._d
-
-    def _row_gates(self, gates, plan, D):
-        """Gate of every set slot of each send row (0 elsewhere), fp32 [D, k]."""
-        k = gates.shape[1]
-        tok = plan.row_token[:D].to(torch.int64)
-        km = plan.row_kmask[:D].to(torch.int32)
-        bits = (km[:, None] >> torch.arange(k, device=km.device, dtype=torch.int32)) & 1
-        return torch.where(bits.bool(), gates[tok], torch.zeros_like(gates[tok])).contiguous()
 
     def _rows_to_dest(self, t: torch.Tensor) -> torch.Tensor:
         """Per-send-row metadata (first dim D) to the destination ranks (first dim n_recv)."""
@@ -301,9 +290,8 @@ class EPLayer:
             d = self._d
             if d is None or d.gates is None:
                 raise ValueError("reduce='rows' needs dispatch(..., gates=...) first")
-            k = gates.shape[1]
             pre = torch.empty((d.rows.shape[0], H), dtype=torch.bfloat16, device=y_recv.device)
-            self.ops.combine_local(y_recv, d.gates, local_slots(d.kmask, k), pre)
+            self.ops.combine_local(y_recv, d.gates, d.slots, pre)
             return self._sum_back(pre, "pre", out)
         if reduce != "expanded":
             raise ValueError("reduce must be 'expanded' or 'rows'")
@@ -328,16 +316,10 @@ class EPLayer:
         g_recv = self._send_rows(grad_out, "grad")
         grad_y = torch.empty_like(y_recv)
         gg = torch.zeros((d.rows.shape[0], k), dtype=torch.float32, device=y_recv.device)
-        self.ops.combine_backward(y_recv, d.gates, local_slots(d.kmask, k), g_recv, grad_y, gg)
+        self.ops.combine_backward(y_recv, d.gates, d.slots, g_recv, grad_y, gg)
         back = self._rows_to_source(gg)                      # [D, k], send-row order
-        D = back.shape[0]
-        tok = plan.row_token[:D].to(torch.int64)
-        km = plan.row_kmask[:D].to(torch.int64)
-        bits = ((km[:, None] >> torch.arange(k, device=km.device)) & 1).bool()
-        grad_gates = torch.zeros((N, k), dtype=torch.float32, device=y_recv.device)
-        cols = torch.arange(k, device=km.device).expand(D, k)
-        grad_gates[tok[:, None].expand(D, k)[bits], cols[bits]] = back[bits]
-        return grad_y, grad_gates
+        grad_gates = torch.empty((N, k), dtype=torch.float32, device=y_recv.device)
+        return grad_y, self.ops.gather_row_slots(back, plan, grad_gates)
 
     def backward_dispatch(self, grad_rows: torch.Tensor,
                           out: Optional[torch.Tensor] = None) -> torch.Tensor:

@@ -103,8 +103,9 @@ int coact_last_cuda_error(void);
  *   1  count, plan, gather, combine, predict_home, placement, two-hop, peer calls, noalloc
  *   2  dispatch_gather_tma, backward (dispatch_gather_backward, combine_scatter_backward),
  *      combine_rows, shuffle_reduce_scatter, assign_replicas, plan_dispatch_slots,
- *      forward_gather_tokens, coact_last_cuda_error; combine_scatter_peer takes NULL gates */
-#define COACT_ABI_VERSION 2
+ *      forward_gather_tokens, coact_last_cuda_error; combine_scatter_peer takes NULL gates
+ *   3  plan_row_meta, gather_row_slots, rebalance_ranks */
+#define COACT_ABI_VERSION 3
 
 /*
  * coact_count -- expert co-activation pair counts and per-expert loads.
@@ -352,7 +353,9 @@ int combine_scatter_backward(const uint16_t *y, int64_t n_rows, const float *gat
  *    enqueued; use plan_dispatch with a workspace for larger batches.
  *  - The first call on each device looks up the scratch array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call before any
- *    stream capture.
+ *    stream capture.  The address is kept per CUDA context: after a device reset (a new
+ *    context, in which the library's module is loaded again) the first call looks it up
+ *    again, so make that call outside a capture too.
  *  - All calls on a device share the one scratch array, and it keeps the last call's
  *    contents.  Nothing in it needs clearing (every entry a call reads is written
  *    earlier in the same call), but calls that overlap on the GPU -- e.g. two streams at
@@ -463,6 +466,48 @@ int combine_scatter_peer(const uint64_t *y_bases, const int32_t *y_row_offset,
                          void *out, int out_dtype, int32_t *err_flag, coact_stream_t stream);
 
 /*
+ * plan_row_meta -- what travels with each send row under expert parallelism besides the
+ * row itself.  Cobalt / Zyphra, English abstracts: each token goes to the ranks holding
+ * its experts (each rank once), which run them and send the results back to be combined;
+ * a deduplicated row serves one or more of the token's k slots.  For
+ * d < n_rows = min(row_capacity, rank_offsets[R]) (read on the device) and j < k, with
+ * t = row_token[d] and r the rank whose segment [rank_offsets[r], rank_offsets[r+1])
+ * holds d:
+ *   bit j of row_kmask[d] set:  row_experts[d,j] = ids[t,j]      (the expert to run)
+ *                               row_gates[d,j]   = gates[t,j]    (for a combine there)
+ *                               row_slots[d,j]   = comb_row[t,j] + slot_base[r]
+ *   otherwise:                  -1, 0.0f, -1
+ * slot_base: DEVICE int32 [R] or NULL (0).  With slot_base[r] = (assignment rows that
+ * earlier sources send rank r) - asg_offsets[r], row_slots[d,j] is the position of slot
+ * j's expert output in rank r's expanded receive order -- the comb_row the receiving
+ * rank's own combine or backward takes.  Inputs are the plan's outputs (row_token,
+ * row_kmask [row_capacity], rank_offsets [R+1], comb_row [N,k]) and the router's ids
+ * int32 / gates fp32 [N,k]; outputs [row_capacity, k] (rows >= n_rows untouched), each
+ * optional (NULL: not computed; its input may then be NULL).  A row whose token is
+ * outside [0, N) gets -1 / 0 / -1 and sets COACT_EFLAG_ROW_RANGE.
+ */
+int plan_row_meta(const int32_t *row_token, const uint8_t *row_kmask, int64_t row_capacity,
+                  const int32_t *rank_offsets, int R,
+                  const int32_t *ids, const float *gates, const int32_t *comb_row,
+                  int64_t N, int k, const int32_t *slot_base,
+                  int32_t *row_experts, float *row_gates, int32_t *row_slots,
+                  int32_t *err_flag, coact_stream_t stream);
+
+/*
+ * gather_row_slots -- the way back of one value per (send row, slot) to token order, e.g.
+ * the gate gradients computed where the experts ran, returned in send-row order:
+ *   out[t,j] = vals[d,j] for the send row d of token t (one of its send_row[t, j0] >= 0)
+ *              whose row_kmask[d] holds bit j,
+ *   out[t,j] = 0 where none does (slots of invalid tokens).
+ * vals: DEVICE fp32 [n_rows, k]; send_row int32 [N,k] and row_kmask uint8 [>= n_rows] of
+ * the plan; out: DEVICE fp32 [N,k], every entry written.  A send row outside [0, n_rows)
+ * is skipped and sets COACT_EFLAG_ROW_RANGE.
+ */
+int gather_row_slots(const float *vals, int64_t n_rows, const int32_t *send_row,
+                     const uint8_t *row_kmask, int64_t N, int k, float *out,
+                     int32_t *err_flag, coact_stream_t stream);
+
+/*
  * shuffle_reduce_scatter -- token shuffling fused into the post-attention reduce-scatter.
  * Zyphra, English abstract: under sequence parallelism each token moves, during the
  * reduce-scatter that follows attention, to the GPU predicted to hold its next-layer
@@ -535,6 +580,22 @@ int coact_place_correlated(const int64_t *pair, int E, int R, int32_t *expert_ra
  */
 int coact_rebalance_ranks(const int64_t *loads, const int32_t *expert_node, int E,
                           const int32_t *rank_node, int R, int32_t *expert_rank);
+
+/*
+ * rebalance_ranks -- the same greedy on the device, for Cobalt's "per-step intra-node
+ * adjustment" (English abstract) without a host round trip: the loads coact_count left on
+ * the device go straight to a placement plan_dispatch can take.  Within each node, its
+ * experts by load descending (ties: lower id) each take the node's least loaded rank
+ * with a free slot (E/R slots per rank; ties: lower rank).  loads: DEVICE int64 [E];
+ * expert_node: DEVICE int32 [E]; rank_node: DEVICE int32 [R] in [0, n_nodes);
+ * expert_rank: DEVICE int32 [E] (out).  Needs E % R == 0 (host check).  An expert whose
+ * node is outside [0, n_nodes) or has no free slot left (a node layout that does not fit
+ * its ranks) gets -1 and sets COACT_EFLAG_ID_RANGE, as does a rank whose node is outside
+ * [0, n_nodes) (it then takes no expert).  One CTA; no host synchronisation.
+ */
+int rebalance_ranks(const int64_t *loads, const int32_t *expert_node, int E,
+                    const int32_t *rank_node, int R, int n_nodes, int32_t *expert_rank,
+                    int32_t *err_flag, coact_stream_t stream);
 
 /*
  * coact_place_replicas -- a replica layout from co-activation and workload statistics

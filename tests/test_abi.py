@@ -76,7 +76,10 @@ def test_strerror_and_version(lib):
     lib.coact_strerror.restype = ctypes.c_char_p
     assert lib.coact_strerror(0) == b"ok"
     assert b"workspace" in lib.coact_strerror(-4)
-    assert lib.coact_abi_version() == 2
+    import re
+    hdr = open(os.path.join(ROOT, "include", "coact.h")).read()
+    assert lib.coact_abi_version() == int(re.search(r"#define COACT_ABI_VERSION (\d+)", hdr).group(1))
+    assert lib.coact_abi_version() == 3
 
 
 P = ctypes.c_void_p
@@ -256,3 +259,45 @@ def test_two_hop_and_planner_reject_bad_arguments(lib):
     bad = (ctypes.c_int32 * 4)(0, 0, 0, 1)                        # node 0 holds 3 of 2 slots
     assert r(loads, bad, 4, rn, 2, out) == -1
     assert r(loads, en, 4, rn, 3, out) == -2                      # 4 % 3 != 0
+
+
+def test_row_meta_calls_reject_bad_arguments(lib):
+    """plan_row_meta / gather_row_slots: host-detectable errors return a status before
+    anything is enqueued (no GPU needed to see them)."""
+    f, g = lib.plan_row_meta, lib.gather_row_slots
+    I64, I32 = ctypes.c_int64, ctypes.c_int
+    f.argtypes = [P, P, I64, P, I32, P, P, P, I64, I32, P, P, P, P, P, P]
+    g.argtypes = [P, I64, P, P, I64, I32, P, P, P]
+    ok = dict(rt=FAKE, km=FAKE, cap=10, ro=FAKE, R=4, ids=FAKE, gates=FAKE, comb=FAKE, N=5, k=2,
+              base=None, ex=FAKE, gt=FAKE, sl=FAKE)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return f(a["rt"], a["km"], a["cap"], a["ro"], a["R"], a["ids"], a["gates"], a["comb"],
+                 a["N"], a["k"], a["base"], a["ex"], a["gt"], a["sl"], None, None)
+
+    assert call(N=-1) == -1 and call(cap=-1) == -1
+    assert call(k=0) == -2 and call(k=9) == -2 and call(R=0) == -2 and call(R=65) == -2
+    assert call(ro=None) == -1
+    assert call(ids=None) == -1 and call(gates=None) == -1 and call(comb=None) == -1
+    assert call(rt=None) == -1 and call(km=None) == -1
+    assert call(cap=0) == 0                                   # nothing to do
+    assert call(ex=None, gt=None, sl=None, rt=None, km=None) == 0
+    assert g(FAKE, 4, FAKE, FAKE, -1, 2, FAKE, None, None) == -1
+    assert g(FAKE, 4, FAKE, FAKE, 5, 0, FAKE, None, None) == -2
+    assert g(FAKE, 4, None, FAKE, 5, 2, FAKE, None, None) == -1
+    assert g(None, 4, FAKE, FAKE, 5, 2, FAKE, None, None) == -1
+    assert g(FAKE, 4, FAKE, FAKE, 0, 2, FAKE, None, None) == 0
+
+
+def test_rebalance_ranks_rejects_bad_arguments(lib):
+    f = lib.rebalance_ranks
+    I32 = ctypes.c_int
+    f.argtypes = [P, P, I32, P, I32, I32, P, P, P]
+    assert f(None, FAKE, 8, FAKE, 4, 2, FAKE, None, None) == -1
+    assert f(FAKE, FAKE, 8, FAKE, 4, 2, None, None, None) == -1
+    assert f(FAKE, FAKE, 9, FAKE, 4, 2, FAKE, None, None) == -2       # E % R != 0
+    assert f(FAKE, FAKE, 1, FAKE, 1, 1, FAKE, None, None) == -2       # E < 2
+    assert f(FAKE, FAKE, 2048, FAKE, 4, 1, FAKE, None, None) == -2    # E > 1024
+    assert f(FAKE, FAKE, 8, FAKE, 4, 0, FAKE, None, None) == -2       # no node
+    assert f(FAKE, FAKE, 128, FAKE, 128, 2, FAKE, None, None) == -2   # R > 64

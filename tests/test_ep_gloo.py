@@ -85,6 +85,22 @@ class OracleOps:
         parts = np.stack([self.o._bits(b) for b in blocks])
         return self._store(out, self.o.shuffle_reduce_f32chain(parts, row_token.numpy()))
 
+    def row_meta(self, plan, ids, gates, slot_base):
+        p = {"D": int(plan.rank_offsets[-1]), "rank_offsets": plan.rank_offsets.numpy(),
+             "row_token": plan.row_token.numpy(), "row_kmask": plan.row_kmask.numpy(),
+             "comb_row": plan.comb_row.numpy()}
+        g = np.zeros(ids.shape, np.float32) if gates is None else gates.numpy()
+        ex, gt, sl, f = self.o.row_meta(p, ids.numpy(), g, slot_base=slot_base.numpy())
+        assert f == 0
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a))
+        return t(ex), (None if gates is None else t(gt)), t(sl)
+
+    def gather_row_slots(self, vals, plan, out):
+        got, f = self.o.gather_row_slots(vals.numpy(), plan.send_row.numpy(), plan.row_kmask.numpy())
+        assert f == 0
+        out.copy_(torch.from_numpy(got))
+        return out
+
     def combine_backward(self, y, gates, comb, g_out, g_y, g_gates):
         gy, gg, _ = self.o.combine_backward(self.o._bits(y), gates.numpy(), comb.numpy(),
                                             self.o._bits(g_out))
@@ -202,11 +218,15 @@ def _worker_backward(rank, world, port, cfg_spec, out):
         seg = slice(ro[rank], ro[rank + 1])
         tok, km = full["row_token"][seg], full["row_kmask"][seg]
         want_g = np.where((km[:, None] >> np.arange(k)) & 1, r.gates[tok], 0).astype(np.float32)
+        # each served slot's output position on this rank: its place in the single-process
+        # plan's rank segment of assignments
+        want_s = np.where((km[:, None] >> np.arange(k)) & 1, full["comb_row"][tok] - ao[rank], -1)
         _, pre_want = oracle.combine_prereduced(y_full, r.gates, full)
         gy_w, gg_w, _ = oracle.combine_backward(y_full, r.gates, full["comb_row"], oracle._bits(g_out))
         gx_w = oracle.gather_backward_f32chain(oracle._bits(G), full["send_row"])
         out[rank] = (
             np.array_equal(got.gates.numpy().view(np.uint32), want_g.view(np.uint32)),
+            np.array_equal(got.slots.numpy(), want_s),
             np.array_equal(pre_out.numpy().view(np.uint32), pre_want[lo:hi].view(np.uint32)),
             np.array_equal(oracle._bits(grad_y), gy_w[ao[rank]:ao[rank + 1]]),
             np.array_equal(grad_gates.numpy(), gg_w[lo:hi].astype(np.float32)),
@@ -228,7 +248,8 @@ def test_ep_prereduced_and_backward_match_single_process(world, spec):
     for p in procs:
         p.join(180)
         assert p.exitcode == 0
-    names = ("exchanged gates", "pre-reduced combine", "grad_y", "grad_gates", "grad_x")
+    names = ("exchanged gates", "output slots", "pre-reduced combine", "grad_y", "grad_gates",
+             "grad_x")
     for r in range(world):
         for name, ok in zip(names, out[r]):
             assert ok, f"rank {r}: {name} differs from the single-process oracle"
