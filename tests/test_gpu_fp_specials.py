@@ -97,7 +97,8 @@ def assert_bits_nan_as_nan(got, want, what):
 def check_tolerance_where_finite(got_f, chain, ref64, mag, bf16):
     ok = (np.isfinite(chain) & np.isfinite(ref64) & np.isfinite(mag)
           & (np.abs(ref64) < 2.0 ** 127) & np.isfinite(got_f))
-    d = np.abs(got_f.astype(np.float64) - ref64)
+    with np.errstate(invalid="ignore", over="ignore"):
+        d = np.abs(got_f.astype(np.float64) - ref64)
     tol = 1e-5 * mag + (ulp_bf16(ref64) if bf16 else 1e-30)
     assert (d[ok] <= tol[ok]).all()
     return int(ok.sum())
@@ -112,8 +113,8 @@ def test_combine_special_values(coact, k, H):
     comb[5, 0] = -1                                    # an absent slot
     chain = oracle.combine_f32chain(y, g, comb)
     ref64 = oracle.combine_f64(y, g, comb)
-    yf = workload.bf16_bits_to_float(y).astype(np.float64)
     with np.errstate(invalid="ignore", over="ignore"):
+        yf = workload.bf16_bits_to_float(y).astype(np.float64)
         mag = np.zeros((N, H))
         for j in range(k):
             v = comb[:, j] >= 0
@@ -133,7 +134,9 @@ def test_combine_special_values(coact, k, H):
             assert_bits_nan_as_nan(got, want, "combine bf16")
             n_ok = check_tolerance_where_finite(workload.bf16_bits_to_float(got), chain, ref64,
                                                 mag, True)
-        assert n_ok > N * H // 4                     # the ordinary part was checked too
+        # the ordinary part was checked too (with k = 8, about a quarter of the elements
+        # have only finite terms and a finite sum)
+        assert n_ok > N * H // 8
     assert np.isnan(chain).any() and np.isinf(chain).any()    # the specials were exercised
 
 
