@@ -131,39 +131,50 @@ def check_gather_complete(send: torch.Tensor, x_bits: np.ndarray, row_token: np.
             raise AssertionError(f"gathered row {d0 + _first_bad_row(got, want)} differs")
 
 
-def check_combine_complete(out: torch.Tensor, y: torch.Tensor, gates: np.ndarray,
-                           comb_row: np.ndarray, chunk: int = 512, workers: int = 0):
-    """Every combined row against the oracle (check_combine_host), in chunks of tokens.
-
-    For each chunk the expert-output rows that the ORACLE's comb_row names are copied from
-    the device (the generated inputs, selected by the oracle's indices), and the chunk is
-    checked on a worker thread (the oracle's C calls release the GIL).  At most
+def for_chunks(n: int, chunk: int, prepare, workers: int = 0):
+    """Runs a check over [0, n) in chunks: prepare(c0, c1) does the device work in this
+    thread (selecting and copying the chunk's rows to the host) and returns a callable
+    that checks them on a worker thread (the oracle's C calls release the GIL).  At most
     2 x workers chunks are in flight, which bounds host memory."""
     import concurrent.futures as cf
     import os
-    N, k = gates.shape
     workers = workers or max(1, min(16, os.cpu_count() or 1))
     pending = []
-
-    def job(t0, got, yh, g, local):
-        try:
-            check_combine_host(got, yh, g, local)
-        except AssertionError as e:
-            raise AssertionError(f"combined rows of tokens [{t0}, {t0 + len(g)}): {e}") from None
-
     with cf.ThreadPoolExecutor(workers) as ex:
-        for t0 in range(0, N, chunk):
-            t1 = min(N, t0 + chunk)
-            rows = comb_row[t0:t1]
-            valid = rows >= 0
-            sel = rows[valid].astype(np.int64)
-            yh = host_bits(y.index_select(0, torch.as_tensor(sel, device=y.device)))
-            local = np.full(rows.shape, -1, np.int32)
-            local[valid] = np.arange(sel.size, dtype=np.int32)
-            o = out[t0:t1]
-            got = o.cpu().numpy() if o.dtype == torch.float32 else host_bits(o)
-            pending.append(ex.submit(job, t0, got, yh, gates[t0:t1], local))
+        for c0 in range(0, n, chunk):
+            pending.append(ex.submit(prepare(c0, min(n, c0 + chunk))))
             if len(pending) >= 2 * workers:
                 pending.pop(0).result()
         for f in pending:
             f.result()
+
+
+def rows_of(t: torch.Tensor, idx: np.ndarray) -> np.ndarray:
+    """Host bf16 bits of the device rows t[idx] (idx: any shape of non-negative ints)."""
+    return host_bits(t.index_select(0, torch.as_tensor(np.ravel(idx).astype(np.int64),
+                                                       device=t.device)))
+
+
+def check_combine_complete(out: torch.Tensor, y: torch.Tensor, gates: np.ndarray,
+                           comb_row: np.ndarray, chunk: int = 512, workers: int = 0):
+    """Every combined row against the oracle (check_combine_host), in chunks of tokens:
+    per chunk, the expert-output rows that the ORACLE's comb_row names are copied from
+    the device (the generated inputs, selected by the oracle's indices)."""
+    def prepare(t0, t1):
+        rows = comb_row[t0:t1]
+        valid = rows >= 0
+        yh = rows_of(y, rows[valid])
+        local = np.full(rows.shape, -1, np.int32)
+        local[valid] = np.arange(int(valid.sum()), dtype=np.int32)
+        o = out[t0:t1]
+        got = o.cpu().numpy() if o.dtype == torch.float32 else host_bits(o)
+        g = gates[t0:t1]
+
+        def job():
+            try:
+                check_combine_host(got, yh, g, local)
+            except AssertionError as e:
+                raise AssertionError(f"combined rows of tokens [{t0}, {t1}): {e}") from None
+        return job
+
+    for_chunks(len(gates), chunk, prepare, workers)

@@ -9,8 +9,8 @@ against the CPU oracle on the same seeded inputs.
   combine_scatter_backward   grad_y bit-exact (fp32 product rounded to bf16); grad_gates
                              within the stated bound of the float64 dot product:
                              (8*ceil(H/256) + 5) * 2^-24 * sum_h |grad_out * y|
-Full-size configurations are checked on sampled tokens / rows, with the launch
-configuration the benchmark uses."""
+Full-size configurations are checked in full (every row and every gate gradient, streamed
+in chunks against the oracle), with the launch configuration the benchmark uses."""
 import math
 
 import numpy as np
@@ -19,7 +19,7 @@ import torch
 
 import oracle
 import workload
-from _gpu_util import DEV, Y_STREAM, cuda, host_bits, run_plan
+from _gpu_util import DEV, Y_STREAM, cuda, for_chunks, host_bits, rows_of, run_plan
 
 pytestmark = pytest.mark.gpu
 
@@ -74,11 +74,6 @@ def check_combine_backward(gy_dev, gg_dev, y_bits, gates, comb_row, go_bits, gy_
     assert (np.abs(gg.astype(np.float64) - gg_o) <= grad_gates_bound(y_bits.shape[1], ga_o)).all()
 
 
-def sample_tokens(N, seed, n=300):
-    rng = np.random.default_rng(seed)
-    return np.unique(np.concatenate([rng.integers(0, N, n), [0, N - 1]]))
-
-
 # ----------------------------------------------------------------------------- transposed dispatch
 
 
@@ -100,22 +95,32 @@ def test_gather_backward_full(coact, cfg, out_dtype):
 
 
 @pytest.mark.parametrize("cfg", [2, 3])
-def test_gather_backward_full_size_sampled(coact, cfg):
+def test_gather_backward_full_size_complete(coact, cfg):
+    """Configs 2 and 3 at full size: every token's gradient row against the oracle's fp32
+    add chain over the rows the oracle's send_row names, in chunks of tokens."""
     r = workload.make_routing(cfg)
     H = r.cfg.H
     plan, _ = run_plan(coact, r)
     o = oracle_plan_for(r)
     g_send = workload.fill_bf16(plan.row_capacity, H, r.seed, G_STREAM, device=DEV)
     gx = torch.empty((r.N, H), dtype=torch.bfloat16, device=DEV)
-    coact.dispatch_gather_backward(g_send, plan.send_row, gx)
+    err = zero_flag()
+    coact.dispatch_gather_backward(g_send, plan.send_row, gx, err_flag=err)
     torch.cuda.synchronize()
-    del g_send
-    toks = sample_tokens(r.N, 20 + cfg)
-    sr = o["send_row"][toks]
-    used = np.unique(sr[sr >= 0])
-    g_local = host_bits(workload.fill_bf16(len(used), H, r.seed, G_STREAM, row_ids=used))
-    local = np.where(sr >= 0, np.searchsorted(used, np.maximum(sr, 0)), -1).astype(np.int32)
-    check_grad_x(gx, g_local, local, tokens=toks)
+    assert err.item() == 0
+
+    def prepare(t0, t1):
+        sr = o["send_row"][t0:t1]
+        valid = sr >= 0
+        g_local = rows_of(g_send, sr[valid])
+        local = np.full(sr.shape, -1, np.int32)
+        local[valid] = np.arange(int(valid.sum()), dtype=np.int32)
+        got = host_bits(gx[t0:t1])
+        return lambda: np.testing.assert_array_equal(
+            got, oracle.bf16_rne(oracle.gather_backward_f32chain(g_local, local)),
+            err_msg=f"tokens [{t0}, {t1})")
+
+    for_chunks(r.N, 1024, prepare)
 
 
 @pytest.mark.parametrize("k", [1, 3, 8])
@@ -206,7 +211,9 @@ def test_combine_rows_device_unit_count(coact):
 
 
 @pytest.mark.parametrize("cfg", [2, 3])
-def test_combine_rows_full_size_sampled(coact, cfg):
+def test_combine_rows_full_size_complete(coact, cfg):
+    """Configs 2 and 3 at full size: every partial row (one per send row) against the
+    oracle's fp32 chain over the unit's slots, in chunks of send rows."""
     r = workload.make_routing(cfg)
     H, nk = r.cfg.H, r.N * r.k
     plan, _ = run_plan(coact, r)
@@ -216,19 +223,23 @@ def test_combine_rows_full_size_sampled(coact, cfg):
     pre = torch.empty((D, H), dtype=torch.float32, device=DEV)
     coact.combine_rows(y, cuda(r.gates), plan.comb_row, plan.row_token, plan.row_kmask, pre)
     torch.cuda.synchronize()
-    del y
-    rng = np.random.default_rng(30 + cfg)
-    units = np.unique(np.concatenate([rng.integers(0, D, 300), [0, D - 1]]))
-    toks = o["row_token"][units]
-    cr = o["comb_row"][toks]
-    used = np.unique(cr)
-    y_local = host_bits(workload.fill_bf16(len(used), H, r.seed, Y_STREAM, row_ids=used))
-    local = np.searchsorted(used, cr).astype(np.int32)
-    want = oracle.combine_units_f32chain(y_local, r.gates[toks], local,
-                                         np.arange(len(units), dtype=np.int32),
-                                         o["row_kmask"][units])
-    got = pre[torch.as_tensor(units, device=DEV)].cpu().numpy()
-    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+    def prepare(u0, u1):
+        toks = o["row_token"][u0:u1]
+        cr = o["comb_row"][toks]
+        y_local = rows_of(y, cr)
+        local = np.arange(cr.size, dtype=np.int32).reshape(cr.shape)
+        got = pre[u0:u1].cpu().numpy()
+        g, km = r.gates[toks], o["row_kmask"][u0:u1]
+
+        def job():
+            want = oracle.combine_units_f32chain(y_local, g, local,
+                                                 np.arange(u1 - u0, dtype=np.int32), km)
+            np.testing.assert_array_equal(got.view(np.uint32), want.view(np.uint32),
+                                          err_msg=f"units [{u0}, {u1})")
+        return job
+
+    for_chunks(D, 1024, prepare)
 
 
 # ----------------------------------------------------------------------------- combine backward
@@ -252,7 +263,10 @@ def test_combine_backward_full(coact, cfg):
 
 
 @pytest.mark.parametrize("cfg", [2, 3])
-def test_combine_backward_full_size_sampled(coact, cfg):
+def test_combine_backward_full_size_complete(coact, cfg):
+    """Configs 2 and 3 at full size: every grad_y row bit for bit and every gate gradient
+    within its bound, in chunks of tokens (each chunk's y rows and grad_y rows are the
+    ones the oracle's comb_row names)."""
     r = workload.make_routing(cfg)
     H, nk = r.cfg.H, r.N * r.k
     plan, _ = run_plan(coact, r)
@@ -263,15 +277,22 @@ def test_combine_backward_full_size_sampled(coact, cfg):
     gg = torch.empty((r.N, r.k), dtype=torch.float32, device=DEV)
     coact.combine_scatter_backward(y, cuda(r.gates), plan.comb_row, g_out, gy, gg)
     torch.cuda.synchronize()
-    del y
-    toks = sample_tokens(r.N, 40 + cfg)
-    cr = o["comb_row"][toks]
-    used = np.unique(cr)
-    y_local = host_bits(workload.fill_bf16(len(used), H, r.seed, Y_STREAM, row_ids=used))
-    go_local = host_bits(g_out[torch.as_tensor(toks, device=DEV)])
-    local = np.searchsorted(used, cr).astype(np.int32)
-    check_combine_backward(gy, gg, y_local, r.gates[toks], local, go_local, gy_rows=used,
-                           gg_tokens=toks)
+    gg_h = gg.cpu().numpy().astype(np.float64)
+
+    def prepare(t0, t1):
+        cr = o["comb_row"][t0:t1]
+        y_local, gy_got = rows_of(y, cr), rows_of(gy, cr)
+        go_local = host_bits(g_out[t0:t1])
+        local = np.arange(cr.size, dtype=np.int32).reshape(cr.shape)
+        g = r.gates[t0:t1]
+
+        def job():
+            gy_o, gg_o, ga_o = oracle.combine_backward(y_local, g, local, go_local)
+            np.testing.assert_array_equal(gy_got, gy_o, err_msg=f"grad_y, tokens [{t0}, {t1})")
+            assert (np.abs(gg_h[t0:t1] - gg_o) <= grad_gates_bound(H, ga_o)).all(), (t0, t1)
+        return job
+
+    for_chunks(r.N, 512, prepare)
 
 
 @pytest.mark.parametrize("cfg", [0, 1, 2])

@@ -10,7 +10,8 @@ import torch
 
 import oracle
 import workload
-from _gpu_util import DEV, assert_plan_equal, cuda, host_bits, plan_to_host
+from _gpu_util import (DEV, assert_plan_equal, cuda, for_chunks, host_bits, plan_to_host,
+                       rows_of)
 
 pytestmark = pytest.mark.gpu
 
@@ -45,9 +46,10 @@ def check_rows(out, parts_bits, row_token_local, rows=None):
         assert np.array_equal(host_bits(got), oracle.bf16_rne(chain))
 
 
-def test_config4_full_size_sampled(coact):
+def test_config4_full_size(coact):
     """Config 4 (N = 65536, H = 4096, R = 16): homes predicted by the library from the
-    calibration counts, the shuffle plan, and the reduce-scatter over 16 partials."""
+    calibration counts, the shuffle plan, and the reduce-scatter over 16 partials, every
+    row checked."""
     tl = workload.make_two_layer(workload.CONFIGS[4])
     c = tl.layer1.cfg
     N, H, R, E = c.N, c.H, c.R, c.E
@@ -77,12 +79,18 @@ def test_config4_full_size_sampled(coact):
     assert err.item() == 0
     for r, seg in segs:
         assert torch.equal(seg.view(torch.int16), out[int(offs[r]):int(offs[r + 1])].view(torch.int16))
-    rng = np.random.default_rng(4)
-    rows = np.unique(np.concatenate([rng.integers(0, N, 200), [0, N - 1]]))
-    toks = o["row_token"][rows]
-    pb = np.stack([host_bits(workload.fill_bf16(len(toks), H, 0, PART_STREAM + q, row_ids=toks))
-                   for q in range(R)])
-    check_rows(out, pb, np.arange(len(toks), dtype=np.int32), rows=rows)
+    # every shuffled row: the 16 partials' rows of the oracle's token order, in chunks
+    def prepare(i0, i1):
+        toks = o["row_token"][i0:i1]
+        pb = np.stack([rows_of(p, toks) for p in parts])
+        got = host_bits(out[i0:i1])
+
+        def job():
+            chain = oracle.shuffle_reduce_f32chain(pb, np.arange(i1 - i0, dtype=np.int32))
+            np.testing.assert_array_equal(got, oracle.bf16_rne(chain), err_msg=f"rows [{i0}, {i1})")
+        return job
+
+    for_chunks(N, 1024, prepare, workers=4)
 
 
 @pytest.mark.parametrize("P,H", [(1, 8), (3, 1000), (16, 256), (64, 64), (5, 2056)])
