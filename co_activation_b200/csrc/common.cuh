@@ -220,6 +220,7 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
 }
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 // NVTX range around each C-ABI call, for timeline profilers (builds with -DCOACT_NVTX; the
 // NVTX v3 headers are header-only and cost nothing when no tool is attached).

@@ -7,11 +7,17 @@
 //
 // Each x row is read from HBM once and written to every distinct destination row, so
 // the algorithmic traffic is (N + D) * H * 2 bytes (+ N*k*4 for send_row).
-//  * k_gather_v16 (default) -- one warp per token, 16-byte vector loads of the x row
-//    into registers (up to 8 per lane in flight) and streaming 16-byte stores to each
-//    destination; a grid of 8 CTAs of 8 warps per SM (4 resident at 60 registers: the
-//    extra waves balance the tail better than one resident wave, measured).  Before its
-//    wait on the predecessor, each warp warms L2 with the x rows it will copy first
+//  * k_gather_v16 (default) -- one warp per token: vector loads of the x row into
+//    registers, then streaming stores of them to each destination row.  Chunks are 32
+//    bytes (one 256-bit access per lane) when the rows and both buffers are 32-byte
+//    aligned, else 16 bytes; 2 (resp. 4) chunks per lane in flight on long rows.  The
+//    kernel is specialised per k: a token's k destination rows are resolved once with k
+//    shuffles and the store loop is unrolled and warp-uniform (no per-chunk shuffle or
+//    data-dependent loop, which kept the MIO queue full).  A grid of 16 CTAs of 8 warps
+//    per SM (3-6 resident): the extra waves balance the tail of tokens with different
+//    fan-outs.  Measured on B200, config 3's gather in the step: 1,677 us with the
+//    earlier 16-byte kernel (one kernel for all k, 8 CTAs per SM) -> 1,591 us.  Before
+//    its wait on the predecessor, each warp warms L2 with the x rows it will copy first
 //    (bulk L2 prefetch): behind the latency-bound plan, whose last kernel lets this one
 //    launch at once, HBM streams x while the plan finishes.
 //  * k_gather_bulk (entry point dispatch_gather_tma) -- TMA bulk copies.  One warp per
@@ -24,6 +30,7 @@
 // All mbarrier waits are bounded by a wall-clock limit; on expiry the kernel raises
 // COACT_EFLAG_TIMEOUT, drains its own copies and returns.
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -32,52 +39,96 @@ namespace {
 
 // ------------------------------------------------------------------ vector path
 
-// n_prefetch: tokens [0, n_prefetch) have their x rows warmed into L2 before the wait on
-// the predecessor (each warp its own tokens, in the order it copies them), so that
-// while a latency-bound predecessor (the plan) runs, HBM already streams x.
-template <int UNROLL>
+// Row chunks of 16 bytes (uint4) or 32 bytes (Row32: one 256-bit access per lane, half the
+// memory instructions of the 16-byte path; used when rows and buffers are 32-byte aligned).
+struct alignas(32) Row32 {
+    uint32_t w[8];
+};
+
+template <typename V>
+__device__ __forceinline__ V ld_chunk(const V *p);
+template <>
+__device__ __forceinline__ uint4 ld_chunk<uint4>(const uint4 *p) {
+    return ld_stream(p);
+}
+template <>
+__device__ __forceinline__ Row32 ld_chunk<Row32>(const Row32 *p) {
+    Row32 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]),
+                   "=r"(v.w[5]), "=r"(v.w[6]), "=r"(v.w[7])
+                 : "l"(p));
+    return v;
+}
+__device__ __forceinline__ void st_chunk(uint4 *p, const uint4 &v) { st_stream(p, v); }
+__device__ __forceinline__ void st_chunk(Row32 *p, const Row32 &v) {
+    asm volatile("st.global.cs.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v.w[0]),
+                 "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]), "r"(v.w[6]),
+                 "r"(v.w[7])
+                 : "memory");
+}
+
+// One warp per token; Hv chunks of type V per row.  K > 0: the token's K destination
+// rows are resolved once (K shuffles) and the store loop is unrolled and warp-uniform;
+// K == 0: k destinations at run time, walked with a ballot mask.  n_prefetch: tokens
+// [0, n_prefetch) have their x rows warmed into L2 before the wait on the predecessor
+// (each warp its own tokens, in the order it copies them), so that while a
+// latency-bound predecessor (the plan) runs, HBM already streams x.
+template <int K, typename V, int UNROLL>
 __global__ void __launch_bounds__(256)
-    k_gather_v16(const uint4 *__restrict__ x, int64_t N, int64_t H16,
-                 const int32_t *__restrict__ send_row, int k, uint4 *__restrict__ send,
-                 int64_t cap, int64_t n_prefetch, int32_t *__restrict__ err) {
+    k_gather_v16(const V *__restrict__ x, int64_t N, int64_t Hv,
+                 const int32_t *__restrict__ send_row, int k, V *__restrict__ send, int64_t cap,
+                 int64_t n_prefetch, int32_t *__restrict__ err) {
     const int lane = threadIdx.x & 31;
     const int64_t gwarp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     if (lane == 0)
         for (int64_t t = gwarp; t < n_prefetch; t += nwarps)
-            prefetch_l2_bulk(x + t * H16, (uint32_t)(H16 * 16));
+            prefetch_l2_bulk(x + t * Hv, (uint32_t)(Hv * sizeof(V)));
     pdl_wait();
     pdl_trigger();
+    const int kk = K > 0 ? K : k;
     int flags = 0;
     for (int64_t t = gwarp; t < N; t += nwarps) {
-        // destinations: lane j < k reads send_row[t, j]; broadcast by shuffles below
+        // destinations: lane j < k reads send_row[t, j]
         int dl = -1;
-        if (lane < k) {
-            dl = __ldg(send_row + t * k + lane);
+        if (lane < kk) {
+            dl = __ldg(send_row + t * kk + lane);
             if (dl >= 0 && (int64_t)dl >= cap) {
                 flags |= COACT_EFLAG_ROW_RANGE;
                 dl = -1;
             }
         }
+        int d[K > 0 ? K : 1];
+        if (K > 0) {
+#pragma unroll
+            for (int j = 0; j < (K > 0 ? K : 1); ++j) d[j] = __shfl_sync(0xffffffffu, dl, j);
+        }
         const unsigned dmask = __ballot_sync(0xffffffffu, dl >= 0);
-        const uint4 *src = x + t * H16;
-        for (int64_t c0 = 0; c0 < H16; c0 += 32 * UNROLL) {
-            uint4 v[UNROLL];
+        const V *src = x + t * Hv + lane;
+        for (int64_t c0 = 0; c0 < Hv; c0 += 32 * UNROLL) {
+            V v[UNROLL];
 #pragma unroll
-            for (int u = 0; u < UNROLL; ++u) {
-                const int64_t c = c0 + u * 32 + lane;
-                if (c < H16) v[u] = ld_stream(src + c);
-            }
-            unsigned m = dmask;
-            while (m) {
-                const int j = __ffs(m) - 1;
-                m &= m - 1;
-                const int d = __shfl_sync(0xffffffffu, dl, j);
-                uint4 *dst = send + (int64_t)d * H16;
+            for (int u = 0; u < UNROLL; ++u)
+                if (c0 + u * 32 + lane < Hv) v[u] = ld_chunk<V>(src + c0 + u * 32);
+            if (K > 0) {
 #pragma unroll
-                for (int u = 0; u < UNROLL; ++u) {
-                    const int64_t c = c0 + u * 32 + lane;
-                    if (c < H16) st_stream(dst + c, v[u]);
+                for (int j = 0; j < (K > 0 ? K : 1); ++j) {
+                    if (d[j] < 0) continue;
+                    V *dst = send + (int64_t)d[j] * Hv + lane + c0;
+#pragma unroll
+                    for (int u = 0; u < UNROLL; ++u)
+                        if (c0 + u * 32 + lane < Hv) st_chunk(dst + u * 32, v[u]);
+                }
+            } else {
+                unsigned m = dmask;
+                while (m) {
+                    const int j = __ffs(m) - 1;
+                    m &= m - 1;
+                    V *dst = send + (int64_t)__shfl_sync(0xffffffffu, dl, j) * Hv + lane + c0;
+#pragma unroll
+                    for (int u = 0; u < UNROLL; ++u)
+                        if (c0 + u * 32 + lane < Hv) st_chunk(dst + u * 32, v[u]);
                 }
             }
         }
@@ -278,14 +329,17 @@ int launch_bulk(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row
 
 int launch_v16(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row, int k,
                uint16_t *send, int64_t cap, int32_t *err, cudaStream_t st, const DeviceInfo &di) {
-    const int64_t H16 = H / 8;
 #ifndef COACT_GATHER_PER_SM
-#define COACT_GATHER_PER_SM 8  // CTAs per SM in the grid (0: one resident wave)
+#define COACT_GATHER_PER_SM 16  // CTAs per SM in the grid (0: one resident wave)
 #endif
-    const uint4 *xv = reinterpret_cast<const uint4 *>(x);
-    uint4 *sv = reinterpret_cast<uint4 *>(send);
 #ifndef COACT_GATHER_UNROLL
-#define COACT_GATHER_UNROLL 8  // 16-byte loads in flight per lane on long rows
+#define COACT_GATHER_UNROLL 4  // chunk loads in flight per lane on long rows
+#endif
+#ifndef COACT_GATHER_VEC
+#define COACT_GATHER_VEC 32  // widest chunk: 32 (256-bit accesses where aligned) or 16
+#endif
+#ifndef COACT_GATHER_KT
+#define COACT_GATHER_KT 1  // 1: kernels specialised per k (unrolled destinations); 0: one kernel
 #endif
 #ifndef COACT_GATHER_PREFETCH_BYTES
 // x bytes warmed into L2 before the wait.  Measured on B200 behind the plan of a
@@ -296,13 +350,41 @@ int launch_v16(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row,
     // the bulk prefetch takes a 32-bit size: rows beyond 16 MB are not prefetched
     const int64_t n_pf =
         H * 2 > (1 << 24) ? 0 : std::min<int64_t>(N, (int64_t)(COACT_GATHER_PREFETCH_BYTES) / (H * 2));
-    auto go = [&](auto kern) {
-        return launch_pdl(kern, grid_for(kern, N, COACT_GATHER_PER_SM, di), 256, 0, st, xv, N,
-                          H16, send_row, k, sv, cap, n_pf, err);
+    const bool wide = COACT_GATHER_VEC == 32 && H % 16 == 0 && aligned32(x) && aligned32(send);
+    auto go = [&](auto kern, auto *xv, auto *sv, int64_t Hv) {
+        return launch_pdl(kern, grid_for(kern, N, COACT_GATHER_PER_SM, di), 256, 0, st, xv, N, Hv,
+                          send_row, k, sv, cap, n_pf, err);
     };
-    if (H16 <= 32) return go(k_gather_v16<1>);
-    if (H16 <= 128) return go(k_gather_v16<4>);
-    return go(k_gather_v16<COACT_GATHER_UNROLL>);
+    auto with_k = [&](auto k_tag) {
+        constexpr int KK = decltype(k_tag)::value;
+        if (wide) {
+            const Row32 *xv = reinterpret_cast<const Row32 *>(x);
+            Row32 *sv = reinterpret_cast<Row32 *>(send);
+            const int64_t Hv = H / 16;
+            if (Hv <= 32) return go(k_gather_v16<KK, Row32, 1>, xv, sv, Hv);
+            return go(k_gather_v16<KK, Row32, (COACT_GATHER_UNROLL + 1) / 2>, xv, sv, Hv);
+        }
+        const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+        uint4 *sv = reinterpret_cast<uint4 *>(send);
+        const int64_t Hv = H / 8;
+        if (Hv <= 32) return go(k_gather_v16<KK, uint4, 1>, xv, sv, Hv);
+        return go(k_gather_v16<KK, uint4, COACT_GATHER_UNROLL>, xv, sv, Hv);
+    };
+#if COACT_GATHER_KT
+    switch (k) {
+        case 1: return with_k(std::integral_constant<int, 1>{});
+        case 2: return with_k(std::integral_constant<int, 2>{});
+        case 3: return with_k(std::integral_constant<int, 3>{});
+        case 4: return with_k(std::integral_constant<int, 4>{});
+        case 5: return with_k(std::integral_constant<int, 5>{});
+        case 6: return with_k(std::integral_constant<int, 6>{});
+        case 7: return with_k(std::integral_constant<int, 7>{});
+        case 8: return with_k(std::integral_constant<int, 8>{});
+    }
+    return COACT_ERR_UNSUPPORTED;
+#else
+    return with_k(std::integral_constant<int, 0>{});
+#endif
 }
 
 }  // namespace
