@@ -17,10 +17,14 @@
 //    (-1 = no row) and unit weights, grad_x[t] = sum of grad_send over the token's send
 //    rows.  fmaf(1, v, acc) rounds exactly like acc + v, so this is the fp32 add chain.
 //
-// k_combine_v16: one warp per token.  Each lane covers 8 hidden elements per 16-byte
-// column chunk and keeps U chunks x K rows of loads in flight before the FMAs.  The K
+// k_combine_v16: one warp per token.  Each lane covers 16 hidden elements per 32-byte
+// column chunk (one 256-bit access; 8 elements per 16-byte chunk where y or out is not
+// 32-byte aligned) and keeps U chunks x K rows of loads in flight before the FMAs.  The K
 // source rows are scattered over y (expanded receive order), the output row is written
 // once with streaming stores.  HBM traffic: N*k*H*2 (y) + N*H*(2|4) (out) + N*k*8.
+// Measured on B200 in the config-3 step (k = 8, 14 KB rows): 2,689 us with 16-byte
+// chunks, 2,418 us with 32-byte chunks -- 7.0 TB/s, above the measured copy bandwidth
+// because the combine's traffic is 89% reads.
 #include <algorithm>
 
 #include <cuda_bf16.h>
@@ -30,12 +34,15 @@
 namespace coact {
 namespace {
 
-// Unit u = token u with all K slots.  gates == nullptr: every weight is 1.
-template <int K, int U, bool F32>
+// Unit u = token u with all K slots.  gates == nullptr: every weight is 1.  Chunks of
+// type V: 16 bytes (uint4, 8 elements) or 32 bytes (Row32, 16 elements per lane, one
+// 256-bit access) when y's rows and out are 32-byte aligned.
+template <int K, int U, bool F32, typename V>
 __global__ void __launch_bounds__(256)
-    k_combine_v16(const uint4 *__restrict__ y, int64_t n_rows, const float *__restrict__ gates,
-                  const int32_t *__restrict__ comb_row, int64_t N, int64_t H16,
+    k_combine_v16(const V *__restrict__ y, int64_t n_rows, const float *__restrict__ gates,
+                  const int32_t *__restrict__ comb_row, int64_t N, int64_t Hv,
                   void *__restrict__ out, int32_t *__restrict__ err) {
+    constexpr int W = sizeof(V) / 4;   // 32-bit words (bf16 pairs) per chunk
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
@@ -59,45 +66,50 @@ __global__ void __launch_bounds__(256)
             row[j] = __shfl_sync(0xffffffffu, rl, j);
             g[j] = __shfl_sync(0xffffffffu, gl, j);
         }
-        for (int64_t c0 = 0; c0 < H16; c0 += 32 * U) {
-            uint4 v[U][K];
+        for (int64_t c0 = 0; c0 < Hv; c0 += 32 * U) {
+            V v[U][K];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int64_t c = c0 + u * 32 + lane;
 #pragma unroll
                 for (int j = 0; j < K; ++j)
-                    if (c < H16 && row[j] >= 0) v[u][j] = ld_stream(y + row[j] * H16 + c);
+                    if (c < Hv && row[j] >= 0) v[u][j] = ld_chunk<V>(y + row[j] * Hv + c);
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int64_t c = c0 + u * 32 + lane;
-                if (c >= H16) continue;
-                float acc[8];
+                if (c >= Hv) continue;
+                float acc[2 * W];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+                for (int e = 0; e < 2 * W; ++e) acc[e] = 0.0f;
 #pragma unroll
                 for (int j = 0; j < K; ++j) {
                     if (row[j] < 0) continue;
-                    const uint32_t w[4] = {v[u][j].x, v[u][j].y, v[u][j].z, v[u][j].w};
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        acc[2 * q] = __fmaf_rn(g[j], bf16lo(w[q]), acc[2 * q]);
-                        acc[2 * q + 1] = __fmaf_rn(g[j], bf16hi(w[q]), acc[2 * q + 1]);
+                    for (int q = 0; q < W; ++q) {
+                        const uint32_t w = chunk_word(v[u][j], q);
+                        acc[2 * q] = __fmaf_rn(g[j], bf16lo(w), acc[2 * q]);
+                        acc[2 * q + 1] = __fmaf_rn(g[j], bf16hi(w), acc[2 * q + 1]);
                     }
                 }
-                if (F32) {
-                    float4 *o = reinterpret_cast<float4 *>(out) + (t * H16 + c) * 2;
-                    __stcs(o, make_float4(acc[0], acc[1], acc[2], acc[3]));
-                    __stcs(o + 1, make_float4(acc[4], acc[5], acc[6], acc[7]));
-                } else {
-                    uint4 p;
-                    uint32_t *pw = &p.x;
+                if (F32) {               // 2W floats: two chunks of V
+                    V p0, p1;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
-                        pw[q] = *reinterpret_cast<const uint32_t *>(&h2);
+                    for (int q = 0; q < W; ++q) {
+                        set_chunk_word(p0, q, __float_as_uint(acc[q]));
+                        set_chunk_word(p1, q, __float_as_uint(acc[W + q]));
                     }
-                    st_stream(reinterpret_cast<uint4 *>(out) + t * H16 + c, p);
+                    V *o = reinterpret_cast<V *>(out) + (t * Hv + c) * 2;
+                    st_chunk(o, p0);
+                    st_chunk(o + 1, p1);
+                } else {
+                    V p;
+#pragma unroll
+                    for (int q = 0; q < W; ++q) {
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+                        set_chunk_word(p, q, *reinterpret_cast<const uint32_t *>(&h2));
+                    }
+                    st_chunk(reinterpret_cast<V *>(out) + t * Hv + c, p);
                 }
             }
         }
@@ -233,7 +245,10 @@ int launch(const uint16_t *y, int64_t n_rows, const float *gates, const int32_t 
 #ifndef COACT_COMBINE_PER_SM
 #define COACT_COMBINE_PER_SM 8  // CTAs per SM in the grid (0: one resident wave)
 #endif
-    const int blocks = grid_for(k_combine_v16<K, U, F32>, n_units, COACT_COMBINE_PER_SM, di);
+#ifndef COACT_COMBINE_VEC
+#define COACT_COMBINE_VEC 32  // 256-bit chunks where y and out are 32-byte aligned (16: never)
+#endif
+    const int blocks = grid_for(k_combine_v16<K, U, F32, uint4>, n_units, COACT_COMBINE_PER_SM, di);
     if (UNITS)
         return launch_pdl(k_combine_units<K, 4, 2, F32, true>, blocks, 256, 0, st,
                           reinterpret_cast<const uint4 *>(y), n_rows, gates, comb_row, N, row_token,
@@ -242,7 +257,21 @@ int launch(const uint16_t *y, int64_t n_rows, const float *gates, const int32_t 
         return launch_pdl(k_combine_units<K, 4, 2, F32, false>, blocks, 256, 0, st,
                           reinterpret_cast<const uint4 *>(y), n_rows, gates, comb_row, N, nullptr,
                           nullptr, n_units, nullptr, H16, out, err);
-    return launch_pdl(k_combine_v16<K, U, F32>, blocks, 256, 0, st,
+    if (COACT_COMBINE_VEC == 32 && H % 16 == 0 && aligned32(y) && aligned32(out)) {
+#if defined(COACT_COMBINE_LOADS)
+        constexpr int UW = (U + 1) / 2;    // the same bytes in flight in 32-byte chunks
+#else
+        // 32-byte chunks per lane: two for k <= 2 and k >= 7, one for k = 3..6.  Measured on
+        // B200 in the step: k = 8 (config 3) two chunks 2,418 us vs one 2,464 us; k = 2
+        // (config 1) two chunks 38.0 us vs eight 51.0 us; k = 6 (config 2) one and three equal.
+        constexpr int UW = (K <= 2 || K >= 7) ? 2 : 1;
+#endif
+        return launch_pdl(k_combine_v16<K, UW, F32, Row32>,
+                          grid_for(k_combine_v16<K, UW, F32, Row32>, n_units, COACT_COMBINE_PER_SM, di),
+                          256, 0, st, reinterpret_cast<const Row32 *>(y), n_rows, gates, comb_row,
+                          N, H / 16, out, err);
+    }
+    return launch_pdl(k_combine_v16<K, U, F32, uint4>, blocks, 256, 0, st,
                       reinterpret_cast<const uint4 *>(y), n_rows, gates, comb_row, N, H16, out, err);
 }
 

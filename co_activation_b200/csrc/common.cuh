@@ -49,6 +49,49 @@ __device__ __forceinline__ void st_stream(uint4 *p, const uint4 &v) {
                  : "memory");
 }
 
+// Row chunks of 16 bytes (uint4) or 32 bytes (Row32: one 256-bit access per lane, half the
+// memory instructions of 16-byte chunks; only for rows and buffers that are 32-byte
+// aligned, which the host checks before choosing it).
+struct alignas(32) Row32 {
+    uint32_t w[8];
+};
+
+template <typename V>
+__device__ __forceinline__ V ld_chunk(const V *p);
+template <>
+__device__ __forceinline__ uint4 ld_chunk<uint4>(const uint4 *p) {
+    return ld_stream(p);
+}
+template <>
+__device__ __forceinline__ Row32 ld_chunk<Row32>(const Row32 *p) {
+    Row32 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]),
+                   "=r"(v.w[5]), "=r"(v.w[6]), "=r"(v.w[7])
+                 : "l"(p));
+    return v;
+}
+__device__ __forceinline__ void st_chunk(uint4 *p, const uint4 &v) { st_stream(p, v); }
+__device__ __forceinline__ void st_chunk(Row32 *p, const Row32 &v) {
+    asm volatile("st.global.cs.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v.w[0]),
+                 "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]), "r"(v.w[6]),
+                 "r"(v.w[7])
+                 : "memory");
+}
+
+// 32-bit word q of a chunk (q a compile-time constant after unrolling)
+__device__ __forceinline__ uint32_t chunk_word(const uint4 &v, int q) {
+    return q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
+}
+__device__ __forceinline__ uint32_t chunk_word(const Row32 &v, int q) { return v.w[q]; }
+__device__ __forceinline__ void set_chunk_word(uint4 &v, int q, uint32_t x) {
+    if (q == 0) v.x = x;
+    else if (q == 1) v.y = x;
+    else if (q == 2) v.z = x;
+    else v.w = x;
+}
+__device__ __forceinline__ void set_chunk_word(Row32 &v, int q, uint32_t x) { v.w[q] = x; }
+
 // Asks the copy engine of the SM (TMA) to bring [p, p + bytes) of this GPU's memory into
 // L2; p 16-byte aligned, bytes a multiple of 16.  A hint with no completion: nothing is
 // returned, no mbarrier is involved and nothing needs waiting for.  L2 is where every

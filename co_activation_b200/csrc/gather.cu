@@ -39,35 +39,6 @@ namespace {
 
 // ------------------------------------------------------------------ vector path
 
-// Row chunks of 16 bytes (uint4) or 32 bytes (Row32: one 256-bit access per lane, half the
-// memory instructions of the 16-byte path; used when rows and buffers are 32-byte aligned).
-struct alignas(32) Row32 {
-    uint32_t w[8];
-};
-
-template <typename V>
-__device__ __forceinline__ V ld_chunk(const V *p);
-template <>
-__device__ __forceinline__ uint4 ld_chunk<uint4>(const uint4 *p) {
-    return ld_stream(p);
-}
-template <>
-__device__ __forceinline__ Row32 ld_chunk<Row32>(const Row32 *p) {
-    Row32 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]),
-                   "=r"(v.w[5]), "=r"(v.w[6]), "=r"(v.w[7])
-                 : "l"(p));
-    return v;
-}
-__device__ __forceinline__ void st_chunk(uint4 *p, const uint4 &v) { st_stream(p, v); }
-__device__ __forceinline__ void st_chunk(Row32 *p, const Row32 &v) {
-    asm volatile("st.global.cs.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v.w[0]),
-                 "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]), "r"(v.w[6]),
-                 "r"(v.w[7])
-                 : "memory");
-}
-
 // One warp per token; Hv chunks of type V per row.  K > 0: the token's K destination
 // rows are resolved once (K shuffles) and the store loop is unrolled and warp-uniform;
 // K == 0: k destinations at run time, walked with a ballot mask.  n_prefetch: tokens
