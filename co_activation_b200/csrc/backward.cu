@@ -11,12 +11,13 @@
 // without row_token, unit u is token u with all k slots.
 //
 // k_combine_bwd: one warp per unit.  The unit's live slots (with a row) are compacted in
-// ascending slot order by a warp ballot.  Each lane owns 8 hidden elements per 16-byte
-// column chunk; per group of U chunks it loads grad_out once, then streams the live rows
-// of y G at a time, writing their scaled grad_y rows and accumulating one dot product per
-// slot (fp32 fma, a lane's elements in ascending order), reduced across the warp by a
-// butterfly at the end.  Summation order of a dot product: each lane's chain of
-// 8 * ceil(H/256) terms, then 5 butterfly levels.
+// ascending slot order by a warp ballot.  Each lane owns 16 hidden elements per 32-byte
+// column chunk (8 per 16-byte chunk where y, grad_out or grad_y is not 32-byte aligned);
+// per group of U chunks it loads grad_out once, then streams the live rows of y G at a
+// time, writing their scaled grad_y rows and accumulating one dot product per slot (fp32
+// fma, a lane's elements in ascending order), reduced across the warp by a butterfly at
+// the end.  Summation order of a dot product: each lane's chain of 16 * ceil(H/512)
+// terms (8 * ceil(H/256) with 16-byte chunks), then 5 butterfly levels.
 // HBM traffic: N*H*2 (grad_out) + N*k*H*2 (y) + N*k*H*2 (grad_y) + N*k*12.
 #include <algorithm>
 
@@ -27,14 +28,15 @@
 namespace coact {
 namespace {
 
-template <int K, int U, int G, bool UNITS>
+template <int K, int U, int G, bool UNITS, typename V>
 __global__ void __launch_bounds__(256)
-    k_combine_bwd(const uint4 *__restrict__ y, int64_t n_rows, const float *__restrict__ gates,
+    k_combine_bwd(const V *__restrict__ y, int64_t n_rows, const float *__restrict__ gates,
                   const int32_t *__restrict__ comb_row, int64_t N,
                   const int32_t *__restrict__ row_token, const uint8_t *__restrict__ row_kmask,
                   int64_t n_units, const int32_t *__restrict__ unit_count,
-                  const uint4 *__restrict__ g_out, int64_t H16, uint4 *__restrict__ g_y,
+                  const V *__restrict__ g_out, int64_t Hv, V *__restrict__ g_y,
                   float *__restrict__ g_gates, int32_t *__restrict__ err) {
+    constexpr int W = sizeof(V) / 4;   // 32-bit words (bf16 pairs) per chunk
     pdl_wait();
     pdl_trigger();
     if (UNITS && unit_count) n_units = min(n_units, (int64_t)max(__ldg(unit_count), 0));
@@ -79,48 +81,46 @@ __global__ void __launch_bounds__(256)
             dot[i] = 0.0f;
             live &= live - 1;
         }
-        const uint4 *go_row = g_out + u * H16;
-        for (int64_t c0 = 0; c0 < H16; c0 += 32 * U) {
-            uint4 vg[U];
+        const V *go_row = g_out + u * Hv;
+        for (int64_t c0 = 0; c0 < Hv; c0 += 32 * U) {
+            V vg[U];
 #pragma unroll
             for (int q = 0; q < U; ++q) {
                 const int64_t c = c0 + q * 32 + lane;
-                if (c < H16) vg[q] = ld_stream(go_row + c);
+                if (c < Hv) vg[q] = ld_chunk<V>(go_row + c);
             }
 #pragma unroll
             for (int i0 = 0; i0 < K; i0 += G) {
                 if (i0 >= m) break;
-                uint4 vy[U][G];
+                V vy[U][G];
 #pragma unroll
                 for (int q = 0; q < U; ++q) {
                     const int64_t c = c0 + q * 32 + lane;
 #pragma unroll
                     for (int gi = 0; gi < G; ++gi)
-                        if (c < H16 && i0 + gi < K && i0 + gi < m)
-                            vy[q][gi] = ld_stream(y + row[i0 + gi] * H16 + c);
+                        if (c < Hv && i0 + gi < K && i0 + gi < m)
+                            vy[q][gi] = ld_chunk<V>(y + row[i0 + gi] * Hv + c);
                 }
 #pragma unroll
                 for (int q = 0; q < U; ++q) {
                     const int64_t c = c0 + q * 32 + lane;
-                    if (c >= H16) continue;
-                    const uint32_t wg[4] = {vg[q].x, vg[q].y, vg[q].z, vg[q].w};
+                    if (c >= Hv) continue;
 #pragma unroll
                     for (int gi = 0; gi < G; ++gi) {
                         const int i = i0 + gi;
                         if (i >= K || i >= m) continue;
-                        const uint32_t w[4] = {vy[q][gi].x, vy[q][gi].y, vy[q][gi].z, vy[q][gi].w};
-                        uint4 p;
-                        uint32_t *pw = &p.x;
+                        V p;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float g0 = bf16lo(wg[e]), g1 = bf16hi(wg[e]);
-                            dot[i] = __fmaf_rn(g0, bf16lo(w[e]), dot[i]);
-                            dot[i] = __fmaf_rn(g1, bf16hi(w[e]), dot[i]);
+                        for (int e = 0; e < W; ++e) {
+                            const uint32_t wg = chunk_word(vg[q], e), w = chunk_word(vy[q][gi], e);
+                            const float g0 = bf16lo(wg), g1 = bf16hi(wg);
+                            dot[i] = __fmaf_rn(g0, bf16lo(w), dot[i]);
+                            dot[i] = __fmaf_rn(g1, bf16hi(w), dot[i]);
                             const __nv_bfloat162 h2 =
                                 __floats2bfloat162_rn(__fmul_rn(g[i], g0), __fmul_rn(g[i], g1));
-                            pw[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                            set_chunk_word(p, e, *reinterpret_cast<const uint32_t *>(&h2));
                         }
-                        st_stream(g_y + row[i] * H16 + c, p);
+                        st_chunk(g_y + row[i] * Hv + c, p);
                     }
                 }
             }
@@ -146,14 +146,20 @@ int launch(const uint16_t *y, int64_t n_rows, const float *gates, const int32_t 
            int64_t N, const int32_t *row_token, const uint8_t *row_kmask, int64_t n_units,
            const int32_t *unit_count, const uint16_t *g_out, int64_t H, uint16_t *g_y,
            float *g_gates, int32_t *err, cudaStream_t st, const DeviceInfo &di) {
-    // loads in flight per lane: U chunks of grad_out + U x G rows of y
+    // loads in flight per lane: U chunks of grad_out + U x G rows of y (16-byte chunks);
+    // one 32-byte chunk per row where y, grad_out and grad_y are 32-byte aligned
     constexpr int U = 2, G = 2;
-    const int64_t H16 = H / 8;
     const int blocks = (int)std::max<int64_t>(
         1, std::min<int64_t>(ceil_div(n_units, 8), (int64_t)di.sm_count * 8));
-    return launch_pdl(k_combine_bwd<K, U, G, UNITS>, blocks, 256, 0, st,
+    if (H % 16 == 0 && aligned32(y) && aligned32(g_out) && aligned32(g_y))
+        return launch_pdl(k_combine_bwd<K, 1, G, UNITS, Row32>, blocks, 256, 0, st,
+                          reinterpret_cast<const Row32 *>(y), n_rows, gates, comb_row, N,
+                          row_token, row_kmask, n_units, unit_count,
+                          reinterpret_cast<const Row32 *>(g_out), H / 16,
+                          reinterpret_cast<Row32 *>(g_y), g_gates, err);
+    return launch_pdl(k_combine_bwd<K, U, G, UNITS, uint4>, blocks, 256, 0, st,
                       reinterpret_cast<const uint4 *>(y), n_rows, gates, comb_row, N, row_token,
-                      row_kmask, n_units, unit_count, reinterpret_cast<const uint4 *>(g_out), H16,
+                      row_kmask, n_units, unit_count, reinterpret_cast<const uint4 *>(g_out), H / 8,
                       reinterpret_cast<uint4 *>(g_y), g_gates, err);
 }
 

@@ -124,13 +124,14 @@ __global__ void __launch_bounds__(256)
 // G rows at a time, U column chunks per lane (U*G loads in flight), accumulating in that
 // order: the same fma chain as k_combine_v16, without registers and issue slots for
 // absent slots.
-template <int K, int U, int G, bool F32, bool UNITS>
+template <int K, int U, int G, bool F32, bool UNITS, typename V>
 __global__ void __launch_bounds__(256)
-    k_combine_units(const uint4 *__restrict__ y, int64_t n_rows, const float *__restrict__ gates,
+    k_combine_units(const V *__restrict__ y, int64_t n_rows, const float *__restrict__ gates,
                     const int32_t *__restrict__ comb_row, int64_t N,
                     const int32_t *__restrict__ row_token, const uint8_t *__restrict__ row_kmask,
-                    int64_t n_units, const int32_t *__restrict__ unit_count, int64_t H16,
+                    int64_t n_units, const int32_t *__restrict__ unit_count, int64_t Hv,
                     void *__restrict__ out, int32_t *__restrict__ err) {
+    constexpr int W = sizeof(V) / 4;   // 32-bit words (bf16 pairs) per chunk
     pdl_wait();
     pdl_trigger();
     if (UNITS && unit_count) n_units = min(n_units, (int64_t)max(__ldg(unit_count), 0));
@@ -170,23 +171,23 @@ __global__ void __launch_bounds__(256)
             g[i] = __shfl_sync(0xffffffffu, gl, l);
             live &= live - 1;
         }
-        for (int64_t c0 = 0; c0 < H16; c0 += 32 * U) {
-            float acc[U][8];
+        for (int64_t c0 = 0; c0 < Hv; c0 += 32 * U) {
+            float acc[U][2 * W];
 #pragma unroll
             for (int q = 0; q < U; ++q)
 #pragma unroll
-                for (int e = 0; e < 8; ++e) acc[q][e] = 0.0f;
+                for (int e = 0; e < 2 * W; ++e) acc[q][e] = 0.0f;
 #pragma unroll
             for (int i0 = 0; i0 < K; i0 += G) {
                 if (i0 >= m) break;
-                uint4 v[U][G];
+                V v[U][G];
 #pragma unroll
                 for (int q = 0; q < U; ++q) {
                     const int64_t c = c0 + q * 32 + lane;
 #pragma unroll
                     for (int gi = 0; gi < G; ++gi)
-                        if (c < H16 && i0 + gi < K && i0 + gi < m)
-                            v[q][gi] = ld_stream(y + row[i0 + gi] * H16 + c);
+                        if (c < Hv && i0 + gi < K && i0 + gi < m)
+                            v[q][gi] = ld_chunk<V>(y + row[i0 + gi] * Hv + c);
                 }
 #pragma unroll
                 for (int q = 0; q < U; ++q) {
@@ -194,11 +195,11 @@ __global__ void __launch_bounds__(256)
                     for (int gi = 0; gi < G; ++gi) {
                         if (i0 + gi >= K || i0 + gi >= m) continue;
                         const float gg = g[i0 + gi];
-                        const uint32_t w[4] = {v[q][gi].x, v[q][gi].y, v[q][gi].z, v[q][gi].w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            acc[q][2 * e] = __fmaf_rn(gg, bf16lo(w[e]), acc[q][2 * e]);
-                            acc[q][2 * e + 1] = __fmaf_rn(gg, bf16hi(w[e]), acc[q][2 * e + 1]);
+                        for (int e = 0; e < W; ++e) {
+                            const uint32_t w = chunk_word(v[q][gi], e);
+                            acc[q][2 * e] = __fmaf_rn(gg, bf16lo(w), acc[q][2 * e]);
+                            acc[q][2 * e + 1] = __fmaf_rn(gg, bf16hi(w), acc[q][2 * e + 1]);
                         }
                     }
                 }
@@ -206,21 +207,26 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
             for (int q = 0; q < U; ++q) {
                 const int64_t c = c0 + q * 32 + lane;
-                if (c >= H16) continue;
-                if (F32) {
-                    float4 *o = reinterpret_cast<float4 *>(out) + (u * H16 + c) * 2;
-                    __stcs(o, make_float4(acc[q][0], acc[q][1], acc[q][2], acc[q][3]));
-                    __stcs(o + 1, make_float4(acc[q][4], acc[q][5], acc[q][6], acc[q][7]));
-                } else {
-                    uint4 p;
-                    uint32_t *pw = &p.x;
+                if (c >= Hv) continue;
+                if (F32) {               // 2W floats: two chunks of V
+                    V p0, p1;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
+                    for (int e = 0; e < W; ++e) {
+                        set_chunk_word(p0, e, __float_as_uint(acc[q][e]));
+                        set_chunk_word(p1, e, __float_as_uint(acc[q][W + e]));
+                    }
+                    V *o = reinterpret_cast<V *>(out) + (u * Hv + c) * 2;
+                    st_chunk(o, p0);
+                    st_chunk(o + 1, p1);
+                } else {
+                    V p;
+#pragma unroll
+                    for (int e = 0; e < W; ++e) {
                         const __nv_bfloat162 h2 =
                             __floats2bfloat162_rn(acc[q][2 * e], acc[q][2 * e + 1]);
-                        pw[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                        set_chunk_word(p, e, *reinterpret_cast<const uint32_t *>(&h2));
                     }
-                    st_stream(reinterpret_cast<uint4 *>(out) + u * H16 + c, p);
+                    st_chunk(reinterpret_cast<V *>(out) + u * Hv + c, p);
                 }
             }
         }
@@ -249,15 +255,23 @@ int launch(const uint16_t *y, int64_t n_rows, const float *gates, const int32_t 
 #define COACT_COMBINE_VEC 32  // 256-bit chunks where y and out are 32-byte aligned (16: never)
 #endif
     const int blocks = grid_for(k_combine_v16<K, U, F32, uint4>, n_units, COACT_COMBINE_PER_SM, di);
-    if (UNITS)
-        return launch_pdl(k_combine_units<K, 4, 2, F32, true>, blocks, 256, 0, st,
-                          reinterpret_cast<const uint4 *>(y), n_rows, gates, comb_row, N, row_token,
-                          row_kmask, n_units, unit_count, H16, out, err);
-    if (SPARSE && K >= 3)      // token rows with absent slots (the transposed dispatch)
-        return launch_pdl(k_combine_units<K, 4, 2, F32, false>, blocks, 256, 0, st,
-                          reinterpret_cast<const uint4 *>(y), n_rows, gates, comb_row, N, nullptr,
-                          nullptr, n_units, nullptr, H16, out, err);
-    if (COACT_COMBINE_VEC == 32 && H % 16 == 0 && aligned32(y) && aligned32(out)) {
+    const bool wide = COACT_COMBINE_VEC == 32 && H % 16 == 0 && aligned32(y) && aligned32(out);
+    if (UNITS || (SPARSE && K >= 3)) {   // sparse slots: units, or token rows with absent slots
+        const int32_t *rt = UNITS ? row_token : nullptr;
+        const uint8_t *km = UNITS ? row_kmask : nullptr;
+        const int32_t *uc = UNITS ? unit_count : nullptr;
+        // 32-byte chunks for k >= 3 (measured in the step: combine_rows 1,061 -> 1,009 us on
+        // config 2, 3,633 -> 3,533 us on config 3); k <= 2 keeps 16-byte chunks (config 1's
+        // combine_rows was not faster with 32-byte ones)
+        if (wide && K >= 3)
+            return launch_pdl(k_combine_units<K, 2, 2, F32, UNITS, Row32>, blocks, 256, 0, st,
+                              reinterpret_cast<const Row32 *>(y), n_rows, gates, comb_row, N, rt,
+                              km, n_units, uc, H / 16, out, err);
+        return launch_pdl(k_combine_units<K, 4, 2, F32, UNITS, uint4>, blocks, 256, 0, st,
+                          reinterpret_cast<const uint4 *>(y), n_rows, gates, comb_row, N, rt, km,
+                          n_units, uc, H16, out, err);
+    }
+    if (wide) {
 #if defined(COACT_COMBINE_LOADS)
         constexpr int UW = (U + 1) / 2;    // the same bytes in flight in 32-byte chunks
 #else

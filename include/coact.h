@@ -326,8 +326,9 @@ int dispatch_gather_backward(const uint16_t *grad_send, int64_t n_rows,
  * grad_out: bf16 [n_units, H] (token mode: [N, H]); grad_y: bf16 [n_rows, H], rows no
  * slot names are not written; grad_gates: fp32 [N, k], slots no unit covers are not
  * written, a covered slot without a row (comb_row -1) gets 0.  The dot product sums, per
- * lane of a warp, 8*ceil(H/256) products in ascending order with fma, then adds the 32
- * lane sums by a 5-level butterfly: its error is at most (8*ceil(H/256) + 5) * 2^-24 *
+ * lane of a warp, m products in ascending order with fma -- m = 16*ceil(H/512) when y,
+ * grad_out and grad_y are 32-byte aligned and H % 16 == 0, else 8*ceil(H/256) -- then
+ * adds the 32 lane sums by a 5-level butterfly: its error is at most (m + 5) * 2^-24 *
  * sum_h |grad_out * y| (first order).  n_units and unit_count are ignored when row_token
  * is NULL.
  */

@@ -8,7 +8,8 @@ against the CPU oracle on the same seeded inputs.
                              dispatch_gather_backward: bit-exact with the oracle's
   combine_scatter_backward   grad_y bit-exact (fp32 product rounded to bf16); grad_gates
                              within the stated bound of the float64 dot product:
-                             (8*ceil(H/256) + 5) * 2^-24 * sum_h |grad_out * y|
+                             (m + 5) * 2^-24 * sum_h |grad_out * y|, m the terms per lane
+                             (max(8*ceil(H/256), 16*ceil(H/512)))
 Full-size configurations are checked in full (every row and every gate gradient, streamed
 in chunks against the oracle), with the launch configuration the benchmark uses."""
 import math
@@ -55,7 +56,8 @@ def check_grad_x(got: torch.Tensor, g_bits: np.ndarray, send_row: np.ndarray, to
 
 
 def grad_gates_bound(H: int, mag: np.ndarray) -> np.ndarray:
-    m = 8 * math.ceil(H / 256)
+    # terms per lane: 8 * ceil(H/256) with 16-byte chunks, 16 * ceil(H/512) with 32-byte ones
+    m = max(8 * math.ceil(H / 256), 16 * math.ceil(H / 512))
     return 1.01 * (m + 5) * 2.0 ** -24 * mag + 1e-30
 
 

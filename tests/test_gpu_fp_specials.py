@@ -243,7 +243,7 @@ def test_combine_backward_special_values(coact, k, H):
                       ("-inf", lambda a: np.isneginf(a))):
         assert np.array_equal(cls(got), cls(gg_o)), f"grad_gates {name}"
     fin = np.isfinite(gg_o)
-    m = 8 * math.ceil(H / 256)
+    m = max(8 * math.ceil(H / 256), 16 * math.ceil(H / 512))
     bound = 1.01 * (m + 5) * 2.0 ** -24 * ga_o + 1e-30
     assert (np.abs(got[fin] - gg_o[fin]) <= bound[fin]).all()
     assert np.isnan(gg_o).any() and fin.sum() > N * k // 4
