@@ -1104,8 +1104,14 @@ def run_e2e(coact, S, args, world, device):
     concurrently with the SMs)."""
     cfg = S.cfg
 
+    kind = {"host": "pinned"}
+
     def pinned(t, fill: bool):
-        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        try:
+            h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        except RuntimeError:            # the host cannot pin this much: pageable buffers
+            kind["host"] = "pageable (pinning failed)"
+            h = torch.empty(t.shape, dtype=t.dtype)
         if fill:
             h.copy_(t)
         return h
@@ -1161,8 +1167,8 @@ def run_e2e(coact, S, args, world, device):
     agg = aggregate(cfg.N * K, a.elapsed_time(b_) / 1e3, world, device)
     return {"value": agg["tokens_per_s"], "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
-            "note": "pinned host buffers; input copy of step i+1 overlaps compute and output "
-                    "copy of step i (two device buffer sets)"}
+            "note": f"{kind['host']} host buffers; input copy of step i+1 overlaps compute and "
+                    "output copy of step i (two device buffer sets)"}
 
 
 # ----------------------------------------------------------------------------- the oracle
