@@ -247,3 +247,35 @@ def test_combine_backward_special_values(coact, k, H):
     bound = 1.01 * (m + 5) * 2.0 ** -24 * ga_o + 1e-30
     assert (np.abs(got[fin] - gg_o[fin]) <= bound[fin]).all()
     assert np.isnan(gg_o).any() and fin.sum() > N * k // 4
+
+
+def test_device_nan_results_are_canonical(coact):
+    """What the device emits for a NaN result, pinned: whatever the NaN's payload or sign in
+    the inputs (signalling, quiet, negative), the fused multiply-adds give the canonical
+    quiet NaN (fp32 0x7FFFFFFF) and its round to bf16 gives 0x7FFF.  The oracle keeps an
+    input's payload instead (C library semantics); the contract compares NaN as NaN."""
+    H = 64
+    nans = np.array([0x7FC0, 0xFFC0, 0x7F81, 0xFF81, 0x7FFF, 0xFFA5, 0x7FAA], np.uint16)
+    rows = np.repeat(nans.reshape(-1, 1), H, axis=1)
+    k1 = len(nans)
+    # k = 1: each token's only row is a NaN row; k = 2: a NaN row after an ordinary one, and
+    # 0 * inf (an invalid operation from non-NaN inputs)
+    ordinary = host_bits(workload.fill_bf16(k1, H, 0, 11))
+    y1 = rows
+    y2 = np.concatenate([ordinary, rows, np.full((1, H), 0x7F80, np.uint16)])
+    comb2 = np.stack([np.arange(k1), k1 + np.arange(k1)], 1).astype(np.int32)
+    comb2 = np.concatenate([comb2, [[0, 2 * k1]]]).astype(np.int32)
+    g2 = np.ones(comb2.shape, np.float32)
+    g2[-1, 1] = 0.0
+    for y, comb, g in ((y1, np.arange(k1, dtype=np.int32).reshape(-1, 1),
+                        np.full((k1, 1), 0.5, np.float32)), (y2, comb2, g2)):
+        f32 = torch.empty((comb.shape[0], H), dtype=torch.float32, device=DEV)
+        b16 = torch.empty((comb.shape[0], H), dtype=torch.bfloat16, device=DEV)
+        coact.combine_scatter(to_dev_bits(y), cuda(g), cuda(comb), f32)
+        coact.combine_scatter(to_dev_bits(y), cuda(g), cuda(comb), b16)
+        torch.cuda.synchronize()
+        got32 = f32.cpu().numpy().view(np.uint32)
+        got16 = host_bits(b16)
+        assert np.isnan(oracle.combine_f32chain(y, g, comb)).all()
+        assert (got32 == 0x7FFFFFFF).all(), sorted({hex(v) for v in got32.ravel()})
+        assert (got16 == 0x7FFF).all(), sorted({hex(v) for v in got16.ravel()})
