@@ -16,10 +16,11 @@
 //    data-dependent loop, which kept the MIO queue full).  A grid of 16 CTAs of 8 warps
 //    per SM (3-6 resident): the extra waves balance the tail of tokens with different
 //    fan-outs.  Measured on B200, config 3's gather in the step: 1,677 us with the
-//    earlier 16-byte kernel (one kernel for all k, 8 CTAs per SM) -> 1,591 us.  Before
-//    its wait on the predecessor, each warp warms L2 with the x rows it will copy first
-//    (bulk L2 prefetch): behind the latency-bound plan, whose last kernel lets this one
-//    launch at once, HBM streams x while the plan finishes.
+//    earlier 16-byte kernel (one kernel for all k, 8 CTAs per SM) -> 1,591 us.  As a build
+//    option (-DCOACT_GATHER_PREFETCH_BYTES), each warp can warm L2 with the x rows it will
+//    copy first before its wait on the predecessor (bulk L2 prefetch, behind the plan whose
+//    last kernel lets this one launch at once); measured without gain on the current
+//    kernel, it is off.
 //  * k_gather_bulk (entry point dispatch_gather_tma) -- TMA bulk copies.  One warp per
 //    CTA; lane 0 streams rows into a ring of shared-memory stages with cp.async.bulk
 //    (global -> shared, completion on an mbarrier), then lanes j < k each issue the
@@ -313,10 +314,11 @@ int launch_v16(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row,
 #define COACT_GATHER_KT 1  // 1: kernels specialised per k (unrolled destinations); 0: one kernel
 #endif
 #ifndef COACT_GATHER_PREFETCH_BYTES
-// x bytes warmed into L2 before the wait.  Measured on B200 behind the plan of a
-// 16K-token, 4 KB-row batch: 16-32 MB took ~1% off the step; 64 MB no longer did (more
-// than the plan's ~8 us of idle HBM time covers).
-#define COACT_GATHER_PREFETCH_BYTES (32ll << 20)
+// x bytes warmed into L2 before the wait (0: none).  With the earlier 16-byte gather, 16-32
+// MB took ~1% off config 1's step behind its plan; with the current kernel it gains nothing
+// (config 1: 72.1 vs 72.2 us, config 3: 4,069 vs 4,070 us per step) and on config 3 costs
+// ~7% extra DRAM reads (prefetched lines evicted by the write stream before use) -> off.
+#define COACT_GATHER_PREFETCH_BYTES 0ll
 #endif
     // the bulk prefetch takes a 32-bit size: rows beyond 16 MB are not prefetched
     const int64_t n_pf =

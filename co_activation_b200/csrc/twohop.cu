@@ -144,12 +144,16 @@ __global__ void __launch_bounds__(256)
 // Token-major forward: one warp per token.  Lane j < K holds the token's rank row
 // d_j = send_row[t, j] (first slot of each rank) and its hop-1 row s_j = fwd_src[d_j];
 // lanes with the same s_j form a group (warp ballots), the group's source row is read
-// once (UNROLL 16-byte loads per lane in flight) and stored to each of its rank rows.
-template <int K, int UNROLL>
+// once (UNROLL chunk loads per lane in flight) and stored to each of its rank rows.
+// Rows of more than 2 KB take four 32-byte chunks per lane where src and dst are 32-byte
+// aligned and H % 16 == 0 (measured on B200, hop 2 of config 3 with the two-stage
+// layout: 2,547 us with eight 16-byte chunks, 2,518 us with four 32-byte ones, 2,686 us
+// with two), else eight 16-byte chunks.
+template <int K, int UNROLL, typename V>
 __global__ void __launch_bounds__(256)
-    k_forward_tokens(const uint4 *__restrict__ src, int64_t n_src, int64_t H16,
+    k_forward_tokens(const V *__restrict__ src, int64_t n_src, int64_t Hv,
                      const int32_t *__restrict__ send_row, int64_t N,
-                     const int32_t *__restrict__ fwd_src, int64_t n_rows, uint4 *__restrict__ dst,
+                     const int32_t *__restrict__ fwd_src, int64_t n_rows, V *__restrict__ dst,
                      int32_t *__restrict__ err) {
     pdl_wait();
     pdl_trigger();
@@ -192,13 +196,13 @@ __global__ void __launch_bounds__(256)
                 drow[i] = __shfl_sync(0xffffffffu, d, l);
                 g &= g - 1;
             }
-            const uint4 *in = src + (int64_t)s0 * H16;
-            for (int64_t c0 = 0; c0 < H16; c0 += 32 * UNROLL) {
-                uint4 v[UNROLL];
+            const V *in = src + (int64_t)s0 * Hv;
+            for (int64_t c0 = 0; c0 < Hv; c0 += 32 * UNROLL) {
+                V v[UNROLL];
 #pragma unroll
                 for (int u = 0; u < UNROLL; ++u) {
                     const int64_t c = c0 + u * 32 + lane;
-                    if (c < H16) v[u] = ld_stream(in + c);
+                    if (c < Hv) v[u] = ld_chunk<V>(in + c);
                 }
 #pragma unroll
                 for (int i = 0; i < K; ++i) {
@@ -206,7 +210,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
                     for (int u = 0; u < UNROLL; ++u) {
                         const int64_t c = c0 + u * 32 + lane;
-                        if (c < H16) st_stream(dst + drow[i] * H16 + c, v[u]);
+                        if (c < Hv) st_chunk(dst + drow[i] * Hv + c, v[u]);
                     }
                 }
             }
@@ -325,12 +329,16 @@ extern "C" int forward_gather_tokens(const uint16_t *src, int64_t n_src_rows, in
 #define COACT_FWT_CASE(KK)                                                                        \
     case KK:                                                                                      \
         if (H16 <= 32)                                                                            \
-            return launch_pdl(k_forward_tokens<KK, 1>, blocks, 256, 0, st, sv, n_src_rows, H16,   \
+            return launch_pdl(k_forward_tokens<KK, 1, uint4>, blocks, 256, 0, st, sv, n_src_rows, H16,   \
                               send_row, N, fwd_src, n_rows, dv, err_flag);                        \
         if (H16 <= 128)                                                                           \
-            return launch_pdl(k_forward_tokens<KK, 4>, blocks, 256, 0, st, sv, n_src_rows, H16,   \
+            return launch_pdl(k_forward_tokens<KK, 4, uint4>, blocks, 256, 0, st, sv, n_src_rows, H16,   \
                               send_row, N, fwd_src, n_rows, dv, err_flag);                        \
-        return launch_pdl(k_forward_tokens<KK, 8>, blocks, 256, 0, st, sv, n_src_rows, H16,       \
+        if (H % 16 == 0 && aligned32(src) && aligned32(dst))                                     \
+            return launch_pdl(k_forward_tokens<KK, 4, Row32>, blocks, 256, 0, st,                 \
+                              reinterpret_cast<const Row32 *>(src), n_src_rows, H / 16, send_row, \
+                              N, fwd_src, n_rows, reinterpret_cast<Row32 *>(dst), err_flag);      \
+        return launch_pdl(k_forward_tokens<KK, 8, uint4>, blocks, 256, 0, st, sv, n_src_rows, H16, \
                           send_row, N, fwd_src, n_rows, dv, err_flag);
     switch (k) {
         COACT_FWT_CASE(1)
