@@ -470,9 +470,10 @@ def row_meta(plan_: dict, ids, gates, slot_base=None, n_rows=None):
     n = plan_["D"] if n_rows is None else int(n_rows)
     ro = _c(plan_["rank_offsets"], np.int32)
     sb = None if slot_base is None else _c(slot_base, np.int32)
-    ex = np.zeros((n, k), np.int32)
-    go = np.zeros((n, k), np.float32)
-    sl = np.zeros((n, k), np.int32)
+    # sentinels, so that every entry must be written by the C code
+    ex = np.full((n, k), -7, np.int32)
+    go = np.full((n, k), np.nan, np.float32)
+    sl = np.full((n, k), -7, np.int32)
     f = _get().oracle_row_meta(_p(_c(plan_["row_token"], np.int32)),
                                _p(_c(plan_["row_kmask"], np.uint8)), n, _p(ro), len(ro) - 1,
                                _p(ids), _p(g), _p(_c(plan_["comb_row"], np.int32)), N, k, _p(sb),
@@ -487,6 +488,6 @@ def gather_row_slots(vals, send_row, row_kmask):
     sr = _c(send_row, np.int32)
     km = _c(row_kmask, np.uint8)
     N, k = sr.shape
-    out = np.zeros((N, k), np.float32)
+    out = np.full((N, k), np.nan, np.float32)     # every entry must be written by the C code
     f = _get().oracle_gather_row_slots(_p(v), v.shape[0], _p(sr), _p(km), N, k, _p(out))
     return out, f
