@@ -1358,6 +1358,92 @@ def run_reference(args):
     }))
 
 
+def run_hbm_mix(args):
+    """What this GPU's HBM delivers per read/write mix, the context of the roofline
+    fractions: the gather over synthetic contiguous destinations at fan-out f (f rows
+    written per row read, f/(1+f) of the bytes written) and the combine over synthetic
+    expert rows at k rows per output row (k/(1+k) read), in contiguous and in seeded random
+    row order, beside torch's copy_ and full-tensor sum.  H = 7,168 (config 3's rows),
+    ~MIX_GB per launch, L2 flushed between launches, CUDA events; one GPU, one JSON line."""
+    import co_activation_b200 as coact
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    reps = max(5, min(args.steps, 20))
+    total = args.mix_gb * 1e9
+    H = 7168
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            flush_buf.zero_()
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush_buf.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) / 1e3)
+        return statistics.mean(ts)
+
+    res = {}
+    clk = ClockSampler(0)
+    clk.start()
+    n = int(total // 4)
+    a = torch.empty(n, dtype=torch.bfloat16, device=dev).normal_()
+    b = torch.empty_like(a)
+    res["torch_copy"] = {"write_share": 0.5, "GBps": 4 * n / timed(lambda: b.copy_(a)) / 1e9}
+    del b
+    s = torch.empty((), dtype=torch.int64, device=dev)
+    res["torch_sum"] = {"write_share": 0.0,
+                        "GBps": 2 * n / timed(lambda: torch.sum(a.view(torch.int64), dim=0,
+                                                                out=s)) / 1e9}
+    del a
+    torch.cuda.empty_cache()
+    gen = torch.Generator(device=dev)
+    for f in (1, 2, 4, 8):
+        N = int(total / ((1 + f) * H * 2))
+        x = torch.empty((N, H), dtype=torch.bfloat16, device=dev).normal_()
+        send_row = (torch.arange(f, dtype=torch.int32, device=dev)[None, :] * N
+                    + torch.arange(N, dtype=torch.int32, device=dev)[:, None]).contiguous()
+        send = torch.empty((N * f, H), dtype=torch.bfloat16, device=dev)
+        byt = (N + N * f) * H * 2 + N * f * 4
+        res[f"gather_fanout{f}"] = {"write_share": round(N * f * H * 2 / byt, 4),
+                                    "GBps": byt / timed(lambda: coact.dispatch_gather(
+                                        x, send_row, send)) / 1e9}
+        del x, send_row, send
+        torch.cuda.empty_cache()
+    for k in (1, 2, 4, 8):
+        N = int(total / ((k + 1) * H * 2))
+        y = torch.empty((N * k, H), dtype=torch.bfloat16, device=dev).normal_()
+        g = torch.rand((N, k), dtype=torch.float32, device=dev)
+        out = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
+        byt = N * k * H * 2 + N * H * 2 + N * k * 8
+        share = round(N * H * 2 / byt, 4)
+        rows = torch.arange(N * k, dtype=torch.int32, device=dev).view(N, k).contiguous()
+        res[f"combine_k{k}"] = {"write_share": share,
+                                "GBps": byt / timed(lambda: coact.combine_scatter(
+                                    y, g, rows, out)) / 1e9}
+        gen.manual_seed(args.seed + k)
+        rows = torch.randperm(N * k, device=dev, generator=gen).to(torch.int32).view(N, k)
+        res[f"combine_k{k}_random_rows"] = {"write_share": share,
+                                            "GBps": byt / timed(lambda: coact.combine_scatter(
+                                                y, g, rows, out)) / 1e9}
+        del y, g, out, rows
+        torch.cuda.empty_cache()
+    clocks = clk.stop()
+    peak, kind = peaks()
+    for v in res.values():
+        v["GBps"] = round(v["GBps"], 1)
+        v["frac_of_copy_peak"] = round(v["GBps"] / peak, 4)
+    print(json.dumps({"hbm_mix": res, "unit": "GB/s", "H": H, "bytes_per_launch": total,
+                      "reps": reps, "warmup": args.warmup, "copy_peak": peak,
+                      "copy_peak_kind": kind, "clocks": clocks}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -1404,10 +1490,17 @@ def main():
                          "(node co-location from the batch's counts, outside the step)")
     ap.add_argument("--two-hop", action="store_true",
                     help="dispatch in two hops: to nodes, then inside the node to ranks")
+    ap.add_argument("--hbm-mix", action="store_true",
+                    help="instead of the step: what the HBM delivers per read/write mix (the "
+                         "gather at fan-out 1-8, the combine at k = 1-8, torch copy and sum)")
+    ap.add_argument("--mix-gb", type=float, default=16.0,
+                    help="--hbm-mix: bytes moved per launch, in GB")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.hbm_mix:
+        run_hbm_mix(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)
