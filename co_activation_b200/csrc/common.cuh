@@ -141,7 +141,8 @@ __device__ __forceinline__ void raise_flag_warp(int32_t *err, int bits) {
 // kernel of the same call starts, every kernel before it has completed: such a kernel
 // may read the call's inputs before waiting.  The first kernel of a call reads no
 // global memory before pdl_wait() (it may warm L2 with prefetch_l2_bulk, which reads
-// nothing into the program), so the last kernel of a call may trigger early.
+// nothing into the program).  The last kernel of plan_dispatch triggers nothing: its
+// successor launches when it completes (see k_plan_scatter).
 __device__ __forceinline__ void pdl_wait() {
 #if !defined(COACT_NO_PDL)
     asm volatile("griddepcontrol.wait;" ::: "memory");

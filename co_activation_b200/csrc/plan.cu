@@ -9,17 +9,21 @@
 // with two bounded grid barriers was measured on B200: slower on N = 16K tokens, 6 us
 // faster on 64-128K, so it was dropped):
 //  1. k_plan_tiles   one thread per token, 256-token tiles: per-token rank mask, per-tile
-//                    per-rank row and assignment counts (warp ballots / redux, no
-//                    atomics) and per-tile statistics partials.
+//                    per-rank row and assignment counts (per-warp bit planes of the
+//                    tokens' rank counts, transposed across the warp; no atomics) and
+//                    per-tile statistics partials.
 //  2. k_plan_scan    R + 1 blocks: block r turns rank r's per-tile counts into exclusive
 //                    per-tile bases (in place) and a total; the last block reduces the
 //                    statistics partials and clears src_dst.
 //     (skipped when R * n_tiles <= COACT_PLAN_SMALL_MAX: k_plan_scatter<SMALL> then sums
 //     the per-tile counts itself, which costs less than a launch at these sizes)
 //  3. k_plan_scatter one thread per token again: rank offsets from the totals, stable
-//                    in-tile positions from per-rank ballots (rows) and 4-bit ballot
-//                    prefix sums (assignments), then row_token / row_kmask / send_row /
-//                    comb_row / rank_mask, and the src x dst split matrix.
+//                    in-tile positions from the same transposed bit planes (popcounts
+//                    of the lane sets below this lane: rows, and count bits weighted by
+//                    2^q: assignments), then row_token / row_kmask / send_row /
+//                    comb_row / rank_mask, and the src x dst split matrix.  It does its
+//                    in-tile work before waiting on its predecessor, and triggers no
+//                    early launch of its own successor.
 // Positions depend only on token order, so every output is deterministic.
 #include <algorithm>
 
@@ -36,9 +40,6 @@ constexpr int kTile = COACT_PLAN_TILE;     // experiment builds (a multiple of 3
 constexpr int kTile = 256;                 // tokens per tile, one per thread
 #endif
 constexpr int kTileWarps = kTile / 32;
-#ifndef COACT_PLAN_EARLY_TRIGGER
-#define COACT_PLAN_EARLY_TRIGGER 1  // k_plan_scatter lets the next call's kernel launch at once
-#endif
 constexpr int kScanThreads = 1024;
 constexpr int kStatSlots = 6;              // per-tile partials (see TileStat)
 enum TileStat { TS_REMOTE_ROWS, TS_XNODE_ROWS, TS_NODE_ROWS, TS_LOCAL_ASG, TS_XNODE_ASG, TS_VALID_ASG };
@@ -115,14 +116,92 @@ __device__ __forceinline__ void load_nodes(int nd, int R, int n_nodes, int *s_no
     __syncthreads();
 }
 
-// Warp-uniform OR of a 64-bit mask.
-__device__ __forceinline__ unsigned long long warp_or64(unsigned long long m) {
-    const unsigned lo = __reduce_or_sync(0xffffffffu, (unsigned)m);
-    const unsigned hi = __reduce_or_sync(0xffffffffu, (unsigned)(m >> 32));
-    return ((unsigned long long)hi << 32) | lo;
+// ---- per-warp rank tables by bit planes
+//
+// A warp holds 32 tokens, one per lane, each with its K slot ranks.  Every per-rank count
+// the planner needs -- rows (lanes holding rank r), assignments (slots on rank r), and
+// their exclusive prefixes over the lanes -- comes from one table: for rank r and bit q,
+// the set of lanes whose slot count c_r has bit q set.  Each lane first writes its own
+// counts as NP bit planes over the ranks (bit r of plane q = bit q of c_r, NW 32-bit words
+// for R <= 32 * NW), then a warp bit-matrix transpose per plane word turns them into the
+// per-rank lane sets, held by lane r % 32.  The cost is independent of how many ranks the
+// warp touches (a loop over the ranks, with a ballot per rank and count bit, costs ~75
+// instructions per rank: ~4,600 per warp at R = 64, k = 8).
+
+// Bits needed to hold a count of 0..K.
+template <int K>
+constexpr int plane_bits() { return K >= 8 ? 4 : K >= 4 ? 3 : K >= 2 ? 2 : 1; }
+
+// This lane's per-rank slot counts as bit planes: bit (r & 31) of p[q][r >> 5] is bit q
+// of #{j : rk[j] == r}.  All zero when !ok.
+// Built by adding one-hot rank vectors with a ripple carry through the planes (the count
+// never exceeds K < 2^NP, so the last carry is always zero).
+template <int K, int NW>
+__device__ __forceinline__ void count_planes(const int (&rk)[K], bool ok,
+                                             uint32_t (&p)[plane_bits<K>()][NW]) {
+    constexpr int NP = plane_bits<K>();
+#pragma unroll
+    for (int q = 0; q < NP; ++q)
+#pragma unroll
+        for (int w = 0; w < NW; ++w) p[q][w] = 0;
+    if (!ok) return;
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            uint32_t carry = (rk[j] >> 5) == w ? 1u << (rk[j] & 31) : 0u;
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+                const uint32_t c = p[q][w] & carry;
+                p[q][w] ^= carry;
+                carry = c;
+            }
+        }
+    }
 }
 
-template <int K>
+// 32 x 32 bit-matrix transpose across the warp: lane i passes row i (bit j = entry (i, j))
+// and gets back column i (bit j = entry (j, i)).  Each of the five butterfly steps swaps
+// the two off-diagonal s x s blocks inside every 2s x 2s block (an exchange with lane
+// i ^ s); together they swap the row and column index bits.
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
+    constexpr uint32_t kHi[5] = {0xFFFF0000u, 0xFF00FF00u, 0xF0F0F0F0u, 0xCCCCCCCCu, 0xAAAAAAAAu};
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+        const int s = 16 >> i;
+        const uint32_t hi = kHi[i];
+        const uint32_t y = __shfl_xor_sync(0xffffffffu, x, s);
+        x = (lane & s) ? ((x & hi) | ((y & hi) >> s)) : ((x & ~hi) | ((y & ~hi) << s));
+    }
+    return x;
+}
+
+// Count planes -> per-rank lane sets in place: afterwards p[q][w] on lane l is the set of
+// lanes whose count of rank 32*w + l has bit q set.
+template <int K, int NW>
+__device__ __forceinline__ void transpose_planes(uint32_t (&p)[plane_bits<K>()][NW], int lane) {
+#pragma unroll
+    for (int q = 0; q < plane_bits<K>(); ++q)
+#pragma unroll
+        for (int w = 0; w < NW; ++w) p[q][w] = warp_transpose32(p[q][w], lane);
+}
+
+// From the lane sets of rank 32*w + lane: the warp's rows on it (lanes holding it) and
+// assignments on it (the sum of the lanes' counts).
+template <int K, int NW>
+__device__ __forceinline__ void rank_totals(const uint32_t (&p)[plane_bits<K>()][NW], int w,
+                                            uint32_t &lanes, int &rows, int &asg) {
+    lanes = 0;
+    asg = 0;
+#pragma unroll
+    for (int q = 0; q < plane_bits<K>(); ++q) {
+        lanes |= p[q][w];
+        asg += __popc(p[q][w]) << q;
+    }
+    rows = __popc(lanes);
+}
+
+template <int K, int NW>
 __global__ void __launch_bounds__(kTile)
     k_plan_tiles(const int32_t *__restrict__ ids, int64_t N, int E,
                  const int32_t *__restrict__ expert_rank, const int32_t *__restrict__ slot_rank,
@@ -137,10 +216,6 @@ __global__ void __launch_bounds__(kTile)
     __shared__ long long s_stat[kTileWarps][kStatSlots];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    for (int i = tid; i < kTileWarps * 64; i += kTile) {
-        (&s_wrows[0][0])[i] = 0;
-        (&s_wasg[0][0])[i] = 0;
-    }
     pdl_wait();
     pdl_trigger();
     if (src_dst && blockIdx.x == 0)   // cleared here; the scatter kernel accumulates into it
@@ -175,19 +250,20 @@ __global__ void __launch_bounds__(kTile)
         st[TS_NODE_ROWS] = __popcll(nmask & ~(1ull << nsrc));
         st[TS_VALID_ASG] = K;
     }
-    // per-rank counts of this warp: rows = lanes holding the rank, asg = slots on it
-    unsigned long long wmask = warp_or64(mask);
-    while (wmask) {
-        const int r = __ffsll(wmask) - 1;
-        wmask &= wmask - 1;
-        int c = 0;
+    // per-rank counts of this warp (every rank < R written): rows = lanes holding the
+    // rank, asg = slots on it; lane l holds ranks l and 32 + l
+    uint32_t pl[plane_bits<K>()][NW];
+    count_planes<K, NW>(rk, ok, pl);
+    transpose_planes<K, NW>(pl, lane);
 #pragma unroll
-        for (int j = 0; j < K; ++j) c += ok && rk[j] == r;
-        const unsigned b = __ballot_sync(0xffffffffu, c > 0);
-        const int a = __reduce_add_sync(0xffffffffu, c);
-        if (lane == 0) {
-            s_wrows[warp][r] = __popc(b);
-            s_wasg[warp][r] = a;
+    for (int w = 0; w < NW; ++w) {
+        const int r = 32 * w + lane;
+        uint32_t lanes;
+        int rows, asg;
+        rank_totals<K, NW>(pl, w, lanes, rows, asg);
+        if (r < R) {
+            s_wrows[warp][r] = rows;
+            s_wasg[warp][r] = asg;
         }
     }
 #pragma unroll
@@ -352,7 +428,7 @@ __device__ __forceinline__ void rank_bases(int R, int tile, const int *tot_row,
 // counts have been scanned in place by k_plan_scan and ws.tot holds the totals.
 // Everything before pdl_wait() reads only this call's inputs (safe: the predecessor is
 // this call's own k_plan_tiles or k_plan_scan, see pdl_wait).
-template <int K, bool SMALL>
+template <int K, bool SMALL, int NW>
 __global__ void __launch_bounds__(kTile)
     k_plan_scatter(const int32_t *__restrict__ ids, int64_t N, int E,
                    const int32_t *__restrict__ expert_rank, const int32_t *__restrict__ slot_rank,
@@ -367,22 +443,20 @@ __global__ void __launch_bounds__(kTile)
     __shared__ int s_rbase[64], s_abase[64];
     __shared__ int s_wrows[kTileWarps][64];
     __shared__ int s_wasg[kTileWarps][64];
+    __shared__ uint32_t s_lanes[kTileWarps][plane_bits<K>()][32 * NW];  // per-warp lane sets
+    __shared__ uint32_t s_pre[(K + 1) / 2][kTile];  // per-slot in-warp prefixes, 16 bits each
     __shared__ int s_tot[2][64], s_before[2][64];
     __shared__ long long s_stat[kTileWarps][kStatSlots];
     extern __shared__ int s_sd[];  // [R*R] when src_dst != NULL
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tile = blockIdx.x;
-#if COACT_PLAN_EARLY_TRIGGER
-    // The last kernel of the call: the next call's first kernel reads nothing before its
-    // own wait, so it may launch now (the dispatch gather then warms L2 with x while the
-    // plan finishes).
-    pdl_trigger();
-#endif
-    for (int i = tid; i < kTileWarps * 64; i += kTile) {
-        (&s_wrows[0][0])[i] = 0;
-        (&s_wasg[0][0])[i] = 0;
-    }
+    // The last kernel of the call does not trigger its dependents: they launch when it
+    // completes.  Launched earlier, the next kernel's CTAs (the dispatch gather) would
+    // share SMs with this kernel's blocks and inherit the shared-memory carveout chosen
+    // for them (~164 KB of 228 at R = 64) for as long as they keep those SMs busy -- the
+    // whole gather -- and the gather's 32-byte loads in flight need the L1 capacity
+    // (config 3 on B200: the step took 4.47 ms instead of 4.06).
     if (src_dst)
         for (int i = tid; i < R * R; i += kTile) s_sd[i] = 0;
     __syncthreads();
@@ -401,42 +475,64 @@ __global__ void __launch_bounds__(kTile)
     }
     // lanes with the same home rank, for the src x dst split counts
     const unsigned same_src = __match_any_sync(0xffffffffu, ok ? src : -1);
-    const bool src_leader = ok && lane == __ffs(same_src) - 1;
 
-    // per slot: in-warp row prefix (< 32) | in-warp assignment prefix (< 256) << 8
-    int pre[K];
+    // per-rank lane sets of this warp (lane l: ranks l and 32 + l), per-warp totals (every
+    // rank < R written) and the sets themselves for the per-slot prefixes below
+    uint32_t pl[plane_bits<K>()][NW];
+    count_planes<K, NW>(rk, ok, pl);
+    transpose_planes<K, NW>(pl, lane);
+    uint32_t holders[NW];
 #pragma unroll
-    for (int j = 0; j < K; ++j) pre[j] = 0;
+    for (int w = 0; w < NW; ++w) {
+        const int r = 32 * w + lane;
+        int rows, asg;
+        rank_totals<K, NW>(pl, w, holders[w], rows, asg);
+        if (r < R) {
+            s_wrows[warp][r] = rows;
+            s_wasg[warp][r] = asg;
+        }
+#pragma unroll
+        for (int q = 0; q < plane_bits<K>(); ++q) s_lanes[warp][q][r] = pl[q][w];
+    }
+    // src x dst split counts: for each group of valid lanes sharing a home rank (usually
+    // one per warp), its rows per destination rank
+    if (src_dst) {
+        unsigned rest = __ballot_sync(0xffffffffu, ok);
+        while (rest) {
+            const int leader = __ffs(rest) - 1;
+            const unsigned grp = __shfl_sync(0xffffffffu, same_src, leader);
+            const int s = __shfl_sync(0xffffffffu, src, leader);
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const int r = 32 * w + lane;
+                const int n = __popc(holders[w] & grp);
+                if (r < R && n) atomicAdd(&s_sd[s * R + r], n);
+            }
+            rest &= ~grp;
+        }
+    }
+    __syncwarp();
+    // per slot, 16 bits (two slots a word, kept in shared memory across the wait below):
+    // in-warp row prefix (< 32) | in-warp assignment prefix (< 256) << 8, from the lanes
+    // below this one in the lane sets of the slot's rank
     const unsigned lt = lanemask_lt();
-    unsigned long long wmask = warp_or64(mask);
-    while (wmask) {
-        const int r = __ffsll(wmask) - 1;
-        wmask &= wmask - 1;
-        int c = 0;
 #pragma unroll
-        for (int j = 0; j < K; ++j) c += ok && rk[j] == r;
-        const unsigned b = __ballot_sync(0xffffffffu, c > 0);
-        // exclusive prefix of c (0..K <= 8, four bits) over the lanes via bit ballots
-        int ap = 0, at = 0;
+    for (int j2 = 0; j2 < (K + 1) / 2; ++j2) {
+        uint32_t packed = 0;
 #pragma unroll
-        for (int bit = 0; bit < 4; ++bit) {
-            if ((K >> bit) == 0) break;
-            const unsigned bb = __ballot_sync(0xffffffffu, (c >> bit) & 1);
-            ap += __popc(bb & lt) << bit;
-            at += __popc(bb) << bit;
-        }
-        const int packed = __popc(b & lt) | (ap << 8);
+        for (int h = 0; h < 2 && 2 * j2 + h < K; ++h) {
+            const int r = ok ? rk[2 * j2 + h] : 0;
+            uint32_t below = 0;
+            int ap = 0;
 #pragma unroll
-        for (int j = 0; j < K; ++j)
-            if (ok && rk[j] == r) pre[j] = packed;
-        if (lane == 0) {
-            s_wrows[warp][r] = __popc(b);
-            s_wasg[warp][r] = at;
+            for (int q = 0; q < plane_bits<K>(); ++q) {
+                const uint32_t m = s_lanes[warp][q][r] & lt;
+                below |= m;
+                ap += __popc(m) << q;
+            }
+            packed |= (uint32_t)(__popc(below) | (ap << 8)) << (16 * h);
         }
-        if (src_dst && src_leader) {
-            const int n = __popc(b & same_src);
-            if (n) atomicAdd(&s_sd[src * R + r], n);
-        }
+        s_pre[j2][tid] = packed;
     }
     __syncthreads();
     if (tid < R) {
@@ -453,9 +549,6 @@ __global__ void __launch_bounds__(kTile)
 
     // ---- cross-tile bases: need the predecessor's results
     pdl_wait();
-#if !COACT_PLAN_EARLY_TRIGGER
-    pdl_trigger();
-#endif
     if (SMALL) {
         // rank r's row and assignment counts read together (one round trip), then reduced
         for (int r = warp; r < R; r += kTileWarps) {
@@ -533,10 +626,11 @@ __global__ void __launch_bounds__(kTile)
 #pragma unroll
                 for (int jj = 0; jj < K; ++jj) km |= (unsigned)(rk[jj] == r) << jj;
                 const unsigned below = km & ((1u << j) - 1);
-                comb_row[t * K + j] = s_abase[r] + s_wasg[warp][r] + (pre[j] >> 8) + __popc(below);
+                const uint32_t pj = (s_pre[j / 2][tid] >> (16 * (j % 2))) & 0xffffu;
+                comb_row[t * K + j] = s_abase[r] + s_wasg[warp][r] + (int)(pj >> 8) + __popc(below);
                 int sr = -1;
                 if (below == 0) {
-                    const int64_t row = (int64_t)s_rbase[r] + s_wrows[warp][r] + (pre[j] & 0xff);
+                    const int64_t row = (int64_t)s_rbase[r] + s_wrows[warp][r] + (int)(pj & 0xff);
                     if (row < cap) {
                         row_token[row] = (int32_t)t;
                         row_kmask[row] = (uint8_t)km;
@@ -563,7 +657,7 @@ __global__ void __launch_bounds__(kTile)
 #define COACT_PLAN_SMALL_MAX 4096  // R * n_tiles up to which the scan kernel is skipped
 #endif
 
-template <int K>
+template <int K, int NW>
 int launch_plan(const int32_t *ids, int64_t N, int E, const int32_t *expert_rank,
                 const int32_t *slot_rank, int R,
                 const int32_t *rank_node, int n_nodes, const int32_t *src_rank,
@@ -576,25 +670,40 @@ int launch_plan(const int32_t *ids, int64_t N, int E, const int32_t *expert_rank
     const size_t sd_smem = src_dst ? sizeof(int) * R * R : 0;
     auto *rm = reinterpret_cast<unsigned long long *>(rank_mask);
     if (n_tiles > 0 && (int64_t)R * n_tiles <= COACT_PLAN_SMALL_MAX) {
-        if (int s = launch_pdl(k_plan_tiles<K>, n_tiles, kTile, 0, st, ids, N, E, expert_rank, slot_rank, R,
+        if (int s = launch_pdl(k_plan_tiles<K, NW>, n_tiles, kTile, 0, st, ids, N, E, expert_rank, slot_rank, R,
                                rank_node, n_nodes, src_rank, n_tiles, ws, src_dst, err))
             return s;
-        return launch_pdl(k_plan_scatter<K, true>, n_tiles, kTile, sd_smem, st, ids, N, E,
+        return launch_pdl(k_plan_scatter<K, true, NW>, n_tiles, kTile, sd_smem, st, ids, N, E,
                           expert_rank, slot_rank, R, src_rank, n_tiles, ws, rank_counts, rank_offsets,
                           asg_offsets, rm, row_token, row_kmask, cap, send_row, comb_row, stats,
                           src_dst, err);
     }
     if (n_tiles > 0)
-        if (int s = launch_pdl(k_plan_tiles<K>, n_tiles, kTile, 0, st, ids, N, E, expert_rank, slot_rank, R,
+        if (int s = launch_pdl(k_plan_tiles<K, NW>, n_tiles, kTile, 0, st, ids, N, E, expert_rank, slot_rank, R,
                                rank_node, n_nodes, src_rank, n_tiles, ws, src_dst, err))
             return s;
     if (int s = launch_pdl(k_plan_scan, R + 1, kScanThreads, 0, st, N, K, R, n_tiles, ws, stats,
                            n_tiles > 0 ? nullptr : src_dst))
         return s;
-    return launch_pdl(k_plan_scatter<K, false>, std::max(n_tiles, 1), kTile, sd_smem, st, ids, N,
+    return launch_pdl(k_plan_scatter<K, false, NW>, std::max(n_tiles, 1), kTile, sd_smem, st, ids, N,
                       E, expert_rank, slot_rank, R, src_rank, n_tiles, ws, rank_counts, rank_offsets,
                       asg_offsets, rm, row_token, row_kmask, cap, send_row, comb_row, stats,
                       src_dst, err);
+}
+
+// R <= 32: one 32-bit word per bit plane; R <= 64: two.
+template <int K>
+int launch_plan_any(const int32_t *ids, int64_t N, int E, const int32_t *expert_rank,
+                    const int32_t *slot_rank, int R, const int32_t *rank_node, int n_nodes,
+                    const int32_t *src_rank, int32_t *rank_counts, int32_t *rank_offsets,
+                    int32_t *asg_offsets, uint64_t *rank_mask, int32_t *row_token,
+                    uint8_t *row_kmask, int64_t cap, int32_t *send_row, int32_t *comb_row,
+                    int64_t *stats, int32_t *src_dst, const Workspace &ws, int32_t *err,
+                    cudaStream_t st, const DeviceInfo &di) {
+    auto *run = R > 32 ? launch_plan<K, 2> : launch_plan<K, 1>;
+    return run(ids, N, E, expert_rank, slot_rank, R, rank_node, n_nodes, src_rank, rank_counts,
+               rank_offsets, asg_offsets, rank_mask, row_token, row_kmask, cap, send_row,
+               comb_row, stats, src_dst, ws, err, st, di);
 }
 
 }  // namespace
@@ -640,7 +749,7 @@ int plan_entry(const int32_t *ids, int64_t N, int k, int E, const int32_t *exper
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 #define COACT_PLAN_CASE(KK)                                                                        \
     case KK:                                                                                       \
-        return launch_plan<KK>(ids, N, E, expert_rank, slot_rank, R, rank_node, n_nodes, src_rank, \
+        return launch_plan_any<KK>(ids, N, E, expert_rank, slot_rank, R, rank_node, n_nodes, src_rank, \
                                rank_counts, rank_offsets, asg_offsets, rank_mask, row_token,       \
                                row_kmask, row_capacity, send_row, comb_row, stats, src_dst, ws,    \
                                err_flag, st, di);
@@ -770,7 +879,7 @@ extern "C" int plan_dispatch_noalloc(const int32_t *ids, int64_t N, int k, int E
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 #define COACT_PLAN_NOALLOC_CASE(KK)                                                                \
     case KK:                                                                                       \
-        return launch_plan<KK>(ids, N, E, expert_rank, nullptr, R, rank_node, n_nodes, src_rank,   \
+        return launch_plan_any<KK>(ids, N, E, expert_rank, nullptr, R, rank_node, n_nodes, src_rank,   \
                                rank_counts, rank_offsets, asg_offsets, rank_mask, row_token,       \
                                row_kmask, row_capacity, send_row, comb_row, stats, src_dst, ws,    \
                                err_flag, st, di);

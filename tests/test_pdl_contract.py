@@ -7,8 +7,9 @@ its predecessor on the stream has finished.  Correctness rests on two rules:
     atomics -- except k_plan_scatter, the second kernel of plan_dispatch, which reads the
     call's own inputs (its predecessor is the call's own k_plan_tiles / k_plan_scan);
     an L2 prefetch (prefetch_l2_bulk) is allowed anywhere, it reads nothing in;
-  * a kernel triggers its dependents only after its own pdl_wait(), except the last
-    kernel of a call whose successors obey the first rule (k_plan_scatter).
+  * a kernel triggers its dependents only after its own pdl_wait(); k_plan_scatter, the
+    last kernel of plan_dispatch, triggers nothing (its successor, usually the dispatch
+    gather, launches when it completes, on SMs free of the scatter's blocks).
 """
 import os
 import re
@@ -16,7 +17,7 @@ import re
 import pytest
 
 CSRC = os.path.join(os.path.dirname(__file__), "..", "co_activation_b200", "csrc")
-EARLY_TRIGGER_OK = {"k_plan_scatter"}
+NO_TRIGGER = {"k_plan_scatter"}
 PRE_WAIT_READS_OK = {"k_plan_scatter"}
 GLOBAL_ACCESS = re.compile(r"__ldg\(|ld_stream\(|st_stream\(|__stcs\(|atomic[A-Z][a-z]+\(|"
                            r"cp\.async\.bulk\.(?!prefetch)|\bld\.global|\bst\.global")
@@ -59,8 +60,10 @@ def test_wait_then_trigger(fn, name, body):
     waits = [m.start() for m in re.finditer(r"\bpdl_wait\(\);", body)]
     trigs = [m.start() for m in re.finditer(r"\bpdl_trigger\(\);", body)]
     assert len(waits) == 1, f"{fn}:{name} waits {len(waits)} times"
-    assert trigs, f"{fn}:{name} never triggers its dependents"
-    if name not in EARLY_TRIGGER_OK:
+    if name in NO_TRIGGER:
+        assert not trigs, f"{fn}:{name} triggers its dependents"
+    else:
+        assert trigs, f"{fn}:{name} never triggers its dependents"
         assert min(trigs) > waits[0], f"{fn}:{name} triggers before its wait"
     pre = body[:waits[0]]
     if name not in PRE_WAIT_READS_OK:
@@ -68,8 +71,10 @@ def test_wait_then_trigger(fn, name, body):
         assert hit is None, f"{fn}:{name} touches global memory before its wait: {hit.group(0)}"
 
 
-def test_early_trigger_only_in_last_kernel_of_plan():
-    """k_plan_scatter is the last launch of plan_dispatch (and of its variants)."""
+def test_scatter_is_last_kernel_of_plan():
+    """k_plan_scatter, which reads its call's inputs before its wait, is the last launch of
+    plan_dispatch (and of its variants): every kernel before it in the call triggers only
+    after its own wait, so when it starts, everything before the call has completed."""
     src = open(os.path.join(CSRC, "plan.cu")).read()
     body = src[src.index("int launch_plan("):]
     body = body[:body.index("\n}\n")]
