@@ -245,6 +245,11 @@ int grid_for(void (*kernel)(KArgs...), int64_t units, int per_sm, const DeviceIn
 template <typename... KArgs, typename... Args>
 int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                Args &&...args) {
+#if defined(COACT_CARVEOUT)   // experiment builds: preferred shared-memory carveout, percent
+    if (cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                             COACT_CARVEOUT))
+        return cuda_fail(e);
+#endif
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;

@@ -21,8 +21,9 @@
  *    and waits for it (griddepcontrol.wait) before touching its outputs.  Work that the
  *    caller enqueues normally after a call sees all of that call's results.  A kernel
  *    of the caller's own that is launched with programmatic stream serialisation right
- *    after a call must likewise wait before reading that call's outputs: the last kernel
- *    of plan_dispatch lets such a successor start while the plan is still running.
+ *    after a call must likewise wait before reading that call's outputs: a library
+ *    kernel lets its successor start once its own wait has returned, before it finishes
+ *    (the last kernel of plan_dispatch excepted: its successor starts when it completes).
  *  - Return value: COACT_OK (0) or a negative coact_status.  A negative status is
  *    decided on the host before anything is enqueued (except COACT_ERR_CUDA, which
  *    reports a failed launch).
@@ -264,6 +265,12 @@ int dispatch_gather_tma(const uint16_t *x, int64_t N, int64_t H,
  * plan); gates: fp32 [N, k]; comb_row: int32 [N, k]; out: [N, H] of bf16 (out_dtype 0)
  * or fp32 (out_dtype 1).  A comb_row entry outside [0, n_rows) is skipped: -1 silently
  * (a slot of an invalid token), any other value with COACT_EFLAG_ROW_RANGE.
+ * Rate: bound by HBM reads, with the loads in flight staged in each SM's L1 data cache,
+ * so it runs at full rate only where the L1 is not given over to shared memory.  Its
+ * CTAs take whatever shared-memory carveout an SM already has when they start beside
+ * another kernel's blocks (after a predecessor that triggers its dependents early, or on
+ * another stream): on B200 the combine of 131,072 tokens with k = 8 and H = 7168 took
+ * 3.0 ms instead of 2.4 under the largest carveout.
  */
 int combine_scatter(const uint16_t *y, int64_t n_rows, const float *gates,
                     const int32_t *comb_row, int64_t N, int k, int64_t H,

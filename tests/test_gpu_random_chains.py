@@ -4,11 +4,10 @@ oracle: counts, every plan output, the gathered rows and the combine.
 
 Three call orders per case:
   0  count -> plan -> gather -> combine               (the step)
-  1  plan -> combine -> gather                        (a combine right after the plan,
-                                                       whose last kernel lets it launch early)
+  1  plan -> combine -> gather                        (a combine right after the plan)
   2  plan(batch A) -> plan(batch B) -> gather -> combine   (the same plan buffers and
-                                                       workspace reused while the first
-                                                       plan's last kernel may still run)
+                                                       workspace reused by the next call
+                                                       on the stream)
 """
 import numpy as np
 import pytest
