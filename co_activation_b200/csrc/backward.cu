@@ -149,8 +149,11 @@ int launch(const uint16_t *y, int64_t n_rows, const float *gates, const int32_t 
     // loads in flight per lane: U chunks of grad_out + U x G rows of y (16-byte chunks);
     // one 32-byte chunk per row where y, grad_out and grad_y are 32-byte aligned
     constexpr int U = 2, G = 2;
+#ifndef COACT_BWD_PER_SM
+#define COACT_BWD_PER_SM 8
+#endif
     const int blocks = (int)std::max<int64_t>(
-        1, std::min<int64_t>(ceil_div(n_units, 8), (int64_t)di.sm_count * 8));
+        1, std::min<int64_t>(ceil_div(n_units, 8), (int64_t)di.sm_count * COACT_BWD_PER_SM));
     if (H % 16 == 0 && aligned32(y) && aligned32(g_out) && aligned32(g_y))
         return launch_pdl(k_combine_bwd<K, 1, G, UNITS, Row32>, blocks, 256, 0, st,
                           reinterpret_cast<const Row32 *>(y), n_rows, gates, comb_row, N,

@@ -257,6 +257,10 @@ int launch(const uint16_t *y, int64_t n_rows, const float *gates, const int32_t 
     const int blocks = grid_for(k_combine_v16<K, U, F32, uint4>, n_units, COACT_COMBINE_PER_SM, di);
     const bool wide = COACT_COMBINE_VEC == 32 && H % 16 == 0 && aligned32(y) && aligned32(out);
     if (UNITS || (SPARSE && K >= 3)) {   // sparse slots: units, or token rows with absent slots
+#ifndef COACT_UNITS_PER_SM
+#define COACT_UNITS_PER_SM COACT_COMBINE_PER_SM
+#endif
+        const int blocks = grid_for(k_combine_v16<K, U, F32, uint4>, n_units, COACT_UNITS_PER_SM, di);
         const int32_t *rt = UNITS ? row_token : nullptr;
         const uint8_t *km = UNITS ? row_kmask : nullptr;
         const int32_t *uc = UNITS ? unit_count : nullptr;

@@ -13,14 +13,16 @@
 //    aligned, else 16 bytes; 2 (resp. 4) chunks per lane in flight on long rows.  The
 //    kernel is specialised per k: a token's k destination rows are resolved once with k
 //    shuffles and the store loop is unrolled and warp-uniform (no per-chunk shuffle or
-//    data-dependent loop, which kept the MIO queue full).  A grid of 16 CTAs of 8 warps
-//    per SM (3-6 resident): the extra waves balance the tail of tokens with different
-//    fan-outs.  Measured on B200, config 3's gather in the step: 1,677 us with the
-//    earlier 16-byte kernel (one kernel for all k, 8 CTAs per SM) -> 1,591 us.  As a build
-//    option (-DCOACT_GATHER_PREFETCH_BYTES), each warp can warm L2 with the x rows it will
-//    copy first before its wait on the predecessor (bulk L2 prefetch, behind the plan whose
-//    last kernel lets this one launch at once); measured without gain on the current
-//    kernel, it is off.
+//    data-dependent loop, which kept the MIO queue full).  The grid has one warp per
+//    token up to 128 CTAs of 8 warps per SM (3-6 resident): tokens have different
+//    fan-outs, and with one token per warp the CTA scheduler balances them to the end,
+//    where a grid-stride loop over several tokens per warp leaves a tail.  Measured on
+//    B200, 131,072 tokens of 14 KB rows, k = 8 (D = 4.33 rows per token) in the step:
+//    1,677 us with the earlier 16-byte kernel (one kernel for all k, 8 CTAs per SM),
+//    1,591-1,607 us with this kernel at 16 CTAs per SM, 1,550 us with one token per warp.
+//    As a build option (-DCOACT_GATHER_PREFETCH_BYTES), each warp can warm L2 with the x
+//    rows it will copy first before its wait on the predecessor (bulk L2 prefetch); it
+//    measured without gain on the current kernel and is off.
 //  * k_gather_bulk (entry point dispatch_gather_tma) -- TMA bulk copies.  One warp per
 //    CTA; lane 0 streams rows into a ring of shared-memory stages with cp.async.bulk
 //    (global -> shared, completion on an mbarrier), then lanes j < k each issue the
@@ -302,7 +304,7 @@ int launch_bulk(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row
 int launch_v16(const uint16_t *x, int64_t N, int64_t H, const int32_t *send_row, int k,
                uint16_t *send, int64_t cap, int32_t *err, cudaStream_t st, const DeviceInfo &di) {
 #ifndef COACT_GATHER_PER_SM
-#define COACT_GATHER_PER_SM 16  // CTAs per SM in the grid (0: one resident wave)
+#define COACT_GATHER_PER_SM 128  // CTAs per SM in the grid at most (0: one resident wave)
 #endif
 #ifndef COACT_GATHER_UNROLL
 #define COACT_GATHER_UNROLL 4  // chunk loads in flight per lane on long rows
