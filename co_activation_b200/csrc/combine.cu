@@ -251,10 +251,18 @@ int launch(const uint16_t *y, int64_t n_rows, const float *gates, const int32_t 
 #ifndef COACT_COMBINE_PER_SM
 #define COACT_COMBINE_PER_SM 8  // CTAs per SM in the grid (0: one resident wave)
 #endif
+#ifndef COACT_COMBINE_PER_SM_K2
+// k <= 2: one warp per token up to 128 CTAs per SM.  Measured on B200 in the step: config
+// 4 (k = 2, 8 KB rows) both combines 495.7 -> 480.6 us, config 1 38.3 -> 37.4 us; over
+// 14 KB rows the k = 1 combine 6.25 -> 6.75 TB/s.  For k >= 3 (one CTA of 184 registers
+// resident per SM) finer grids were no faster.
+#define COACT_COMBINE_PER_SM_K2 128
+#endif
+    constexpr int kPerSm = K <= 2 ? COACT_COMBINE_PER_SM_K2 : COACT_COMBINE_PER_SM;
 #ifndef COACT_COMBINE_VEC
 #define COACT_COMBINE_VEC 32  // 256-bit chunks where y and out are 32-byte aligned (16: never)
 #endif
-    const int blocks = grid_for(k_combine_v16<K, U, F32, uint4>, n_units, COACT_COMBINE_PER_SM, di);
+    const int blocks = grid_for(k_combine_v16<K, U, F32, uint4>, n_units, kPerSm, di);
     const bool wide = COACT_COMBINE_VEC == 32 && H % 16 == 0 && aligned32(y) && aligned32(out);
     if (UNITS || (SPARSE && K >= 3)) {   // sparse slots: units, or token rows with absent slots
 #ifndef COACT_UNITS_PER_SM
@@ -285,7 +293,7 @@ int launch(const uint16_t *y, int64_t n_rows, const float *gates, const int32_t 
         constexpr int UW = (K <= 2 || K >= 7) ? 2 : 1;
 #endif
         return launch_pdl(k_combine_v16<K, UW, F32, Row32>,
-                          grid_for(k_combine_v16<K, UW, F32, Row32>, n_units, COACT_COMBINE_PER_SM, di),
+                          grid_for(k_combine_v16<K, UW, F32, Row32>, n_units, kPerSm, di),
                           256, 0, st, reinterpret_cast<const Row32 *>(y), n_rows, gates, comb_row,
                           N, H / 16, out, err);
     }
