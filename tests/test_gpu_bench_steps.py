@@ -113,3 +113,27 @@ def test_bench_two_layer_step_config4(coact, bench):
     # the point of the prediction: more layer-2 assignments served on the token's rank
     base = oracle.plan(l2.ids, E, l2.expert_rank, R, rank_node=l2.rank_node, n_nodes=c.n_nodes)
     assert p2["stats"][5] > 2 * base["stats"][5]
+
+
+def test_bench_hbm_mix_line():
+    """`bench.py --hbm-mix` (the per-mix HBM figures behind the roofline's context) runs
+    through the library's gather and combine and prints one JSON line with every mix."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    p = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--hbm-mix",
+                        "--mix-gb", "0.5", "--steps", "5", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=600, cwd=root)
+    assert p.returncode == 0, p.stderr[-2000:]
+    line = json.loads(p.stdout.strip().splitlines()[-1])
+    mix = line["hbm_mix"]
+    want = {"torch_copy", "torch_sum"} | {f"gather_fanout{f}" for f in (1, 2, 4, 8)} | \
+        {f"combine_k{k}{s}" for k in (1, 2, 4, 8) for s in ("", "_random_rows")}
+    assert set(mix) == want
+    for name, v in mix.items():
+        assert 0 <= v["write_share"] <= 0.5 or name.startswith("gather")
+        assert v["GBps"] > 500, (name, v)     # half a GB per launch still streams at TB/s
+    f8 = mix["gather_fanout8"]["write_share"]
+    assert abs(f8 - 8 / 9) < 0.01 and abs(mix["combine_k8"]["write_share"] - 1 / 9) < 0.01
