@@ -231,7 +231,16 @@ extern "C" int dispatch_gather_peer(const uint16_t *x, int64_t N, int64_t H, con
     DeviceInfo di;
     if (int s = device_info(&di)) return s;
     const int64_t H16 = H / 8;
-    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(N, 8), di.sm_count * 8));
+#ifndef COACT_PEER_PER_SM
+// CTAs per SM in the peer gather's grid at most: one warp per token up to 128 per SM, as
+// in dispatch_gather (tokens differ in fan-out).  Measured on B200 with every destination
+// buffer in the GPU's own memory, one source holding a whole batch: 131,072 tokens, k = 8,
+// 14 KB rows 2,693 -> 2,597 us; 65,536 tokens, k = 6, 8 KB rows 612 -> 587 us (8 per SM
+// with a grid-stride loop before).
+#define COACT_PEER_PER_SM 128
+#endif
+    const int blocks = (int)std::max<int64_t>(
+        1, std::min<int64_t>(ceil_div(N, 8), (int64_t)di.sm_count * COACT_PEER_PER_SM));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const uint4 *xv = reinterpret_cast<const uint4 *>(x);
     auto *b = reinterpret_cast<const unsigned long long *>(dst_bases);
