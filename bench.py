@@ -245,10 +245,11 @@ def plan_launches(R: int, N: int) -> int:
 
 
 class OneLayerStep:
-    """count (side stream, overlapped with the plan: it depends on nothing the other
-    calls produce) -> plan -> gather -> combine."""
+    """plan -> gather -> combine, with the count on a side stream beside the gather (it
+    depends on nothing the other calls produce; beside the HBM-bound gather it takes SMs
+    the copy leaves idle, where beside the latency-bound plan it slowed the plan)."""
     n_events = 5
-    phases = {"coact_count": (0, 1), "plan_dispatch": (0, 2), "dispatch_gather": (2, 3),
+    phases = {"coact_count": (2, 1), "plan_dispatch": (0, 2), "dispatch_gather": (2, 3),
               "combine_scatter": (3, 4)}
     host_inputs = ("ids", "gates", "expert_rank", "rank_node", "x", "y")
 
@@ -268,15 +269,20 @@ class OneLayerStep:
         c = OneLayerStep(coact, self.L.r, device, fill=False)
         return c
 
-    def step(self, ev=None):
-        main = torch.cuda.current_stream()
+    def count_beside(self, main, ev, i_end):
+        """The count on the side stream from this point of the main stream; ev[i_end]
+        marks its end."""
         self.side.wait_stream(main)
-        if ev: ev[0].record()
         with torch.cuda.stream(self.side):
             self.L.count()
-            if ev: ev[1].record()
+            if ev: ev[i_end].record()
+
+    def step(self, ev=None):
+        main = torch.cuda.current_stream()
+        if ev: ev[0].record()
         self.L.plan_()
         if ev: ev[2].record()
+        self.count_beside(main, ev, 1)
         self.L.gather()
         if ev: ev[3].record()
         self.L.combine()
@@ -401,13 +407,13 @@ class TwoLayerStep:
 
 
 class TwoHopStep(OneLayerStep):
-    """One layer with the two-hop dispatch (Cobalt: fewer remote nodes): count (side
-    stream) -> node-level plan + rank-level plan + forward map -> hop-1 gather into node
-    segments -> hop-2 forward into rank segments -> combine.  The forward runs in token
+    """One layer with the two-hop dispatch (Cobalt: fewer remote nodes): node-level plan +
+    rank-level plan + forward map -> hop-1 gather into node segments (count beside it on a
+    side stream) -> hop-2 forward into rank segments -> combine.  The forward runs in token
     order (forward_gather_tokens: each hop-1 row read once) unless forward = "rows"."""
     forward = "tokens"
     n_events = 6
-    phases = {"coact_count": (0, 1), "plan_two_hop": (0, 2), "gather_hop1": (2, 3),
+    phases = {"coact_count": (2, 1), "plan_two_hop": (0, 2), "gather_hop1": (2, 3),
               "forward_hop2": (3, 4), "combine_scatter": (4, 5)}
 
     def __init__(self, coact, r: workload.Routing, device, fill: bool = True):
@@ -426,14 +432,11 @@ class TwoHopStep(OneLayerStep):
     def step(self, ev=None):
         L, c = self.L, self.cfg
         main = torch.cuda.current_stream()
-        self.side.wait_stream(main)
         if ev: ev[0].record()
-        with torch.cuda.stream(self.side):
-            L.count()
-            if ev: ev[1].record()
         L.coact.plan_two_hop(L.ids, c.E, L.expert_rank, c.R, L.rank_node, c.n_nodes, self.th,
                              err_flag=L.err)
         if ev: ev[2].record()
+        self.count_beside(main, ev, 1)
         L.coact.dispatch_gather(L.x, self.th.node.send_row, self.hop1, err_flag=L.err,
                                 tma=L.tma)
         if ev: ev[3].record()
@@ -545,13 +548,16 @@ class RebalanceStep(OneLayerStep):
 
 
 class PreReducedStep(OneLayerStep):
-    """One layer with the pre-reduced reverse path: count (side stream) -> plan -> gather
-    -> combine_rows over the send rows (one bf16 partial row per (token, rank), D rows
-    instead of N*k) -> dispatch_gather_backward adds each token's partial rows."""
+    """One layer with the pre-reduced reverse path: count (side stream, beside the plan) ->
+    plan -> gather -> combine_rows over the send rows (one bf16 partial row per (token,
+    rank), D rows instead of N*k) -> dispatch_gather_backward adds each token's partial
+    rows.  Here the count stays beside the plan: run beside the gather, its shared-memory
+    carveout outlasted it on SMs the gather kept busy, and combine_rows, whose loads in
+    flight are staged in L1, lost more than the plan gained (config 3: 6,644 vs 6,622 us)."""
     n_events = 6
     phases = {"coact_count": (0, 1), "plan_dispatch": (0, 2), "dispatch_gather": (2, 3),
               "combine_rows": (3, 4), "reduce_rows": (4, 5)}
-    step_desc = ("coact_count (side stream) + plan_dispatch + dispatch_gather + combine_rows "
+    step_desc = ("coact_count (side stream, beside the plan) + plan_dispatch + dispatch_gather + combine_rows "
                  "(partial rows per send row) + dispatch_gather_backward (sum per token, bf16 out)")
 
     def __init__(self, coact, r: workload.Routing, device, fill: bool = True):
@@ -566,11 +572,8 @@ class PreReducedStep(OneLayerStep):
     def step(self, ev=None):
         L, c = self.L, self.L.coact
         main = torch.cuda.current_stream()
-        self.side.wait_stream(main)
         if ev: ev[0].record()
-        with torch.cuda.stream(self.side):
-            L.count()
-            if ev: ev[1].record()
+        self.count_beside(main, ev, 1)
         L.plan_()
         if ev: ev[2].record()
         L.gather()
@@ -593,12 +596,12 @@ class PreReducedStep(OneLayerStep):
 
 class ReplicaStep(OneLayerStep):
     """One layer over an expert layout with replicas (Cobalt: EP distributes expert
-    replicas across GPUs; task assignment routes tokens to fewer remote nodes): count
-    (side stream) -> assign_replicas -> plan over the chosen per-slot ranks -> gather ->
-    combine.  The n_hot most loaded experts of the batch have a second replica on another
-    node (workload.replicate_hot)."""
+    replicas across GPUs; task assignment routes tokens to fewer remote nodes):
+    assign_replicas -> plan over the chosen per-slot ranks -> gather (count beside it on a
+    side stream) -> combine.  The n_hot most loaded experts of the batch have a second
+    replica on another node (workload.replicate_hot)."""
     n_events = 6
-    phases = {"coact_count": (0, 1), "assign_replicas": (0, 2), "plan_dispatch": (2, 3),
+    phases = {"coact_count": (3, 1), "assign_replicas": (0, 2), "plan_dispatch": (2, 3),
               "dispatch_gather": (3, 4), "combine_scatter": (4, 5)}
 
     layout_kind = "hot"        # "hot": workload.replicate_hot; "planned": coact_place_replicas
@@ -626,8 +629,9 @@ class ReplicaStep(OneLayerStep):
         self.kernels_per_step = 1 + 1 + plan_launches(c.R, self.N) + 1 + 1
         layout = ("coact_place_replicas over the batch's counts" if self.layout_kind == "planned"
                   else "the hottest experts with a second replica on another node")
-        self.step_desc = (f"coact_count (side stream) + assign_replicas ({n_hot} replicas: {layout})"
-                          " + plan_dispatch_slots + dispatch_gather + combine_scatter (bf16 out)")
+        self.step_desc = (f"assign_replicas ({n_hot} replicas: {layout}) + plan_dispatch_slots + "
+                          "dispatch_gather (coact_count beside it, side stream) + combine_scatter "
+                          "(bf16 out)")
 
     def clone_for_copy(self, coact, device):
         return ReplicaStep(coact, self.L.r, device, self.n_hot, fill=False)
@@ -635,17 +639,14 @@ class ReplicaStep(OneLayerStep):
     def step(self, ev=None):
         L, c, cfg = self.L, self.L.coact, self.cfg
         main = torch.cuda.current_stream()
-        self.side.wait_stream(main)
         if ev: ev[0].record()
-        with torch.cuda.stream(self.side):
-            L.count()
-            if ev: ev[1].record()
         c.assign_replicas(L.ids, cfg.E, self.rep, self.nrep, cfg.R, self.slot, rank_node=L.rank_node,
                           n_nodes=cfg.n_nodes, err_flag=L.err)
         if ev: ev[2].record()
         c.plan_dispatch(L.ids, cfg.E, None, cfg.R, L.plan, rank_node=L.rank_node,
                         n_nodes=cfg.n_nodes, err_flag=L.err, slot_rank=self.slot)
         if ev: ev[3].record()
+        self.count_beside(main, ev, 1)
         L.gather()
         if ev: ev[4].record()
         L.combine()
@@ -1048,17 +1049,18 @@ def run_gpu(args):
                    "placement": placement,
                    "pass": mode,
                    "gather": ("dispatch_gather_tma (TMA bulk copies)" if LayerBuffers.tma
-                              else "dispatch_gather (16-byte vector copies)"),
+                              else "dispatch_gather (vector copies, 32-byte where aligned, one "
+                                   "warp per token)"),
                    "step": getattr(S, "step_desc", None) or ("two layers: counts + cross-layer counts + predict_home (side stream, "
                             "beside layer 1); plan, gather, combine of layer 1; plan, gather, "
                             "combine of layer 2"
                             if cfg.two_layer else
-                            "coact_count (side stream) + two-hop plan (node and rank plans, "
-                            f"forward map) + hop-1 gather + hop-2 forward ({args.forward}) + "
+                            "two-hop plan (node and rank plans, forward map) + hop-1 gather "
+                            f"(coact_count beside it, side stream) + hop-2 forward ({args.forward}) + "
                             "combine_scatter"
                             if args.two_hop else
-                            "coact_count (side stream, overlapped with plan) + plan_dispatch + "
-                            "dispatch_gather + combine_scatter (bf16 out)"),
+                            "plan_dispatch + dispatch_gather (coact_count beside it, side "
+                            "stream) + combine_scatter (bf16 out)"),
                    "l2": "flushed between timed steps (write of 2x L2, then a read of another 2x L2 "
                          "buffer so no dirty line is left), outside the step events",
                    "timing": timing,
