@@ -124,8 +124,12 @@ __global__ void __launch_bounds__(256)
 // G rows at a time, U column chunks per lane (U*G loads in flight), accumulating in that
 // order: the same fma chain as k_combine_v16, without registers and issue slots for
 // absent slots.
+// Three CTAs per SM (at most 85 registers): 79 for k = 6-8 without spills, against 128 (two
+// CTAs per SM) unbounded.  Measured on B200, combine_rows + the transposed dispatch of the
+// pre-reduced step: 65,536 tokens, k = 6: 1,011 + 542 -> 968 + 531 us; 131,072 tokens, k =
+// 8: 3,531 + 1,516 -> 3,472 + 1,474 us; 16,384 tokens, k = 2: 50.9 -> 49.9 us.
 template <int K, int U, int G, bool F32, bool UNITS, typename V>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 3)
     k_combine_units(const V *__restrict__ y, int64_t n_rows, const float *__restrict__ gates,
                     const int32_t *__restrict__ comb_row, int64_t N,
                     const int32_t *__restrict__ row_token, const uint8_t *__restrict__ row_kmask,
